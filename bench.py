@@ -1,0 +1,385 @@
+#!/usr/bin/env python3
+"""Benchmark of the S + U Vᵀ hot path on one B200 (or N independent replicas).
+
+One step = one pass of every hot-path stage over the 70B-MLP-shaped layer
+(W 28672×8192 bf16, Student-t ν=3 ×0.02, seeded):
+  1. magnitude top-k split at 5 % (CSR S + residual)        [split, unstructured]
+  2. 2:4 split (values + in-group indices + residual)        [split, structured]
+  3. pack of the 2:4 S and the rank-256 factors U, V         [pack]
+  4. prefill apply, 4096 tokens                              [apply, large batch]
+  5. decode apply, batch 1                                    [apply, batch 1]
+Inputs are resident in HBM when the timed region starts; every input of a
+stage (W 470 MB, S 264 MB, ...) is larger than the 126 MB L2, and stage 4
+writes 235 MB just before stage 5 reads S, so stage 5 streams from DRAM.
+
+`value` is the headline metric: streamed-weight GB/s of the batch-1 apply
+(algorithmic bytes = 2:4 values + metadata + U + V + x + y, per call, over its
+CUDA-event time).  The other stages are reported under "stages".  `e2e` is
+the same metric through the C ABI with host X/Y buffers (copies inside the
+timed region).  `--impl reference` times the float64 CPU oracle on a bounded
+row sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+M, N, R_RANK = 28672, 8192, 256
+T_PREFILL = 4096
+TOPK_FRAC = 0.05
+SEED = 5000
+METRIC = "S+UVᵀ apply: streamed-weight GB/s (batch 1) & TFLOP/s (prefill) vs roofline"
+WORKLOAD = "mlp_70b_28672x8192_bf16_2to4_r256"
+
+
+def decode_bytes(m=M, n=N, r=R_RANK, batch=1) -> int:
+    vals = m * (n // 2) * 2
+    meta = m * (n // 4) // 2          # 4 bits per group of four
+    uv = (m + n) * r * 2
+    return vals + meta + uv + batch * (n + m) * 2
+
+
+def prefill_flops(m=M, n=N, r=R_RANK, t=T_PREFILL) -> int:
+    return 2 * t * (m * (n // 2) + r * (m + n))
+
+
+def split_topk_bytes(m=M, n=N, frac=TOPK_FRAC) -> int:
+    k = int(np.floor(frac * m * n))
+    return 2 * m * n * 2 + k * (4 + 2) + (m + 1) * 4      # read W, write R, S (i32 col + bf16 val)
+
+
+def split_24_bytes(m=M, n=N) -> int:
+    return 2 * m * n * 2 + m * (n // 2) * 2 + m * (n // 4)  # read W, write R, values, index bytes
+
+
+def peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm": d["hbm_gbs"], "bf16": d["bf16_tflops"],
+                "bf16_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", self.gpu_id],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                self.out = ""
+
+    def summary(self) -> dict:
+        rows = []
+        for line in (self.out or "").splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i in range(4) if r[i] == "Active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": rows[0][1],
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def dist_setup(ngpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def dist_max(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ CPU oracle arm
+
+def oracle_sample(target_s: float = 12.0, rows_cap: int = M):
+    """Time the float64 oracle apply (dense Ŵ rows + product) on a row sample
+    of the batch-1 workload; returns (GB/s-equivalent, rows, seconds, cores)."""
+    import oracle
+    from sparse_rank_linear_03_b200 import synth
+    cores = len(os.sched_getaffinity(0))
+    rng = np.random.default_rng(SEED + 11)
+    Uf, Vf = synth.stand_in_factors(M, N, R_RANK, SEED + 2)
+    U64 = oracle.bits_to_f64(synth.to_bf16_bits(Uf), "bf16")
+    V64 = oracle.bits_to_f64(synth.to_bf16_bits(Vf), "bf16")
+    x64 = oracle.bits_to_f64(synth.to_bf16_bits(synth.normal_f32(1, N, SEED + 1)), "bf16")
+
+    def run(nrows):
+        rows = np.sort(rng.choice(M, size=nrows, replace=False))
+        Wr = synth.to_bf16_bits((0.02 * np.random.default_rng(SEED).standard_t(3, size=(nrows, N)))
+                                .astype(np.float32))
+        t0 = time.perf_counter()
+        s = oracle.split_24(Wr, "bf16")
+        S = oracle.nm24_to_dense(oracle.bits_to_f64(s["val"], "bf16"), s["idx"])
+        oracle.apply_rows(rows, S, U64, V64, x64)
+        return time.perf_counter() - t0
+
+    dt = run(64)
+    nrows = int(min(rows_cap, max(64, 64 * target_s / max(dt, 1e-3))))
+    dt = run(nrows)
+    frac = nrows / M
+    gb = decode_bytes() * frac / 1e9
+    return gb / dt, nrows, dt, cores
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def run_gpu(args, world, rank, local):
+    import torch
+    from sparse_rank_linear_03_b200 import hsl, synth
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    pk = peaks()
+
+    # inputs (host-generated once, resident in HBM before timing)
+    W = synth.torch_from_storage(synth.to_bf16_bits(synth.student_t_f32(M, N, SEED)), "bf16", dev)
+    Uf, Vf = synth.stand_in_factors(M, N, R_RANK, SEED + 2)
+    U = synth.torch_from_storage(synth.to_bf16_bits(Uf), "bf16", dev)
+    V = synth.torch_from_storage(synth.to_bf16_bits(Vf), "bf16", dev)
+    x1 = synth.torch_from_storage(synth.to_bf16_bits(synth.normal_f32(1, N, SEED + 1)), "bf16", dev)
+    Xp = torch.randn(T_PREFILL, N, generator=torch.Generator().manual_seed(SEED + 3)).to(
+        torch.bfloat16).to(dev)
+    y1 = torch.empty(1, M, dtype=torch.bfloat16, device=dev)
+    Yp = torch.empty(T_PREFILL, M, dtype=torch.bfloat16, device=dev)
+    R_csr = torch.empty_like(W)
+    R_24 = torch.empty_like(W)
+    csr = hsl.Layer(M, N, 0, "csr", "bf16")
+    nm = hsl.Layer(M, N, R_RANK, "nm24", "bf16")
+
+    stages = ["split_topk", "split_24", "pack", "apply_prefill", "apply_decode"]
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        csr.split(W, TOPK_FRAC, R_csr)
+        if ev:
+            ev[1].record(stream)
+        nm.split(W, 0.5, R_24)
+        if ev:
+            ev[2].record(stream)
+        nm.pack(U, V)
+        if ev:
+            ev[3].record(stream)
+        nm.apply(Xp, Yp)
+        if ev:
+            ev[4].record(stream)
+        nm.apply(x1, y1)
+        if ev:
+            ev[5].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    csr.check()
+    nm.check()
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    barrier(world)
+    torch.cuda.synchronize()
+    launches0 = hsl.launch_count()
+    with ClockSampler(gpu_id) as clk:
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_stop = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for k in range(args.steps):
+            step(events[k])
+        t_stop.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    launches = hsl.launch_count() - launches0
+    total_ms = dist_max(t_start.elapsed_time(t_stop), world)
+    per = {s: [] for s in stages}
+    for ev in events:
+        for i, s in enumerate(stages):
+            per[s].append(ev[i].elapsed_time(ev[i + 1]))
+    avg = {s: dist_max(sum(v) / len(v), world) for s, v in per.items()}
+
+    dec_bytes = decode_bytes()
+    dec_gbs = dec_bytes / (avg["apply_decode"] * 1e-3) / 1e9
+    pre_tf = prefill_flops() / (avg["apply_prefill"] * 1e-3) / 1e12
+    split_gbs = split_topk_bytes() / (avg["split_topk"] * 1e-3) / 1e9
+    s24_gbs = split_24_bytes() / (avg["split_24"] * 1e-3) / 1e9
+
+    # end to end through the C ABI with host buffers (pinned)
+    xh = x1.cpu().pin_memory()
+    yh = torch.empty(1, M, dtype=torch.bfloat16).pin_memory()
+    for _ in range(3):
+        nm.apply(xh, yh)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 20
+    e0.record(stream)
+    for _ in range(reps):
+        nm.apply(xh, yh)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = dist_max(e0.elapsed_time(e1) / reps, world)
+    e2e_gbs = dec_bytes / (e2e_ms * 1e-3) / 1e9 * world
+
+    clocks = clk.summary()
+    result = {
+        "metric": METRIC,
+        "value": round(dec_gbs * world, 1),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded Student-t nu=3 W, N(0,1) X, Gaussian stand-in U/V)",
+        "config": {"workload": WORKLOAD, "m": M, "n": N, "r": R_RANK, "decode_batch": 1,
+                   "prefill_tokens": T_PREFILL, "topk_frac": TOPK_FRAC,
+                   "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2 (W 470 MB, S 264 MB); prefill writes 235 MB "
+                         "before the decode apply"},
+        "stages": {
+            "split_topk": {"ms": round(avg["split_topk"], 4), "GB/s": round(split_gbs, 1),
+                           "frac_hbm": round(split_gbs / pk["hbm"], 3)},
+            "split_24": {"ms": round(avg["split_24"], 4), "GB/s": round(s24_gbs, 1),
+                         "frac_hbm": round(s24_gbs / pk["hbm"], 3)},
+            "pack": {"ms": round(avg["pack"], 4)},
+            "apply_prefill": {"ms": round(avg["apply_prefill"], 4), "TFLOP/s": round(pre_tf, 2),
+                              "frac_tensor": round(pre_tf / pk["bf16_sustained"], 4)},
+            "apply_decode": {"ms": round(avg["apply_decode"], 4), "GB/s": round(dec_gbs, 1),
+                             "frac_hbm": round(dec_gbs / pk["hbm"], 3)},
+        },
+        "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1), "peak": pk["hbm"],
+                     "unit": "GB/s", "frac": round(dec_gbs / pk["hbm"], 4),
+                     "traffic": None, "kernel": "decode apply (z + fused sparse/U·z)",
+                     "peak_source": pk["source"]},
+        "e2e": {"value": round(e2e_gbs, 1), "unit": "GB/s", "h2d_bytes_per_step": N * 2,
+                "d2h_bytes_per_step": M * 2},
+        "gpu_launches": int(launches),
+        "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
+                   "reasons": clocks["reasons"]},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs, rows, dt, cores = oracle_sample(args.cpu_seconds)
+        result["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores,
+                                  "kind": "oracle",
+                                  "sample": f"{rows} of {M} rows, batch 1: float64 2:4 split of "
+                                            f"the rows + dense Ŵ rows + product, {dt:.1f} s"}
+    return result
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    vals = []
+    for _ in range(args.warmup):
+        oracle_sample(args.cpu_seconds / 4, rows_cap=256)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        gbs, rows, dt, cores = oracle_sample(args.cpu_seconds, rows_cap=M)
+        vals.append(gbs)
+    wall = time.perf_counter() - t0
+    v = statistics.mean(vals)
+    return {"metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(wall / args.steps * 1e3, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": WORKLOAD, "m": M, "n": N, "r": R_RANK, "decode_batch": 1},
+            "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{rows} of {M} rows per step (float64 CPU oracle)"},
+            "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="hsl", choices=["hsl", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        res = run_reference(args, world, rank)
+        if res is not None:
+            print(json.dumps(res, ensure_ascii=False))
+        return
+    world, rank, local = dist_setup(args.gpus)
+    res = run_gpu(args, world, rank, local)
+    if rank == 0:
+        print(json.dumps(res, ensure_ascii=False))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

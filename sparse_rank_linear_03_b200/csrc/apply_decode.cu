@@ -1,0 +1,438 @@
+// Decode-batch apply: y = S x + U (Vᵀ x) for batch ≤ 16 per pass.
+//
+// "Hierarchical Sparse + Low-Rank Compression of LLMs", §Implementation and
+// operational patterns: the forward is a sparse product plus two small dense
+// products, never forming Ŵ.  SqueezeLLM article (aibr.jp/archives/208940),
+// §1: at batch 1 the cost is reading the weights, so both kernels below are
+// built to stream S, U and V from HBM once, with 16-byte vector loads.
+//
+//   k_lowrank_z   z = Vᵀ x.  Each CTA reduces a slab of V rows into fp32
+//                 partials; the last CTA to finish (ticket) sums the partials
+//                 in a fixed order, so z is deterministic.  It triggers the
+//                 dependent launch at its start.
+//   k_apply_csr   persistent CTAs over row ranges of equal bytes (all layers
+//   k_apply_nm24  of a group concatenated).  x is staged in shared memory as
+//                 [column][token]; S rows are streamed (CSR: G lanes per row;
+//                 2:4: a warp per row) into fp32 sums kept in shared memory;
+//                 then griddepcontrol.wait (programmatic dependent launch:
+//                 the S stream overlaps the z kernel), z is staged, and each
+//                 row adds U[i,:]·z and stores y.
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace hsl {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kSeg = 256;  // rows per shared-memory segment
+
+struct ApplyArgs {
+  const ApplyProblem* probs;
+  const int64_t* prob_row0;
+  const int64_t* cta_rows;
+  const void* x0;
+  void* y0;
+  const void* const* xy;  // device table: x[count] then y[count]; null for one layer
+  int32_t count, slices;
+  int32_t b0, bc;
+  int32_t r_pad_max;
+};
+
+template <typename T>
+__device__ __forceinline__ const T* x_of(const ApplyArgs& a, int p) {
+  return static_cast<const T*>(a.xy ? a.xy[p] : a.x0);
+}
+template <typename T>
+__device__ __forceinline__ T* y_of(const ApplyArgs& a, int p) {
+  return static_cast<T*>(const_cast<void*>(a.xy ? a.xy[a.count + p] : a.y0));
+}
+
+// 8 consecutive values of T as fp32 (16 bytes of bf16 or 32 bytes of fp32).
+template <typename T> __device__ __forceinline__ void load8(const T* p, float (&v)[8]);
+template <> __device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, float (&v)[8]) {
+  const uint4 q = ld_stream16(p);
+  v[0] = bf_lo(q.x); v[1] = bf_hi(q.x); v[2] = bf_lo(q.y); v[3] = bf_hi(q.y);
+  v[4] = bf_lo(q.z); v[5] = bf_hi(q.z); v[6] = bf_lo(q.w); v[7] = bf_hi(q.w);
+}
+template <> __device__ __forceinline__ void load8<float>(const float* p, float (&v)[8]) {
+  const uint4 a = ld_stream16(p), b = ld_stream16(p + 4);
+  v[0] = __uint_as_float(a.x); v[1] = __uint_as_float(a.y);
+  v[2] = __uint_as_float(a.z); v[3] = __uint_as_float(a.w);
+  v[4] = __uint_as_float(b.x); v[5] = __uint_as_float(b.y);
+  v[6] = __uint_as_float(b.z); v[7] = __uint_as_float(b.w);
+}
+
+template <typename T>
+__device__ __forceinline__ float ldx(const T* p) { return VT<T>::f(*p); }
+
+// ---- z = Vᵀ x ----------------------------------------------------------------
+template <typename T, int BCZ>
+__global__ void __launch_bounds__(kThreads) k_lowrank_z(ApplyArgs a) {
+  pdl_trigger();
+  extern __shared__ __align__(16) float red[];  // [rows per iter][BCZ][r_pad]
+  __shared__ int sh_last;
+  // layer of this CTA
+  int lo = 0, hi = a.count - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (a.probs[mid].z_cta0 <= int(blockIdx.x)) lo = mid; else hi = mid - 1;
+  }
+  const ApplyProblem& P = a.probs[lo];
+  const int local = int(blockIdx.x) - P.z_cta0;
+  const int n = P.n, rp = P.r_pad;
+  const int64_t j0 = int64_t(local) * n / P.z_ncta, j1 = int64_t(local + 1) * n / P.z_ncta;
+  const int LV = rp / 8;
+  const int RPI = kThreads / LV;
+  const int tr = threadIdx.x / LV, tc = threadIdx.x % LV;
+  const bool active = tr < RPI;
+  const T* x = x_of<T>(a, lo);
+  const T* V = static_cast<const T*>(P.V);
+
+  for (int bb = 0; bb < a.bc; bb += BCZ) {
+    float acc[BCZ][8];
+#pragma unroll
+    for (int b = 0; b < BCZ; ++b)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[b][e] = 0.f;
+    if (active) {
+      for (int64_t j = j0 + tr; j < j1; j += RPI) {
+        float v[8];
+        load8<T>(V + j * rp + tc * 8, v);
+#pragma unroll
+        for (int b = 0; b < BCZ; ++b) {
+          const float xv = (bb + b < a.bc) ? ldx<T>(x + int64_t(a.b0 + bb + b) * n + j) : 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[b][e] = fmaf(v[e], xv, acc[b][e]);
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < BCZ; ++b)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) red[(tr * BCZ + b) * rp + tc * 8 + e] = acc[b][e];
+    }
+    __syncthreads();
+    for (int o = threadIdx.x; o < BCZ * rp; o += kThreads) {
+      const int b = o / rp, c = o % rp;
+      float s = 0.f;
+      for (int r = 0; r < RPI; ++r) s += red[(r * BCZ + b) * rp + c];
+      if (bb + b < a.bc) P.zpart[(int64_t(local) * 16 + bb + b) * rp + c] = s;
+    }
+    __syncthreads();
+  }
+  // the last CTA of this layer sums the partials in CTA order
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) sh_last = (atomicAdd(P.zcount, 1u) == unsigned(P.z_ncta - 1));
+  __syncthreads();
+  if (sh_last) {
+    __threadfence();
+    for (int o = threadIdx.x; o < a.bc * rp; o += kThreads) {
+      const int b = o / rp, c = o % rp;
+      float s = 0.f;
+      for (int q = 0; q < P.z_ncta; ++q) s += __ldcg(&P.zpart[(int64_t(q) * 16 + b) * rp + c]);
+      P.z[b * rp + c] = s;
+    }
+    if (threadIdx.x == 0) *P.zcount = 0u;
+  }
+}
+
+// ---- shared pieces of the apply kernels ----------------------------------------
+template <typename T, int BC>
+__device__ __forceinline__ void stage_x(T* xs, const T* x, int n, int b0, int bc) {
+  if (BC == 1 && (n % 8) == 0 && (reinterpret_cast<uintptr_t>(x + int64_t(b0) * n) % 16) == 0) {
+    const uint4* src = reinterpret_cast<const uint4*>(x + int64_t(b0) * n);
+    uint4* dst = reinterpret_cast<uint4*>(xs);
+    const int nv = n * int(sizeof(T)) / 16;
+    for (int i = threadIdx.x; i < nv; i += kThreads) dst[i] = src[i];
+    if (threadIdx.x == 0) xs[n] = VT<T>::from_f(0.f);
+    return;
+  }
+  for (int idx = threadIdx.x; idx < (n + 1) * BC; idx += kThreads) {
+    const int c = idx / BC, b = idx % BC;
+    xs[idx] = (c < n && b < bc) ? x[int64_t(b0 + b) * n + c] : VT<T>::from_f(0.f);
+  }
+}
+
+template <typename T, int BC>
+__device__ __forceinline__ void xcol(const T* xs, int c, float (&xv)[BC]) {
+#pragma unroll
+  for (int b = 0; b < BC; ++b) xv[b] = VT<T>::f(xs[c * BC + b]);
+}
+
+// y[row] = ysp[row] + U[row,:]·z for rows [s0, s1) of layer P.
+template <typename T, int BC>
+__device__ __forceinline__ void urows(const ApplyProblem& P, const float* zs, const float* ysp,
+                                      int s0, int s1, T* y, int bc) {
+  const int rp = P.r_pad;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int GU = 1;
+  while (GU * 8 < rp) GU <<= 1;  // lanes per row, power of two ≤ 32
+  const int rpw = 32 / GU;        // rows per warp pass
+  const T* U = static_cast<const T*>(P.U);
+  for (int ib = s0 + warp * rpw; ib < s1; ib += (kThreads / 32) * rpw) {
+    const int i = ib + lane / GU, gl = lane % GU;
+    float acc[BC];
+#pragma unroll
+    for (int b = 0; b < BC; ++b) acc[b] = 0.f;
+    if (i < s1 && gl * 8 < rp) {
+      float u[8];
+      load8<T>(U + int64_t(i) * rp + gl * 8, u);
+#pragma unroll
+      for (int b = 0; b < BC; ++b)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[b] = fmaf(u[e], zs[b * rp + gl * 8 + e], acc[b]);
+    }
+    for (int o = GU >> 1; o; o >>= 1)
+#pragma unroll
+      for (int b = 0; b < BC; ++b) acc[b] += __shfl_xor_sync(0xffffffffu, acc[b], o);
+    if (gl == 0 && i < s1) {
+#pragma unroll
+      for (int b = 0; b < BC; ++b)
+        if (b < bc) y[int64_t(b) * P.m + i] = VT<T>::from_f(acc[b] + ysp[(i - s0) * BC + b]);
+    }
+  }
+}
+
+// ---- sparse row sums -------------------------------------------------------------
+template <typename T, int BC>
+__device__ __forceinline__ void csr_rows(const ApplyProblem& P, const T* xs, float* ysp, int s0,
+                                         int s1) {
+  const int G = P.group;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int gl = lane & (G - 1);
+  const int rpw = 32 / G;
+  const T* pval = static_cast<const T*>(P.pval);
+  for (int ib = s0 + warp * rpw; ib < s1; ib += (kThreads / 32) * rpw) {
+    const int i = ib + lane / G;
+    float acc[BC];
+#pragma unroll
+    for (int b = 0; b < BC; ++b) acc[b] = 0.f;
+    if (i < s1) {
+      const int32_t e1 = P.prow[i + 1];
+      for (int32_t e = P.prow[i] + 8 * gl; e < e1; e += 8 * G) {
+        const uint4 cv = ld_stream16(P.pcol + e);
+        float v[8];
+        load8<T>(pval + e, v);
+        const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const int c = int((cw[t >> 1] >> ((t & 1) * 16)) & 0xFFFFu);
+          float xv[BC];
+          xcol<T, BC>(xs, c, xv);
+#pragma unroll
+          for (int b = 0; b < BC; ++b) acc[b] = fmaf(v[t], xv[b], acc[b]);
+        }
+      }
+    }
+    for (int o = G >> 1; o; o >>= 1)
+#pragma unroll
+      for (int b = 0; b < BC; ++b) acc[b] += __shfl_xor_sync(0xffffffffu, acc[b], o);
+    if (gl == 0 && i < s1)
+#pragma unroll
+      for (int b = 0; b < BC; ++b) ysp[(i - s0) * BC + b] = acc[b];
+  }
+}
+
+template <typename T, int BC>
+__device__ __forceinline__ void nm24_rows(const ApplyProblem& P, const T* xs, float* ysp, int s0,
+                                          int s1) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int n = P.n;
+  const int64_t half = n / 2;
+  const T* pval = static_cast<const T*>(P.pval);
+  const bool vec = (n % 16) == 0;
+  const int nq = (n + 15) / 16;
+  for (int i = s0 + warp; i < s1; i += kThreads / 32) {
+    const T* vrow = pval + int64_t(i) * half;
+    const uint16_t* mrow = P.pmeta + int64_t(i) * P.meta_stride;
+    float acc[BC];
+#pragma unroll
+    for (int b = 0; b < BC; ++b) acc[b] = 0.f;
+    if (vec) {
+      for (int sup = 0; sup * 256 < nq; ++sup) {
+        const uint4 mw = ld_stream16(mrow + sup * 256 + lane * 8);
+        const uint32_t mws[4] = {mw.x, mw.y, mw.z, mw.w};
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const int q = (sup * 8 + t) * 32 + lane;
+          if (q < nq) {
+            float v[8];
+            load8<T>(vrow + int64_t(q) * 8, v);
+            const uint32_t meta = (mws[t >> 1] >> ((t & 1) * 16)) & 0xFFFFu;
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              const uint32_t nib = (meta >> (4 * g)) & 0xFu;
+              const int base = q * 16 + g * 4;
+              float x0[BC], x1[BC];
+              xcol<T, BC>(xs, base + int(nib & 3u), x0);
+              xcol<T, BC>(xs, base + int(nib >> 2), x1);
+#pragma unroll
+              for (int b = 0; b < BC; ++b)
+                acc[b] = fmaf(v[2 * g + 1], x1[b], fmaf(v[2 * g], x0[b], acc[b]));
+            }
+          }
+        }
+      }
+    } else {
+      const int groups = n / 4;
+      for (int gi = lane; gi < groups; gi += 32) {
+        const int q = gi >> 2, g = gi & 3;
+        const int sup = q >> 8, rem = q & 255;
+        const uint32_t meta = mrow[sup * 256 + (rem & 31) * 8 + (rem >> 5)];
+        const uint32_t nib = (meta >> (4 * g)) & 0xFu;
+        const float v0 = VT<T>::f(vrow[2 * gi]), v1 = VT<T>::f(vrow[2 * gi + 1]);
+        float x0[BC], x1[BC];
+        xcol<T, BC>(xs, gi * 4 + int(nib & 3u), x0);
+        xcol<T, BC>(xs, gi * 4 + int(nib >> 2), x1);
+#pragma unroll
+        for (int b = 0; b < BC; ++b) acc[b] = fmaf(v1, x1[b], fmaf(v0, x0[b], acc[b]));
+      }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1)
+#pragma unroll
+      for (int b = 0; b < BC; ++b) acc[b] += __shfl_xor_sync(0xffffffffu, acc[b], o);
+    if (lane == 0)
+#pragma unroll
+      for (int b = 0; b < BC; ++b) ysp[(i - s0) * BC + b] = acc[b];
+  }
+}
+
+// ---- the persistent apply kernel ---------------------------------------------------
+template <typename T, int BC, bool CSR>
+__global__ void __launch_bounds__(kThreads) k_apply_decode(ApplyArgs a) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  float* zs = reinterpret_cast<float*>(smem);                 // [BC][r_pad_max]
+  float* ysp = zs + BC * a.r_pad_max;                          // [kSeg][BC]
+  T* xs = reinterpret_cast<T*>(ysp + kSeg * BC);               // [(n+1)][BC]
+
+  const int64_t slo = int64_t(blockIdx.x) * a.slices / gridDim.x;
+  const int64_t shi = int64_t(blockIdx.x + 1) * a.slices / gridDim.x;
+  int64_t row = a.cta_rows[slo];
+  const int64_t row_end = a.cta_rows[shi];
+  if (row >= row_end) return;
+  int p = 0;
+  {
+    int lo = 0, hi = a.count - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (a.prob_row0[mid] <= row) lo = mid; else hi = mid - 1;
+    }
+    p = lo;
+  }
+  bool waited = false;
+  while (row < row_end) {
+    const ApplyProblem P = a.probs[p];
+    const int64_t p_end = a.prob_row0[p + 1];
+    const int l0 = int(row - P.row0);
+    const int l1 = int(min(row_end, p_end) - P.row0);
+    __syncthreads();
+    stage_x<T, BC>(xs, x_of<T>(a, p), P.n, a.b0, a.bc);
+    __syncthreads();
+    T* y = y_of<T>(a, p) + int64_t(a.b0) * P.m;
+    for (int s0 = l0; s0 < l1; s0 += kSeg) {
+      const int s1 = min(s0 + kSeg, l1);
+      if (CSR) csr_rows<T, BC>(P, xs, ysp, s0, s1);
+      else nm24_rows<T, BC>(P, xs, ysp, s0, s1);
+      __syncthreads();
+      if (!waited) {
+        pdl_wait();
+        waited = true;
+      }
+      if (s0 == l0 && P.r_pad > 0) {
+        for (int o = threadIdx.x; o < a.bc * P.r_pad; o += kThreads) zs[o] = __ldcg(P.z + o);
+        for (int o = a.bc * P.r_pad + threadIdx.x; o < BC * P.r_pad; o += kThreads) zs[o] = 0.f;
+      }
+      __syncthreads();
+      urows<T, BC>(P, zs, ysp, s0, s1, y, a.bc);
+      __syncthreads();
+    }
+    row = P.row0 + l1;
+    ++p;
+  }
+}
+
+template <typename T, int BC>
+size_t apply_smem(const ApplyPlan& plan) {
+  return size_t(BC) * plan.r_pad_max * 4 + size_t(kSeg) * BC * 4 +
+         round_up(size_t(plan.n_max + 1) * BC * sizeof(T), 16);
+}
+
+template <typename T, int BC>
+hsl_status launch_chunk(ApplyPlan& plan, ApplyArgs a, int num_sms, cudaStream_t s) {
+  // z = Vᵀ x, normal launch (waits for everything before it on the stream)
+  if (plan.z_grid > 0) {
+    constexpr int BCZ = BC < 8 ? BC : 8;
+    const size_t zsm = size_t(kThreads) * 8 * BCZ * 4;
+    auto zk = k_lowrank_z<T, BCZ>;
+    cudaFuncSetAttribute(zk, cudaFuncAttributeMaxDynamicSharedMemorySize, int(zsm));
+    zk<<<plan.z_grid, kThreads, zsm, s>>>(a);
+    note_launch();
+    if (hsl_status e = cuda_fail(cudaGetLastError(), "z launch")) return e;
+  }
+  const size_t sm = apply_smem<T, BC>(plan);
+  auto ak = plan.fmt == HSL_FMT_CSR ? k_apply_decode<T, BC, true> : k_apply_decode<T, BC, false>;
+  if (cudaError_t e = cudaFuncSetAttribute(ak, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm)))
+    return cuda_fail(e, "apply smem attribute");
+  int occ = 0;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, ak, kThreads, sm);
+  occ = std::max(1, std::min(occ, 24));
+  while (24 % occ) --occ;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(num_sms * occ));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = sm;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = plan.z_grid > 0 ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  note_launch();
+  return cuda_fail(cudaLaunchKernelEx(&cfg, ak, a), "apply launch");
+}
+
+template <typename T>
+hsl_status run_typed(ApplyPlan& plan, ApplyArgs a, int64_t batch, int num_sms, cudaStream_t s) {
+  const int eb = sizeof(T);
+  // largest batch chunk whose staged x fits comfortably in shared memory
+  int bcmax = 16;
+  while (bcmax > 1 && size_t(plan.n_max + 1) * bcmax * eb > 96 * 1024) bcmax >>= 1;
+  for (int64_t b0 = 0; b0 < batch; b0 += bcmax) {
+    const int bc = int(std::min<int64_t>(bcmax, batch - b0));
+    a.b0 = int32_t(b0);
+    a.bc = bc;
+    hsl_status st;
+    if (bc == 1) st = launch_chunk<T, 1>(plan, a, num_sms, s);
+    else if (bc == 2) st = launch_chunk<T, 2>(plan, a, num_sms, s);
+    else if (bc <= 4) st = launch_chunk<T, 4>(plan, a, num_sms, s);
+    else if (bc <= 8) st = launch_chunk<T, 8>(plan, a, num_sms, s);
+    else st = launch_chunk<T, 16>(plan, a, num_sms, s);
+    if (st) return st;
+  }
+  return HSL_OK;
+}
+
+}  // namespace
+
+hsl_status apply_decode_run(ApplyPlan& plan, const void* X, void* Y, const void* const* xy_dev,
+                            int64_t batch, int num_sms, cudaStream_t s) {
+  ApplyArgs a;
+  a.probs = static_cast<const ApplyProblem*>(plan.probs.p);
+  a.prob_row0 = static_cast<const int64_t*>(plan.prob_row0.p);
+  a.cta_rows = static_cast<const int64_t*>(plan.cta_rows.p);
+  a.x0 = X;
+  a.y0 = Y;
+  a.xy = xy_dev;
+  a.count = plan.count;
+  a.slices = plan.slices;
+  a.b0 = 0;
+  a.bc = 0;
+  a.r_pad_max = plan.r_pad_max;
+  if (plan.dtype == HSL_BF16) return run_typed<__nv_bfloat16>(plan, a, batch, num_sms, s);
+  return run_typed<float>(plan, a, batch, num_sms, s);
+}
+
+}  // namespace hsl

@@ -1,0 +1,109 @@
+// Host-side internals of libhsl: the handle, device buffers, kernel launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+#include <string>
+
+#include "hsl.h"
+
+namespace hsl {
+
+// ---- bookkeeping -----------------------------------------------------------
+extern std::atomic<uint64_t> g_launches;
+inline void note_launch(int n = 1) { g_launches.fetch_add(uint64_t(n), std::memory_order_relaxed); }
+void set_message(const std::string& s);
+hsl_status cuda_fail(cudaError_t e, const char* what);
+
+// Grow-only device allocation.
+struct DevBuf {
+  void* p = nullptr;
+  size_t bytes = 0;
+};
+hsl_status ensure(DevBuf& b, size_t bytes, const char* what);
+void release(DevBuf& b);
+
+inline int dtype_bytes(hsl_dtype d) { return d == HSL_F32 ? 4 : 2; }
+inline int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
+
+// ---- the apply problem descriptor (device-resident, one per layer) --------
+struct ApplyProblem {
+  const int32_t* prow;    // CSR: packed row starts (elements, multiples of 8), m+1
+  const uint16_t* pcol;   // CSR: packed 16-bit columns (pad = n)
+  const void* pval;       // CSR: packed values; NM24: values [m][n/2]
+  const uint16_t* pmeta;  // NM24: metadata, interleaved per lane (see pack.cu)
+  const void* U;          // [m][r_pad]
+  const void* V;          // [n][r_pad]
+  float* zpart;           // [z_ncta][16][r_pad]
+  float* z;               // [16][r_pad]
+  unsigned* zcount;       // last-CTA ticket of the z reduction
+  int32_t m, n, r_pad;
+  int32_t group;          // CSR: lanes per row (4..32)
+  int32_t meta_stride;    // NM24: u16 metadata words per row
+  int32_t z_cta0, z_ncta; // this layer's CTAs in the z launch
+  int64_t row0;           // first row of this layer in the concatenated row space
+};
+
+// Launch plan for one or more layers applied together.
+struct ApplyPlan {
+  int count = 0;
+  hsl_format fmt = HSL_FMT_CSR;
+  hsl_dtype dtype = HSL_F32;
+  int32_t n_max = 0, r_pad_max = 0;
+  int64_t rows_total = 0;
+  int z_grid = 0;       // CTAs of the z launch (0 when r == 0)
+  int slices = 0;       // equal-byte row ranges the apply grid divides among CTAs
+  DevBuf probs;         // ApplyProblem[count]
+  DevBuf prob_row0;     // int64[count+1]
+  DevBuf cta_rows;      // int64[apply_grid+1]
+  DevBuf xy_ptrs;       // const void*[2*count] (group calls)
+  const void* const* last_x = nullptr;  // host cache of the uploaded pointers
+  std::string host_xy;  // bytes of the last uploaded pointer table
+};
+
+struct Handle {
+  int64_t m = 0, n = 0;
+  int32_t r = 0, r_pad = 0;
+  hsl_format fmt = HSL_FMT_CSR;
+  hsl_dtype dtype = HSL_F32;
+  int device = 0;
+  int num_sms = 148;
+
+  // canonical S
+  DevBuf row_ptr, col, val;   // CSR
+  DevBuf nm_val, nm_idx;      // NM24
+  int64_t nnz = 0;
+  bool has_sparse = false;
+
+  // packed layouts
+  DevBuf prow, pcol, pval, pmeta, U, V, Vt;
+  int32_t group = 8, meta_stride = 0;
+  int64_t pack_cap = 0;
+  bool packed = false;
+
+  // workspace
+  DevBuf zpart, z, zcount, err, split_ws, flags;
+  DevBuf xstage, ystage;
+  int z_ncta = 0;
+  ApplyPlan plan;  // the single-layer plan, built by hsl_pack
+};
+
+// ---- launchers (each returns HSL_OK or an error already described) ------
+hsl_status split_topk_run(Handle& h, const void* W, hsl_dtype wdt, int64_t k, void* R,
+                          cudaStream_t s);
+hsl_status split_24_run(Handle& h, const void* W, hsl_dtype wdt, void* R, cudaStream_t s);
+hsl_status pack_sparse_run(Handle& h, cudaStream_t s);
+hsl_status pack_factors_run(Handle& h, const void* U, const void* V, cudaStream_t s);
+hsl_status csr_convert_run(Handle& h, const int32_t* row_ptr, const int32_t* col,
+                           const void* val, cudaStream_t s);
+hsl_status plan_build(ApplyPlan& plan, Handle* const* hs, int count, cudaStream_t s);
+hsl_status apply_run(ApplyPlan& plan, const void* X, void* Y, const void* const* Xs,
+                     void* const* Ys, int64_t batch, cudaStream_t s);
+
+}  // namespace hsl
+
+struct hsl_handle_s {
+  hsl::Handle h;
+};

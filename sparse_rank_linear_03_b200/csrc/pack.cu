@@ -1,0 +1,344 @@
+// Packing: canonical S → the layouts the apply kernels stream, padded factor
+// copies, and the launch plan (row ranges of equal streamed bytes per CTA).
+//
+// "Hierarchical Sparse + Low-Rank Compression of LLMs", §Implementation and
+// operational patterns (from theory to production), mixed precision: the
+// pages store factors in 16 bits and sparse indices in narrow integers.  The
+// packed CSR uses 16-bit column indices (n < 65535) and pads each row to a
+// multiple of 8 entries so every lane reads whole 16-byte vectors; padding
+// entries point at column n, a zero kept at the end of the staged x.
+//
+// Packed 2:4 metadata: one 16-bit word per chunk of 8 kept values (4 groups,
+// 4 bits each = i0 | i1 << 2).  Within a row, chunk q = (8·s + t)·32 + l is
+// stored at word s·256 + l·8 + t, so lane l of a warp fetches the metadata of
+// its next 8 chunks with a single 16-byte load.
+#include <algorithm>
+#include <vector>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace hsl {
+namespace {
+
+__device__ __forceinline__ int32_t pad8(int32_t v) { return (v + 7) & ~7; }
+
+// One CTA: prow = exclusive scan of the padded row lengths; prow[m] = total.
+// A row whose bounds are not 0 <= row_ptr[i] <= row_ptr[i+1] <= nnz is taken
+// as empty and flagged; starts are clamped to cap so no later read or write
+// leaves the packed arrays, whatever an imported row_ptr holds.
+__device__ __forceinline__ int32_t row_len_checked(const int32_t* row_ptr, int64_t i, int64_t nnz,
+                                                   bool& bad) {
+  const int32_t a = row_ptr[i], b = row_ptr[i + 1];
+  if (a < 0 || b < a || int64_t(b) > nnz) {
+    bad = true;
+    return 0;
+  }
+  return b - a;
+}
+
+__global__ void __launch_bounds__(1024) k_csr_prow(const int32_t* __restrict__ row_ptr, int64_t m,
+                                                   int64_t nnz, int64_t cap,
+                                                   int32_t* __restrict__ prow, uint32_t* err) {
+  __shared__ int64_t wsum[32];
+  const int t = threadIdx.x, nt = blockDim.x;
+  const int64_t per = (m + nt - 1) / nt;
+  const int64_t lo = int64_t(t) * per < m ? int64_t(t) * per : m;
+  const int64_t hi = lo + per < m ? lo + per : m;
+  bool bad = false;
+  int64_t s = 0;
+  for (int64_t i = lo; i < hi; ++i) s += pad8(row_len_checked(row_ptr, i, nnz, bad));
+  int64_t incl = s;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int64_t v = __shfl_up_sync(0xffffffffu, incl, o);
+    if ((t & 31) >= o) incl += v;
+  }
+  if ((t & 31) == 31) wsum[t >> 5] = incl;
+  __syncthreads();
+  if (t < 32) {
+    const int64_t w = t < (nt >> 5) ? wsum[t] : 0;
+    int64_t wi = w;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t v = __shfl_up_sync(0xffffffffu, wi, o);
+      if (t >= o) wi += v;
+    }
+    wsum[t] = wi - w;
+  }
+  __syncthreads();
+  int64_t off = wsum[t >> 5] + incl - s;
+  for (int64_t i = lo; i < hi; ++i) {
+    prow[i] = int32_t(off < cap ? off : cap);
+    off += pad8(row_len_checked(row_ptr, i, nnz, bad));
+  }
+  if (hi == m && lo < hi) {
+    if (off > cap) bad = true;
+    prow[m] = int32_t(off < cap ? off : cap);
+  }
+  if (m == 0 && t == 0) prow[0] = 0;
+  if (t == 0 && row_ptr[0] != 0) bad = true;
+  if (bad) set_error(err, kErrBadIndex);
+}
+
+// Warp per row: copy columns (int32 → u16) and values; pad with (n, 0).
+template <typename SB>
+__global__ void __launch_bounds__(256) k_csr_fill(const int32_t* __restrict__ row_ptr,
+                                                  const int32_t* __restrict__ col,
+                                                  const SB* __restrict__ val,
+                                                  const int32_t* __restrict__ prow, int64_t m,
+                                                  int64_t nnz, int32_t n, uint16_t* __restrict__ pcol,
+                                                  SB* __restrict__ pval, uint32_t* err) {
+  const int lane = threadIdx.x & 31;
+  bool bad = false;
+  for (int64_t i = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; i < m;
+       i += (int64_t(gridDim.x) * blockDim.x) >> 5) {
+    bool badrow = false;
+    const int32_t len = row_len_checked(row_ptr, i, nnz, badrow);
+    const int32_t s0 = row_ptr[i];
+    const int32_t d0 = prow[i], plen = prow[i + 1] - d0;
+    for (int32_t e = lane; e < plen; e += 32) {
+      bool in = e < len;
+      const int32_t c = in ? col[s0 + e] : n;
+      if (in && (c < 0 || c >= n)) {  // never index outside the staged x
+        bad = true;
+        in = false;
+      }
+      pcol[d0 + e] = in ? uint16_t(c) : uint16_t(n);
+      pval[d0 + e] = in ? val[s0 + e] : SB(0);
+    }
+  }
+  if (bad) set_error(err, kErrBadIndex);
+}
+
+__global__ void k_nm24_meta(const uint8_t* __restrict__ idx, int64_t m, int64_t n,
+                            int32_t meta_stride, uint16_t* __restrict__ pmeta) {
+  const int64_t words = m * meta_stride;
+  const int64_t groups = n / 4;
+  for (int64_t w = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; w < words;
+       w += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t row = w / meta_stride;
+    const int32_t pos = int32_t(w % meta_stride);
+    const int32_t s = pos >> 8, l = (pos & 255) >> 3, t = pos & 7;
+    const int64_t q = int64_t(s * 8 + t) * 32 + l;
+    uint32_t word = 0;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      const int64_t grp = 4 * q + g;
+      if (grp < groups) word |= uint32_t(idx[row * groups + grp] & 0xF) << (4 * g);
+    }
+    pmeta[w] = uint16_t(word);
+  }
+}
+
+template <typename SB>
+__global__ void k_pad_cols(const SB* __restrict__ src, int64_t rows, int32_t r, int32_t r_pad,
+                           SB* __restrict__ dst) {
+  const int64_t total = rows * r_pad;
+  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
+       e += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t i = e / r_pad;
+    const int32_t c = int32_t(e % r_pad);
+    dst[e] = c < r ? src[i * r + c] : SB(0);
+  }
+}
+
+// One CTA: boundaries of `slices` row ranges of equal streamed bytes over the
+// concatenated rows of all layers.  Cost of the first i rows of layer p:
+//   CSR : prow[i]·(value + 2 index bytes) + i·(U row bytes + 8)
+//   NM24: i·(n/2 value bytes + n/8 metadata bytes + U row bytes + 8)
+__global__ void __launch_bounds__(1024) k_partition(const ApplyProblem* __restrict__ probs,
+                                                    int count, int fmt_csr, int eb,
+                                                    int64_t* __restrict__ cost0, int slices,
+                                                    int64_t* __restrict__ cta_rows) {
+  auto row_cost = [&](const ApplyProblem& P, int64_t i) -> int64_t {
+    const int64_t u = int64_t(P.r_pad) * eb + 8;
+    if (fmt_csr) return int64_t(P.prow[i]) * (eb + 2) + i * u;
+    return i * (int64_t(P.n / 2) * eb + P.n / 8 + u);
+  };
+  if (threadIdx.x == 0) {
+    int64_t acc = 0;
+    for (int p = 0; p < count; ++p) {
+      cost0[p] = acc;
+      acc += row_cost(probs[p], probs[p].m);
+    }
+    cost0[count] = acc;
+  }
+  __syncthreads();
+  const int64_t total = cost0[count];
+  for (int c = threadIdx.x; c <= slices; c += blockDim.x) {
+    if (c == slices) {
+      cta_rows[c] = probs[count - 1].row0 + probs[count - 1].m;
+      continue;
+    }
+    const int64_t target = total / slices * c + (total % slices) * c / slices;
+    // layer: last p with cost0[p] <= target
+    int lo = 0, hi = count - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (cost0[mid] <= target) lo = mid; else hi = mid - 1;
+    }
+    const ApplyProblem& P = probs[lo];
+    const int64_t want = target - cost0[lo];
+    // first row i in [0, m] with row_cost(i) >= want
+    int64_t a = 0, b = P.m;
+    while (a < b) {
+      const int64_t mid = (a + b) >> 1;
+      if (row_cost(P, mid) >= want) b = mid; else a = mid + 1;
+    }
+    cta_rows[c] = P.row0 + a;
+  }
+}
+
+}  // namespace
+
+// Slices per SM in a plan; the apply grid (SMs × resident CTAs) divides it for
+// every residency 1, 2, 3, 4, 6, 8, 12, 24.
+constexpr int kSlicesPerSM = 24;
+
+hsl_status pack_sparse_run(Handle& h, cudaStream_t s) {
+  const int eb = dtype_bytes(h.dtype);
+  if (h.fmt == HSL_FMT_CSR) {
+    const int64_t cap = round_up(h.nnz + 7 * h.m + 8, 8);  // multiple of 8: every row start stays 16-byte aligned
+    if (hsl_status e = ensure(h.prow, size_t(h.m + 1) * 4, "packed row starts")) return e;
+    if (hsl_status e = ensure(h.pcol, size_t(cap) * 2, "packed columns")) return e;
+    if (hsl_status e = ensure(h.pval, size_t(cap) * eb, "packed values")) return e;
+    h.pack_cap = cap;
+    k_csr_prow<<<1, 1024, 0, s>>>(static_cast<const int32_t*>(h.row_ptr.p), h.m, h.nnz, cap,
+                                  static_cast<int32_t*>(h.prow.p), static_cast<uint32_t*>(h.err.p));
+    note_launch();
+    const int64_t grid = std::min<int64_t>((h.m * 32 + 255) / 256, int64_t(h.num_sms) * 8);
+    if (eb == 2)
+      k_csr_fill<uint16_t><<<unsigned(std::max<int64_t>(grid, 1)), 256, 0, s>>>(
+          static_cast<const int32_t*>(h.row_ptr.p), static_cast<const int32_t*>(h.col.p),
+          static_cast<const uint16_t*>(h.val.p), static_cast<const int32_t*>(h.prow.p), h.m,
+          h.nnz, int32_t(h.n), static_cast<uint16_t*>(h.pcol.p), static_cast<uint16_t*>(h.pval.p),
+          static_cast<uint32_t*>(h.err.p));
+    else
+      k_csr_fill<uint32_t><<<unsigned(std::max<int64_t>(grid, 1)), 256, 0, s>>>(
+          static_cast<const int32_t*>(h.row_ptr.p), static_cast<const int32_t*>(h.col.p),
+          static_cast<const uint32_t*>(h.val.p), static_cast<const int32_t*>(h.prow.p), h.m,
+          h.nnz, int32_t(h.n), static_cast<uint16_t*>(h.pcol.p), static_cast<uint32_t*>(h.pval.p),
+          static_cast<uint32_t*>(h.err.p));
+    note_launch();
+    // lanes per row: about two 8-entry vectors per lane on an average row
+    const double avg_vec = double(h.nnz) / double(std::max<int64_t>(h.m, 1)) / 8.0;
+    int g = 4;
+    while (g < 32 && g * 2 < avg_vec) g *= 2;
+    h.group = g;
+    return cuda_fail(cudaGetLastError(), "CSR pack launch");
+  }
+  // NM24
+  const int64_t nq = (h.n + 15) / 16;  // chunks of 8 kept values per row
+  h.meta_stride = int32_t(round_up(nq, 256));
+  if (hsl_status e = ensure(h.pmeta, size_t(h.m) * h.meta_stride * 2, "2:4 metadata")) return e;
+  const int64_t words = h.m * h.meta_stride;
+  const int64_t grid = std::min<int64_t>((words + 255) / 256, int64_t(h.num_sms) * 16);
+  k_nm24_meta<<<unsigned(std::max<int64_t>(grid, 1)), 256, 0, s>>>(
+      static_cast<const uint8_t*>(h.nm_idx.p), h.m, h.n, h.meta_stride,
+      static_cast<uint16_t*>(h.pmeta.p));
+  note_launch();
+  return cuda_fail(cudaGetLastError(), "2:4 pack launch");
+}
+
+hsl_status pack_factors_run(Handle& h, const void* U, const void* V, cudaStream_t s) {
+  const int eb = dtype_bytes(h.dtype);
+  if (h.r == 0) return HSL_OK;
+  if (hsl_status e = ensure(h.U, size_t(h.m) * h.r_pad * eb, "U copy")) return e;
+  if (hsl_status e = ensure(h.V, size_t(h.n) * h.r_pad * eb, "V copy")) return e;
+  for (int which = 0; which < 2; ++which) {
+    const int64_t rows = which ? h.n : h.m;
+    const void* src = which ? V : U;
+    void* dst = which ? h.V.p : h.U.p;
+    const int64_t grid = std::min<int64_t>((rows * h.r_pad + 255) / 256, int64_t(h.num_sms) * 16);
+    if (eb == 2)
+      k_pad_cols<uint16_t><<<unsigned(grid), 256, 0, s>>>(static_cast<const uint16_t*>(src), rows,
+                                                          h.r, h.r_pad, static_cast<uint16_t*>(dst));
+    else
+      k_pad_cols<uint32_t><<<unsigned(grid), 256, 0, s>>>(static_cast<const uint32_t*>(src), rows,
+                                                          h.r, h.r_pad, static_cast<uint32_t*>(dst));
+    note_launch();
+  }
+  return cuda_fail(cudaGetLastError(), "factor pack launch");
+}
+
+hsl_status plan_build(ApplyPlan& plan, Handle* const* hs, int count, cudaStream_t s) {
+  plan.count = count;
+  plan.fmt = hs[0]->fmt;
+  plan.dtype = hs[0]->dtype;
+  plan.n_max = 0;
+  plan.r_pad_max = 0;
+  const int eb = dtype_bytes(plan.dtype);
+  std::vector<ApplyProblem> probs(count);
+  int64_t row0 = 0;
+  int zc = 0;
+  for (int i = 0; i < count; ++i) {
+    Handle& h = *hs[i];
+    ApplyProblem& P = probs[i];
+    P.prow = static_cast<const int32_t*>(h.prow.p);
+    P.pcol = static_cast<const uint16_t*>(h.pcol.p);
+    P.pval = h.fmt == HSL_FMT_CSR ? h.pval.p : h.nm_val.p;
+    P.pmeta = static_cast<const uint16_t*>(h.pmeta.p);
+    P.U = h.U.p;
+    P.V = h.V.p;
+    P.m = int32_t(h.m);
+    P.n = int32_t(h.n);
+    P.r_pad = h.r_pad;
+    P.group = h.group;
+    P.meta_stride = h.meta_stride;
+    P.row0 = row0;
+    row0 += h.m;
+    // z: about 32 KB of V per CTA, at most 2 CTAs per SM for one layer
+    int zn = 0;
+    if (h.r_pad > 0) {
+      const int64_t vbytes = h.n * int64_t(h.r_pad) * eb;
+      zn = int(std::min<int64_t>(std::max<int64_t>((vbytes + 32767) / 32768, 1),
+                                 std::min<int64_t>(h.n, 2 * h.num_sms)));
+      if (hsl_status e = ensure(h.zpart, size_t(zn) * 16 * h.r_pad * 4, "z partials")) return e;
+      if (hsl_status e = ensure(h.z, size_t(16) * h.r_pad * 4, "z")) return e;
+      if (h.zcount.p == nullptr) {
+        if (hsl_status e = ensure(h.zcount, 256, "z ticket")) return e;
+        if (cudaError_t ce = cudaMemsetAsync(h.zcount.p, 0, 256, s)) return cuda_fail(ce, "memset");
+      }
+    }
+    h.z_ncta = zn;
+    P.zpart = static_cast<float*>(h.zpart.p);
+    P.z = static_cast<float*>(h.z.p);
+    P.zcount = static_cast<unsigned*>(h.zcount.p);
+    P.z_cta0 = zc;
+    P.z_ncta = zn;
+    zc += zn;
+    plan.n_max = std::max(plan.n_max, int32_t(h.n));
+    plan.r_pad_max = std::max(plan.r_pad_max, h.r_pad);
+  }
+  plan.rows_total = row0;
+  plan.z_grid = zc;
+  const int slices = hs[0]->num_sms * kSlicesPerSM;
+  plan.slices = slices;
+  if (hsl_status e = ensure(plan.probs, sizeof(ApplyProblem) * count, "plan")) return e;
+  if (hsl_status e = ensure(plan.prob_row0, sizeof(int64_t) * (count + 1), "plan")) return e;
+  if (hsl_status e = ensure(plan.cta_rows, sizeof(int64_t) * (slices + 1), "plan")) return e;
+  std::vector<int64_t> pr0(count + 1);
+  for (int i = 0; i < count; ++i) pr0[i] = probs[i].row0;
+  pr0[count] = row0;
+  if (cudaError_t e = cudaMemcpyAsync(plan.probs.p, probs.data(), sizeof(ApplyProblem) * count,
+                                      cudaMemcpyHostToDevice, s))
+    return cuda_fail(e, "plan upload");
+  if (cudaError_t e = cudaMemcpyAsync(plan.prob_row0.p, pr0.data(), sizeof(int64_t) * (count + 1),
+                                      cudaMemcpyHostToDevice, s))
+    return cuda_fail(e, "plan upload");
+  DevBuf cost0;
+  if (hsl_status e = ensure(cost0, sizeof(int64_t) * (count + 1), "plan")) return e;
+  k_partition<<<1, 1024, 0, s>>>(static_cast<const ApplyProblem*>(plan.probs.p), count,
+                                 plan.fmt == HSL_FMT_CSR ? 1 : 0, eb,
+                                 static_cast<int64_t*>(cost0.p), slices,
+                                 static_cast<int64_t*>(plan.cta_rows.p));
+  note_launch();
+  hsl_status st = cuda_fail(cudaGetLastError(), "partition launch");
+  // the vectors above are pageable: the copies have completed on return, and
+  // the kernel's scratch can be freed once the stream reaches this point
+  cudaStreamSynchronize(s);
+  release(cost0);
+  plan.host_xy.clear();
+  return st;
+}
+
+}  // namespace hsl
