@@ -227,8 +227,14 @@ def lowrank_svd(R64: np.ndarray, r: int) -> tuple[np.ndarray, np.ndarray]:
     if r == 0:
         return np.zeros((m, 0)), np.zeros((n, 0))
     Uf, s, Vt = np.linalg.svd(R64, full_matrices=False)
-    root = np.sqrt(s[:r])
-    return Uf[:, :r] * root, Vt[:r, :].T * root
+    q = min(r, len(s))
+    root = np.sqrt(s[:q])
+    U = np.zeros((m, r))
+    V = np.zeros((n, r))
+    # a rank above min(m, n) is exact: the extra factor columns are zero
+    U[:, :q] = Uf[:, :q] * root
+    V[:, :q] = Vt[:q, :].T * root
+    return U, V
 
 
 def lowrank_randomized(R64: np.ndarray, r: int, omega: np.ndarray,

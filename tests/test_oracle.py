@@ -283,6 +283,14 @@ def test_eckart_young_with_eigvalsh():
     assert np.allclose(V.T @ V, np.diag(sig), atol=1e-10)
 
 
+def test_lowrank_rank_above_min_dimension_is_exact_and_zero_padded():
+    R = np.random.default_rng(17).standard_normal((5, 12))
+    U, V = oracle.lowrank_svd(R, 9)
+    assert U.shape == (5, 9) and V.shape == (12, 9)
+    assert not U[:, 5:].any() and not V[:, 5:].any()
+    assert np.abs(U @ V.T - R).max() < 1e-12
+
+
 def test_randomized_matches_exact_on_low_rank():
     rng = np.random.default_rng(8)
     R = rng.standard_normal((60, 5)) @ rng.standard_normal((5, 50))
