@@ -95,6 +95,16 @@ def _ptr(t) -> int | None:
     return int(t)
 
 
+def _need(t, numel: int, what: str) -> None:
+    if t is not None and isinstance(t, torch.Tensor) and t.numel() != numel:
+        raise ValueError(f"{what} has {t.numel()} elements, expected {numel}")
+
+
+def _dtype_of(t, want: str, what: str) -> None:
+    if isinstance(t, torch.Tensor) and t.dtype != TORCH_DTYPE[want]:
+        raise ValueError(f"{what} is {t.dtype}, the layer stores {want}")
+
+
 def launch_count() -> int:
     """Kernels libhsl has launched in this process."""
     return int(lib.hsl_launch_count())
@@ -128,7 +138,8 @@ class Layer:
     def split(self, W: torch.Tensor, frac: float, residual: torch.Tensor | None = None,
               stream=None) -> None:
         wdt = {torch.float32: "f32", torch.bfloat16: "bf16"}[W.dtype]
-        if residual is not None and (residual.dtype != W.dtype or residual.shape != W.shape):
+        _need(W, self.m * self.n, "W")
+        if residual is not None and (residual.dtype != W.dtype or residual.numel() != W.numel()):
             raise ValueError("residual must match W")
         _ok(lib.hsl_split_topk(self._h, _ptr(W), DTYPE[wdt], float(frac), _ptr(residual),
                                _stream(stream)), "hsl_split_topk")
@@ -156,19 +167,34 @@ class Layer:
         return {"val": val, "idx": idx}
 
     def set_sparse_csr(self, row_ptr, col, val, stream=None) -> None:
+        _need(row_ptr, self.m + 1, "row_ptr")
+        _need(val, col.numel(), "val")
+        _dtype_of(val, self.dtype, "val")
         _ok(lib.hsl_set_sparse_csr(self._h, int(col.numel()), _ptr(row_ptr), _ptr(col), _ptr(val),
                                    _stream(stream)), "hsl_set_sparse_csr")
 
     def set_sparse_nm24(self, val, idx, stream=None) -> None:
+        _need(val, self.m * (self.n // 2), "val")
+        _need(idx, self.m * (self.n // 4), "idx")
+        _dtype_of(val, self.dtype, "val")
         _ok(lib.hsl_set_sparse_nm24(self._h, _ptr(val), _ptr(idx), _stream(stream)),
             "hsl_set_sparse_nm24")
 
     # -- pack + apply -------------------------------------------------------
     def pack(self, U, V, stream=None) -> None:
+        _need(U, self.m * self.r, "U")
+        _need(V, self.n * self.r, "V")
+        _dtype_of(U, self.dtype, "U")
+        _dtype_of(V, self.dtype, "V")
         _ok(lib.hsl_pack(self._h, _ptr(U), _ptr(V), _stream(stream)), "hsl_pack")
 
     def apply(self, X: torch.Tensor, Y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
         batch = X.shape[0] if X.dim() == 2 else 1
+        _need(X, batch * self.n, "X")
+        _dtype_of(X, self.dtype, "X")
+        if Y is not None:
+            _need(Y, batch * self.m, "Y")
+            _dtype_of(Y, self.dtype, "Y")
         if Y is None:
             Y = torch.empty(batch, self.m, dtype=X.dtype, device=X.device,
                             pin_memory=(X.device.type == "cpu"))
@@ -193,6 +219,11 @@ class Group:
 
     def apply(self, Xs: list[torch.Tensor], Ys: list[torch.Tensor], stream=None) -> None:
         batch = Xs[0].shape[0]
+        if len(Xs) != len(self.layers) or len(Ys) != len(self.layers):
+            raise ValueError("one X and one Y per layer")
+        for l, x, y in zip(self.layers, Xs, Ys):
+            _need(x, batch * l.n, "X")
+            _need(y, batch * l.m, "Y")
         xa = (ctypes.c_void_p * len(Xs))(*[_ptr(x) for x in Xs])
         ya = (ctypes.c_void_p * len(Ys))(*[_ptr(y) for y in Ys])
         _ok(lib.hsl_group_apply(self._g, xa, ya, batch, _stream(stream)), "hsl_group_apply")
