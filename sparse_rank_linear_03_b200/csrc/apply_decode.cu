@@ -97,6 +97,7 @@ __global__ void __launch_bounds__(kThreads) k_lowrank_z(ApplyArgs a) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[b][e] = 0.f;
     if (active) {
+#pragma unroll 4
       for (int64_t j = j0 + tr; j < j1; j += RPI) {
         float v[8];
         load8<T>(V + j * rp + tc * 8, v);
@@ -130,9 +131,17 @@ __global__ void __launch_bounds__(kThreads) k_lowrank_z(ApplyArgs a) {
     __threadfence();
     for (int o = threadIdx.x; o < a.bc * rp; o += kThreads) {
       const int b = o / rp, c = o % rp;
-      float s = 0.f;
-      for (int q = 0; q < P.z_ncta; ++q) s += __ldcg(&P.zpart[(int64_t(q) * 16 + b) * rp + c]);
-      P.z[b * rp + c] = s;
+      const float* src = P.zpart + int64_t(b) * rp + c;
+      const int64_t step = int64_t(16) * rp;
+      // eight independent partial sums keep eight loads in flight; the final
+      // combination order is fixed, so z is deterministic
+      float s8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      int q = 0;
+      for (; q + 8 <= P.z_ncta; q += 8)
+#pragma unroll
+        for (int u = 0; u < 8; ++u) s8[u] += __ldcg(src + (q + u) * step);
+      for (; q < P.z_ncta; ++q) s8[q & 7] += __ldcg(src + q * step);
+      P.z[b * rp + c] = ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
     }
     if (threadIdx.x == 0) *P.zcount = 0u;
   }
@@ -250,7 +259,40 @@ __device__ __forceinline__ void nm24_rows(const ApplyProblem& P, const T* xs, fl
     float acc[BC];
 #pragma unroll
     for (int b = 0; b < BC; ++b) acc[b] = 0.f;
-    if (vec) {
+    if (BC == 1 && sizeof(T) == 2 && vec) {
+      // Batch-1 bf16: lane's chunk q needs x[16q, 16q+16) = two 16-byte units
+      // of the staged x.  Lanes 4-7 of each quarter-warp read the two units in
+      // the opposite order, which makes both loads bank-conflict free.  The two
+      // kept x of a group come out of one byte permute (bf16 pair i0, i1).
+      const uint4* xs4 = reinterpret_cast<const uint4*>(xs);
+      const int hsw = (lane >> 2) & 1;
+      float a0 = 0.f, a1 = 0.f;
+      for (int sup = 0; sup * 256 < nq; ++sup) {
+        const uint4 mw = ld_stream16(mrow + sup * 256 + lane * 8);
+        const uint32_t mws[4] = {mw.x, mw.y, mw.z, mw.w};
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const int q = (sup * 8 + t) * 32 + lane;
+          if (q < nq) {
+            const uint4 v = ld_stream16(vrow + int64_t(q) * 8);
+            const uint4 ua = xs4[2 * q + hsw], ub = xs4[2 * q + (hsw ^ 1)];
+            const uint4 xl = hsw ? ub : ua, xh = hsw ? ua : ub;
+            const uint32_t xw[8] = {xl.x, xl.y, xl.z, xl.w, xh.x, xh.y, xh.z, xh.w};
+            const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+            const uint32_t meta = (mws[t >> 1] >> ((t & 1) * 16)) & 0xFFFFu;
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              const uint32_t nib = (meta >> (4 * g)) & 0xFu;
+              const uint32_t sel = 0x1010u + (nib & 3u) * 0x22u + (nib >> 2) * 0x2200u;
+              const uint32_t xp = __byte_perm(xw[2 * g], xw[2 * g + 1], sel);
+              a0 = fmaf(bf_lo(vw[g]), bf_lo(xp), a0);
+              a1 = fmaf(bf_hi(vw[g]), bf_hi(xp), a1);
+            }
+          }
+        }
+      }
+      acc[0] = a0 + a1;
+    } else if (vec) {
       for (int sup = 0; sup * 256 < nq; ++sup) {
         const uint4 mw = ld_stream16(mrow + sup * 256 + lane * 8);
         const uint32_t mws[4] = {mw.x, mw.y, mw.z, mw.w};

@@ -1,0 +1,459 @@
+// Large-batch (prefill) apply on tcgen05 tensor cores, 2:4 S, bf16.
+//
+// "Hierarchical Sparse + Low-Rank Compression of LLMs", §Implementation and
+// operational patterns: y = S x + U (Vᵀ x).  With many tokens both products
+// are dense contractions, so they run on the 5th-generation tensor cores:
+//
+//   k_prefill_z    Z = X·V  ([T][r16] bf16).  M = 128 tokens per CTA, N = r16,
+//                  K = n, operands by TMA (128-byte swizzle), fp32 accumulator
+//                  in TMEM, bf16 epilogue.  Triggers the dependent launch at
+//                  its start.
+//   k_prefill_24   Yᵀ tile [128 rows of W × 256 tokens] in ONE TMEM
+//                  accumulator: first K = n with A = S (the 2:4 tile is
+//                  expanded to dense bf16 in shared memory by four warps from
+//                  the TMA-loaded values and index bytes), B = X; then
+//                  K = r16 with A = U, B = Z (TMA).  The producer waits for
+//                  the Z kernel (griddepcontrol.wait) only before the first Z
+//                  tile, so the S·Xᵀ part overlaps it.  Epilogue: tcgen05.ld,
+//                  bf16, stores of Y[t][i].
+//
+// Warp roles (192 threads): warp 0 lane 0 issues TMA; warp 1 owns TMEM and
+// lane 0 issues MMAs; warps 2-5 expand S and run the epilogue.  All waits are
+// bounded (kSpinLimit polls); a wait that gives up sets the error word and
+// the CTA drains its copies, frees TMEM and exits.
+#include <cuda.h>
+
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc.cuh"
+
+namespace hsl {
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 3;
+constexpr int A_BYTES = BM * BK * 2;             // 16 KB dense A tile
+constexpr int B_BYTES = BN * BK * 2;             // 32 KB B tile
+constexpr int SV_BYTES = BM * (BK / 2) * 2;      // 8 KB compressed values
+constexpr int SI_BYTES = BM * (BK / 4);          // 2 KB index bytes
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SV_BYTES + SI_BYTES;
+constexpr int PREFILL_SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+
+// Z kernel: A = X tile [128 × 64], B = Vt tile [r16 × 64]
+constexpr int ZSTAGES = 4;
+constexpr int ZA_BYTES = 128 * BK * 2;
+constexpr int ZB_MAX = 256 * BK * 2;
+constexpr int Z_SMEM = ZSTAGES * (ZA_BYTES + ZB_MAX) + 1024 + 256;
+
+struct PrefillMaps {
+  CUtensorMap x;    // X  [T][n]      box {64, 256}  (main) / {64, 128} (z)
+  CUtensorMap xz;   // X  [T][n]      box {64, 128}
+  CUtensorMap sv;   // S values [m][n/2] box {32, 128}
+  CUtensorMap si;   // S index bytes [m][n/4] box {16, 128}
+  CUtensorMap u;    // U  [m][r_pad]  box {64, 128}
+  CUtensorMap z;    // Z  [T][r16]    box {64, 256}
+  CUtensorMap vt;   // Vt [r16][n]    box {64, r16}
+};
+
+// ---- 2:4 expansion: byte selectors for __byte_perm(vals, 0, sel) ----------
+// vals = v0 | v1 << 16 (the two kept values of a group), nibble = i0 | i1 << 2.
+// Returns (sel_lo | sel_hi << 16): the dense elements {e0,e1} and {e2,e3}.
+__host__ __device__ constexpr uint32_t expand_sel(uint32_t nib) {
+  uint32_t i0 = nib & 3u, i1 = nib >> 2;
+  uint32_t s = 0;
+  for (uint32_t k = 0; k < 4; ++k) {
+    uint32_t lo_byte = (k == i0) ? 0u : (k == i1) ? 2u : 4u;  // byte 4+ of the second operand = 0
+    uint32_t two = lo_byte | ((lo_byte + 1u) << 4);
+    s |= two << (8 * k);
+  }
+  return s;
+}
+
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, uint32_t* err,
+                                              volatile int* abort_flag) {
+  if (*abort_flag) return false;
+  if (tc::mbar_wait(bar, parity, err)) return true;
+  *abort_flag = 1;
+  return false;
+}
+
+__global__ void __launch_bounds__(192, 1)
+    k_prefill_24(const __grid_constant__ PrefillMaps maps, __nv_bfloat16* __restrict__ Y, int m,
+                 int n, int T, int r16, uint32_t* err) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sA = smem;
+  unsigned char* sB = sA + STAGES * A_BYTES;
+  unsigned char* sV = sB + STAGES * B_BYTES;
+  unsigned char* sI = sV + STAGES * SV_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sI + STAGES * SI_BYTES);
+  uint64_t* expd = full + STAGES;
+  uint64_t* empty = expd + STAGES;
+  uint64_t* accf = empty + STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  __shared__ uint32_t sel_tab[16];
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ntn = (T + BN - 1) / BN;
+  const int mt = blockIdx.x / ntn, nt = blockIdx.x % ntn;
+  const int i0 = mt * BM, t0 = nt * BN;
+  const int nkS = (n + BK - 1) / BK;
+  const int nkL = (r16 + BK - 1) / BK;
+  const int nk = nkS + nkL;
+
+  if (threadIdx.x < 16) sel_tab[threadIdx.x] = expand_sel(threadIdx.x);
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int s = 0; s < STAGES; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&expd[s], 128);
+      tc::mbar_init(&empty[s], 1);
+    }
+    tc::mbar_init(accf, 1);
+    tc::fence_mbar_init();
+    tc::prefetch_tmap(&maps.x);
+    tc::prefetch_tmap(&maps.sv);
+    tc::prefetch_tmap(&maps.si);
+    if (r16 > 0) {
+      tc::prefetch_tmap(&maps.u);
+      tc::prefetch_tmap(&maps.z);
+    }
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_slot, BN);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  volatile int* abrt = &abort_flag;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int issued[STAGES] = {0, 0, 0};
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % STAGES;
+        const uint32_t ph = (kb / STAGES) & 1;
+        if (!wait_or_abort(&empty[s], ph ^ 1, err, abrt)) break;
+        if (kb < nkS) {
+          tc::mbar_expect_tx(&full[s], B_BYTES + SV_BYTES + SI_BYTES);
+          tc::tma_load_2d(sB + s * B_BYTES, &maps.x, kb * BK, t0, &full[s]);
+          tc::tma_load_2d(sV + s * SV_BYTES, &maps.sv, kb * (BK / 2), i0, &full[s]);
+          tc::tma_load_2d(sI + s * SI_BYTES, &maps.si, kb * (BK / 4), i0, &full[s]);
+        } else {
+          if (kb == nkS) pdl_wait();  // Z is written by the preceding kernel
+          const int kl = kb - nkS;
+          tc::mbar_expect_tx(&full[s], A_BYTES + B_BYTES);
+          tc::tma_load_2d(sA + s * A_BYTES, &maps.u, kl * BK, i0, &full[s]);
+          tc::tma_load_2d(sB + s * B_BYTES, &maps.z, kl * BK, t0, &full[s]);
+        }
+        ++issued[s];
+      }
+      // drain: every copy this thread started has landed before the CTA exits
+      for (int s = 0; s < STAGES; ++s)
+        if (issued[s]) tc::mbar_wait(&full[s], (issued[s] - 1) & 1, err);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = tc::idesc_bf16(BM, BN);
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % STAGES;
+        const uint32_t ph = (kb / STAGES) & 1;
+        const bool ok = kb < nkS ? wait_or_abort(&expd[s], ph, err, abrt)
+                                 : wait_or_abort(&full[s], ph, err, abrt);
+        if (!ok) break;
+        tc::tc_fence_after();
+        const uint64_t ad = tc::desc_sw128(sA + s * A_BYTES);
+        const uint64_t bd = tc::desc_sw128(sB + s * B_BYTES);
+#pragma unroll
+        for (int k = 0; k < BK / 16; ++k)
+          tc::mma_bf16(tmem, tc::desc_advance(ad, k * 32), tc::desc_advance(bd, k * 32), idesc,
+                       (kb > 0 || k > 0) ? 1u : 0u);
+        tc::mma_commit(&empty[s]);
+      }
+      tc::mma_commit(accf);
+    }
+  } else {
+    // warps 2..5: expansion of S, then the epilogue.  Row = TMEM lane.
+    const int row = ((warp & 3) << 5) | lane;
+    for (int kb = 0; kb < nkS; ++kb) {
+      const int s = kb % STAGES;
+      const uint32_t ph = (kb / STAGES) & 1;
+      if (!wait_or_abort(&full[s], ph, err, abrt)) break;
+      const uint4* vsrc = reinterpret_cast<const uint4*>(sV + s * SV_BYTES + row * 64);
+      const uint4 ib = *reinterpret_cast<const uint4*>(sI + s * SI_BYTES + row * 16);
+      const uint32_t ibw[4] = {ib.x, ib.y, ib.z, ib.w};
+      unsigned char* arow = sA + s * A_BYTES + (row >> 3) * 1024 + (row & 7) * 128;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {  // 16 bytes of values = 4 groups = 2 chunks of 8 dense
+        const uint4 v = vsrc[q];
+        const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int c = 2 * q + h;  // dense chunk (8 columns)
+          uint32_t d[4];
+#pragma unroll
+          for (int g = 0; g < 2; ++g) {
+            const int grp = 2 * c + g;  // group within the 64-column block
+            const uint32_t nib = (ibw[grp >> 2] >> (8 * (grp & 3))) & 0xFu;
+            const uint32_t sel = sel_tab[nib];
+            const uint32_t w = vw[2 * h + g];
+            d[2 * g] = __byte_perm(w, 0u, sel & 0xFFFFu);
+            d[2 * g + 1] = __byte_perm(w, 0u, sel >> 16);
+          }
+          *reinterpret_cast<uint4*>(arow + ((c ^ (row & 7)) << 4)) = make_uint4(d[0], d[1], d[2], d[3]);
+        }
+      }
+      tc::fence_async_smem();
+      tc::mbar_arrive(&expd[s]);
+    }
+    // epilogue
+    if (tc::mbar_wait(accf, 0, err) && !*abrt) {
+      tc::tc_fence_after();
+      const int i = i0 + row;
+      const uint32_t tbase = tmem + (uint32_t((warp & 3) * 32) << 16);
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        float v[32];
+        tc::tmem_ld32(tbase + c0, v);
+        if (i < m) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int t = t0 + c0 + j;
+            if (t < T) Y[int64_t(t) * m + i] = __float2bfloat16_rn(v[j]);
+          }
+        }
+      }
+    } else {
+      *abrt = 1;
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, BN);
+  }
+}
+
+// Z = X·V : one CTA per 128 tokens, N = r16 (16..256).
+__global__ void __launch_bounds__(192, 1)
+    k_prefill_z(const __grid_constant__ PrefillMaps maps, __nv_bfloat16* __restrict__ Z, int n,
+                int T, int r16, uint32_t* err) {
+  pdl_trigger();
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sA = smem;
+  unsigned char* sB = sA + ZSTAGES * ZA_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + ZSTAGES * ZB_MAX);
+  uint64_t* empty = full + ZSTAGES;
+  uint64_t* accf = empty + ZSTAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t0 = blockIdx.x * 128;
+  const int nk = (n + BK - 1) / BK;
+  const uint32_t ncols = r16 <= 32 ? 32u : r16 <= 64 ? 64u : r16 <= 128 ? 128u : 256u;
+  const int b_bytes = r16 * BK * 2;
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int s = 0; s < ZSTAGES; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    tc::mbar_init(accf, 1);
+    tc::fence_mbar_init();
+    tc::prefetch_tmap(&maps.xz);
+    tc::prefetch_tmap(&maps.vt);
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_slot, ncols);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  volatile int* abrt = &abort_flag;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int issued[ZSTAGES] = {0, 0, 0, 0};
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % ZSTAGES;
+        const uint32_t ph = (kb / ZSTAGES) & 1;
+        if (!wait_or_abort(&empty[s], ph ^ 1, err, abrt)) break;
+        tc::mbar_expect_tx(&full[s], ZA_BYTES + b_bytes);
+        tc::tma_load_2d(sA + s * ZA_BYTES, &maps.xz, kb * BK, t0, &full[s]);
+        tc::tma_load_2d(sB + s * ZB_MAX, &maps.vt, kb * BK, 0, &full[s]);
+        ++issued[s];
+      }
+      for (int s = 0; s < ZSTAGES; ++s)
+        if (issued[s]) tc::mbar_wait(&full[s], (issued[s] - 1) & 1, err);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = tc::idesc_bf16(128, r16);
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % ZSTAGES;
+        const uint32_t ph = (kb / ZSTAGES) & 1;
+        if (!wait_or_abort(&full[s], ph, err, abrt)) break;
+        tc::tc_fence_after();
+        const uint64_t ad = tc::desc_sw128(sA + s * ZA_BYTES);
+        const uint64_t bd = tc::desc_sw128(sB + s * ZB_MAX);
+#pragma unroll
+        for (int k = 0; k < BK / 16; ++k)
+          tc::mma_bf16(tmem, tc::desc_advance(ad, k * 32), tc::desc_advance(bd, k * 32), idesc,
+                       (kb > 0 || k > 0) ? 1u : 0u);
+        tc::mma_commit(&empty[s]);
+      }
+      tc::mma_commit(accf);
+    }
+  } else {
+    const int row = ((warp & 3) << 5) | lane;  // token within the tile
+    if (tc::mbar_wait(accf, 0, err) && !*abrt) {
+      tc::tc_fence_after();
+      const int t = t0 + row;
+      const uint32_t tbase = tmem + (uint32_t((warp & 3) * 32) << 16);
+      for (int c0 = 0; c0 < r16; c0 += 32) {
+        float v[32];
+        tc::tmem_ld32(tbase + c0, v);
+        if (t < T) {
+          __nv_bfloat16* zr = Z + int64_t(t) * r16 + c0;
+#pragma unroll
+          for (int j = 0; j < 32; j += 8) {
+            if (c0 + j < r16) {
+              uint4 o;
+              o.x = __bfloat16_as_ushort(__float2bfloat16_rn(v[j])) |
+                    (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(v[j + 1]))) << 16);
+              o.y = __bfloat16_as_ushort(__float2bfloat16_rn(v[j + 2])) |
+                    (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(v[j + 3]))) << 16);
+              o.z = __bfloat16_as_ushort(__float2bfloat16_rn(v[j + 4])) |
+                    (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(v[j + 5]))) << 16);
+              o.w = __bfloat16_as_ushort(__float2bfloat16_rn(v[j + 6])) |
+                    (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(v[j + 7]))) << 16);
+              *reinterpret_cast<uint4*>(zr + j) = o;
+            }
+          }
+        }
+      }
+    } else {
+      *abrt = 1;
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, ncols);
+  }
+}
+
+// ---- host: tensor maps through the driver entry point (no libcuda link) -----
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+// 2-D row-major map: `rows` × `cols` elements, box {box_cols, box_rows}.
+bool make_map(CUtensorMap* map, CUtensorMapDataType dt, int esize, const void* base, int64_t rows,
+              int64_t cols, int64_t row_stride_elems, int box_cols, int box_rows,
+              CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(row_stride_elems * esize)};
+  cuuint32_t box[2] = {cuuint32_t(box_cols), cuuint32_t(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+// Z workspace and Vt come from the handle (Vt built by prefill_pack_run).
+bool prefill_supported(const Handle& h, const void* X) {
+  return h.fmt == HSL_FMT_NM24 && h.dtype == HSL_BF16 && h.n % 64 == 0 &&
+         (reinterpret_cast<uintptr_t>(X) % 16) == 0 && encode_fn() != nullptr;
+}
+
+hsl_status apply_prefill_run(Handle& h, const void* X, void* Y, int64_t T, cudaStream_t s) {
+  const int r16 = int(round_up(h.r, 16));
+  if (r16 > 256) return HSL_ERR_UNSUPPORTED;
+  const int64_t m = h.m, n = h.n;
+  if (r16 > 0) {
+    if (hsl_status e = ensure(h.zpre, size_t(T) * r16 * 2, "prefill Z")) return e;
+  }
+  PrefillMaps maps;
+  memset(&maps, 0, sizeof(maps));
+  const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const auto SW = CU_TENSOR_MAP_SWIZZLE_128B, NO = CU_TENSOR_MAP_SWIZZLE_NONE;
+  bool ok = make_map(&maps.x, BF, 2, X, T, n, n, 64, 256, SW) &&
+            make_map(&maps.xz, BF, 2, X, T, n, n, 64, 128, SW) &&
+            make_map(&maps.sv, BF, 2, h.nm_val.p, m, n / 2, n / 2, 32, 128, NO) &&
+            make_map(&maps.si, U8, 1, h.nm_idx.p, m, n / 4, n / 4, 16, 128, NO);
+  if (ok && r16 > 0)
+    ok = make_map(&maps.u, BF, 2, h.U.p, m, h.r_pad, h.r_pad, 64, 128, SW) &&
+         make_map(&maps.z, BF, 2, h.zpre.p, T, r16, r16, 64, 256, SW) &&
+         make_map(&maps.vt, BF, 2, h.Vt.p, r16, n, n, 64, r16, SW);
+  if (!ok) {
+    set_message("tensor map encoding failed");
+    return HSL_ERR_CUDA;
+  }
+  uint32_t* err = static_cast<uint32_t*>(h.err.p);
+  if (r16 > 0) {
+    cudaFuncSetAttribute(k_prefill_z, cudaFuncAttributeMaxDynamicSharedMemorySize, Z_SMEM);
+    k_prefill_z<<<unsigned((T + 127) / 128), 192, Z_SMEM, s>>>(
+        maps, static_cast<__nv_bfloat16*>(h.zpre.p), int(n), int(T), r16, err);
+    note_launch();
+    if (hsl_status e = cuda_fail(cudaGetLastError(), "prefill z launch")) return e;
+  }
+  if (cudaError_t e = cudaFuncSetAttribute(k_prefill_24, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           PREFILL_SMEM))
+    return cuda_fail(e, "prefill smem attribute");
+  const int64_t tiles = ((m + BM - 1) / BM) * ((T + BN - 1) / BN);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(tiles));
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = PREFILL_SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = r16 > 0 ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  note_launch();
+  return cuda_fail(cudaLaunchKernelEx(&cfg, k_prefill_24, maps,
+                                      static_cast<__nv_bfloat16*>(Y), int(m), int(n), int(T),
+                                      r16, err),
+                   "prefill launch");
+}
+
+}  // namespace hsl

@@ -59,9 +59,6 @@ void release(DevBuf& b) {
   b.bytes = 0;
 }
 
-hsl_status apply_decode_run(ApplyPlan& plan, const void* X, void* Y, const void* const* xy_dev,
-                            int64_t batch, int num_sms, cudaStream_t s);
-
 namespace {
 
 hsl_status invalid(const std::string& why) {
@@ -108,7 +105,7 @@ hsl_status ensure_err_word(Handle& h, cudaStream_t s) {
 void free_all(Handle& h) {
   DevBuf* bufs[] = {&h.row_ptr, &h.col, &h.val, &h.nm_val, &h.nm_idx, &h.prow, &h.pcol,
                     &h.pval, &h.pmeta, &h.U, &h.V, &h.Vt, &h.zpart, &h.z, &h.zcount,
-                    &h.err, &h.split_ws, &h.flags, &h.xstage, &h.ystage, &h.plan.probs,
+                    &h.err, &h.split_ws, &h.flags, &h.xstage, &h.ystage, &h.zpre, &h.plan.probs,
                     &h.plan.prob_row0, &h.plan.cta_rows, &h.plan.xy_ptrs};
   for (DevBuf* b : bufs) release(*b);
 }
@@ -376,7 +373,11 @@ hsl_status hsl_apply(hsl_handle h, const void* X, void* Y, int64_t batch, hsl_st
     if (hsl_status e = ensure(H.ystage, size_t(batch) * H.m * eb, "Y staging")) return e;
     Yd = H.ystage.p;
   }
-  if (hsl_status e = apply_decode_run(H.plan, Xd, Yd, nullptr, batch, H.num_sms, s)) return e;
+  if (batch >= kPrefillMinBatch && prefill_supported(H, Xd)) {
+    if (hsl_status e = apply_prefill_run(H, Xd, Yd, batch, s)) return e;
+  } else {
+    if (hsl_status e = apply_decode_run(H.plan, Xd, Yd, nullptr, batch, H.num_sms, s)) return e;
+  }
   if (yh)
     return cuda_fail(cudaMemcpyAsync(Y, Yd, size_t(batch) * H.m * eb, cudaMemcpyDeviceToHost, s),
                      "Y device-to-host");

@@ -85,7 +85,7 @@ struct Handle {
 
   // workspace
   DevBuf zpart, z, zcount, err, split_ws, flags;
-  DevBuf xstage, ystage;
+  DevBuf xstage, ystage, zpre;
   int z_ncta = 0;
   ApplyPlan plan;  // the single-layer plan, built by hsl_pack
 };
@@ -99,8 +99,12 @@ hsl_status pack_factors_run(Handle& h, const void* U, const void* V, cudaStream_
 hsl_status csr_convert_run(Handle& h, const int32_t* row_ptr, const int32_t* col,
                            const void* val, cudaStream_t s);
 hsl_status plan_build(ApplyPlan& plan, Handle* const* hs, int count, cudaStream_t s);
-hsl_status apply_run(ApplyPlan& plan, const void* X, void* Y, const void* const* Xs,
-                     void* const* Ys, int64_t batch, cudaStream_t s);
+hsl_status apply_decode_run(ApplyPlan& plan, const void* X, void* Y, const void* const* xy_dev,
+                            int64_t batch, int num_sms, cudaStream_t s);
+// tensor-core path for large batches (2:4, bf16, n % 64 == 0)
+constexpr int64_t kPrefillMinBatch = 64;
+bool prefill_supported(const Handle& h, const void* X);
+hsl_status apply_prefill_run(Handle& h, const void* X, void* Y, int64_t T, cudaStream_t s);
 
 }  // namespace hsl
 

@@ -141,6 +141,17 @@ __global__ void k_pad_cols(const SB* __restrict__ src, int64_t rows, int32_t r, 
   }
 }
 
+// Vt[c][j] = V[j][c] for c < r_pad, zero rows up to r16 (prefill B operand).
+__global__ void k_transpose_v(const uint16_t* __restrict__ V, int64_t n, int32_t r_pad, int32_t r16,
+                              uint16_t* __restrict__ Vt) {
+  const int64_t total = int64_t(r16) * n;
+  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
+       e += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t c = e / n, j = e % n;
+    Vt[e] = c < r_pad ? V[j * r_pad + c] : uint16_t(0);
+  }
+}
+
 // One CTA: boundaries of `slices` row ranges of equal streamed bytes over the
 // concatenated rows of all layers.  Cost of the first i rows of layer p:
 //   CSR : prow[i]·(value + 2 index bytes) + i·(U row bytes + 8)
@@ -257,6 +268,14 @@ hsl_status pack_factors_run(Handle& h, const void* U, const void* V, cudaStream_
                                                           h.r, h.r_pad, static_cast<uint32_t*>(dst));
     note_launch();
   }
+  if (h.fmt == HSL_FMT_NM24 && h.dtype == HSL_BF16 && h.n % 64 == 0) {
+    const int32_t r16 = int32_t(round_up(h.r, 16));
+    if (hsl_status e = ensure(h.Vt, size_t(r16) * h.n * 2, "V transpose")) return e;
+    const int64_t grid = std::min<int64_t>((r16 * h.n + 255) / 256, int64_t(h.num_sms) * 16);
+    k_transpose_v<<<unsigned(grid), 256, 0, s>>>(static_cast<const uint16_t*>(h.V.p), h.n, h.r_pad,
+                                                 r16, static_cast<uint16_t*>(h.Vt.p));
+    note_launch();
+  }
   return cuda_fail(cudaGetLastError(), "factor pack launch");
 }
 
@@ -286,12 +305,13 @@ hsl_status plan_build(ApplyPlan& plan, Handle* const* hs, int count, cudaStream_
     P.meta_stride = h.meta_stride;
     P.row0 = row0;
     row0 += h.m;
-    // z: about 32 KB of V per CTA, at most 2 CTAs per SM for one layer
+    // z: about 128 KB of V per CTA (at most 64 CTAs per layer), so the final
+    // reduction over the CTAs' partials stays short
     int zn = 0;
     if (h.r_pad > 0) {
       const int64_t vbytes = h.n * int64_t(h.r_pad) * eb;
-      zn = int(std::min<int64_t>(std::max<int64_t>((vbytes + 32767) / 32768, 1),
-                                 std::min<int64_t>(h.n, 2 * h.num_sms)));
+      zn = int(std::min<int64_t>(std::max<int64_t>((vbytes + 131071) / 131072, 1),
+                                 std::min<int64_t>(h.n, 64)));
       if (hsl_status e = ensure(h.zpart, size_t(zn) * 16 * h.r_pad * 4, "z partials")) return e;
       if (hsl_status e = ensure(h.z, size_t(16) * h.r_pad * 4, "z")) return e;
       if (h.zcount.p == nullptr) {
