@@ -93,6 +93,15 @@ def test_topk_tie_heavy(hsl, dtype, shape, frac):
     assert_topk_parity(hsl, W, dtype, dtype, frac)
 
 
+@pytest.mark.parametrize("dtype,shape", [("bf16", (3, 40000)), ("f32", (5, 20000)),
+                                         ("bf16", (70, 32768)), ("f32", (33, 16384))])
+@pytest.mark.parametrize("frac", [0.01, 0.5])
+def test_topk_wide_rows(hsl, dtype, shape, frac):
+    """Rows wider than one register block (per-row emit) and exactly one block."""
+    W = tie_heavy(*shape, seed=shape[1], dtype=dtype)
+    assert_topk_parity(hsl, W, dtype, dtype, frac)
+
+
 def test_topk_unaligned_input_pointer(hsl):
     """W and R starting 4 bytes past an allocation (scalar path)."""
     W = synth.student_t_f32(64, 130, 3)
