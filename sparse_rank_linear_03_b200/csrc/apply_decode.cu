@@ -270,11 +270,17 @@ __device__ __forceinline__ void nm24_rows(const ApplyProblem& P, const T* xs, fl
       for (int sup = 0; sup * 256 < nq; ++sup) {
         const uint4 mw = ld_stream16(mrow + sup * 256 + lane * 8);
         const uint32_t mws[4] = {mw.x, mw.y, mw.z, mw.w};
+        uint4 vv[8];  // all eight value chunks of this lane in flight at once
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const int q = (sup * 8 + t) * 32 + lane;
+          if (q < nq) vv[t] = ld_stream16(vrow + int64_t(q) * 8);
+        }
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
           const int q = (sup * 8 + t) * 32 + lane;
           if (q < nq) {
-            const uint4 v = ld_stream16(vrow + int64_t(q) * 8);
+            const uint4 v = vv[t];
             const uint4 ua = xs4[2 * q + hsw], ub = xs4[2 * q + (hsw ^ 1)];
             const uint4 xl = hsw ? ub : ua, xh = hsw ? ua : ub;
             const uint32_t xw[8] = {xl.x, xl.y, xl.z, xl.w, xh.x, xh.y, xh.z, xh.w};

@@ -136,6 +136,10 @@ __global__ void __launch_bounds__(192, 1)
 
   if (warp == 0) {
     if (lane == 0) {
+      // X and Z tiles are re-read by every 128-row tile: keep them in L2;
+      // S and U are read by few CTAs in a row: let them leave L2 first.
+      const uint64_t keep = tc::make_policy_evict_last();
+      const uint64_t stream = tc::make_policy_evict_first();
       int issued[STAGES] = {0, 0, 0};
       for (int kb = 0; kb < nk; ++kb) {
         const int s = kb % STAGES;
@@ -143,15 +147,15 @@ __global__ void __launch_bounds__(192, 1)
         if (!wait_or_abort(&empty[s], ph ^ 1, err, abrt)) break;
         if (kb < nkS) {
           tc::mbar_expect_tx(&full[s], B_BYTES + SV_BYTES + SI_BYTES);
-          tc::tma_load_2d(sB + s * B_BYTES, &maps.x, kb * BK, t0, &full[s]);
-          tc::tma_load_2d(sV + s * SV_BYTES, &maps.sv, kb * (BK / 2), i0, &full[s]);
-          tc::tma_load_2d(sI + s * SI_BYTES, &maps.si, kb * (BK / 4), i0, &full[s]);
+          tc::tma_load_2d_hint(sB + s * B_BYTES, &maps.x, kb * BK, t0, &full[s], keep);
+          tc::tma_load_2d_hint(sV + s * SV_BYTES, &maps.sv, kb * (BK / 2), i0, &full[s], stream);
+          tc::tma_load_2d_hint(sI + s * SI_BYTES, &maps.si, kb * (BK / 4), i0, &full[s], stream);
         } else {
           if (kb == nkS) pdl_wait();  // Z is written by the preceding kernel
           const int kl = kb - nkS;
           tc::mbar_expect_tx(&full[s], A_BYTES + B_BYTES);
-          tc::tma_load_2d(sA + s * A_BYTES, &maps.u, kl * BK, i0, &full[s]);
-          tc::tma_load_2d(sB + s * B_BYTES, &maps.z, kl * BK, t0, &full[s]);
+          tc::tma_load_2d_hint(sA + s * A_BYTES, &maps.u, kl * BK, i0, &full[s], stream);
+          tc::tma_load_2d_hint(sB + s * B_BYTES, &maps.z, kl * BK, t0, &full[s], keep);
         }
         ++issued[s];
       }
@@ -186,13 +190,17 @@ __global__ void __launch_bounds__(192, 1)
       const int s = kb % STAGES;
       const uint32_t ph = (kb / STAGES) & 1;
       if (!wait_or_abort(&full[s], ph, err, abrt)) break;
-      const uint4* vsrc = reinterpret_cast<const uint4*>(sV + s * SV_BYTES + row * 64);
+      // values arrive with the 64-byte TMA swizzle: 16-byte chunk q of a row
+      // sits at chunk q ^ ((row >> 1) & 3), which spreads a quarter-warp over
+      // all banks
+      const unsigned char* vrow_s = sV + s * SV_BYTES + row * 64;
+      const int vsw = (row >> 1) & 3;
       const uint4 ib = *reinterpret_cast<const uint4*>(sI + s * SI_BYTES + row * 16);
       const uint32_t ibw[4] = {ib.x, ib.y, ib.z, ib.w};
       unsigned char* arow = sA + s * A_BYTES + (row >> 3) * 1024 + (row & 7) * 128;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {  // 16 bytes of values = 4 groups = 2 chunks of 8 dense
-        const uint4 v = vsrc[q];
+        const uint4 v = *reinterpret_cast<const uint4*>(vrow_s + ((q ^ vsw) << 4));
         const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -417,7 +425,8 @@ hsl_status apply_prefill_run(Handle& h, const void* X, void* Y, int64_t T, cudaS
   const auto SW = CU_TENSOR_MAP_SWIZZLE_128B, NO = CU_TENSOR_MAP_SWIZZLE_NONE;
   bool ok = make_map(&maps.x, BF, 2, X, T, n, n, 64, 256, SW) &&
             make_map(&maps.xz, BF, 2, X, T, n, n, 64, 128, SW) &&
-            make_map(&maps.sv, BF, 2, h.nm_val.p, m, n / 2, n / 2, 32, 128, NO) &&
+            make_map(&maps.sv, BF, 2, h.nm_val.p, m, n / 2, n / 2, 32, 128,
+                     CU_TENSOR_MAP_SWIZZLE_64B) &&
             make_map(&maps.si, U8, 1, h.nm_idx.p, m, n / 4, n / 4, 16, 128, NO);
   if (ok && r16 > 0)
     ok = make_map(&maps.u, BF, 2, h.U.p, m, h.r_pad, h.r_pad, 64, 128, SW) &&

@@ -38,9 +38,11 @@ __device__ __forceinline__ float bf_hi(uint32_t u) { return __uint_as_float(u & 
 
 // ---- memory -------------------------------------------------------------
 // 16-byte streaming load that does not allocate in L1 (weights are read once).
+// Not volatile: the data is read-only for the kernel's lifetime, so the
+// compiler may batch these loads ahead of the arithmetic that consumes them.
 __device__ __forceinline__ uint4 ld_stream16(const void* p) {
   uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "l"(p));
   return v;
