@@ -105,6 +105,33 @@ hsl_status hsl_destroy(hsl_handle h);
 hsl_status hsl_split_topk(hsl_handle h, const void* W, hsl_dtype w_dtype,
                           double frac, void* residual, hsl_stream s);
 
+/* Top-k split that allocates no device memory.  The source pages have no
+ * counterpart of this entry point: it exists for callers that may not call
+ * cudaMalloc — code inside a serving runtime or plugin host that owns all
+ * device memory and hands out pre-planned buffers, code that must not risk the
+ * device-wide synchronisation of cudaMalloc/cudaFree, or callers without a
+ * handle to keep workspace alive.  It computes exactly what hsl_split_topk
+ * computes on a CSR handle (same kernels, bit-identical results), with every
+ * input and output owned by the caller and no handle:
+ *   W:        device, m×n row-major, element type w_dtype.
+ *   frac:     k = floor(frac·m·n) kept (frac ≤ 0 → 0, frac ≥ 1 → m·n).
+ *   row_ptr:  device int32[m+1];  col: device int32[k];  val: device, k values
+ *             of val_dtype (f32 → bf16 rounds to nearest even).  col/val may
+ *             be NULL when k == 0.
+ *   residual: device m×n of w_dtype, or NULL.
+ *   status:   device uint32 or NULL; cleared, then OR-ed with 1 for a NaN in
+ *             W and 2 for a device wait that gave up.
+ * Scratch: one fixed static device array of about 640 KB per GPU (held until
+ * the process exits).  Limits: m ≤ 65536 and m·n < 2^31, else
+ * HSL_ERR_UNSUPPORTED.  The first call on a device looks the array up with
+ * that device current (make it before any stream capture).  All calls share
+ * the array, so calls that can overlap on the GPU race: serialise them on one
+ * stream.  Asynchronous on s, like the other entry points. */
+hsl_status hsl_split_topk_noalloc(const void* W, int64_t m, int64_t n, hsl_dtype w_dtype,
+                                  double frac, int32_t* row_ptr, int32_t* col, void* val,
+                                  hsl_dtype val_dtype, void* residual, uint32_t* status,
+                                  hsl_stream s);
+
 /* Number of stored sparse values (k for CSR, m·n/2 for NM24; 0 before any
  * split/set).  Host-only, no synchronisation (k is known on the host). */
 hsl_status hsl_get_nnz(hsl_handle h, int64_t* nnz);

@@ -26,7 +26,7 @@ EXPORTS = (
     "hsl_create", "hsl_destroy", "hsl_split_topk", "hsl_get_nnz", "hsl_get_sparse",
     "hsl_set_sparse_csr", "hsl_set_sparse_nm24", "hsl_pack", "hsl_apply",
     "hsl_group_create", "hsl_group_apply", "hsl_group_destroy", "hsl_check",
-    "hsl_status_str", "hsl_last_message", "hsl_launch_count",
+    "hsl_status_str", "hsl_last_message", "hsl_launch_count", "hsl_split_topk_noalloc",
 )
 
 
@@ -60,6 +60,7 @@ def _load() -> ctypes.CDLL:
         "hsl_status_str": [ctypes.c_int],
         "hsl_last_message": [],
         "hsl_launch_count": [],
+        "hsl_split_topk_noalloc": [P, I64, I64, ctypes.c_int, D, P, P, P, ctypes.c_int, P, P, P],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
