@@ -75,7 +75,7 @@ def peaks() -> dict:
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -87,7 +87,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100", "-i", self.gpu_id],
+                 "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
@@ -107,7 +107,7 @@ class ClockSampler:
         rows = []
         for line in (self.out or "").splitlines():
             parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
+            if len(parts) < 9 or parts[0].lower() != self.gpu_id.lower():
                 continue
             try:
                 rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
@@ -137,13 +137,21 @@ def dist_setup(ngpus: int):
 
 
 def dist_max(x: float, world: int) -> float:
+    """Max over ranks (the step time every rank reports is the slowest rank's)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cpu" if dist.get_backend() == "gloo" else "cuda"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_value(per_rank_units: float, max_seconds: float, world: int) -> float:
+    """Whole-job throughput of independent replicas: all ranks' units over the
+    slowest rank's time (weak scaling: every rank runs the same workload)."""
+    return per_rank_units * world / max_seconds
 
 
 def barrier(world: int):

@@ -244,6 +244,66 @@ __device__ __forceinline__ void csr_rows(const ApplyProblem& P, const T* xs, flo
   }
 }
 
+// Batch-1 bf16 2:4 rows.  A warp takes a row; lane l handles value chunks
+// q = (8·s + t)·32 + l (8 values = 4 groups each) and, per super-chunk s,
+// issues its metadata load and all eight 16-byte value loads before using any.
+// x is staged with its 16-byte unit U stored at U ^ ((U >> 3) & 1), so the two
+// units of a chunk's 16-element window come back in order and every
+// quarter-warp's loads hit distinct banks.  The two kept x of a group are
+// picked with one byte permute whose selector comes from a 16-entry table.
+__device__ __forceinline__ void stage_x_nm24_b1(__nv_bfloat16* xs, const __nv_bfloat16* x, int n) {
+  const uint4* src = reinterpret_cast<const uint4*>(x);
+  uint4* dst = reinterpret_cast<uint4*>(xs);
+  const int nu = n / 8;
+  for (int U = threadIdx.x; U < nu; U += kThreads) dst[U ^ ((U >> 3) & 1)] = src[U];
+}
+
+__device__ __forceinline__ void nm24_rows_b1(const ApplyProblem& P, const __nv_bfloat16* xs,
+                                             const uint32_t* sel_lut, float* ysp, int s0, int s1) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int n = P.n;
+  const int64_t half = n / 2;
+  const int nq = n / 16;
+  const __nv_bfloat16* pval = static_cast<const __nv_bfloat16*>(P.pval);
+  const uint4* xs4 = reinterpret_cast<const uint4*>(xs);
+  for (int i = s0 + warp; i < s1; i += kThreads / 32) {
+    const __nv_bfloat16* vrow = pval + int64_t(i) * half;
+    const uint16_t* mrow = P.pmeta + int64_t(i) * P.meta_stride;
+    float a0 = 0.f, a1 = 0.f;
+    for (int sup = 0; sup * 256 < nq; ++sup) {
+      const uint4 mw = ld_stream16(mrow + sup * 256 + lane * 8);
+      uint4 vv[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const int q = (sup * 8 + t) * 32 + lane;
+        if (q < nq) vv[t] = ld_stream16(vrow + int64_t(q) * 8);
+      }
+      const uint32_t mws[4] = {mw.x, mw.y, mw.z, mw.w};
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const int q = (sup * 8 + t) * 32 + lane;
+        if (q < nq) {
+          const int sw = (q >> 2) & 1;
+          const uint4 xl = xs4[(2 * q) ^ sw], xh = xs4[(2 * q + 1) ^ sw];
+          const uint32_t xw[8] = {xl.x, xl.y, xl.z, xl.w, xh.x, xh.y, xh.z, xh.w};
+          const uint32_t vw[4] = {vv[t].x, vv[t].y, vv[t].z, vv[t].w};
+          const uint32_t meta = mws[t >> 1] >> ((t & 1) * 16);
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const uint32_t xp = __byte_perm(xw[2 * g], xw[2 * g + 1], sel_lut[(meta >> (4 * g)) & 0xFu]);
+            a0 = fmaf(bf_lo(vw[g]), bf_lo(xp), a0);
+            a1 = fmaf(bf_hi(vw[g]), bf_hi(xp), a1);
+          }
+        }
+      }
+    }
+    float acc = a0 + a1;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) ysp[i - s0] = acc;
+  }
+}
+
 template <typename T, int BC>
 __device__ __forceinline__ void nm24_rows(const ApplyProblem& P, const T* xs, float* ysp, int s0,
                                           int s1) {
@@ -259,46 +319,7 @@ __device__ __forceinline__ void nm24_rows(const ApplyProblem& P, const T* xs, fl
     float acc[BC];
 #pragma unroll
     for (int b = 0; b < BC; ++b) acc[b] = 0.f;
-    if (BC == 1 && sizeof(T) == 2 && vec) {
-      // Batch-1 bf16: lane's chunk q needs x[16q, 16q+16) = two 16-byte units
-      // of the staged x.  Lanes 4-7 of each quarter-warp read the two units in
-      // the opposite order, which makes both loads bank-conflict free.  The two
-      // kept x of a group come out of one byte permute (bf16 pair i0, i1).
-      const uint4* xs4 = reinterpret_cast<const uint4*>(xs);
-      const int hsw = (lane >> 2) & 1;
-      float a0 = 0.f, a1 = 0.f;
-      for (int sup = 0; sup * 256 < nq; ++sup) {
-        const uint4 mw = ld_stream16(mrow + sup * 256 + lane * 8);
-        const uint32_t mws[4] = {mw.x, mw.y, mw.z, mw.w};
-        uint4 vv[8];  // all eight value chunks of this lane in flight at once
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          const int q = (sup * 8 + t) * 32 + lane;
-          if (q < nq) vv[t] = ld_stream16(vrow + int64_t(q) * 8);
-        }
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          const int q = (sup * 8 + t) * 32 + lane;
-          if (q < nq) {
-            const uint4 v = vv[t];
-            const uint4 ua = xs4[2 * q + hsw], ub = xs4[2 * q + (hsw ^ 1)];
-            const uint4 xl = hsw ? ub : ua, xh = hsw ? ua : ub;
-            const uint32_t xw[8] = {xl.x, xl.y, xl.z, xl.w, xh.x, xh.y, xh.z, xh.w};
-            const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
-            const uint32_t meta = (mws[t >> 1] >> ((t & 1) * 16)) & 0xFFFFu;
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              const uint32_t nib = (meta >> (4 * g)) & 0xFu;
-              const uint32_t sel = 0x1010u + (nib & 3u) * 0x22u + (nib >> 2) * 0x2200u;
-              const uint32_t xp = __byte_perm(xw[2 * g], xw[2 * g + 1], sel);
-              a0 = fmaf(bf_lo(vw[g]), bf_lo(xp), a0);
-              a1 = fmaf(bf_hi(vw[g]), bf_hi(xp), a1);
-            }
-          }
-        }
-      }
-      acc[0] = a0 + a1;
-    } else if (vec) {
+    if (vec) {
       for (int sup = 0; sup * 256 < nq; ++sup) {
         const uint4 mw = ld_stream16(mrow + sup * 256 + lane * 8);
         const uint32_t mws[4] = {mw.x, mw.y, mw.z, mw.w};
@@ -350,8 +371,11 @@ __device__ __forceinline__ void nm24_rows(const ApplyProblem& P, const T* xs, fl
 
 // ---- the persistent apply kernel ---------------------------------------------------
 template <typename T, int BC, bool CSR>
-__global__ void __launch_bounds__(kThreads) k_apply_decode(ApplyArgs a) {
+__global__ void __launch_bounds__(kThreads, 2) k_apply_decode(ApplyArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ uint32_t sel_lut[16];  // byte-permute selector of a 2:4 nibble (x[i0], x[i1])
+  if (threadIdx.x < 16)
+    sel_lut[threadIdx.x] = 0x1010u + (threadIdx.x & 3u) * 0x22u + (threadIdx.x >> 2) * 0x2200u;
   float* zs = reinterpret_cast<float*>(smem);                 // [BC][r_pad_max]
   float* ysp = zs + BC * a.r_pad_max;                          // [kSeg][BC]
   T* xs = reinterpret_cast<T*>(ysp + kSeg * BC);               // [(n+1)][BC]
@@ -376,13 +400,23 @@ __global__ void __launch_bounds__(kThreads) k_apply_decode(ApplyArgs a) {
     const int64_t p_end = a.prob_row0[p + 1];
     const int l0 = int(row - P.row0);
     const int l1 = int(min(row_end, p_end) - P.row0);
+    // the batch-1 bf16 2:4 fast path needs a 16-byte aligned x and n % 16 == 0
+    const bool fast24 = !CSR && BC == 1 && sizeof(T) == 2 && P.n % 16 == 0 &&
+                        (reinterpret_cast<uintptr_t>(x_of<T>(a, p) + int64_t(a.b0) * P.n) % 16) == 0;
     __syncthreads();
-    stage_x<T, BC>(xs, x_of<T>(a, p), P.n, a.b0, a.bc);
+    if (fast24)
+      stage_x_nm24_b1(reinterpret_cast<__nv_bfloat16*>(xs),
+                      reinterpret_cast<const __nv_bfloat16*>(x_of<T>(a, p) + int64_t(a.b0) * P.n),
+                      P.n);
+    else
+      stage_x<T, BC>(xs, x_of<T>(a, p), P.n, a.b0, a.bc);
     __syncthreads();
     T* y = y_of<T>(a, p) + int64_t(a.b0) * P.m;
     for (int s0 = l0; s0 < l1; s0 += kSeg) {
       const int s1 = min(s0 + kSeg, l1);
       if (CSR) csr_rows<T, BC>(P, xs, ysp, s0, s1);
+      else if (fast24)
+        nm24_rows_b1(P, reinterpret_cast<const __nv_bfloat16*>(xs), sel_lut, ysp, s0, s1);
       else nm24_rows<T, BC>(P, xs, ysp, s0, s1);
       __syncthreads();
       if (!waited) {
@@ -428,8 +462,13 @@ hsl_status launch_chunk(ApplyPlan& plan, ApplyArgs a, int num_sms, cudaStream_t 
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, ak, kThreads, sm);
   occ = std::max(1, std::min(occ, 24));
   while (24 % occ) --occ;
+  // every CTA stages the whole x of its layers: keep at least ~64 rows per CTA
+  // so small layers are not dominated by that staging
+  int grid = num_sms * occ;
+  const int64_t row_cap = std::max<int64_t>(1, plan.rows_total / 64);
+  if (grid > row_cap) grid = int(row_cap);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(unsigned(num_sms * occ));
+  cfg.gridDim = dim3(unsigned(grid));
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = sm;
   cfg.stream = s;

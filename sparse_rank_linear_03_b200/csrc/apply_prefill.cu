@@ -8,22 +8,34 @@
 //                  K = n, operands by TMA (128-byte swizzle), fp32 accumulator
 //                  in TMEM, bf16 epilogue.  Triggers the dependent launch at
 //                  its start.
-//   k_prefill_24   Yᵀ tile [128 rows of W × 256 tokens] in ONE TMEM
-//                  accumulator: first K = n with A = S (the 2:4 tile is
-//                  expanded to dense bf16 in shared memory by four warps from
-//                  the TMA-loaded values and index bytes), B = X; then
-//                  K = r16 with A = U, B = Z (TMA).  The producer waits for
-//                  the Z kernel (griddepcontrol.wait) only before the first Z
-//                  tile, so the S·Xᵀ part overlaps it.  Epilogue: tcgen05.ld,
-//                  bf16, stores of Y[t][i].
+//   k_prefill_24sp the default: Yᵀ tile [256 rows of W × 192 tokens], two
+//                  128-row TMEM accumulators sharing every X tile; the 2:4
+//                  part runs on the sparse MMA (tcgen05.mma.sp, compressed
+//                  values straight from TMA, metadata in TMEM), the low-rank
+//                  part on dense MMAs (A = U, B = Z) into the same
+//                  accumulators.  See the comment above the kernel.
+//   k_prefill_24   the same product with each 2:4 tile expanded to dense bf16
+//                  in shared memory (twice the S work on the dense MMA), one
+//                  128×256 accumulator.  Kept as a cross-check of the sparse
+//                  kernel (selected by HSL_PREFILL_EXPAND=1).
+//   In both, the producer waits for the Z kernel (griddepcontrol.wait) only
+//   before the first Z tile, so the S·Xᵀ part overlaps it; the epilogue reads
+//   TMEM (tcgen05.ld), rounds to bf16 and stores Y[t][i] with streaming stores.
+//
+// Why 256×192 tiles: with a 2:4 sparse MMA the tensor work per byte of X halves,
+// so the X traffic per flop decides whether L2 can feed the MMAs; sharing each
+// X tile across 256 rows of W lowers the bytes per flop about 1.6× against a
+// 128×256 tile.  TMEM holds 2×192 accumulator columns plus 4-column-aligned
+// metadata slots (the sparse MMA requires that alignment).
 //
 // Warp roles (192 threads): warp 0 lane 0 issues TMA; warp 1 owns TMEM and
-// lane 0 issues MMAs; warps 2-5 expand S and run the epilogue.  All waits are
-// bounded (kSpinLimit polls); a wait that gives up sets the error word and
-// the CTA drains its copies, frees TMEM and exits.
+// lane 0 issues MMAs; warps 2-5 move metadata (or expand S) and run the
+// epilogue.  All waits are bounded (kSpinLimit polls); a wait that gives up sets
+// the error word and the CTA drains its copies, frees TMEM and exits.
 #include <cuda.h>
 
 #include <algorithm>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -234,7 +246,8 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const int t = t0 + c0 + j;
-            if (t < T) Y[int64_t(t) * m + i] = __float2bfloat16_rn(v[j]);
+            // streaming store: Y is written once; keep X and Z resident in L2
+            if (t < T) __stcs(Y + int64_t(t) * m + i, __float2bfloat16_rn(v[j]));
           }
         }
       }
@@ -336,20 +349,25 @@ __global__ void __launch_bounds__(192, 1)
         float v[32];
         tc::tmem_ld32(tbase + c0, v);
         if (t < T) {
+          // Z as a bf16 pair: hi = bf16(z), lo = bf16(z − hi); U·(hi + lo)
+          // keeps the low-rank product accurate to ~2⁻¹⁷ of |U·z|
           __nv_bfloat16* zr = Z + int64_t(t) * r16 + c0;
+          __nv_bfloat16* zl = Z + int64_t(T) * r16 + int64_t(t) * r16 + c0;
 #pragma unroll
           for (int j = 0; j < 32; j += 8) {
             if (c0 + j < r16) {
-              uint4 o;
-              o.x = __bfloat16_as_ushort(__float2bfloat16_rn(v[j])) |
-                    (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(v[j + 1]))) << 16);
-              o.y = __bfloat16_as_ushort(__float2bfloat16_rn(v[j + 2])) |
-                    (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(v[j + 3]))) << 16);
-              o.z = __bfloat16_as_ushort(__float2bfloat16_rn(v[j + 4])) |
-                    (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(v[j + 5]))) << 16);
-              o.w = __bfloat16_as_ushort(__float2bfloat16_rn(v[j + 6])) |
-                    (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(v[j + 7]))) << 16);
-              *reinterpret_cast<uint4*>(zr + j) = o;
+              uint32_t hw[4], lw[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const __nv_bfloat16 h0 = __float2bfloat16_rn(v[j + 2 * e]);
+                const __nv_bfloat16 h1 = __float2bfloat16_rn(v[j + 2 * e + 1]);
+                const __nv_bfloat16 l0 = __float2bfloat16_rn(v[j + 2 * e] - __bfloat162float(h0));
+                const __nv_bfloat16 l1 = __float2bfloat16_rn(v[j + 2 * e + 1] - __bfloat162float(h1));
+                hw[e] = __bfloat16_as_ushort(h0) | (uint32_t(__bfloat16_as_ushort(h1)) << 16);
+                lw[e] = __bfloat16_as_ushort(l0) | (uint32_t(__bfloat16_as_ushort(l1)) << 16);
+              }
+              *reinterpret_cast<uint4*>(zr + j) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+              *reinterpret_cast<uint4*>(zl + j) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
             }
           }
         }
@@ -363,6 +381,220 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 1) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, ncols);
+  }
+}
+
+// ---- sparse tensor-core prefill -------------------------------------------------
+// Yᵀ tile [256 rows of W × 192 tokens]: two 128-row accumulators in TMEM share
+// every X tile (half the X traffic of one 128-row tile per flop).  K-blocks of
+// 64 logical columns: A = the compressed 2:4 values (TMA, 64-byte swizzle,
+// 32 values per row), B = X (TMA, 128-byte swizzle), two tcgen05.mma.sp of
+// K = 32 per half.  The metadata of a K-block is copied into TMEM by four warps
+// (tcgen05.st) from a layout built at pack time, one 8-byte word pair per TMEM
+// lane; each MMA's metadata column is 4-column aligned (a requirement of the
+// sparse MMA's metadata address).  The low-rank tail runs dense MMAs on
+// U [256 × 32] and Z [192 × 32] K-blocks (64-byte swizzle) into the same
+// accumulators.
+constexpr int SP_BN = 192, SP_STAGES = 5;
+constexpr int SP_A_HALF = 128 * 64;        // 128 rows × 64 bytes
+constexpr int SP_A = 2 * SP_A_HALF;        // 16 KB
+constexpr int SP_B = SP_BN * 128;          // 24 KB (X: 192 rows × 64 bf16)
+constexpr int SP_B_Z = SP_BN * 64;         // Z: 192 rows × 32 bf16
+constexpr int SP_M = 2 * 128 * 8;           // metadata of the stage: 2 halves × 128 lanes × 8 B
+constexpr int SP_STAGE = SP_A + SP_B + SP_M;
+constexpr int SP_SMEM = SP_STAGES * SP_STAGE + 1024 + 256;
+// TMEM columns: accumulator 0 [0, 192), accumulator 1 [256, 448); metadata
+// slots of 4 columns, one per (stage, half, MMA): 16 in [192, 256), the rest in
+// [448, 512).
+constexpr uint32_t SP_ACC1_COL = 256;
+__device__ __forceinline__ uint32_t sp_meta_col(int s, int h, int i) {
+  const uint32_t slot = uint32_t(s * 4 + h * 2 + i);
+  return slot < 16 ? 192u + 4u * slot : 448u + 4u * (slot - 16u);
+}
+static_assert(SP_STAGES * 4 <= 32, "metadata slots");
+
+struct SpMaps {
+  CUtensorMap x;   // X [T][n]       box {64, 192} SW128
+  CUtensorMap sv;  // S values [m][n/2] box {32, 128} SW64
+  CUtensorMap u;   // U [m][r_pad]   box {32, 128} SW64
+  CUtensorMap z;   // Z hi [T][r16]  box {32, 192} SW64
+  CUtensorMap zlo; // Z lo [T][r16]  box {32, 192} SW64
+};
+
+__global__ void __launch_bounds__(192, 1)
+    k_prefill_24sp(const __grid_constant__ SpMaps maps, const uint2* __restrict__ meta,
+                   __nv_bfloat16* __restrict__ Y, int m, int n, int T, int r16, uint32_t* err) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sA = smem;
+  unsigned char* sB = sA + SP_STAGES * SP_A;
+  unsigned char* sM = sB + SP_STAGES * SP_B;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sM + SP_STAGES * SP_M);
+  uint64_t* mfull = full + SP_STAGES;
+  uint64_t* empty = mfull + SP_STAGES;
+  uint64_t* accf = empty + SP_STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ntn = (T + SP_BN - 1) / SP_BN;
+  const int mt = blockIdx.x / ntn, nt = blockIdx.x % ntn;
+  const int i0 = mt * 256, t0 = nt * SP_BN;
+  const int nkS = n / 64;
+  const int nkL = (r16 + 31) / 32;
+  const int nk = nkS + nkL;
+  const int mtiles128 = (m + 127) / 128;
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int s = 0; s < SP_STAGES; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&mfull[s], 128);
+      tc::mbar_init(&empty[s], 1);
+    }
+    tc::mbar_init(accf, 1);
+    tc::fence_mbar_init();
+    tc::prefetch_tmap(&maps.x);
+    tc::prefetch_tmap(&maps.sv);
+    if (r16 > 0) {
+      tc::prefetch_tmap(&maps.u);
+      tc::prefetch_tmap(&maps.z);
+    }
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_slot, 512);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  volatile int* abrt = &abort_flag;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t keep = tc::make_policy_evict_last();
+      const uint64_t stream = tc::make_policy_evict_first();
+      int issued[SP_STAGES] = {0, 0, 0, 0, 0};
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % SP_STAGES;
+        const uint32_t ph = (kb / SP_STAGES) & 1;
+        if (!wait_or_abort(&empty[s], ph ^ 1, err, abrt)) break;
+        unsigned char* a = sA + s * SP_A;
+        unsigned char* b = sB + s * SP_B;
+        if (kb < nkS) {
+          // the metadata of both halves rides on the same barrier (1 KB each)
+          const int mt0 = i0 / 128;
+          const int nmeta = (mt0 < mtiles128) + (mt0 + 1 < mtiles128);
+          tc::mbar_expect_tx(&full[s], SP_A + SP_B + nmeta * 1024);
+          tc::tma_load_2d_hint(a, &maps.sv, kb * 32, i0, &full[s], stream);
+          tc::tma_load_2d_hint(a + SP_A_HALF, &maps.sv, kb * 32, i0 + 128, &full[s], stream);
+          tc::tma_load_2d_hint(b, &maps.x, kb * 64, t0, &full[s], keep);
+          for (int h = 0; h < 2; ++h)
+            if (mt0 + h < mtiles128)
+              tc::bulk_load(sM + s * SP_M + h * 1024, meta + (int64_t(mt0 + h) * nkS + kb) * 128,
+                            1024, &full[s]);
+        } else {
+          if (kb == nkS) pdl_wait();  // Z is written by the preceding kernel
+          const int kl = kb - nkS;
+          tc::mbar_expect_tx(&full[s], SP_A + 2 * SP_B_Z);
+          tc::tma_load_2d_hint(a, &maps.u, kl * 32, i0, &full[s], stream);
+          tc::tma_load_2d_hint(a + SP_A_HALF, &maps.u, kl * 32, i0 + 128, &full[s], stream);
+          tc::tma_load_2d_hint(b, &maps.z, kl * 32, t0, &full[s], keep);
+          tc::tma_load_2d_hint(b + SP_B_Z, &maps.zlo, kl * 32, t0, &full[s], keep);
+        }
+        ++issued[s];
+      }
+      for (int s = 0; s < SP_STAGES; ++s)
+        if (issued[s]) tc::mbar_wait(&full[s], (issued[s] - 1) & 1, err);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc_sp = tc::idesc_bf16(128, SP_BN) | (1u << 2);
+      const uint32_t idesc_d = tc::idesc_bf16(128, SP_BN);
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % SP_STAGES;
+        const uint32_t ph = (kb / SP_STAGES) & 1;
+        if (!wait_or_abort(&full[s], ph, err, abrt)) break;
+        if (kb < nkS && !wait_or_abort(&mfull[s], ph, err, abrt)) break;
+        tc::tc_fence_after();
+        const unsigned char* a = sA + s * SP_A;
+        const unsigned char* b = sB + s * SP_B;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t d = tmem + (h ? SP_ACC1_COL : 0u);
+          const uint64_t ad = tc::desc_sw64(a + h * SP_A_HALF);
+          if (kb < nkS) {
+            const uint64_t bd = tc::desc_sw128(b);
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+              tc::mma_bf16_sp(d, tc::desc_advance(ad, 32 * i), tc::desc_advance(bd, 64 * i),
+                              tmem + sp_meta_col(s, h, i), idesc_sp,
+                              (kb > 0 || i > 0) ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {  // Z hi, then Z lo
+              const uint64_t bd = tc::desc_sw64(b + part * SP_B_Z);
+#pragma unroll
+              for (int i = 0; i < 2; ++i)
+                tc::mma_bf16(d, tc::desc_advance(ad, 32 * i), tc::desc_advance(bd, 32 * i), idesc_d,
+                             1u);
+            }
+          }
+        }
+        tc::mma_commit(&empty[s]);
+      }
+      tc::mma_commit(accf);
+    }
+  } else {
+    // warps 2..5: metadata into TMEM, then the epilogue.  TMEM lane = L.
+    const int L = ((warp & 3) << 5) | lane;
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    for (int kb = 0; kb < nkS; ++kb) {
+      const int s = kb % SP_STAGES;
+      const uint32_t ph = (kb / SP_STAGES) & 1;
+      // the stage's bytes (metadata included) have landed: its previous MMAs are done
+      if (!wait_or_abort(&full[s], ph, err, abrt)) break;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int mt128 = i0 / 128 + h;
+        uint2 w = make_uint2(0x44444444u, 0x44444444u);  // rows past m: a valid pattern, zero values
+        if (mt128 < mtiles128) w = *reinterpret_cast<const uint2*>(sM + s * SP_M + h * 1024 + L * 8);
+        tc::tmem_st1(tmem + lane_base + sp_meta_col(s, h, 0), w.x);
+        tc::tmem_st1(tmem + lane_base + sp_meta_col(s, h, 1), w.y);
+      }
+      tc::tmem_st_wait();
+      tc::tc_fence_before();
+      tc::mbar_arrive(&mfull[s]);
+    }
+    if (tc::mbar_wait(accf, 0, err) && !*abrt) {
+      tc::tc_fence_after();
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        const int i = i0 + 128 * h + L;
+#pragma unroll 1
+        for (int c0 = 0; c0 < SP_BN; c0 += 32) {
+          float v[32];
+          tc::tmem_ld32(tmem + lane_base + (h ? SP_ACC1_COL : 0u) + c0, v);
+          if (i < m) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int t = t0 + c0 + j;
+              if (c0 + j < SP_BN && t < T) __stcs(Y + int64_t(t) * m + i, __float2bfloat16_rn(v[j]));
+            }
+          }
+        }
+      }
+    } else {
+      *abrt = 1;
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 512);
   }
 }
 
@@ -416,7 +648,58 @@ hsl_status apply_prefill_run(Handle& h, const void* X, void* Y, int64_t T, cudaS
   if (r16 > 256) return HSL_ERR_UNSUPPORTED;
   const int64_t m = h.m, n = h.n;
   if (r16 > 0) {
-    if (hsl_status e = ensure(h.zpre, size_t(T) * r16 * 2, "prefill Z")) return e;
+    if (hsl_status e = ensure(h.zpre, size_t(T) * r16 * 2 * 2, "prefill Z (hi, lo)")) return e;
+  }
+  uint32_t* err0 = static_cast<uint32_t*>(h.err.p);
+  if (h.pmeta_tc.p && std::getenv("HSL_PREFILL_EXPAND") == nullptr) {
+    // sparse tensor-core path
+    SpMaps sm;
+    memset(&sm, 0, sizeof(sm));
+    const auto BFs = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    bool ok = make_map(&sm.x, BFs, 2, X, T, n, n, 64, SP_BN, CU_TENSOR_MAP_SWIZZLE_128B) &&
+              make_map(&sm.sv, BFs, 2, h.nm_val.p, m, n / 2, n / 2, 32, 128,
+                       CU_TENSOR_MAP_SWIZZLE_64B);
+    if (ok && r16 > 0)
+      ok = make_map(&sm.u, BFs, 2, h.U.p, m, h.r_pad, h.r_pad, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B) &&
+           make_map(&sm.z, BFs, 2, h.zpre.p, T, r16, r16, 32, SP_BN, CU_TENSOR_MAP_SWIZZLE_64B) &&
+           make_map(&sm.zlo, BFs, 2, static_cast<__nv_bfloat16*>(h.zpre.p) + T * r16, T, r16, r16,
+                    32, SP_BN, CU_TENSOR_MAP_SWIZZLE_64B);
+    PrefillMaps zm;
+    memset(&zm, 0, sizeof(zm));
+    if (ok && r16 > 0)
+      ok = make_map(&zm.xz, BFs, 2, X, T, n, n, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
+           make_map(&zm.vt, BFs, 2, h.Vt.p, r16, n, n, 64, r16, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!ok) {
+      set_message("tensor map encoding failed");
+      return HSL_ERR_CUDA;
+    }
+    if (r16 > 0) {
+      cudaFuncSetAttribute(k_prefill_z, cudaFuncAttributeMaxDynamicSharedMemorySize, Z_SMEM);
+      k_prefill_z<<<unsigned((T + 127) / 128), 192, Z_SMEM, s>>>(
+          zm, static_cast<__nv_bfloat16*>(h.zpre.p), int(n), int(T), r16, err0);
+      note_launch();
+      if (hsl_status e = cuda_fail(cudaGetLastError(), "prefill z launch")) return e;
+    }
+    if (cudaError_t e = cudaFuncSetAttribute(k_prefill_24sp,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, SP_SMEM))
+      return cuda_fail(e, "prefill smem attribute");
+    const int64_t tiles = ((m + 255) / 256) * ((T + SP_BN - 1) / SP_BN);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(tiles));
+    cfg.blockDim = dim3(192);
+    cfg.dynamicSmemBytes = SP_SMEM;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = r16 > 0 ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    note_launch();
+    return cuda_fail(cudaLaunchKernelEx(&cfg, k_prefill_24sp, sm,
+                                        static_cast<const uint2*>(h.pmeta_tc.p),
+                                        static_cast<__nv_bfloat16*>(Y), int(m), int(n), int(T),
+                                        r16, err0),
+                     "sparse prefill launch");
   }
   PrefillMaps maps;
   memset(&maps, 0, sizeof(maps));

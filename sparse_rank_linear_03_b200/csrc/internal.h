@@ -78,7 +78,7 @@ struct Handle {
   bool has_sparse = false;
 
   // packed layouts
-  DevBuf prow, pcol, pval, pmeta, U, V, Vt;
+  DevBuf prow, pcol, pval, pmeta, pmeta_tc, U, V, Vt;
   int32_t group = 8, meta_stride = 0;
   int64_t pack_cap = 0;
   bool packed = false;
@@ -102,7 +102,7 @@ hsl_status plan_build(ApplyPlan& plan, Handle* const* hs, int count, cudaStream_
 hsl_status apply_decode_run(ApplyPlan& plan, const void* X, void* Y, const void* const* xy_dev,
                             int64_t batch, int num_sms, cudaStream_t s);
 // tensor-core path for large batches (2:4, bf16, n % 64 == 0)
-constexpr int64_t kPrefillMinBatch = 64;
+constexpr int64_t kPrefillMinBatch = 16;
 bool prefill_supported(const Handle& h, const void* X);
 hsl_status apply_prefill_run(Handle& h, const void* X, void* Y, int64_t T, cudaStream_t s);
 

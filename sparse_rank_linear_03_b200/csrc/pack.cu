@@ -152,6 +152,41 @@ __global__ void k_transpose_v(const uint16_t* __restrict__ V, int64_t n, int32_t
   }
 }
 
+// 2:4 metadata for the sparse tensor-core prefill: one uint2 per (128-row
+// tile, 64-column K-block, TMEM lane L).  Word i feeds the sparse MMA over
+// logical columns [64·kb + 32·i, +32).  Lane L = 16·m2 + 8·k1 + m0 holds in its
+// low / high 16 bits the four nibbles (16 columns, half k1) of tile rows
+// m0 + 16·m2 and m0 + 8 + 16·m2 — rows i and i + 8 share a word, the pairing
+// of the warp-level sparse MMAs.  Rows past m get the valid pattern 0x4
+// (their values are zero).
+__device__ __forceinline__ uint32_t nib4(const uint8_t* idx, int64_t groups, int64_t row, int64_t g0,
+                                         int64_t m) {
+  if (row >= m) return 0x4444u;
+  const uint8_t* p = idx + row * groups + g0;
+  return uint32_t(p[0] & 0xF) | (uint32_t(p[1] & 0xF) << 4) | (uint32_t(p[2] & 0xF) << 8) |
+         (uint32_t(p[3] & 0xF) << 12);
+}
+
+__global__ void k_meta_tc(const uint8_t* __restrict__ idx, int64_t m, int64_t n,
+                          uint2* __restrict__ out) {
+  const int64_t nkb = n / 64, groups = n / 4;
+  const int64_t total = ((m + 127) / 128) * nkb * 128;
+  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
+       e += int64_t(gridDim.x) * blockDim.x) {
+    const int L = int(e % 128);
+    const int64_t kb = (e / 128) % nkb, mt = e / (128 * nkb);
+    const int m0 = L & 7, k1 = (L >> 3) & 1, m2 = L >> 4;
+    const int64_t rlo = mt * 128 + m0 + 16 * m2, rhi = rlo + 8;
+    uint32_t w[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int64_t g0 = 16 * kb + 8 * i + 4 * k1;
+      w[i] = nib4(idx, groups, rlo, g0, m) | (nib4(idx, groups, rhi, g0, m) << 16);
+    }
+    out[e] = make_uint2(w[0], w[1]);
+  }
+}
+
 // One CTA: boundaries of `slices` row ranges of equal streamed bytes over the
 // concatenated rows of all layers.  Cost of the first i rows of layer p:
 //   CSR : prow[i]·(value + 2 index bytes) + i·(U row bytes + 8)
@@ -238,6 +273,14 @@ hsl_status pack_sparse_run(Handle& h, cudaStream_t s) {
     return cuda_fail(cudaGetLastError(), "CSR pack launch");
   }
   // NM24
+  if (h.dtype == HSL_BF16 && h.n % 64 == 0) {
+    const int64_t tot = ((h.m + 127) / 128) * (h.n / 64) * 128;
+    if (hsl_status e = ensure(h.pmeta_tc, size_t(tot) * 8, "2:4 tensor-core metadata")) return e;
+    const int64_t g = std::min<int64_t>((tot + 255) / 256, int64_t(h.num_sms) * 16);
+    k_meta_tc<<<unsigned(std::max<int64_t>(g, 1)), 256, 0, s>>>(
+        static_cast<const uint8_t*>(h.nm_idx.p), h.m, h.n, static_cast<uint2*>(h.pmeta_tc.p));
+    note_launch();
+  }
   const int64_t nq = (h.n + 15) / 16;  // chunks of 8 kept values per row
   h.meta_stride = int32_t(round_up(nq, 256));
   if (hsl_status e = ensure(h.pmeta, size_t(h.m) * h.meta_stride * 2, "2:4 metadata")) return e;

@@ -431,6 +431,43 @@ __device__ __forceinline__ void lookback(unsigned long long* flags, int64_t blk,
   if (lane == 0) st_release_u64(&flags[blk], pack_flag(kFlagInc, xg + agg_gt, xe + agg_eq));
 }
 
+// Masks of one 16-byte vector: bit e = element e has key > T (gm) / key == T (em).
+// bf16: two 15-bit keys per word, compared without branches by one packed
+// subtraction per threshold: with k' = key | 0x8000 in each half and t ≤ 0x8000,
+// bit 15 of (k' − t) is set iff key ≥ t, and no half ever borrows from the next.
+template <typename KT>
+__device__ __forceinline__ void vec_masks(const uint4& q, uint32_t T, uint32_t& gm, uint32_t& em);
+template <>
+__device__ __forceinline__ void vec_masks<uint16_t>(const uint4& q, uint32_t T, uint32_t& gm,
+                                                    uint32_t& em) {
+  const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+  const uint32_t T0 = T <= 0x7FFFu ? T : 0x8000u;  // T above every key: nothing ≥ T
+  const uint32_t TT = T0 * 0x00010001u, TT1 = (T0 + 1u) * 0x00010001u;
+  uint32_t ge = 0, gt = 0;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const uint32_t k = (w4[u] & 0x7FFF7FFFu) | 0x80008000u;
+    const uint32_t a = (k - TT) & 0x80008000u;
+    const uint32_t b = T0 >= 0x7FFFu ? 0u : ((k - TT1) & 0x80008000u);
+    ge |= (((a >> 15) | (a >> 30)) & 3u) << (2 * u);
+    gt |= (((b >> 15) | (b >> 30)) & 3u) << (2 * u);
+  }
+  gm = gt;
+  em = ge & ~gt;
+}
+template <>
+__device__ __forceinline__ void vec_masks<uint32_t>(const uint4& q, uint32_t T, uint32_t& gm,
+                                                    uint32_t& em) {
+  const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+  gm = em = 0;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const uint32_t k = w4[u] & 0x7FFFFFFFu;
+    gm |= uint32_t(k > T) << u;
+    em |= uint32_t(k == T) << u;
+  }
+}
+
 template <typename KT, typename SB>
 __global__ void __launch_bounds__(kEmitThreads) k_split_emit_blk(
     const KT* __restrict__ W, int64_t m, int64_t n, int rb, int64_t nblk,
@@ -439,6 +476,7 @@ __global__ void __launch_bounds__(kEmitThreads) k_split_emit_blk(
     int32_t* __restrict__ col, SB* __restrict__ val, KT* __restrict__ R, int64_t k,
     uint32_t* __restrict__ err) {
   constexpr int EPV = 16 / sizeof(KT);
+  constexpr uint32_t STEP = kEmitThreads * EPV;  // elements between a thread's vectors
   __shared__ uint32_t wt[kVPT][kEmitThreads / 32];
   __shared__ int64_t sh_blk;
   __shared__ uint32_t sh_ex[2];
@@ -458,30 +496,21 @@ __global__ void __launch_bounds__(kEmitThreads) k_split_emit_blk(
     const uint32_t nv = uint32_t(rows * n / EPV);
     const KT* Wb = W + e0;
 
+    // phase 1: load the block (coalesced, k-major), masks, ranks inside the block
     uint4 q[kVPT];
     uint32_t ex[kVPT];
+    uint32_t mk[kVPT / 2];  // (gm | em << 8) of vector kk in half kk & 1
 #pragma unroll
     for (int kk = 0; kk < kVPT; ++kk) {
       const uint32_t v = uint32_t(kk * kEmitThreads + t);
-      uint32_t pk = 0;
+      uint32_t pk = 0, gm = 0, em = 0;
       if (v < nv) {
         q[kk] = ld_stream16(Wb + int64_t(v) * EPV);
-        const uint32_t w4[4] = {q[kk].x, q[kk].y, q[kk].z, q[kk].w};
-        uint32_t g = 0, e = 0;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          if (sizeof(KT) == 2) {
-            const uint32_t k0 = w4[u] & 0x7FFFu, k1 = (w4[u] >> 16) & 0x7FFFu;
-            g += (k0 > T) + (k1 > T);
-            e += (k0 == T) + (k1 == T);
-          } else {
-            const uint32_t k0 = w4[u] & 0x7FFFFFFFu;
-            g += (k0 > T);
-            e += (k0 == T);
-          }
-        }
-        pk = (g << 16) | e;
+        vec_masks<KT>(q[kk], T, gm, em);
+        pk = (uint32_t(__popc(gm)) << 16) | uint32_t(__popc(em));
       }
+      const uint32_t m16 = gm | (em << 8);
+      if (kk & 1) mk[kk >> 1] |= m16 << 16; else mk[kk >> 1] = m16;
       const uint32_t incl = warp_incl_scan(pk);
       ex[kk] = incl - pk;
       if (lane == 31) wt[kk][warp] = incl;
@@ -513,53 +542,64 @@ __global__ void __launch_bounds__(kEmitThreads) k_split_emit_blk(
       }
     }
     __syncthreads();
-    // kept before an element = keys > T before it + the first `need` ties in
-    // linear order that come before it
+    // phase 2: kept before an element = keys > T before it + the first `need`
+    // ties in linear order that come before it
     const uint32_t ex_gt = sh_ex[0], ex_eq = sh_ex[1];
+    uint32_t j0 = uint32_t(t) * EPV;  // column of this thread's first vector, no division
+    int64_t row = row0;
+    while (j0 >= n32) {
+      j0 -= n32;
+      ++row;
+    }
 #pragma unroll
     for (int kk = 0; kk < kVPT; ++kk) {
       const uint32_t v = uint32_t(kk * kEmitThreads + t);
-      if (v >= nv) continue;
-      const uint32_t base = wt[kk][warp] + ex[kk];
-      uint32_t cg = base >> 16, ce = base & 0xFFFFu;
-      const uint32_t flat = v * EPV;
-      const uint32_t j0 = flat % n32;
-      const int64_t row = row0 + flat / n32;
-      if (j0 == 0)
-        row_ptr[row] = int32_t(ex_gt + cg + min(need, ex_eq + ce));
-      const uint32_t w4[4] = {q[kk].x, q[kk].y, q[kk].z, q[kk].w};
-      uint32_t b[EPV];
-#pragma unroll
-      for (int e = 0; e < EPV; ++e)
-        b[e] = sizeof(KT) == 2 ? ((w4[e >> 1] >> ((e & 1) * 16)) & 0xFFFFu) : w4[e % 4];
-      uint32_t rbits[EPV];
-#pragma unroll
-      for (int e = 0; e < EPV; ++e) {
-        const uint32_t key = b[e] & KeyTraits<KT>::kMask;
-        const bool g = key > T, qq = key == T;
-        const bool sel = g || (qq && (ex_eq + ce) < need);
+      if (v < nv) {
+        const uint32_t m16 = (mk[kk >> 1] >> ((kk & 1) * 16)) & 0xFFFFu;
+        const uint32_t gm = m16 & 0xFFu, em = m16 >> 8;
+        const uint32_t base = wt[kk][warp] + ex[kk];
+        const uint32_t cg = base >> 16, ce = base & 0xFFFFu;
+        const uint32_t pos0 = ex_gt + cg + min(need, ex_eq + ce);
+        if (j0 == 0) row_ptr[row] = int32_t(pos0);
+        // ties kept in this vector: the first `allow` set bits of em
+        uint32_t allow = need > ex_eq + ce ? min(need - (ex_eq + ce), uint32_t(__popc(em))) : 0u;
+        uint32_t keq = 0, rest = em;
+        for (; allow; --allow) {
+          keq |= rest & (0u - rest);
+          rest &= rest - 1u;
+        }
+        const uint32_t sel = gm | keq;
+        uint4 o = q[kk];
         if (sel) {
-          const int64_t pos = int64_t(ex_gt) + cg + min(need, ex_eq + ce);
-          if (pos < k) {
-            col[pos] = int32_t(j0 + e);
-            val[pos] = conv_val<SB>(b[e], sizeof(KT));
+          for (uint32_t s2 = sel; s2; s2 &= s2 - 1u) {
+            const int e = __ffs(s2) - 1;
+            const int64_t pos = int64_t(pos0) + __popc(sel & ((1u << e) - 1u));
+            const uint32_t w = (&o.x)[sizeof(KT) == 2 ? (e >> 1) : e];
+            const uint32_t bits = sizeof(KT) == 2 ? ((w >> ((e & 1) * 16)) & 0xFFFFu) : w;
+            if (pos < k) {
+              col[pos] = int32_t(j0 + e);
+              val[pos] = conv_val<SB>(bits, sizeof(KT));
+            }
+          }
+          // zero the kept elements in the residual
+          uint32_t* ow = &o.x;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            uint32_t z;
+            if (sizeof(KT) == 2)
+              z = (((sel >> (2 * u)) & 1u) ? 0x0000FFFFu : 0u) |
+                  (((sel >> (2 * u + 1)) & 1u) ? 0xFFFF0000u : 0u);
+            else
+              z = ((sel >> u) & 1u) ? 0xFFFFFFFFu : 0u;
+            ow[u] &= ~z;
           }
         }
-        rbits[e] = sel ? 0u : b[e];
-        cg += g;
-        ce += qq;
+        if (R) st_stream16(R + e0 + int64_t(v) * EPV, o);
       }
-      if (R) {
-        uint4 o;
-        if (sizeof(KT) == 2) {
-          o.x = rbits[0] | (rbits[1 % EPV] << 16);
-          o.y = rbits[2 % EPV] | (rbits[3 % EPV] << 16);
-          o.z = rbits[4 % EPV] | (rbits[5 % EPV] << 16);
-          o.w = rbits[6 % EPV] | (rbits[7 % EPV] << 16);
-        } else {
-          o = make_uint4(rbits[0], rbits[1 % EPV], rbits[2 % EPV], rbits[3 % EPV]);
-        }
-        st_stream16(R + e0 + int64_t(v) * EPV, o);
+      j0 += STEP;
+      while (j0 >= n32) {
+        j0 -= n32;
+        ++row;
       }
     }
     if (t == 0 && blk == nblk - 1) row_ptr[m] = int32_t(k);

@@ -12,14 +12,18 @@
 //      bf16 keys have 15 bits: ONE streaming pass with a 32768-bin histogram
 //      per CTA in shared memory (128 KB) finds the threshold key T exactly.
 //      fp32 keys (31 bits) take three passes of 11/11/9 bits.
-//   2. One emit pass over W, persistent CTAs taking rows in ticket order.  Per
-//      row the CTA counts keys > T and keys == T, publishes them, and gets the
-//      exclusive prefix over earlier rows by a decoupled look-back (bounded
-//      spin; CTAs only wait on rows whose tickets were taken earlier, so they
-//      are running).  The row's CSR offset is  gt_before + min(need, eq_before)
-//      where need = k − #(key > T): ties are taken in linear order.  A block
-//      scan gives each element its rank inside the row; the pass writes the
-//      CSR columns/values and the residual (bit copy, +0.0 where kept).
+//   2. One emit pass over W, persistent CTAs taking blocks of rows (up to 32K
+//      elements, held in registers) in ticket order.  Each block's counts of
+//      keys > T and keys == T are published and the exclusive prefix over
+//      earlier blocks comes from a decoupled look-back, 32 predecessors per
+//      poll (bounded spin; CTAs only wait on blocks whose tickets were taken
+//      earlier, so they are running).  An element's CSR position is
+//      gt_before + min(need, eq_before), need = k − #(key > T): ties are taken
+//      in linear order.  Per 16-byte vector the masks of keys > T / == T come
+//      from one carry-free packed subtraction per threshold (bf16); the kept
+//      elements are walked by their set bits; the residual is the vector with
+//      those elements zeroed (bit copy, +0.0 where kept).  Rows wider than a
+//      register block use a per-row variant of the same scheme.
 //   HBM traffic: bf16 2 reads of W + 1 write of R + S; fp32 4 reads.
 #include <algorithm>
 

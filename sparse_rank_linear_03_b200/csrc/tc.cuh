@@ -59,6 +59,14 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
 }
+// Plain 1-D bulk copy global → shared (16-byte aligned, size a multiple of 16).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
 // Same load with an L2 eviction-priority policy (from make_policy_*).
 __device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* map, int32_t x,
                                                  int32_t y, uint64_t* bar, uint64_t policy) {
@@ -117,6 +125,28 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// Sparse A (2:4 along K, compressed in smem), metadata in TMEM at `meta`.
+__device__ __forceinline__ void mma_bf16_sp(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t meta_tmem, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.sp.cta_group::1.kind::f16 [%0], %1, %2, [%5], %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(meta_tmem)
+      : "memory");
+}
+// One / two 32-bit columns of this thread's TMEM lane (32 lanes per warp).
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t a) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(a) : "memory");
+}
+__device__ __forceinline__ void tmem_st2(uint32_t taddr, uint32_t a, uint32_t b) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1, %2};" ::"r"(taddr), "r"(a), "r"(b)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
 // Arrive on an mbarrier once all MMAs issued so far by this thread complete.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile(
@@ -154,6 +184,17 @@ __device__ __forceinline__ uint64_t desc_sw128(const void* smem_tile) {
   d |= uint64_t(1024 >> 4) << 32;       // stride byte offset: next 8-row atom
   d |= uint64_t(1) << 46;               // descriptor version (sm_100)
   d |= uint64_t(2) << 61;               // SWIZZLE_128B
+  return d;
+}
+// Same for the 64-byte swizzle (rows of 32 bf16 = 64 bytes, 8-row atoms of 512 bytes).
+__device__ __forceinline__ uint64_t desc_sw64(const void* smem_tile) {
+  const uint64_t addr = smem_u32(smem_tile);
+  uint64_t d = 0;
+  d |= (addr >> 4) & 0x3FFFull;
+  d |= uint64_t(1) << 16;
+  d |= uint64_t(512 >> 4) << 32;        // stride byte offset: next 8-row atom
+  d |= uint64_t(1) << 46;
+  d |= uint64_t(4) << 61;               // SWIZZLE_64B
   return d;
 }
 // Advance a K-major SW128 descriptor by `bytes` along K inside the 128-byte row.

@@ -1,6 +1,6 @@
 """Parity of the tensor-core (large-batch) 2:4 apply with the float64 oracle.
 
-Batches of 64 tokens or more on bf16 2:4 layers with n % 64 == 0 take the
+Batches of 16 tokens or more on bf16 2:4 layers with n % 64 == 0 take the
 tcgen05 path: Z = X·V, then S·Xᵀ + U·Zᵀ in one TMEM accumulator.  Z is rounded
 to bf16 before the second product, well inside the 1e-2 bound."""
 import numpy as np
@@ -63,12 +63,12 @@ def test_prefill_small_shapes(hsl, m, n, r, T):
 
 def test_prefill_matches_decode_path(hsl):
     """Same layer, same tokens: tensor-core path (one call of 128 tokens) and
-    CUDA-core path (eight calls of 16) agree to bf16 output rounding."""
+    CUDA-core path (sixteen calls of 8) agree to bf16 output rounding."""
     L, W, U, V = build(hsl, 512, 512, 32, 7)
     X = synth.to_bf16_bits(synth.normal_f32(128, 512, 1))
     Xd = dev(X, "bf16")
     Yp = L.apply(Xd)
-    Yd = torch.cat([L.apply(Xd[i:i + 16].contiguous()) for i in range(0, 128, 16)])
+    Yd = torch.cat([L.apply(Xd[i:i + 8].contiguous()) for i in range(0, 128, 8)])
     a, b = f64(host(Yp)), f64(host(Yd))
     assert oracle.rel_err(a, b) <= 2 * TOL["bf16"]
 
@@ -96,3 +96,18 @@ def test_prefill_mlp_70b_4096_tokens_sampled(hsl):
     toks = np.sort(np.random.default_rng(5).choice(4096, 512, replace=False))
     got = f64(host(Y))[np.ix_(toks, rows)]
     assert oracle.rel_err(got, ref_rows(W, U, V, X[toks], rows)) <= TOL["bf16"]
+
+
+def test_sparse_mma_matches_expansion_path(hsl, monkeypatch):
+    """The 2:4 sparse tensor-core kernel and the kernel that expands each 2:4
+    tile to dense in shared memory compute the same product."""
+    L, W, U, V = build(hsl, 640, 512, 48, 13)
+    X = synth.to_bf16_bits(synth.normal_f32(300, 512, 2))
+    Xd = dev(X, "bf16")
+    Ys = L.apply(Xd)
+    monkeypatch.setenv("HSL_PREFILL_EXPAND", "1")
+    Ye = L.apply(Xd)
+    monkeypatch.delenv("HSL_PREFILL_EXPAND")
+    L.check()
+    assert oracle.rel_err(f64(host(Ys)), f64(host(Ye))) <= 2 * TOL["bf16"]
+    assert oracle.rel_err(f64(host(Ys)), ref_rows(W, U, V, X, np.arange(640))) <= TOL["bf16"]
