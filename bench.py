@@ -25,6 +25,7 @@ import argparse
 import json
 import os
 import statistics
+import threading
 import subprocess
 import sys
 import time
@@ -75,50 +76,67 @@ def peaks() -> dict:
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event reasons of one GPU, read through NVML every
+    ~2 ms on a thread while the timed region runs (nvidia-smi's own sampling
+    is too coarse for a region of tens of milliseconds).  `nvml` is the NVML
+    module (pynvml) or a stand-in with the same calls; reading only, no
+    setting of the GPU is touched."""
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+               ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4))
 
-    def __init__(self, gpu_id: str):
-        self.gpu_id = gpu_id
-        self.proc = None
+    def __init__(self, gpu_uuid: str, nvml=None, period_s: float = 0.002):
+        self.gpu_uuid = gpu_uuid
+        self.nvml = nvml
+        self.period = period_s
+        self.samples = []
+        self.sm_max = None
+        self._stop = threading.Event()
+        self._thread = None
+
+    def _read(self):
+        clk = self.nvml.nvmlDeviceGetClockInfo(self.h, self.nvml.NVML_CLOCK_SM)
+        rs = self.nvml.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        self.samples.append((float(clk), int(rs)))
+
+    def _loop(self):
+        while not self._stop.is_set():
+            try:
+                self._read()
+            except Exception:
+                return
+            self._stop.wait(self.period)
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            if self.nvml is None:
+                import pynvml
+                self.nvml = pynvml
+            self.nvml.nvmlInit()
+            self.h = self.nvml.nvmlDeviceGetHandleByUUID(self.gpu_uuid)
+            self.sm_max = float(self.nvml.nvmlDeviceGetMaxClockInfo(self.h, self.nvml.NVML_CLOCK_SM))
+            self._read()  # one sample before the region starts: the thread is live
+            self.samples.clear()
+            self._thread = threading.Thread(target=self._loop, daemon=True)
+            self._thread.start()
         except Exception:
-            self.proc = None
+            self._thread = None
         return self
 
     def __exit__(self, *exc):
-        self.out = ""
-        if self.proc is not None:
-            self.proc.terminate()
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
             try:
-                self.out, _ = self.proc.communicate(timeout=5)
+                self.nvml.nvmlShutdown()
             except Exception:
-                self.proc.kill()
-                self.out = ""
+                pass
 
     def summary(self) -> dict:
-        rows = []
-        for line in (self.out or "").splitlines():
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9 or parts[0].lower() != self.gpu_id.lower():
-                continue
-            try:
-                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
-            except ValueError:
-                continue
-        if not rows:
+        if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for _, _, r in rows for i in range(4) if r[i] == "Active"})
-        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": rows[0][1],
-                "reasons": reasons, "samples": len(rows)}
+        reasons = sorted({name for _, rs in self.samples for name, bit in self.REASONS if rs & bit})
+        return {"sm_mhz": statistics.median(c for c, _ in self.samples), "sm_max_mhz": self.sm_max,
+                "reasons": reasons, "samples": len(self.samples)}
 
 
 # ------------------------------------------------------------------ distributed plumbing

@@ -121,7 +121,7 @@ hsl_status hsl_split_topk(hsl_handle h, const void* W, hsl_dtype w_dtype,
  *   residual: device m×n of w_dtype, or NULL.
  *   status:   device uint32 or NULL; cleared, then OR-ed with 1 for a NaN in
  *             W and 2 for a device wait that gave up.
- * Scratch: one fixed static device array of about 640 KB per GPU (held until
+ * Scratch: one fixed static device array of about 2.2 MB per GPU (held until
  * the process exits).  Limits: m ≤ 65536 and m·n < 2^31, else
  * HSL_ERR_UNSUPPORTED.  The first call on a device looks the array up with
  * that device current (make it before any stream capture).  All calls share

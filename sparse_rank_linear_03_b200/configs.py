@@ -39,7 +39,7 @@ ATTN4096 = Workload("attn4096_csr2_bf16", "csr", "bf16", "f32", 0.02, 128, (1, 4
                     (Layer("o_proj", 4096, 4096, 2000),))
 
 MLP_UP_11008 = Workload("mlp_up_11008x4096_nm24_bf16", "nm24", "bf16", "bf16", 0.5, 64,
-                        (16, 2048), (Layer("up_proj", 11008, 4096, 3000),))
+                        (1, 16, 2048), (Layer("up_proj", 11008, 4096, 3000),))
 
 _7B_SHAPES = (("q", 4096, 4096), ("k", 4096, 4096), ("v", 4096, 4096), ("o", 4096, 4096),
               ("gate", 11008, 4096), ("up", 11008, 4096), ("down", 4096, 11008))

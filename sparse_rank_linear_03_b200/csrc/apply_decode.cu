@@ -17,10 +17,17 @@
 //                 then griddepcontrol.wait (programmatic dependent launch:
 //                 the S stream overlaps the z kernel), z is staged, and each
 //                 row adds U[i,:]·z and stores y.
+//   k_apply_24_b1_tma  batch 1, bf16 2:4: one CTA of 16 warps per SM; each
+//                 warp pulls (row, super-chunk) units into shared memory with
+//                 1-D bulk copies, two in flight; same partition, z overlap
+//                 and epilogue.
 #include <algorithm>
+#include <cstdlib>
+#include <cstring>
 
 #include "common.cuh"
 #include "internal.h"
+#include "tc.cuh"
 
 namespace hsl {
 namespace {
@@ -38,6 +45,7 @@ struct ApplyArgs {
   int32_t count, slices;
   int32_t b0, bc;
   int32_t r_pad_max;
+  uint32_t* err;  // error word (bounded waits that gave up)
 };
 
 template <typename T>
@@ -171,7 +179,7 @@ __device__ __forceinline__ void xcol(const T* xs, int c, float (&xv)[BC]) {
 }
 
 // y[row] = ysp[row] + U[row,:]·z for rows [s0, s1) of layer P.
-template <typename T, int BC>
+template <typename T, int BC, int NT = kThreads>
 __device__ __forceinline__ void urows(const ApplyProblem& P, const float* zs, const float* ysp,
                                       int s0, int s1, T* y, int bc) {
   const int rp = P.r_pad;
@@ -180,7 +188,7 @@ __device__ __forceinline__ void urows(const ApplyProblem& P, const float* zs, co
   while (GU * 8 < rp) GU <<= 1;  // lanes per row, power of two ≤ 32
   const int rpw = 32 / GU;        // rows per warp pass
   const T* U = static_cast<const T*>(P.U);
-  for (int ib = s0 + warp * rpw; ib < s1; ib += (kThreads / 32) * rpw) {
+  for (int ib = s0 + warp * rpw; ib < s1; ib += (NT / 32) * rpw) {
     const int i = ib + lane / GU, gl = lane % GU;
     float acc[BC];
 #pragma unroll
@@ -251,11 +259,12 @@ __device__ __forceinline__ void csr_rows(const ApplyProblem& P, const T* xs, flo
 // units of a chunk's 16-element window come back in order and every
 // quarter-warp's loads hit distinct banks.  The two kept x of a group are
 // picked with one byte permute whose selector comes from a 16-entry table.
+template <int NT = kThreads>
 __device__ __forceinline__ void stage_x_nm24_b1(__nv_bfloat16* xs, const __nv_bfloat16* x, int n) {
   const uint4* src = reinterpret_cast<const uint4*>(x);
   uint4* dst = reinterpret_cast<uint4*>(xs);
   const int nu = n / 8;
-  for (int U = threadIdx.x; U < nu; U += kThreads) dst[U ^ ((U >> 3) & 1)] = src[U];
+  for (int U = threadIdx.x; U < nu; U += NT) dst[U ^ ((U >> 3) & 1)] = src[U];
 }
 
 __device__ __forceinline__ void nm24_rows_b1(const ApplyProblem& P, const __nv_bfloat16* xs,
@@ -436,6 +445,230 @@ __global__ void __launch_bounds__(kThreads, 2) k_apply_decode(ApplyArgs a) {
   }
 }
 
+// ---- batch-1 bf16 2:4, rows fed by bulk copies ---------------------------------
+// The work of a layer is cut into units of one row × one super-chunk (256
+// chunks: 4 KB of values, 512 B of interleaved metadata, 4096 columns).  Each
+// of the 16 warps of the CTA double-buffers units in shared memory: two 1-D
+// bulk copies (values, metadata) per unit complete on a per-(warp, slot)
+// mbarrier, and while the warp computes one unit from shared memory the copy
+// of its next unit lands in the other slot.  A warp takes units w, w+16, ...
+// of the layer's row range, so the prefetch runs across the 256-row segments
+// whose flush (sum of a row's super-chunk partials in a fixed order, then
+// U·z and the y stores) only needs barriers.  Arithmetic per chunk as in
+// nm24_rows_b1.
+constexpr int kB1Threads = 512;
+constexpr int kB1Warps = kB1Threads / 32;
+constexpr int kSupChunks = 256;                  // chunks of a super-chunk
+constexpr int kUnitVBytes = kSupChunks * 16;     // values of a full unit
+constexpr int kUnitMBytes = kSupChunks * 2;      // metadata of a unit
+constexpr int kUnitSlot = kUnitVBytes + kUnitMBytes;
+
+struct B1Layout {
+  int32_t xs;     // bytes of the staged x
+  int32_t nsup;   // super-chunks of the widest row
+  int32_t total;  // dynamic shared memory of the launch
+};
+
+B1Layout b1_layout(int n_max, int r_pad_max) {
+  B1Layout L;
+  L.xs = int32_t(round_up(int64_t(n_max) * 2, 16));
+  L.nsup = int32_t(((n_max + 15) / 16 + kSupChunks - 1) / kSupChunks);
+  L.total = int32_t(int64_t(2 * kB1Warps) * kUnitSlot + L.xs + int64_t(kSeg) * L.nsup * 4 +
+                    int64_t(r_pad_max) * 4 + 2 * kB1Warps * 8 + 16);
+  return L;
+}
+
+__global__ void __launch_bounds__(kB1Threads, 1) k_apply_24_b1_tma(ApplyArgs a, B1Layout lay) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ uint32_t sel_lut[16];
+  __shared__ int abort_flag;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  unsigned char* const slot0 = smem + (2 * warp) * kUnitSlot;
+  __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(smem + 2 * kB1Warps * kUnitSlot);
+  float* ysp = reinterpret_cast<float*>(smem + 2 * kB1Warps * kUnitSlot + lay.xs);  // [kSeg][nsup]
+  float* zs = ysp + kSeg * lay.nsup;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(
+      (reinterpret_cast<uintptr_t>(zs + a.r_pad_max) + 7) & ~uintptr_t(7));
+  uint64_t* const mybar = bars + 2 * warp;
+  if (threadIdx.x < 16)
+    sel_lut[threadIdx.x] = 0x1010u + (threadIdx.x & 3u) * 0x22u + (threadIdx.x >> 2) * 0x2200u;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int i = 0; i < 2 * kB1Warps; ++i) tc::mbar_init(&bars[i], 1);
+    tc::fence_mbar_init();
+  }
+  __syncthreads();
+  volatile int* abrt = &abort_flag;
+  uint32_t ph = 0u, pending = 0u;  // per-slot bits: mbarrier parity, copy in flight
+  const uint64_t policy = tc::make_policy_evict_first();
+
+  const int64_t slo = int64_t(blockIdx.x) * a.slices / gridDim.x;
+  const int64_t shi = int64_t(blockIdx.x + 1) * a.slices / gridDim.x;
+  int64_t row = a.cta_rows[slo];
+  const int64_t row_end = a.cta_rows[shi];
+  if (row >= row_end) return;
+  int p = 0;
+  {
+    int lo = 0, hi = a.count - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (a.prob_row0[mid] <= row) lo = mid; else hi = mid - 1;
+    }
+    p = lo;
+  }
+  // the abort flag is read by lane 0 and broadcast, so a warp decides as one
+  auto aborted = [&]() { return __shfl_sync(0xffffffffu, *abrt, 0) != 0; };
+  bool waited = false;
+  while (row < row_end) {
+    const ApplyProblem P = a.probs[p];
+    const int64_t p_end = a.prob_row0[p + 1];
+    const int l0 = int(row - P.row0);
+    const int l1 = int(min(row_end, p_end) - P.row0);
+    const int n = P.n, nq = n / 16;
+    const int nsup = (nq + kSupChunks - 1) / kSupChunks;
+    // u / nsup as mulhi(u, ceil(2^32 / nsup)): exact for u < 2^32 / nsup
+    const uint32_t nsup_magic = nsup > 1 ? 0xFFFFFFFFu / uint32_t(nsup) + 1u : 0u;
+    const int units = (l1 - l0) * nsup;
+    const int nu = warp < units ? (units - warp + kB1Warps - 1) / kB1Warps : 0;
+    const int useg = kSeg * nsup / kB1Warps;  // units of a warp in one segment
+    const uint32_t mstride = uint32_t(P.meta_stride) * 2u;
+    const unsigned char* pval = static_cast<const unsigned char*>(P.pval);
+    const unsigned char* pmeta = reinterpret_cast<const unsigned char*>(P.pmeta);
+    // unit u = (row l0 + u / nsup, super-chunk u % nsup)
+    auto unit_of = [&](int u, int& r, int& sp) {
+      r = nsup > 1 ? int(__umulhi(uint32_t(u), nsup_magic)) : u;
+      sp = u - r * nsup;
+    };
+    // unit w + 16·j into slot j & 1
+    auto issue = [&](int j) {
+      if (aborted()) return;
+      const int sl = j & 1;
+      if (lane == 0) {
+        int r, sp;
+        unit_of(warp + kB1Warps * j, r, sp);
+        const int64_t i = int64_t(l0) + r;
+        const uint32_t vb = uint32_t(min(kSupChunks, nq - sp * kSupChunks)) * 16u;
+        unsigned char* dst = slot0 + sl * kUnitSlot;
+        tc::fence_async_smem();
+        tc::mbar_expect_tx(mybar + sl, vb + kUnitMBytes);
+        tc::bulk_load_hint(dst, pval + i * n + int64_t(sp) * kUnitVBytes, vb, mybar + sl, policy);
+        tc::bulk_load_hint(dst + kUnitVBytes, pmeta + i * mstride + sp * kUnitMBytes, kUnitMBytes,
+                           mybar + sl, policy);
+      }
+      pending |= 1u << sl;
+    };
+    if (nu > 0) issue(0);  // lands while x is staged
+    const __nv_bfloat16* x = x_of<__nv_bfloat16>(a, p) + int64_t(a.b0) * n;
+    __syncthreads();
+    if ((reinterpret_cast<uintptr_t>(x) & 15) == 0) {
+      stage_x_nm24_b1<kB1Threads>(xs, x, n);
+    } else {
+      for (int c = threadIdx.x; c < n; c += kB1Threads) {
+        const int U = c >> 3;
+        xs[((U ^ ((U >> 3) & 1)) << 3) | (c & 7)] = x[c];
+      }
+    }
+    __syncthreads();
+    const uint4* xs4 = reinterpret_cast<const uint4*>(xs);
+    __nv_bfloat16* y = y_of<__nv_bfloat16>(a, p) + int64_t(a.b0) * P.m;
+    for (int s0 = l0, seg = 0; s0 < l1; s0 += kSeg, ++seg) {
+      const int s1 = min(s0 + kSeg, l1);
+      const int jend = min(nu, (seg + 1) * useg);
+      for (int j = seg * useg; j < jend; ++j) {
+        const int sl = j & 1;
+        if (j + 1 < nu) issue(j + 1);
+        bool ok = ((pending >> sl) & 1u) && !aborted();
+        if (ok) {
+          ok = tc::mbar_wait(mybar + sl, (ph >> sl) & 1u, a.err);
+          if (ok) {
+            ph ^= 1u << sl;
+            pending &= ~(1u << sl);
+          } else {
+            *abrt = 1;  // the copy stays pending; the exit drain waits for it
+          }
+        }
+        int r, sp;
+        unit_of(warp + kB1Warps * j, r, sp);
+        float acc = 0.f;
+        if (ok) {
+          const uint4* vs = reinterpret_cast<const uint4*>(slot0 + sl * kUnitSlot);
+          const uint4 mw = reinterpret_cast<const uint4*>(slot0 + sl * kUnitSlot + kUnitVBytes)[lane];
+          const uint32_t mws[4] = {mw.x, mw.y, mw.z, mw.w};
+          const int nch = min(kSupChunks, nq - sp * kSupChunks);
+          float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const int ql = t * 32 + lane;
+            if (ql < nch) {
+              const int q = sp * kSupChunks + ql;
+              const uint4 v = vs[ql];
+              const int sw = (q >> 2) & 1;
+              const uint4 xl = xs4[(2 * q) ^ sw], xh = xs4[(2 * q + 1) ^ sw];
+              const uint32_t xw[8] = {xl.x, xl.y, xl.z, xl.w, xh.x, xh.y, xh.z, xh.w};
+              const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+              const uint32_t meta = mws[t >> 1] >> ((t & 1) * 16);
+#pragma unroll
+              for (int g = 0; g < 4; ++g) {
+                const uint32_t xp =
+                    __byte_perm(xw[2 * g], xw[2 * g + 1], sel_lut[(meta >> (4 * g)) & 0xFu]);
+                a0 = fmaf(bf_lo(vw[g]), bf_lo(xp), a0);
+                a1 = fmaf(bf_hi(vw[g]), bf_hi(xp), a1);
+              }
+            }
+          }
+          acc = a0 + a1;
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) ysp[(l0 + r - s0) * nsup + sp] = acc;
+        __syncwarp();  // every lane is done with the slot before its next copy
+      }
+      __syncthreads();
+      // a row's partials, summed in super-chunk order
+      float yrow = 0.f;
+      const int i = threadIdx.x;
+      if (i < s1 - s0)
+        for (int q = 0; q < nsup; ++q) yrow += ysp[i * nsup + q];
+      if (!waited) {
+        pdl_wait();
+        waited = true;
+      }
+      if (s0 == l0 && P.r_pad > 0)
+        for (int o = threadIdx.x; o < P.r_pad; o += kB1Threads) zs[o] = __ldcg(P.z + o);
+      __syncthreads();
+      if (i < s1 - s0) ysp[i] = yrow;
+      __syncthreads();
+      urows<__nv_bfloat16, 1, kB1Threads>(P, zs, ysp, s0, s1, y, 1);
+      __syncthreads();
+    }
+    row = P.row0 + l1;
+    ++p;
+  }
+  // after an abort, copies still in flight land before the CTA exits
+  for (int sl = 0; sl < 2; ++sl)
+    if ((pending >> sl) & 1u) tc::mbar_wait(mybar + sl, (ph >> sl) & 1u, a.err);
+}
+
+// Shared memory a CTA of the current device may opt in to.
+int max_dyn_smem() {
+  int dev = 0, v = 0;
+  cudaGetDevice(&dev);
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return v - 1024;  // room for the kernels' static shared memory
+}
+
+// HSL_DECODE_B1=regs keeps batch-1 2:4 on the register-fed kernel (a cross-check).
+bool decode_b1_bulk_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("HSL_DECODE_B1");
+    return !(e && std::strcmp(e, "regs") == 0);
+  }();
+  return on;
+}
+
 template <typename T, int BC>
 size_t apply_smem(const ApplyPlan& plan) {
   return size_t(BC) * plan.r_pad_max * 4 + size_t(kSeg) * BC * 4 +
@@ -450,9 +683,40 @@ hsl_status launch_chunk(ApplyPlan& plan, ApplyArgs a, int num_sms, cudaStream_t 
     const size_t zsm = size_t(kThreads) * 8 * BCZ * 4;
     auto zk = k_lowrank_z<T, BCZ>;
     cudaFuncSetAttribute(zk, cudaFuncAttributeMaxDynamicSharedMemorySize, int(zsm));
+    // the apply CTAs start beside the z CTAs (programmatic dependent launch):
+    // an SM configured for z's small shared memory could not take one
+    cudaFuncSetAttribute(zk, cudaFuncAttributePreferredSharedMemoryCarveout,
+                         cudaSharedmemCarveoutMaxShared);
     zk<<<plan.z_grid, kThreads, zsm, s>>>(a);
     note_launch();
     if (hsl_status e = cuda_fail(cudaGetLastError(), "z launch")) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kThreads);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = plan.z_grid > 0 ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // every CTA stages the whole x of its layers: keep at least ~64 rows per CTA
+  // so small layers are not dominated by that staging
+  const int64_t row_cap = std::max<int64_t>(1, plan.rows_total / 64);
+  if (BC == 1 && sizeof(T) == 2 && plan.fmt == HSL_FMT_NM24 && plan.vec16 &&
+      decode_b1_bulk_enabled()) {
+    const B1Layout lay = b1_layout(plan.n_max, plan.r_pad_max);
+    // unit indices stay below 2^26, where the unit → (row, super-chunk) split is exact
+    if (lay.total <= max_dyn_smem() && plan.rows_total * lay.nsup < (int64_t(1) << 26)) {
+      auto bk = k_apply_24_b1_tma;
+      if (cudaError_t e =
+              cudaFuncSetAttribute(bk, cudaFuncAttributeMaxDynamicSharedMemorySize, lay.total))
+        return cuda_fail(e, "apply smem attribute");
+      cfg.gridDim = dim3(unsigned(std::min<int64_t>(num_sms, row_cap)));
+      cfg.blockDim = dim3(kB1Threads);
+      cfg.dynamicSmemBytes = size_t(lay.total);
+      note_launch();
+      return cuda_fail(cudaLaunchKernelEx(&cfg, bk, a, lay), "apply launch");
+    }
   }
   const size_t sm = apply_smem<T, BC>(plan);
   auto ak = plan.fmt == HSL_FMT_CSR ? k_apply_decode<T, BC, true> : k_apply_decode<T, BC, false>;
@@ -462,21 +726,10 @@ hsl_status launch_chunk(ApplyPlan& plan, ApplyArgs a, int num_sms, cudaStream_t 
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, ak, kThreads, sm);
   occ = std::max(1, std::min(occ, 24));
   while (24 % occ) --occ;
-  // every CTA stages the whole x of its layers: keep at least ~64 rows per CTA
-  // so small layers are not dominated by that staging
   int grid = num_sms * occ;
-  const int64_t row_cap = std::max<int64_t>(1, plan.rows_total / 64);
   if (grid > row_cap) grid = int(row_cap);
-  cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(grid));
-  cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = sm;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = plan.z_grid > 0 ? 1 : 0;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   note_launch();
   return cuda_fail(cudaLaunchKernelEx(&cfg, ak, a), "apply launch");
 }
@@ -518,6 +771,7 @@ hsl_status apply_decode_run(ApplyPlan& plan, const void* X, void* Y, const void*
   a.b0 = 0;
   a.bc = 0;
   a.r_pad_max = plan.r_pad_max;
+  a.err = plan.err;
   if (plan.dtype == HSL_BF16) return run_typed<__nv_bfloat16>(plan, a, batch, num_sms, s);
   return run_typed<float>(plan, a, batch, num_sms, s);
 }

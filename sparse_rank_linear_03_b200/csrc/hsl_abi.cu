@@ -105,7 +105,7 @@ hsl_status ensure_err_word(Handle& h, cudaStream_t s) {
 void free_all(Handle& h) {
   DevBuf* bufs[] = {&h.row_ptr, &h.col, &h.val, &h.nm_val, &h.nm_idx, &h.prow, &h.pcol,
                     &h.pval, &h.pmeta, &h.pmeta_tc, &h.U, &h.V, &h.Vt, &h.zpart, &h.z, &h.zcount,
-                    &h.err, &h.split_ws, &h.flags, &h.xstage, &h.ystage, &h.zpre, &h.plan.probs,
+                    &h.err, &h.split_ws, &h.flags, &h.tiles, &h.xstage, &h.ystage, &h.zpre, &h.plan.probs,
                     &h.plan.prob_row0, &h.plan.cta_rows, &h.plan.xy_ptrs};
   for (DevBuf* b : bufs) release(*b);
 }

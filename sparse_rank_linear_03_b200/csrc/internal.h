@@ -55,6 +55,8 @@ struct ApplyPlan {
   int64_t rows_total = 0;
   int z_grid = 0;       // CTAs of the z launch (0 when r == 0)
   int slices = 0;       // equal-byte row ranges the apply grid divides among CTAs
+  bool vec16 = false;   // every layer has n % 16 == 0 (16-byte aligned 2:4 rows)
+  uint32_t* err = nullptr;  // error word the apply kernels report to (first member's)
   DevBuf probs;         // ApplyProblem[count]
   DevBuf prob_row0;     // int64[count+1]
   DevBuf cta_rows;      // int64[apply_grid+1]
@@ -85,6 +87,7 @@ struct Handle {
 
   // workspace
   DevBuf zpart, z, zcount, err, split_ws, flags;
+  DevBuf tiles;  // per-tile counts of the sampled-bracket split
   DevBuf xstage, ystage, zpre;
   int z_ncta = 0;
   ApplyPlan plan;  // the single-layer plan, built by hsl_pack

@@ -328,6 +328,8 @@ hsl_status plan_build(ApplyPlan& plan, Handle* const* hs, int count, cudaStream_
   plan.dtype = hs[0]->dtype;
   plan.n_max = 0;
   plan.r_pad_max = 0;
+  plan.vec16 = true;
+  plan.err = static_cast<uint32_t*>(hs[0]->err.p);
   const int eb = dtype_bytes(plan.dtype);
   std::vector<ApplyProblem> probs(count);
   int64_t row0 = 0;
@@ -370,6 +372,7 @@ hsl_status plan_build(ApplyPlan& plan, Handle* const* hs, int count, cudaStream_
     P.z_ncta = zn;
     zc += zn;
     plan.n_max = std::max(plan.n_max, int32_t(h.n));
+    plan.vec16 = plan.vec16 && h.n % 16 == 0;
     plan.r_pad_max = std::max(plan.r_pad_max, h.r_pad);
   }
   plan.rows_total = row0;

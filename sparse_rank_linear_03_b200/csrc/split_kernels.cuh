@@ -5,6 +5,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "tc.cuh"
 
 namespace hsl {
 namespace {
@@ -15,6 +16,13 @@ struct SelState {
   uint32_t gt;      // keys strictly above the prefix range so far
   uint32_t pad;
 };
+
+// Emit tiles: W is processed in tiles of kTileBytes by CTAs of kTileThreads.
+constexpr int kTileThreads = 256;
+constexpr int kTileBytes = 32768;
+constexpr int kStages = 3;
+constexpr int kTileVPT = kTileBytes / 16 / kTileThreads;  // vectors per thread
+constexpr int kStageOutBytes = 12288;                     // gathered (col, val) of a tile
 
 template <typename KT> struct KeyTraits;
 template <> struct KeyTraits<uint16_t> {
@@ -37,7 +45,9 @@ template <typename KT, int BITS>
 __global__ void __launch_bounds__(1024) k_split_hist(const KT* __restrict__ W, int64_t count,
                                                      const SelState* __restrict__ st, int shift,
                                                      unsigned* __restrict__ ghist,
-                                                     uint32_t* __restrict__ err, int vec_ok) {
+                                                     uint32_t* __restrict__ err, int vec_ok,
+                                                     const uint32_t* __restrict__ skip) {
+  if (skip && *skip) return;  // the threshold is already known
   constexpr int NB = 1 << BITS;
   constexpr int EPV = 16 / sizeof(KT);
   extern __shared__ unsigned sh[];
@@ -93,7 +103,9 @@ __global__ void __launch_bounds__(1024) k_split_hist(const KT* __restrict__ W, i
 
 // One CTA: locate the digit holding the rem-th largest matching key.
 __global__ void __launch_bounds__(1024) k_split_select(const unsigned* __restrict__ ghist, int nb,
-                                                       int shift, SelState* st) {
+                                                       int shift, SelState* st,
+                                                       const uint32_t* __restrict__ skip) {
+  if (skip && *skip) return;
   __shared__ unsigned warp_tot[32];
   const int t = threadIdx.x, nt = blockDim.x;
   const int per = (nb + nt - 1) / nt;
@@ -133,6 +145,376 @@ __global__ void __launch_bounds__(1024) k_split_select(const unsigned* __restric
         break;
       }
       acc += h;
+    }
+  }
+}
+
+// ---- bf16 threshold from a sampled bracket ------------------------------------
+// A sample of W (one run of kSampleRun vectors at a hashed offset in every
+// stratum of kSampleStride vectors) brackets the key of the k-th largest
+// magnitude: [lo, hi] around the sample's rank k·S/count with a wide margin.
+// One pass over W then counts keys > hi and histograms only the keys inside
+// the bracket (a few percent of W), replacing a shared-memory atomic per
+// element by two packed compares.  If the true threshold is not inside the
+// bracket (the sample misled), the full histogram pass runs instead; the
+// result is exact either way.
+constexpr int kSampleRun = 32;        // vectors of 8 bf16 per sampled run
+constexpr int kSampleStride = 2048;   // vectors per stratum (one run each)
+
+struct Bracket {
+  uint32_t lo, hi;  // keys in [lo, hi] are histogrammed, keys > hi counted
+  uint32_t above;   // number of keys > hi
+  uint32_t ok;      // 1 when the threshold was found inside the bracket
+};
+
+__device__ __forceinline__ uint32_t mix32(uint32_t x) {  // integer hash (lowbias32)
+  x ^= x >> 16;
+  x *= 0x7feb352dU;
+  x ^= x >> 15;
+  x *= 0x846ca68bU;
+  x ^= x >> 16;
+  return x;
+}
+
+// Histogram of the sampled 15-bit keys (NaN keys left out).
+__global__ void __launch_bounds__(1024) k_sample_hist(const uint16_t* __restrict__ W,
+                                                      int64_t nstrata,
+                                                      unsigned* __restrict__ shist) {
+  extern __shared__ unsigned sh[];
+  for (int i = threadIdx.x; i < 32768; i += blockDim.x) sh[i] = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int64_t gw = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = (int64_t(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t c = gw; c < nstrata; c += nw) {  // one warp per run, a vector per lane
+    const int64_t v0 = c * kSampleStride + mix32(uint32_t(c)) % uint32_t(kSampleStride - kSampleRun + 1);
+    const uint4 q = ld_stream16(W + (v0 + lane) * 8);
+    const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t k0 = w4[u] & 0x7FFFu, k1 = (w4[u] >> 16) & 0x7FFFu;
+      if (k0 <= 0x7F80u) atomicAdd(&sh[k0], 1u);
+      if (k1 <= 0x7F80u) atomicAdd(&sh[k1], 1u);
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < 32768; i += blockDim.x)
+    if (sh[i]) atomicAdd(&shist[i], sh[i]);
+}
+
+// One CTA: per thread 32 bins counted from the top key down; returns through
+// `rank_key` the key at which the inclusive count from the top first reaches
+// each target rank (lo for r_lo, hi for r_hi).
+__global__ void __launch_bounds__(1024) k_bracket_select(const unsigned* __restrict__ shist,
+                                                         uint32_t r_hi, uint32_t r_lo,
+                                                         Bracket* __restrict__ br) {
+  __shared__ unsigned warp_tot[32];
+  __shared__ uint32_t key_hi, key_lo;
+  const int t = threadIdx.x;
+  constexpr int PER = 32768 / 1024;
+  if (t == 0) {
+    key_hi = 0x7FFFu;  // r_hi == 0: nothing is certainly above the threshold
+    key_lo = 0u;       // r_lo beyond the sample: keep every key in the bracket
+  }
+  const int top = 32767 - t * PER;  // this thread's bins: top, top−1, ..., top−PER+1
+  unsigned s = 0;
+  for (int b = 0; b < PER; ++b) s += shist[top - b];
+  unsigned incl = s;
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned v = __shfl_up_sync(0xffffffffu, incl, o);
+    if ((t & 31) >= o) incl += v;
+  }
+  if ((t & 31) == 31) warp_tot[t >> 5] = incl;
+  __syncthreads();
+  if (t < 32) {
+    const unsigned w = warp_tot[t];
+    unsigned wi = w;
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned v = __shfl_up_sync(0xffffffffu, wi, o);
+      if (t >= o) wi += v;
+    }
+    warp_tot[t] = wi - w;
+  }
+  __syncthreads();
+  const unsigned before = warp_tot[t >> 5] + incl - s;
+  // hi: the largest key with more than r_hi sample keys at or above it, so at
+  // most r_hi sample keys lie strictly above hi
+  if (r_hi > 0 && r_hi >= before && r_hi < before + s) {
+    unsigned acc = before;
+    for (int b = 0; b < PER; ++b) {
+      acc += shist[top - b];
+      if (acc > r_hi) {
+        key_hi = uint32_t(top - b);
+        break;
+      }
+    }
+  }
+  // lo: the largest key with at least r_lo sample keys at or above it
+  if (r_lo > before && r_lo <= before + s) {
+    unsigned acc = before;
+    for (int b = 0; b < PER; ++b) {
+      acc += shist[top - b];
+      if (acc >= r_lo) {
+        key_lo = uint32_t(top - b);
+        break;
+      }
+    }
+  }
+  __syncthreads();
+  if (t == 0) {
+    br->hi = key_hi;
+    br->lo = min(key_lo, key_hi);
+    br->above = 0;
+    br->ok = 0;
+  }
+}
+
+// Full pass: count keys > hi, histogram keys in [lo, hi] into ghist[key],
+// flag NaN.  bf16 pairs are compared by packed subtraction (see vec_masks).
+// When the bracket spans at most kTileBins keys and tile_hist is given, each
+// warp takes whole emit tiles (kTileBytes of W) and also records, per tile,
+// the count above the bracket and the tile's bracket histogram; with the
+// threshold known, those give every tile's exact (above T, equal to T) counts,
+// so the emit pass needs no look-back.
+constexpr int kTileBins = 64;
+
+__global__ void __launch_bounds__(1024) k_count_bracket(const uint16_t* __restrict__ W,
+                                                        int64_t nvec, Bracket* __restrict__ br,
+                                                        unsigned* __restrict__ ghist,
+                                                        uint32_t* __restrict__ err,
+                                                        uint32_t* __restrict__ tile_above,
+                                                        uint32_t* __restrict__ tile_hist) {
+  extern __shared__ unsigned sh[];
+  __shared__ unsigned warp_above[32];
+  __shared__ unsigned wh[32][kTileBins];
+  const uint32_t lo = br->lo, hi = br->hi;
+  const int nb = int(hi - lo) + 1;
+  const bool record = tile_hist != nullptr && nb <= kTileBins;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < nb; i += blockDim.x) sh[i] = 0;
+  for (int i = lane; i < kTileBins; i += 32) wh[warp][i] = 0;
+  __syncthreads();
+  unsigned* bins = record ? wh[warp] : sh;
+  const uint32_t H = 0x80008000u;
+  const uint32_t HI1 = (hi + 1u) * 0x00010001u, LO = lo * 0x00010001u, NAN1 = 0x7F81u * 0x00010001u;
+  unsigned above = 0;
+  uint32_t nan = 0;  // bit 15 / 31 set once some key ≥ 0x7F81 (a NaN)
+  // one 16-byte vector: keys above hi add to two 16-bit counters in `cnt`
+  // (flushed by the caller before either could reach 2^16), keys inside the
+  // bracket (rare) go to the histogram
+  auto vec = [&](const uint4& q, uint32_t& cnt) {
+    const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+    uint32_t in4[4], any = 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t kw = w4[u] | H;
+      const uint32_t dh = kw - HI1;
+      nan |= kw - NAN1;
+      cnt += (dh & H) >> 15;
+      in4[u] = (kw - LO) & ~dh & H;
+      any |= in4[u];
+    }
+    if (any) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (in4[u] & 0x8000u) atomicAdd(&bins[(w4[u] & 0x7FFFu) - lo], 1u);
+        if (in4[u] & 0x80000000u) atomicAdd(&bins[((w4[u] >> 16) & 0x7FFFu) - lo], 1u);
+      }
+    }
+  };
+  auto flush = [&](uint32_t& cnt) {
+    above += (cnt & 0xFFFFu) + (cnt >> 16);
+    cnt = 0;
+  };
+  if (record) {
+    constexpr int VPT = kTileBytes / 16;  // vectors of a tile
+    const int64_t ntiles = (nvec + VPT - 1) / VPT;
+    const int64_t gw = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nw = (int64_t(gridDim.x) * blockDim.x) >> 5;
+    unsigned above_all = 0;
+    for (int64_t tile = gw; tile < ntiles; tile += nw) {
+      const int64_t v0 = tile * VPT, vend = min(v0 + VPT, nvec);
+      above = 0;
+      uint32_t cnt = 0;  // ≤ 64 vectors · 4 words per lane and tile: no overflow
+      for (int it = 0; it < VPT / 32; it += 8) {
+        uint4 q[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int64_t v = v0 + (it + u) * 32 + lane;
+          if (v < vend) q[u] = ld_stream16(W + v * 8);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (v0 + (it + u) * 32 + lane < vend) vec(q[u], cnt);
+      }
+      flush(cnt);
+      for (int o = 16; o; o >>= 1) above += __shfl_xor_sync(0xffffffffu, above, o);
+      __syncwarp();
+      for (int b = lane; b < kTileBins; b += 32) {
+        const unsigned c = wh[warp][b];
+        tile_hist[tile * kTileBins + b] = c;
+        if (c) atomicAdd(&sh[b], c);
+        wh[warp][b] = 0;
+      }
+      if (lane == 0) tile_above[tile] = above;
+      above_all += above;
+      __syncwarp();
+    }
+    above = lane == 0 ? above_all : 0u;
+  } else {
+    const int64_t gtid = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t gstride = int64_t(gridDim.x) * blockDim.x;
+    for (int64_t v = gtid; v < nvec; v += 4 * gstride) {
+      uint4 q[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t iv = v + u * gstride;
+        if (iv < nvec) q[u] = ld_stream16(W + iv * 8);
+      }
+      uint32_t cnt = 0;  // 16 words at most before the flush
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (v + u * gstride < nvec) vec(q[u], cnt);
+      flush(cnt);
+    }
+  }
+  for (int o = 16; o; o >>= 1) above += __shfl_xor_sync(0xffffffffu, above, o);
+  if (lane == 0) warp_above[warp] = above;
+  if (__syncthreads_or((nan & H) != 0) && threadIdx.x == 0) set_error(err, kErrNaN);
+  if (threadIdx.x == 0) {
+    unsigned a = 0;
+    for (int w = 0; w < int(blockDim.x >> 5); ++w) a += warp_above[w];
+    atomicAdd(&br->above, a);
+  }
+  for (int i = threadIdx.x; i < nb; i += blockDim.x)
+    if (sh[i]) atomicAdd(&ghist[lo + i], sh[i]);
+}
+
+// Whether the tile counts recorded by k_count_bracket give the emit its
+// prefixes: the bracket held the threshold and was narrow enough to record.
+__device__ __forceinline__ bool tile_counts_usable(const Bracket* br) {
+  return br->ok && br->hi - br->lo + 1u <= uint32_t(kTileBins);
+}
+
+// Per tile: (keys > T) << 32 | (keys == T), one warp per tile.
+__global__ void __launch_bounds__(256) k_tile_counts(const uint32_t* __restrict__ tile_above,
+                                                     const uint32_t* __restrict__ tile_hist,
+                                                     int64_t ntiles, const Bracket* __restrict__ br,
+                                                     const SelState* __restrict__ st,
+                                                     unsigned long long* __restrict__ tile_cnt) {
+  if (!tile_counts_usable(br)) return;
+  const uint32_t T = st->prefix, lo = br->lo;
+  const int lane = threadIdx.x & 31;
+  const int64_t gw = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = (int64_t(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t tile = gw; tile < ntiles; tile += nw) {
+    unsigned gt = 0, eq = 0;
+    for (int b = lane; b < kTileBins; b += 32) {
+      const unsigned c = tile_hist[tile * kTileBins + b];
+      gt += lo + uint32_t(b) > T ? c : 0u;
+      eq += lo + uint32_t(b) == T ? c : 0u;
+    }
+    for (int o = 16; o; o >>= 1) {
+      gt += __shfl_xor_sync(0xffffffffu, gt, o);
+      eq += __shfl_xor_sync(0xffffffffu, eq, o);
+    }
+    if (lane == 0)
+      tile_cnt[tile] = ((unsigned long long)(tile_above[tile] + gt) << 32) | eq;
+  }
+}
+
+// One CTA: exclusive prefix of the packed tile counts (both halves stay below
+// 2^32 because W has fewer than 2^32 elements on this path).
+__global__ void __launch_bounds__(1024) k_tile_scan(const unsigned long long* __restrict__ tile_cnt,
+                                                    int64_t ntiles, const Bracket* __restrict__ br,
+                                                    unsigned long long* __restrict__ tile_pre) {
+  if (!tile_counts_usable(br)) return;
+  __shared__ unsigned long long warp_tot[32];
+  const int t = threadIdx.x;
+  const int64_t per = (ntiles + 1023) / 1024;
+  const int64_t a = min(int64_t(t) * per, ntiles), b = min(a + per, ntiles);
+  unsigned long long s = 0;
+  for (int64_t i = a; i < b; ++i) s += tile_cnt[i];
+  unsigned long long incl = s;
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long v = __shfl_up_sync(0xffffffffu, incl, o);
+    if ((t & 31) >= o) incl += v;
+  }
+  if ((t & 31) == 31) warp_tot[t >> 5] = incl;
+  __syncthreads();
+  if (t < 32) {
+    const unsigned long long w = warp_tot[t];
+    unsigned long long wi = w;
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned long long v = __shfl_up_sync(0xffffffffu, wi, o);
+      if (t >= o) wi += v;
+    }
+    warp_tot[t] = wi - w;
+  }
+  __syncthreads();
+  unsigned long long run = warp_tot[t >> 5] + incl - s;
+  for (int64_t i = a; i < b; ++i) {
+    tile_pre[i] = run;
+    run += tile_cnt[i];
+  }
+}
+
+// One CTA: the threshold from the bracket, or (threshold outside it) a clean
+// state and histogram for the full pass.
+__global__ void __launch_bounds__(1024) k_bracket_finish(unsigned* __restrict__ ghist,
+                                                         Bracket* __restrict__ br,
+                                                         SelState* __restrict__ st, uint32_t k) {
+  __shared__ unsigned warp_tot[32];
+  __shared__ int found;
+  const int t = threadIdx.x;
+  const uint32_t lo = br->lo, hi = br->hi, above = br->above;
+  const int nb = int(hi - lo) + 1;
+  const int per = (nb + 1023) / 1024;
+  if (t == 0) found = 0;
+  const int top = int(hi) - t * per;  // bins top, top−1, ... (≥ lo)
+  unsigned s = 0;
+  for (int b = 0; b < per; ++b)
+    if (top - b >= int(lo)) s += ghist[top - b];
+  unsigned incl = s;
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned v = __shfl_up_sync(0xffffffffu, incl, o);
+    if ((t & 31) >= o) incl += v;
+  }
+  if ((t & 31) == 31) warp_tot[t >> 5] = incl;
+  __syncthreads();
+  if (t < 32) {
+    const unsigned w = warp_tot[t];
+    unsigned wi = w;
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned v = __shfl_up_sync(0xffffffffu, wi, o);
+      if (t >= o) wi += v;
+    }
+    warp_tot[t] = wi - w;
+  }
+  __syncthreads();
+  const unsigned before = above + warp_tot[t >> 5] + incl - s;
+  if (k > before && k <= before + s) {
+    unsigned acc = before;
+    for (int b = 0; b < per && top - b >= int(lo); ++b) {
+      const unsigned h = ghist[top - b];
+      if (acc + h >= k) {
+        st->prefix = uint32_t(top - b);
+        st->rem = k - acc;
+        st->gt = acc;
+        found = 1;
+        break;
+      }
+      acc += h;
+    }
+  }
+  __syncthreads();
+  if (t == 0) br->ok = uint32_t(found);
+  if (!found) {  // back to the state the full histogram pass expects
+    for (int i = t; i < nb; i += 1024) ghist[lo + i] = 0;
+    if (t == 0) {
+      st->prefix = 0;
+      st->rem = k;
+      st->gt = 0;
     }
   }
 }
@@ -363,25 +745,6 @@ __global__ void __launch_bounds__(kEmitThreads) k_split_emit(
   }
 }
 
-// ---- emit over blocks of rows held in registers ---------------------------------
-// A CTA takes a ticket for `rb` consecutive rows (rb·n ≤ 256·kVPT·EPV elements),
-// loads them once into registers (coalesced 16-byte vectors, vector v of the
-// block at k-major position v = kk·256 + t), ranks every element inside the
-// block with warp scans per kk plus one scan of the (kk, warp) totals, and
-// gets the block's exclusive prefix by a warp-parallel decoupled look-back
-// (32 predecessor flags per poll).
-constexpr int kVPT = 16;
-
-__device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t u = __shfl_up_sync(0xffffffffu, v, o);
-    if (lane >= o) v += u;
-  }
-  return v;
-}
-
 // Warp 0 only.  Publishes the block aggregate, returns the exclusive prefix.
 __device__ __forceinline__ void lookback(unsigned long long* flags, int64_t blk, uint32_t agg_gt,
                                          uint32_t agg_eq, uint32_t* err, uint32_t& ex_gt,
@@ -468,141 +831,242 @@ __device__ __forceinline__ void vec_masks<uint32_t>(const uint4& q, uint32_t T, 
   }
 }
 
+// ---- emit over element tiles staged by bulk copies -----------------------------
+// W is cut into tiles of kTileBytes (any number of rows or part of one).  A
+// persistent CTA takes tiles in ticket order and keeps kStages of them in
+// flight: a 1-D bulk copy brings each into shared memory; the residual goes
+// back with a bulk store from the same buffer.  Thread t owns the vectors
+// [8t, 8t + 8) of its tile and visits them starting at slot t & 7, so at every
+// step the eight threads of a quarter-warp read eight different bank groups.
+// The kept entries of a tile (a contiguous range of S) are gathered in shared
+// memory and written out with coalesced stores.
+
+// Unsigned 32-bit division by an invariant divisor d (1 ≤ d < 2^31): with
+// l = ceil(log2 d) and mult = floor(2^32·(2^l − d)/d) + 1,
+// q = (t + ((x − t) >> s1)) >> s2, t = mulhi(mult, x), s1 = min(l, 1),
+// s2 = max(l − 1, 0), exact for every 32-bit x (Granlund & Montgomery 1994).
+struct FastDiv {
+  uint32_t d, mult, s1, s2;
+};
+inline FastDiv make_fastdiv(uint32_t d) {
+  FastDiv f;
+  f.d = d;
+  uint32_t l = 0;
+  while ((uint64_t(1) << l) < d) ++l;
+  f.mult = uint32_t(((uint64_t(1) << 32) * ((uint64_t(1) << l) - d)) / d + 1);
+  f.s1 = l < 1 ? l : 1;
+  f.s2 = l > 1 ? l - 1 : 0;
+  return f;
+}
+__device__ __forceinline__ uint32_t fdiv(const FastDiv& f, uint32_t x) {
+  const uint32_t t = __umulhi(f.mult, x);
+  return (t + ((x - t) >> f.s1)) >> f.s2;
+}
+
+template <typename KT>
+__device__ __forceinline__ void zero_kept(uint4& q, uint32_t sel);
+template <>
+__device__ __forceinline__ void zero_kept<uint16_t>(uint4& q, uint32_t sel) {
+  uint32_t* w = &q.x;
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+    w[u] &= ~((((sel >> (2 * u)) & 1u) * 0x0000FFFFu) | (((sel >> (2 * u + 1)) & 1u) * 0xFFFF0000u));
+}
+template <>
+__device__ __forceinline__ void zero_kept<uint32_t>(uint4& q, uint32_t sel) {
+  uint32_t* w = &q.x;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) w[u] = ((sel >> u) & 1u) ? 0u : w[u];
+}
+
+template <typename KT>
+__device__ __forceinline__ uint32_t vec_elem(const uint4& q, int e) {
+  const uint32_t w0 = (e & (sizeof(KT) == 2 ? 4 : 2)) ? ((e & (sizeof(KT) == 2 ? 2 : 1)) ? q.w : q.z)
+                                                      : ((e & (sizeof(KT) == 2 ? 2 : 1)) ? q.y : q.x);
+  return sizeof(KT) == 2 ? ((w0 >> ((e & 1) * 16)) & 0xFFFFu) : w0;
+}
+
 template <typename KT, typename SB>
-__global__ void __launch_bounds__(kEmitThreads) k_split_emit_blk(
-    const KT* __restrict__ W, int64_t m, int64_t n, int rb, int64_t nblk,
+__global__ void __launch_bounds__(kTileThreads, 2) k_split_emit_tile(
+    const KT* __restrict__ W, int64_t m, int64_t count, FastDiv nd, int64_t ntiles,
     const SelState* __restrict__ st, unsigned* __restrict__ ticket,
     unsigned long long* __restrict__ flags, int32_t* __restrict__ row_ptr,
     int32_t* __restrict__ col, SB* __restrict__ val, KT* __restrict__ R, int64_t k,
-    uint32_t* __restrict__ err) {
+    uint32_t* __restrict__ err, const Bracket* __restrict__ br,
+    const unsigned long long* __restrict__ tile_pre) {
   constexpr int EPV = 16 / sizeof(KT);
-  constexpr uint32_t STEP = kEmitThreads * EPV;  // elements between a thread's vectors
-  __shared__ uint32_t wt[kVPT][kEmitThreads / 32];
-  __shared__ int64_t sh_blk;
+  constexpr int TE = kTileBytes / sizeof(KT);
+  constexpr int CAP = kStageOutBytes / (4 + sizeof(SB));
+  extern __shared__ __align__(16) unsigned char smem[];
+  uint4* tiles = reinterpret_cast<uint4*>(smem);
+  int32_t* o_col = reinterpret_cast<int32_t*>(smem + kStages * kTileBytes);
+  SB* o_val = reinterpret_cast<SB*>(o_col + CAP);
+  __shared__ uint64_t bar[kStages];
+  __shared__ int64_t s_tile[kStages];
+  __shared__ uint32_t sh_warp[kTileThreads / 32 + 1];
   __shared__ uint32_t sh_ex[2];
+  __shared__ int s_abort;
+  __shared__ uint32_t s_late;  // stages whose wait gave up (bit sg) and its parity (bit 8 + sg)
+
   const uint32_t T = st->prefix;
   const uint32_t need = st->rem;
-  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const uint32_t n32 = uint32_t(n);
+  const int t = threadIdx.x;
+  const int64_t n = nd.d;
+  // tile prefixes from the recorded counts when available, else look-back
+  const bool pre = tile_pre != nullptr && tile_counts_usable(br);
+  const uint64_t policy = tc::make_policy_evict_first();
 
-  for (;;) {
-    if (t == 0) sh_blk = int64_t(atomicAdd(ticket, 1u));
-    __syncthreads();
-    const int64_t blk = sh_blk;
-    if (blk >= nblk) break;
-    const int64_t row0 = blk * rb;
-    const int64_t rows = min(int64_t(rb), m - row0);
-    const int64_t e0 = row0 * n;
-    const uint32_t nv = uint32_t(rows * n / EPV);
-    const KT* Wb = W + e0;
-
-    // phase 1: load the block (coalesced, k-major), masks, ranks inside the block
-    uint4 q[kVPT];
-    uint32_t ex[kVPT];
-    uint32_t mk[kVPT / 2];  // (gm | em << 8) of vector kk in half kk & 1
-#pragma unroll
-    for (int kk = 0; kk < kVPT; ++kk) {
-      const uint32_t v = uint32_t(kk * kEmitThreads + t);
-      uint32_t pk = 0, gm = 0, em = 0;
-      if (v < nv) {
-        q[kk] = ld_stream16(Wb + int64_t(v) * EPV);
-        vec_masks<KT>(q[kk], T, gm, em);
-        pk = (uint32_t(__popc(gm)) << 16) | uint32_t(__popc(em));
-      }
-      const uint32_t m16 = gm | (em << 8);
-      if (kk & 1) mk[kk >> 1] |= m16 << 16; else mk[kk >> 1] = m16;
-      const uint32_t incl = warp_incl_scan(pk);
-      ex[kk] = incl - pk;
-      if (lane == 31) wt[kk][warp] = incl;
+  auto fetch = [&](int sg) {  // thread 0: next ticket into stage sg
+    const int64_t id = s_abort ? ntiles : int64_t(atomicAdd(ticket, 1u));
+    if (id < ntiles) {
+      const int64_t e0 = id * TE;
+      const uint32_t bytes = uint32_t((count - e0 < TE ? count - e0 : int64_t(TE)) * int64_t(sizeof(KT)));
+      tc::mbar_expect_tx(&bar[sg], bytes);
+      tc::bulk_load_hint(tiles + sg * (kTileBytes / 16), W + e0, bytes, &bar[sg], policy);
     }
-    __syncthreads();
-    if (warp == 0) {
-      // exclusive scan of the kVPT × 8 totals in k-major order: lane takes 4
-      uint32_t a[4], local = 0;
+    s_tile[sg] = id < ntiles ? id : -1;
+  };
+  if (t == 0) {
+    s_abort = 0;
+    s_late = 0;
+    for (int sg = 0; sg < kStages; ++sg) tc::mbar_init(&bar[sg], 1);
+    tc::fence_mbar_init();
+    // the last stage is filled at the end of the first iteration
+    for (int sg = 0; sg < kStages - 1; ++sg) fetch(sg);
+  }
+  __syncthreads();
+
+  const int r0 = t & (kTileVPT - 1);
+  for (int it = 0;; ++it) {
+    const int sg = it % kStages;
+    const int64_t tile = s_tile[sg];
+    if (tile < 0) break;
+    // every thread observes the copy's completion on the mbarrier itself
+    if (!tc::mbar_wait(&bar[sg], uint32_t(it / kStages) & 1u, err) && t == 0) {
+      s_abort = 1;
+      s_late |= (1u << sg) | ((uint32_t(it / kStages) & 1u) << (8 + sg));
+    }
+    const int64_t e0 = tile * TE;
+    const int nv = int((count - e0 < TE ? count - e0 : int64_t(TE)) / EPV);
+    uint4* tv = tiles + sg * (kTileBytes / 16);
+
+    // phase 1: masks and counts of the thread's vectors, slot order r0, r0+1, ...
+    uint32_t msk[kTileVPT], cnt[kTileVPT];
+    uint32_t tot = 0, lo = 0;  // lo: counts of the slots before r0
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int idx = 4 * lane + u;
-        a[u] = wt[idx >> 3][idx & 7];
-        local += a[u];
+    for (int kk = 0; kk < kTileVPT; ++kk) {
+      const int s = (kk + r0) & (kTileVPT - 1);
+      const int v = t * kTileVPT + s;
+      uint32_t gm = 0, em = 0;
+      if (v < nv) vec_masks<KT>(tv[v], T, gm, em);
+      msk[kk] = gm | (em << 8);
+      cnt[kk] = (uint32_t(__popc(gm)) << 16) | uint32_t(__popc(em));
+      tot += cnt[kk];
+      if (s < r0) lo += cnt[kk];
+    }
+    uint32_t total;
+    const uint32_t ex = block_excl_scan(tot, sh_warp, total);
+    if (pre) {
+      if (t == 0) {
+        const unsigned long long p = tile_pre[tile];
+        sh_ex[0] = uint32_t(p >> 32);
+        sh_ex[1] = uint32_t(p);
       }
-      const uint32_t incl = warp_incl_scan(local);
-      uint32_t run = incl - local;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int idx = 4 * lane + u;
-        wt[idx >> 3][idx & 7] = run;
-        run += a[u];
-      }
-      const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
+    } else if (t < 32) {
       uint32_t xg, xe;
-      lookback(flags, blk, total >> 16, total & 0xFFFFu, err, xg, xe);
-      if (lane == 0) {
+      lookback(flags, tile, total >> 16, total & 0xFFFFu, err, xg, xe);
+      if (t == 0) {
         sh_ex[0] = xg;
         sh_ex[1] = xe;
       }
     }
     __syncthreads();
-    // phase 2: kept before an element = keys > T before it + the first `need`
-    // ties in linear order that come before it
-    const uint32_t ex_gt = sh_ex[0], ex_eq = sh_ex[1];
-    uint32_t j0 = uint32_t(t) * EPV;  // column of this thread's first vector, no division
-    int64_t row = row0;
-    while (j0 >= n32) {
-      j0 -= n32;
-      ++row;
-    }
+    const uint32_t tg = sh_ex[0], te = sh_ex[1];
+    const uint32_t P0 = tg + min(need, te);  // first S position of this tile
+    const uint32_t ex_gt = tg + (ex >> 16), ex_eq = te + (ex & 0xFFFFu);
+    // the tile's columns: x = c0 + offset, row = row0 + x / n
+    const int64_t row0 = e0 / n;
+    const uint32_t c0 = uint32_t(e0 - row0 * n);
+
+    // phase 2: positions, gathered S entries, residual in place
+    uint32_t run = lo;
 #pragma unroll
-    for (int kk = 0; kk < kVPT; ++kk) {
-      const uint32_t v = uint32_t(kk * kEmitThreads + t);
+    for (int kk = 0; kk < kTileVPT; ++kk) {
+      const int s = (kk + r0) & (kTileVPT - 1);
+      if (s == 0) run = 0;
+      const int v = t * kTileVPT + s;
       if (v < nv) {
-        const uint32_t m16 = (mk[kk >> 1] >> ((kk & 1) * 16)) & 0xFFFFu;
-        const uint32_t gm = m16 & 0xFFu, em = m16 >> 8;
-        const uint32_t base = wt[kk][warp] + ex[kk];
-        const uint32_t cg = base >> 16, ce = base & 0xFFFFu;
-        const uint32_t pos0 = ex_gt + cg + min(need, ex_eq + ce);
-        if (j0 == 0) row_ptr[row] = int32_t(pos0);
+        const uint32_t gm = msk[kk] & 0xFFu, em = msk[kk] >> 8;
+        const uint32_t cg = ex_gt + (run >> 16), ce = ex_eq + (run & 0xFFFFu);
+        const uint32_t pos0 = cg + min(need, ce);
+        const uint32_t x = c0 + uint32_t(v) * EPV;
+        const uint32_t q = fdiv(nd, x);
+        const uint32_t j0 = x - q * uint32_t(n);
+        if (j0 == 0) row_ptr[row0 + q] = int32_t(pos0);
         // ties kept in this vector: the first `allow` set bits of em
-        uint32_t allow = need > ex_eq + ce ? min(need - (ex_eq + ce), uint32_t(__popc(em))) : 0u;
-        uint32_t keq = 0, rest = em;
-        for (; allow; --allow) {
-          keq |= rest & (0u - rest);
-          rest &= rest - 1u;
+        uint32_t keq = 0;
+        if (need > ce && em) {
+          uint32_t allow = min(need - ce, uint32_t(__popc(em))), rest = em;
+          for (; allow; --allow) {
+            keq |= rest & (0u - rest);
+            rest &= rest - 1u;
+          }
         }
         const uint32_t sel = gm | keq;
-        uint4 o = q[kk];
         if (sel) {
-          for (uint32_t s2 = sel; s2; s2 &= s2 - 1u) {
+          uint4 qv = tv[v];
+          uint32_t p = pos0;
+          for (uint32_t s2 = sel; s2; s2 &= s2 - 1u, ++p) {
             const int e = __ffs(s2) - 1;
-            const int64_t pos = int64_t(pos0) + __popc(sel & ((1u << e) - 1u));
-            const uint32_t w = (&o.x)[sizeof(KT) == 2 ? (e >> 1) : e];
-            const uint32_t bits = sizeof(KT) == 2 ? ((w >> ((e & 1) * 16)) & 0xFFFFu) : w;
-            if (pos < k) {
-              col[pos] = int32_t(j0 + e);
-              val[pos] = conv_val<SB>(bits, sizeof(KT));
+            const uint32_t bits = vec_elem<KT>(qv, e);
+            const uint32_t loc = p - P0;
+            if (loc < uint32_t(CAP)) {
+              o_col[loc] = int32_t(j0 + e);
+              o_val[loc] = conv_val<SB>(bits, sizeof(KT));
+            } else if (p < k) {
+              col[p] = int32_t(j0 + e);
+              val[p] = conv_val<SB>(bits, sizeof(KT));
             }
           }
-          // zero the kept elements in the residual
-          uint32_t* ow = &o.x;
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            uint32_t z;
-            if (sizeof(KT) == 2)
-              z = (((sel >> (2 * u)) & 1u) ? 0x0000FFFFu : 0u) |
-                  (((sel >> (2 * u + 1)) & 1u) ? 0xFFFF0000u : 0u);
-            else
-              z = ((sel >> u) & 1u) ? 0xFFFFFFFFu : 0u;
-            ow[u] &= ~z;
+          if (R) {
+            zero_kept<KT>(qv, sel);
+            tv[v] = qv;
           }
         }
-        if (R) st_stream16(R + e0 + int64_t(v) * EPV, o);
       }
-      j0 += STEP;
-      while (j0 >= n32) {
-        j0 -= n32;
-        ++row;
+      run += cnt[kk];
+    }
+    if (R) tc::fence_async_smem();
+    __syncthreads();
+    if (t == 0) {
+      if (R) {
+        tc::bulk_store(R + e0, tv, uint32_t(nv) * 16u);
+        tc::bulk_commit();
+      }
+      if (tile == ntiles - 1) row_ptr[m] = int32_t(k);
+    }
+    // the tile's S entries, gathered above, in coalesced stores
+    const uint32_t kept = (total >> 16) + min(need, te + (total & 0xFFFFu)) - min(need, te);
+    const uint32_t nout = min(kept, uint32_t(CAP));
+    for (uint32_t i = t; i < nout; i += kTileThreads) {
+      if (P0 + i < k) {
+        col[P0 + i] = o_col[i];
+        val[P0 + i] = o_val[i];
       }
     }
-    if (t == 0 && blk == nblk - 1) row_ptr[m] = int32_t(k);
+    if (t == 0) {
+      // the stage of the previous tile is free once its store has read it
+      // (this tile's store may still be reading its own stage)
+      if (R) tc::bulk_wait_read_but_one();
+      fetch((it + kStages - 1) % kStages);
+    }
+    __syncthreads();
+  }
+  if (t == 0) {
+    tc::bulk_wait_all();
+    // a copy whose wait gave up may still land: give it one more bounded wait
+    for (int sg = 0; sg < kStages; ++sg)
+      if ((s_late >> sg) & 1u) tc::mbar_wait(&bar[sg], (s_late >> (8 + sg)) & 1u, err);
   }
 }
 

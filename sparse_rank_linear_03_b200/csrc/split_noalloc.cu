@@ -11,7 +11,7 @@
 // __device__ array of fixed size, so it allocates nothing.
 //
 // Costs and rules that come with that:
-//   * the array (kNoAllocBytes, about 640 KB) exists on every GPU that loads
+//   * the array (kNoAllocBytes, about 2.2 MB) exists on every GPU that loads
 //     libhsl, for the life of the process;
 //   * all calls share it: calls that can overlap on the GPU (different
 //     streams, or different host threads on one device) race and corrupt each
@@ -37,7 +37,9 @@ namespace {
 constexpr int64_t kNoAllocMaxRows = 65536;
 constexpr size_t kNoAllocHist = 32768 * sizeof(unsigned);
 constexpr size_t kNoAllocState = 256;  // SelState at +0, row ticket at +64
-constexpr size_t kNoAllocBytes = kNoAllocHist + kNoAllocState + size_t(kNoAllocMaxRows) * 8;
+// look-back flags: one per row (per-row emit) or per 32 KB tile of W, m·n < 2^31
+constexpr int64_t kNoAllocFlags = std::max<int64_t>(kNoAllocMaxRows, (int64_t(4) << 31) / kTileBytes);
+constexpr size_t kNoAllocBytes = kNoAllocHist + kNoAllocState + size_t(kNoAllocFlags) * 8;
 }  // namespace
 }  // namespace hsl
 
@@ -99,6 +101,7 @@ hsl_status run_noalloc(const KT* W, int64_t m, int64_t n, int64_t k, int32_t* ro
   const int passes = sizeof(KT) == 2 ? 1 : 3;
   const int bits[3] = {sizeof(KT) == 2 ? 15 : 11, 11, 9};
   const int shifts[3] = {sizeof(KT) == 2 ? 0 : 20, 9, 0};
+  const uint32_t* skip = nullptr;  // no sampled bracket here: every pass runs
   for (int p = 0; p < passes; ++p) {
     if (k == 0 && p > 0) break;
     if (cudaError_t e = cudaMemsetAsync(hist, 0, kNoAllocHist, s)) return cuda_fail(e, "memset");
@@ -106,35 +109,40 @@ hsl_status run_noalloc(const KT* W, int64_t m, int64_t n, int64_t k, int32_t* ro
     if (bits[p] == 15) {
       auto kern = k_split_hist<KT, 15>;
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-      kern<<<d.sms, 1024, smem, s>>>(W, count, st, shifts[p], hist, err, vec_ok ? 1 : 0);
+      kern<<<d.sms, 1024, smem, s>>>(W, count, st, shifts[p], hist, err, vec_ok ? 1 : 0, skip);
     } else if (bits[p] == 11) {
       k_split_hist<KT, 11><<<d.sms * 2, 1024, smem, s>>>(W, count, st, shifts[p], hist, err,
-                                                          vec_ok ? 1 : 0);
+                                                          vec_ok ? 1 : 0, skip);
     } else {
       k_split_hist<KT, 9><<<d.sms * 2, 1024, smem, s>>>(W, count, st, shifts[p], hist, err,
-                                                         vec_ok ? 1 : 0);
+                                                         vec_ok ? 1 : 0, skip);
     }
     note_launch();
     if (hsl_status e = cuda_fail(cudaGetLastError(), "split histogram launch")) return e;
     if (k > 0) {
-      k_split_select<<<1, 1024, 0, s>>>(hist, 1 << bits[p], shifts[p], st);
+      k_split_select<<<1, 1024, 0, s>>>(hist, 1 << bits[p], shifts[p], st, skip);
       note_launch();
       if (hsl_status e = cuda_fail(cudaGetLastError(), "split select launch")) return e;
     }
   }
   // the ticket and the look-back flags must start at zero
   if (cudaError_t e = cudaMemsetAsync(ticket, 0, 4, s)) return cuda_fail(e, "memset");
-  if (cudaError_t e = cudaMemsetAsync(flags, 0, size_t(m) * 8, s)) return cuda_fail(e, "memset");
-  constexpr int EPV = 16 / sizeof(KT);
-  const int64_t cap = int64_t(kEmitThreads) * kVPT * EPV;
-  if (vec_ok && n <= cap) {
-    const int rb = int(cap / n);
-    const int64_t nblk = (m + rb - 1) / rb;
+  const int64_t nflags = std::max<int64_t>(m, (count * int64_t(sizeof(KT)) + kTileBytes - 1) / kTileBytes);
+  if (cudaError_t e = cudaMemsetAsync(flags, 0, size_t(nflags) * 8, s)) return cuda_fail(e, "memset");
+  if (vec_ok) {
+    constexpr int TE = kTileBytes / int(sizeof(KT));
+    const int64_t ntiles = (count + TE - 1) / TE;
+    const size_t smem = size_t(kStages) * kTileBytes + kStageOutBytes;
+    auto kern = k_split_emit_tile<KT, SB>;
+    if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             int(smem)))
+      return cuda_fail(e, "split emit smem attribute");
     int occ = 0;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_split_emit_blk<KT, SB>, kEmitThreads, 0);
-    const int64_t grid = std::min<int64_t>(nblk, int64_t(d.sms) * std::max(occ, 1));
-    k_split_emit_blk<KT, SB><<<unsigned(grid), kEmitThreads, 0, s>>>(
-        W, m, n, rb, nblk, st, ticket, flags, row_ptr, col, val, R, k, err);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kTileThreads, smem);
+    const int64_t grid = std::min<int64_t>(ntiles, int64_t(d.sms) * std::max(occ, 1));
+    kern<<<unsigned(std::max<int64_t>(grid, 1)), kTileThreads, smem, s>>>(
+        W, m, count, make_fastdiv(uint32_t(n)), ntiles, st, ticket, flags, row_ptr, col, val, R,
+        k, err, nullptr, nullptr);
   } else {
     int occ = 0;
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_split_emit<KT, SB>, kEmitThreads, 0);

@@ -97,9 +97,52 @@ def test_topk_tie_heavy(hsl, dtype, shape, frac):
                                          ("bf16", (70, 32768)), ("f32", (33, 16384))])
 @pytest.mark.parametrize("frac", [0.01, 0.5])
 def test_topk_wide_rows(hsl, dtype, shape, frac):
-    """Rows wider than one register block (per-row emit) and exactly one block."""
+    """Rows wider than one 32 KB tile, and rows of exactly one tile."""
     W = tie_heavy(*shape, seed=shape[1], dtype=dtype)
     assert_topk_parity(hsl, W, dtype, dtype, frac)
+
+
+@pytest.mark.parametrize("dtype,shape", [("bf16", (20000, 16)), ("bf16", (3000, 24)),
+                                         ("f32", (5000, 12)), ("f32", (999, 8200))])
+@pytest.mark.parametrize("frac", [0.05, 0.9])
+def test_topk_tiles_across_many_rows(hsl, dtype, shape, frac):
+    """Tiles that hold many short rows or start inside a row; at 0.9 a tile
+    keeps more entries than it gathers in shared memory (the rest go straight
+    to S)."""
+    W = synth.as_storage(synth.student_t_f32(*shape, seed=shape[1]), dtype)
+    assert_topk_parity(hsl, W, dtype, dtype, frac)
+
+
+def test_topk_bf16_sampled_bracket_exact(hsl):
+    """4M-element bf16 split: the threshold comes from the sampled bracket."""
+    W = synth.to_bf16_bits(synth.student_t_f32(2048, 2048, seed=21))
+    assert_topk_parity(hsl, W, "bf16", "bf16", 0.05)
+
+
+def _sampled_positions(count):
+    """Element indices the bf16 split samples (runs of 256 elements at a hashed
+    offset in every stratum of 16384), restated here only to build an input
+    whose sample misleads the bracket."""
+    def mix32(x):
+        x ^= x >> 16
+        x = (x * 0x7FEB352D) & 0xFFFFFFFF
+        x ^= x >> 15
+        x = (x * 0x846CA68B) & 0xFFFFFFFF
+        return x ^ (x >> 16)
+    idx = []
+    for c in range(count // 8 // 2048):
+        v0 = c * 2048 + mix32(c) % (2048 - 32 + 1)
+        idx.append(np.arange(v0 * 8, (v0 + 32) * 8))
+    return np.concatenate(idx)
+
+
+def test_topk_bf16_misleading_sample_falls_back(hsl):
+    """Every sampled element is large and nothing else is: the bracket cannot
+    hold the threshold, the full histogram pass runs, the split stays exact."""
+    m, n = 2048, 2048
+    W = synth.to_bf16_bits(synth.student_t_f32(m, n, seed=22) * np.float32(1e-3)).reshape(-1)
+    W[_sampled_positions(m * n)] = 0x4700  # 32768.0
+    assert_topk_parity(hsl, W.reshape(m, n), "bf16", "bf16", 0.05)
 
 
 def test_topk_unaligned_input_pointer(hsl):
