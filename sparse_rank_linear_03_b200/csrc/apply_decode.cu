@@ -6,10 +6,9 @@
 // §1: at batch 1 the cost is reading the weights, so both kernels below are
 // built to stream S, U and V from HBM once, with 16-byte vector loads.
 //
-//   k_lowrank_z   z = Vᵀ x.  Each CTA reduces a slab of V rows into fp32
-//                 partials; the last CTA to finish (ticket) sums the partials
-//                 in a fixed order, so z is deterministic.  It triggers the
-//                 dependent launch at its start.
+//   k_lowrank_z   z = Vᵀ x from V stored transposed: a warp per row of Vt,
+//                 16-byte loads, a fixed shuffle-tree sum (deterministic).
+//                 It triggers the dependent launch at its start.
 //   k_apply_csr   persistent CTAs over row ranges of equal bytes (all layers
 //   k_apply_nm24  of a group concatenated).  x is staged in shared memory as
 //                 [column][token]; S rows are streamed (CSR: G lanes per row;
@@ -45,7 +44,8 @@ struct ApplyArgs {
   int32_t count, slices;
   int32_t b0, bc;
   int32_t r_pad_max;
-  uint32_t* err;  // error word (bounded waits that gave up)
+  int32_t z_items;  // z work items (rows of Vt) over all layers
+  uint32_t* err;    // error word (bounded waits that gave up)
 };
 
 template <typename T>
@@ -76,82 +76,84 @@ template <typename T>
 __device__ __forceinline__ float ldx(const T* p) { return VT<T>::f(*p); }
 
 // ---- z = Vᵀ x ----------------------------------------------------------------
-template <typename T, int BCZ>
-__global__ void __launch_bounds__(kThreads) k_lowrank_z(ApplyArgs a) {
-  pdl_trigger();
-  extern __shared__ __align__(16) float red[];  // [rows per iter][BCZ][r_pad]
-  __shared__ int sh_last;
-  // layer of this CTA
-  int lo = 0, hi = a.count - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (a.probs[mid].z_cta0 <= int(blockIdx.x)) lo = mid; else hi = mid - 1;
-  }
-  const ApplyProblem& P = a.probs[lo];
-  const int local = int(blockIdx.x) - P.z_cta0;
-  const int n = P.n, rp = P.r_pad;
-  const int64_t j0 = int64_t(local) * n / P.z_ncta, j1 = int64_t(local + 1) * n / P.z_ncta;
-  const int LV = rp / 8;
-  const int RPI = kThreads / LV;
-  const int tr = threadIdx.x / LV, tc = threadIdx.x % LV;
-  const bool active = tr < RPI;
-  const T* x = x_of<T>(a, lo);
-  const T* V = static_cast<const T*>(P.V);
+// One work item per row c of a layer's Vt: a warp computes z[b][c] =
+// Σ_j Vt[c][j]·x[b][j] for the chunk's tokens with 16-byte loads, eight in
+// flight per lane, and a fixed shuffle tree (deterministic).  Small CTAs over
+// all SMs, so the kernel ends within a few microseconds and hardly disturbs the
+// apply kernel that starts beside it (programmatic dependent launch).
+constexpr int kZThreads = 128;
 
-  for (int bb = 0; bb < a.bc; bb += BCZ) {
-    float acc[BCZ][8];
+template <typename T, int BC>
+__global__ void __launch_bounds__(kZThreads) k_lowrank_z(ApplyArgs a) {
+  pdl_trigger();
+  const int lane = threadIdx.x & 31;
+  const int64_t nw = (int64_t(gridDim.x) * kZThreads) >> 5;
+  for (int64_t it = (int64_t(blockIdx.x) * kZThreads + threadIdx.x) >> 5; it < a.z_items; it += nw) {
+    int lo = 0, hi = a.count - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (a.probs[mid].z_item0 <= it) lo = mid; else hi = mid - 1;
+    }
+    const ApplyProblem& P = a.probs[lo];
+    const int c = int(it - P.z_item0), n = P.n;
+    const T* vrow = static_cast<const T*>(P.Vt) + int64_t(c) * n;
+    const T* x = x_of<T>(a, lo) + int64_t(a.b0) * n;
+    float acc[BC];
 #pragma unroll
-    for (int b = 0; b < BCZ; ++b)
+    for (int b = 0; b < BC; ++b) acc[b] = 0.f;
+    const bool vec = (int64_t(n) * int64_t(sizeof(T))) % 16 == 0 &&
+                     (reinterpret_cast<uintptr_t>(vrow) % 16) == 0 &&
+                     (reinterpret_cast<uintptr_t>(x) % 16) == 0;
+    int j = 0;
+    if (vec) {
+      constexpr int U = 8;  // vectors of 8 elements in flight per lane
+      for (; j + 32 * 8 * U <= n; j += 32 * 8 * U) {
+        float v[U][8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[b][e] = 0.f;
-    if (active) {
-#pragma unroll 4
-      for (int64_t j = j0 + tr; j < j1; j += RPI) {
-        float v[8];
-        load8<T>(V + j * rp + tc * 8, v);
+        for (int u = 0; u < U; ++u) load8<T>(vrow + j + (u * 32 + lane) * 8, v[u]);
 #pragma unroll
-        for (int b = 0; b < BCZ; ++b) {
-          const float xv = (bb + b < a.bc) ? ldx<T>(x + int64_t(a.b0 + bb + b) * n + j) : 0.f;
+        for (int b = 0; b < BC; ++b) {
+          if (b < a.bc) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) acc[b][e] = fmaf(v[e], xv, acc[b][e]);
+            for (int u = 0; u < U; ++u) {
+              float xv[8];
+              load8<T>(x + int64_t(b) * n + j + (u * 32 + lane) * 8, xv);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) acc[b] = fmaf(v[u][e], xv[e], acc[b]);
+            }
+          }
         }
       }
+      for (; j + 8 <= n; j += 32 * 8) {
+        const int jj = j + lane * 8;
+        if (jj + 8 <= n) {
+          float v[8];
+          load8<T>(vrow + jj, v);
 #pragma unroll
-      for (int b = 0; b < BCZ; ++b)
+          for (int b = 0; b < BC; ++b) {
+            if (b < a.bc) {
+              float xv[8];
+              load8<T>(x + int64_t(b) * n + jj, xv);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) red[(tr * BCZ + b) * rp + tc * 8 + e] = acc[b][e];
+              for (int e = 0; e < 8; ++e) acc[b] = fmaf(v[e], xv[e], acc[b]);
+            }
+          }
+        }
+      }
+      j = n - n % 8;
     }
-    __syncthreads();
-    for (int o = threadIdx.x; o < BCZ * rp; o += kThreads) {
-      const int b = o / rp, c = o % rp;
-      float s = 0.f;
-      for (int r = 0; r < RPI; ++r) s += red[(r * BCZ + b) * rp + c];
-      if (bb + b < a.bc) P.zpart[(int64_t(local) * 16 + bb + b) * rp + c] = s;
-    }
-    __syncthreads();
-  }
-  // the last CTA of this layer sums the partials in CTA order
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) sh_last = (atomicAdd(P.zcount, 1u) == unsigned(P.z_ncta - 1));
-  __syncthreads();
-  if (sh_last) {
-    __threadfence();
-    for (int o = threadIdx.x; o < a.bc * rp; o += kThreads) {
-      const int b = o / rp, c = o % rp;
-      const float* src = P.zpart + int64_t(b) * rp + c;
-      const int64_t step = int64_t(16) * rp;
-      // eight independent partial sums keep eight loads in flight; the final
-      // combination order is fixed, so z is deterministic
-      float s8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      int q = 0;
-      for (; q + 8 <= P.z_ncta; q += 8)
+    for (int jj = j + lane; jj < n; jj += 32) {
+      const float v = ldx<T>(vrow + jj);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) s8[u] += __ldcg(src + (q + u) * step);
-      for (; q < P.z_ncta; ++q) s8[q & 7] += __ldcg(src + q * step);
-      P.z[b * rp + c] = ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
+      for (int b = 0; b < BC; ++b)
+        if (b < a.bc) acc[b] = fmaf(v, ldx<T>(x + int64_t(b) * n + jj), acc[b]);
     }
-    if (threadIdx.x == 0) *P.zcount = 0u;
+#pragma unroll
+    for (int b = 0; b < BC; ++b) {
+#pragma unroll
+      for (int o = 16; o; o >>= 1) acc[b] += __shfl_xor_sync(0xffffffffu, acc[b], o);
+      if (lane == 0 && b < a.bc) P.z[b * P.r_pad + c] = acc[b];
+    }
   }
 }
 
@@ -678,16 +680,15 @@ size_t apply_smem(const ApplyPlan& plan) {
 template <typename T, int BC>
 hsl_status launch_chunk(ApplyPlan& plan, ApplyArgs a, int num_sms, cudaStream_t s) {
   // z = Vᵀ x, normal launch (waits for everything before it on the stream)
-  if (plan.z_grid > 0) {
-    constexpr int BCZ = BC < 8 ? BC : 8;
-    const size_t zsm = size_t(kThreads) * 8 * BCZ * 4;
-    auto zk = k_lowrank_z<T, BCZ>;
-    cudaFuncSetAttribute(zk, cudaFuncAttributeMaxDynamicSharedMemorySize, int(zsm));
+  if (plan.z_items > 0) {
+    auto zk = k_lowrank_z<T, BC>;
     // the apply CTAs start beside the z CTAs (programmatic dependent launch):
-    // an SM configured for z's small shared memory could not take one
+    // an SM configured for a small shared-memory carveout could not take one
     cudaFuncSetAttribute(zk, cudaFuncAttributePreferredSharedMemoryCarveout,
                          cudaSharedmemCarveoutMaxShared);
-    zk<<<plan.z_grid, kThreads, zsm, s>>>(a);
+    const int64_t zgrid = std::min<int64_t>((int64_t(plan.z_items) * 32 + kZThreads - 1) / kZThreads,
+                                            int64_t(num_sms) * 8);
+    zk<<<unsigned(zgrid), kZThreads, 0, s>>>(a);
     note_launch();
     if (hsl_status e = cuda_fail(cudaGetLastError(), "z launch")) return e;
   }
@@ -696,7 +697,7 @@ hsl_status launch_chunk(ApplyPlan& plan, ApplyArgs a, int num_sms, cudaStream_t 
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = plan.z_grid > 0 ? 1 : 0;
+  attr[0].val.programmaticStreamSerializationAllowed = plan.z_items > 0 ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   // every CTA stages the whole x of its layers: keep at least ~64 rows per CTA
@@ -771,6 +772,7 @@ hsl_status apply_decode_run(ApplyPlan& plan, const void* X, void* Y, const void*
   a.b0 = 0;
   a.bc = 0;
   a.r_pad_max = plan.r_pad_max;
+  a.z_items = plan.z_items;
   a.err = plan.err;
   if (plan.dtype == HSL_BF16) return run_typed<__nv_bfloat16>(plan, a, batch, num_sms, s);
   return run_typed<float>(plan, a, batch, num_sms, s);

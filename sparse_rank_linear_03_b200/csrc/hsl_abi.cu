@@ -104,9 +104,9 @@ hsl_status ensure_err_word(Handle& h, cudaStream_t s) {
 
 void free_all(Handle& h) {
   DevBuf* bufs[] = {&h.row_ptr, &h.col, &h.val, &h.nm_val, &h.nm_idx, &h.prow, &h.pcol,
-                    &h.pval, &h.pmeta, &h.pmeta_tc, &h.U, &h.V, &h.Vt, &h.zpart, &h.z, &h.zcount,
+                    &h.pval, &h.pmeta, &h.pmeta_tc, &h.U, &h.Vt, &h.z,
                     &h.err, &h.split_ws, &h.flags, &h.tiles, &h.xstage, &h.ystage, &h.zpre, &h.plan.probs,
-                    &h.plan.prob_row0, &h.plan.cta_rows, &h.plan.xy_ptrs};
+                    &h.plan.prob_row0, &h.plan.cta_rows, &h.plan.xy_ptrs, &h.plan.zsync};
   for (DevBuf* b : bufs) release(*b);
 }
 
@@ -408,7 +408,8 @@ hsl_status hsl_group_create(const hsl_handle* hs, int32_t count, hsl_group* out,
   std::vector<Handle*> hh(count);
   for (int i = 0; i < count; ++i) hh[i] = &hs[i]->h;
   if (hsl_status e = plan_build(g->plan, hh.data(), count, static_cast<cudaStream_t>(stream))) {
-    DevBuf* bufs[] = {&g->plan.probs, &g->plan.prob_row0, &g->plan.cta_rows, &g->plan.xy_ptrs};
+    DevBuf* bufs[] = {&g->plan.probs, &g->plan.prob_row0, &g->plan.cta_rows, &g->plan.xy_ptrs,
+                      &g->plan.zsync};
     for (DevBuf* b : bufs) release(*b);
     delete g;
     return e;
@@ -454,7 +455,8 @@ hsl_status hsl_group_destroy(hsl_group g) {
   {
     DeviceGuard dg(g->device);
     if (g->plan.probs.p) cudaDeviceSynchronize();
-    DevBuf* bufs[] = {&g->plan.probs, &g->plan.prob_row0, &g->plan.cta_rows, &g->plan.xy_ptrs};
+    DevBuf* bufs[] = {&g->plan.probs, &g->plan.prob_row0, &g->plan.cta_rows, &g->plan.xy_ptrs,
+                      &g->plan.zsync};
     for (DevBuf* b : bufs) release(*b);
     cudaGetLastError();
   }

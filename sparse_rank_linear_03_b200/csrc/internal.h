@@ -35,14 +35,12 @@ struct ApplyProblem {
   const void* pval;       // CSR: packed values; NM24: values [m][n/2]
   const uint16_t* pmeta;  // NM24: metadata, interleaved per lane (see pack.cu)
   const void* U;          // [m][r_pad]
-  const void* V;          // [n][r_pad]
-  float* zpart;           // [z_ncta][16][r_pad]
-  float* z;               // [16][r_pad]
-  unsigned* zcount;       // last-CTA ticket of the z reduction
+  const void* Vt;         // [r16][n]: V transposed, zero rows past r
+  float* z;               // [16][r_pad]: z = Vᵀx per token of the batch chunk
   int32_t m, n, r_pad;
   int32_t group;          // CSR: lanes per row (4..32)
   int32_t meta_stride;    // NM24: u16 metadata words per row
-  int32_t z_cta0, z_ncta; // this layer's CTAs in the z launch
+  int32_t z_item0;        // this layer's first z work item (one per row of Vt)
   int64_t row0;           // first row of this layer in the concatenated row space
 };
 
@@ -53,7 +51,7 @@ struct ApplyPlan {
   hsl_dtype dtype = HSL_F32;
   int32_t n_max = 0, r_pad_max = 0;
   int64_t rows_total = 0;
-  int z_grid = 0;       // CTAs of the z launch (0 when r == 0)
+  int z_items = 0;      // z work items over all layers (0 when r == 0)
   int slices = 0;       // equal-byte row ranges the apply grid divides among CTAs
   bool vec16 = false;   // every layer has n % 16 == 0 (16-byte aligned 2:4 rows)
   uint32_t* err = nullptr;  // error word the apply kernels report to (first member's)
@@ -61,6 +59,7 @@ struct ApplyPlan {
   DevBuf prob_row0;     // int64[count+1]
   DevBuf cta_rows;      // int64[apply_grid+1]
   DevBuf xy_ptrs;       // const void*[2*count] (group calls)
+  DevBuf zsync;         // two u64 counters: CTAs done with z, CTAs done with the call
   const void* const* last_x = nullptr;  // host cache of the uploaded pointers
   std::string host_xy;  // bytes of the last uploaded pointer table
 };
@@ -80,16 +79,15 @@ struct Handle {
   bool has_sparse = false;
 
   // packed layouts
-  DevBuf prow, pcol, pval, pmeta, pmeta_tc, U, V, Vt;
+  DevBuf prow, pcol, pval, pmeta, pmeta_tc, U, Vt;
   int32_t group = 8, meta_stride = 0;
   int64_t pack_cap = 0;
   bool packed = false;
 
   // workspace
-  DevBuf zpart, z, zcount, err, split_ws, flags;
+  DevBuf z, err, split_ws, flags;
   DevBuf tiles;  // per-tile counts of the sampled-bracket split
   DevBuf xstage, ystage, zpre;
-  int z_ncta = 0;
   ApplyPlan plan;  // the single-layer plan, built by hsl_pack
 };
 

@@ -141,14 +141,30 @@ __global__ void k_pad_cols(const SB* __restrict__ src, int64_t rows, int32_t r, 
   }
 }
 
-// Vt[c][j] = V[j][c] for c < r_pad, zero rows up to r16 (prefill B operand).
-__global__ void k_transpose_v(const uint16_t* __restrict__ V, int64_t n, int32_t r_pad, int32_t r16,
-                              uint16_t* __restrict__ Vt) {
-  const int64_t total = int64_t(r16) * n;
-  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
-       e += int64_t(gridDim.x) * blockDim.x) {
-    const int64_t c = e / n, j = e % n;
-    Vt[e] = c < r_pad ? V[j * r_pad + c] : uint16_t(0);
+// Vt[c][j] = V[j][c] for c < r, zero rows up to r16: V as given ([n][r],
+// row-major) transposed through 32×32 shared-memory tiles so both sides are
+// coalesced.  The decode z = Vᵀx reads whole rows of Vt, the prefill Z = X·V
+// takes it as its B operand.
+template <typename SB>
+__global__ void k_transpose_pad(const SB* __restrict__ V, int64_t n, int32_t r, int32_t r16,
+                                SB* __restrict__ Vt) {
+  __shared__ SB tile[32][33];
+  const int64_t tiles_j = (n + 31) / 32, tiles_c = (r16 + 31) / 32;
+  for (int64_t tt = blockIdx.x; tt < tiles_j * tiles_c; tt += gridDim.x) {
+    const int64_t j0 = (tt % tiles_j) * 32;
+    const int32_t c0 = int32_t(tt / tiles_j) * 32;
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {  // rows j of V, columns c
+      const int64_t j = j0 + i;
+      const int32_t c = c0 + int32_t(threadIdx.x);
+      tile[i][threadIdx.x] = (j < n && c < r) ? V[j * r + c] : SB(0);
+    }
+    __syncthreads();
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {  // rows c of Vt, columns j
+      const int32_t c = c0 + i;
+      const int64_t j = j0 + threadIdx.x;
+      if (c < r16 && j < n) Vt[int64_t(c) * n + j] = tile[threadIdx.x][i];
+    }
+    __syncthreads();
   }
 }
 
@@ -297,28 +313,23 @@ hsl_status pack_factors_run(Handle& h, const void* U, const void* V, cudaStream_
   const int eb = dtype_bytes(h.dtype);
   if (h.r == 0) return HSL_OK;
   if (hsl_status e = ensure(h.U, size_t(h.m) * h.r_pad * eb, "U copy")) return e;
-  if (hsl_status e = ensure(h.V, size_t(h.n) * h.r_pad * eb, "V copy")) return e;
-  for (int which = 0; which < 2; ++which) {
-    const int64_t rows = which ? h.n : h.m;
-    const void* src = which ? V : U;
-    void* dst = which ? h.V.p : h.U.p;
-    const int64_t grid = std::min<int64_t>((rows * h.r_pad + 255) / 256, int64_t(h.num_sms) * 16);
-    if (eb == 2)
-      k_pad_cols<uint16_t><<<unsigned(grid), 256, 0, s>>>(static_cast<const uint16_t*>(src), rows,
-                                                          h.r, h.r_pad, static_cast<uint16_t*>(dst));
-    else
-      k_pad_cols<uint32_t><<<unsigned(grid), 256, 0, s>>>(static_cast<const uint32_t*>(src), rows,
-                                                          h.r, h.r_pad, static_cast<uint32_t*>(dst));
-    note_launch();
+  const int32_t r16 = int32_t(round_up(h.r, 16));
+  if (hsl_status e = ensure(h.Vt, size_t(r16) * h.n * eb, "V transpose")) return e;
+  const int64_t grid = std::min<int64_t>((h.m * h.r_pad + 255) / 256, int64_t(h.num_sms) * 16);
+  const int64_t tgrid =
+      std::min<int64_t>(((h.n + 31) / 32) * ((r16 + 31) / 32), int64_t(h.num_sms) * 16);
+  if (eb == 2) {
+    k_pad_cols<uint16_t><<<unsigned(grid), 256, 0, s>>>(static_cast<const uint16_t*>(U), h.m, h.r,
+                                                        h.r_pad, static_cast<uint16_t*>(h.U.p));
+    k_transpose_pad<uint16_t><<<unsigned(tgrid), dim3(32, 8), 0, s>>>(
+        static_cast<const uint16_t*>(V), h.n, h.r, r16, static_cast<uint16_t*>(h.Vt.p));
+  } else {
+    k_pad_cols<uint32_t><<<unsigned(grid), 256, 0, s>>>(static_cast<const uint32_t*>(U), h.m, h.r,
+                                                        h.r_pad, static_cast<uint32_t*>(h.U.p));
+    k_transpose_pad<uint32_t><<<unsigned(tgrid), dim3(32, 8), 0, s>>>(
+        static_cast<const uint32_t*>(V), h.n, h.r, r16, static_cast<uint32_t*>(h.Vt.p));
   }
-  if (h.fmt == HSL_FMT_NM24 && h.dtype == HSL_BF16 && h.n % 64 == 0) {
-    const int32_t r16 = int32_t(round_up(h.r, 16));
-    if (hsl_status e = ensure(h.Vt, size_t(r16) * h.n * 2, "V transpose")) return e;
-    const int64_t grid = std::min<int64_t>((r16 * h.n + 255) / 256, int64_t(h.num_sms) * 16);
-    k_transpose_v<<<unsigned(grid), 256, 0, s>>>(static_cast<const uint16_t*>(h.V.p), h.n, h.r_pad,
-                                                 r16, static_cast<uint16_t*>(h.Vt.p));
-    note_launch();
-  }
+  note_launch(2);
   return cuda_fail(cudaGetLastError(), "factor pack launch");
 }
 
@@ -342,7 +353,7 @@ hsl_status plan_build(ApplyPlan& plan, Handle* const* hs, int count, cudaStream_
     P.pval = h.fmt == HSL_FMT_CSR ? h.pval.p : h.nm_val.p;
     P.pmeta = static_cast<const uint16_t*>(h.pmeta.p);
     P.U = h.U.p;
-    P.V = h.V.p;
+    P.Vt = h.Vt.p;
     P.m = int32_t(h.m);
     P.n = int32_t(h.n);
     P.r_pad = h.r_pad;
@@ -350,33 +361,22 @@ hsl_status plan_build(ApplyPlan& plan, Handle* const* hs, int count, cudaStream_
     P.meta_stride = h.meta_stride;
     P.row0 = row0;
     row0 += h.m;
-    // z: about 128 KB of V per CTA (at most 64 CTAs per layer), so the final
-    // reduction over the CTAs' partials stays short
-    int zn = 0;
-    if (h.r_pad > 0) {
-      const int64_t vbytes = h.n * int64_t(h.r_pad) * eb;
-      zn = int(std::min<int64_t>(std::max<int64_t>((vbytes + 131071) / 131072, 1),
-                                 std::min<int64_t>(h.n, 64)));
-      if (hsl_status e = ensure(h.zpart, size_t(zn) * 16 * h.r_pad * 4, "z partials")) return e;
+    // z = Vᵀx: one work item per row of Vt (a warp each, inside the apply kernel)
+    if (h.r_pad > 0)
       if (hsl_status e = ensure(h.z, size_t(16) * h.r_pad * 4, "z")) return e;
-      if (h.zcount.p == nullptr) {
-        if (hsl_status e = ensure(h.zcount, 256, "z ticket")) return e;
-        if (cudaError_t ce = cudaMemsetAsync(h.zcount.p, 0, 256, s)) return cuda_fail(ce, "memset");
-      }
-    }
-    h.z_ncta = zn;
-    P.zpart = static_cast<float*>(h.zpart.p);
     P.z = static_cast<float*>(h.z.p);
-    P.zcount = static_cast<unsigned*>(h.zcount.p);
-    P.z_cta0 = zc;
-    P.z_ncta = zn;
-    zc += zn;
+    P.z_item0 = zc;
+    zc += h.r_pad;
     plan.n_max = std::max(plan.n_max, int32_t(h.n));
     plan.vec16 = plan.vec16 && h.n % 16 == 0;
     plan.r_pad_max = std::max(plan.r_pad_max, h.r_pad);
   }
   plan.rows_total = row0;
-  plan.z_grid = zc;
+  plan.z_items = zc;
+  if (zc > 0 && plan.zsync.p == nullptr) {
+    if (hsl_status e = ensure(plan.zsync, 256, "z barrier")) return e;
+    if (cudaError_t ce = cudaMemsetAsync(plan.zsync.p, 0, 256, s)) return cuda_fail(ce, "memset");
+  }
   const int slices = hs[0]->num_sms * kSlicesPerSM;
   plan.slices = slices;
   if (hsl_status e = ensure(plan.probs, sizeof(ApplyProblem) * count, "plan")) return e;

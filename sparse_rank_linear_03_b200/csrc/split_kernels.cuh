@@ -149,6 +149,15 @@ __global__ void __launch_bounds__(1024) k_split_select(const unsigned* __restric
   }
 }
 
+// The eight flags at bits 15 / 31 of four words (element 2u / 2u + 1 of word
+// u) as an 8-bit mask in element order: one byte permute per word pair puts
+// the flags at the top bit of each byte, and a multiply by 2^0 + 2^7 + 2^14 +
+// 2^21 gathers the four byte-top bits into bits 28..31 (no two partial
+// products meet, so nothing carries).
+__device__ __forceinline__ uint32_t gather_flags8(const uint32_t (&f)[4]) {
+  const uint32_t lo = __byte_perm(f[0], f[1], 0x7531), hi = __byte_perm(f[2], f[3], 0x7531);
+  return ((lo * 0x00204081u) >> 28) | (((hi * 0x00204081u) >> 24) & 0xF0u);
+}
 // ---- bf16 threshold from a sampled bracket ------------------------------------
 // A sample of W (one run of kSampleRun vectors at a hashed offset in every
 // stratum of kSampleStride vectors) brackets the key of the k-th largest
@@ -314,11 +323,11 @@ __global__ void __launch_bounds__(1024) k_count_bracket(const uint16_t* __restri
       in4[u] = (kw - LO) & ~dh & H;
       any |= in4[u];
     }
-    if (any) {
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        if (in4[u] & 0x8000u) atomicAdd(&bins[(w4[u] & 0x7FFFu) - lo], 1u);
-        if (in4[u] & 0x80000000u) atomicAdd(&bins[((w4[u] >> 16) & 0x7FFFu) - lo], 1u);
+    if (any) {  // usually one element of the lane: walk the set bits
+      for (uint32_t mk = gather_flags8(in4); mk; mk &= mk - 1u) {
+        const int e = __ffs(mk) - 1;
+        const uint32_t w = (e & 4) ? ((e & 2) ? w4[3] : w4[2]) : ((e & 2) ? w4[1] : w4[0]);
+        atomicAdd(&bins[((w >> ((e & 1) * 16)) & 0x7FFFu) - lo], 1u);
       }
     }
   };
@@ -806,17 +815,16 @@ __device__ __forceinline__ void vec_masks<uint16_t>(const uint4& q, uint32_t T, 
   const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
   const uint32_t T0 = T <= 0x7FFFu ? T : 0x8000u;  // T above every key: nothing ≥ T
   const uint32_t TT = T0 * 0x00010001u, TT1 = (T0 + 1u) * 0x00010001u;
-  uint32_t ge = 0, gt = 0;
+  uint32_t a[4], b[4];
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
-    const uint32_t k = (w4[u] & 0x7FFF7FFFu) | 0x80008000u;
-    const uint32_t a = (k - TT) & 0x80008000u;
-    const uint32_t b = T0 >= 0x7FFFu ? 0u : ((k - TT1) & 0x80008000u);
-    ge |= (((a >> 15) | (a >> 30)) & 3u) << (2 * u);
-    gt |= (((b >> 15) | (b >> 30)) & 3u) << (2 * u);
+    const uint32_t k = w4[u] | 0x80008000u;
+    a[u] = (k - TT) & 0x80008000u;
+    b[u] = T0 >= 0x7FFFu ? 0u : ((k - TT1) & 0x80008000u);
   }
-  gm = gt;
-  em = ge & ~gt;
+  const uint32_t ge = gather_flags8(a);
+  gm = gather_flags8(b);
+  em = ge & ~gm;
 }
 template <>
 __device__ __forceinline__ void vec_masks<uint32_t>(const uint4& q, uint32_t T, uint32_t& gm,
@@ -865,12 +873,22 @@ __device__ __forceinline__ uint32_t fdiv(const FastDiv& f, uint32_t x) {
 
 template <typename KT>
 __device__ __forceinline__ void zero_kept(uint4& q, uint32_t sel);
+// bf16: element e's flag goes to the top bit of byte e & 3 of one word (a
+// multiply by 2^7 + 2^14 + 2^21 + 2^28, no carries), and a sign-replicating
+// byte permute widens each flag to the element's two bytes.
+__device__ __forceinline__ uint32_t prmt_sign(uint32_t a, uint32_t sel) {
+  uint32_t r;  // generic prmt: a selector nibble with its top bit set replicates the byte's sign
+  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(r) : "r"(a), "r"(sel));
+  return r;
+}
 template <>
 __device__ __forceinline__ void zero_kept<uint16_t>(uint4& q, uint32_t sel) {
-  uint32_t* w = &q.x;
-#pragma unroll
-  for (int u = 0; u < 4; ++u)
-    w[u] &= ~((((sel >> (2 * u)) & 1u) * 0x0000FFFFu) | (((sel >> (2 * u + 1)) & 1u) * 0xFFFF0000u));
+  const uint32_t f03 = ((sel & 0xFu) * 0x10204080u) & 0x80808080u;
+  const uint32_t f47 = (((sel >> 4) & 0xFu) * 0x10204080u) & 0x80808080u;
+  q.x &= ~prmt_sign(f03, 0x9988u);
+  q.y &= ~prmt_sign(f03, 0xBBAAu);
+  q.z &= ~prmt_sign(f47, 0x9988u);
+  q.w &= ~prmt_sign(f47, 0xBBAAu);
 }
 template <>
 __device__ __forceinline__ void zero_kept<uint32_t>(uint4& q, uint32_t sel) {
