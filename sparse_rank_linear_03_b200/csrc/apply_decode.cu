@@ -180,36 +180,47 @@ __device__ __forceinline__ void xcol(const T* xs, int c, float (&xv)[BC]) {
   for (int b = 0; b < BC; ++b) xv[b] = VT<T>::f(xs[c * BC + b]);
 }
 
-// y[row] = ysp[row] + U[row,:]·z for rows [s0, s1) of layer P.
+// y[row] = ysp[row] + U[row,:]·z for rows [s0, s1) of layer P.  GU lanes
+// share a row (8 elements each); a warp takes R row groups per pass and issues
+// all their U loads before using any, so the pass costs one load latency.
 template <typename T, int BC, int NT = kThreads>
 __device__ __forceinline__ void urows(const ApplyProblem& P, const float* zs, const float* ysp,
                                       int s0, int s1, T* y, int bc) {
+  constexpr int R = BC <= 2 ? 4 : 1;
   const int rp = P.r_pad;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int GU = 1;
   while (GU * 8 < rp) GU <<= 1;  // lanes per row, power of two ≤ 32
   const int rpw = 32 / GU;        // rows per warp pass
+  const int gl = lane % GU;
   const T* U = static_cast<const T*>(P.U);
-  for (int ib = s0 + warp * rpw; ib < s1; ib += (NT / 32) * rpw) {
-    const int i = ib + lane / GU, gl = lane % GU;
-    float acc[BC];
+  for (int ib = s0 + warp * rpw * R; ib < s1; ib += (NT / 32) * rpw * R) {
+    float u[R][8];
 #pragma unroll
-    for (int b = 0; b < BC; ++b) acc[b] = 0.f;
-    if (i < s1 && gl * 8 < rp) {
-      float u[8];
-      load8<T>(U + int64_t(i) * rp + gl * 8, u);
-#pragma unroll
-      for (int b = 0; b < BC; ++b)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[b] = fmaf(u[e], zs[b * rp + gl * 8 + e], acc[b]);
+    for (int q = 0; q < R; ++q) {
+      const int i = ib + q * rpw + lane / GU;
+      if (i < s1 && gl * 8 < rp) load8<T>(U + int64_t(i) * rp + gl * 8, u[q]);
     }
-    for (int o = GU >> 1; o; o >>= 1)
 #pragma unroll
-      for (int b = 0; b < BC; ++b) acc[b] += __shfl_xor_sync(0xffffffffu, acc[b], o);
-    if (gl == 0 && i < s1) {
+    for (int q = 0; q < R; ++q) {
+      const int i = ib + q * rpw + lane / GU;
+      float acc[BC];
 #pragma unroll
-      for (int b = 0; b < BC; ++b)
-        if (b < bc) y[int64_t(b) * P.m + i] = VT<T>::from_f(acc[b] + ysp[(i - s0) * BC + b]);
+      for (int b = 0; b < BC; ++b) acc[b] = 0.f;
+      if (i < s1 && gl * 8 < rp) {
+#pragma unroll
+        for (int b = 0; b < BC; ++b)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[b] = fmaf(u[q][e], zs[b * rp + gl * 8 + e], acc[b]);
+      }
+      for (int o = GU >> 1; o; o >>= 1)
+#pragma unroll
+        for (int b = 0; b < BC; ++b) acc[b] += __shfl_xor_sync(0xffffffffu, acc[b], o);
+      if (gl == 0 && i < s1) {
+#pragma unroll
+        for (int b = 0; b < BC; ++b)
+          if (b < bc) y[int64_t(b) * P.m + i] = VT<T>::from_f(acc[b] + ysp[(i - s0) * BC + b]);
+      }
     }
   }
 }
@@ -456,8 +467,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_apply_decode(ApplyArgs a) {
 // of its next unit lands in the other slot.  A warp takes units w, w+16, ...
 // of the layer's row range, so the prefetch runs across the 256-row segments
 // whose flush (sum of a row's super-chunk partials in a fixed order, then
-// U·z and the y stores) only needs barriers.  Arithmetic per chunk as in
-// nm24_rows_b1.
+// U·z and the y stores) only needs barriers.  Per chunk see chunk24.
 constexpr int kB1Threads = 512;
 constexpr int kB1Warps = kB1Threads / 32;
 constexpr int kSupChunks = 256;                  // chunks of a super-chunk
@@ -480,9 +490,42 @@ B1Layout b1_layout(int n_max, int r_pad_max) {
   return L;
 }
 
-__global__ void __launch_bounds__(kB1Threads, 1) k_apply_24_b1_tma(ApplyArgs a, B1Layout lay) {
+// One chunk of a 2:4 row: 8 kept bf16 values (v), the 16-element x window
+// (xl, xh) and the chunk's 16 metadata bits (low half of meta).  The byte
+// permute selector of group g, 0x1010 + 0x22·i0 + 0x2200·i1 for the kept
+// indices i0 < i1, is itself a byte permute of 0x76543210 by the selector
+// i0 | i1 << 4; the metadata nibbles i0 | i1 << 2 are spread into those bytes
+// with shifts and masks.  Products accumulate in fp32 (a bf16 × bf16 product
+// is exact in fp32; one rounding per fused multiply-add).
+__device__ __forceinline__ void fma2_bf16(float& a0, float& a1, uint32_t v, uint32_t x) {
+  asm("{\n\t.reg .b16 vl, vh, xl, xh;\n\t"
+      "mov.b32 {vl, vh}, %2;\n\t"
+      "mov.b32 {xl, xh}, %3;\n\t"
+      "fma.rn.f32.bf16 %0, vl, xl, %0;\n\t"
+      "fma.rn.f32.bf16 %1, vh, xh, %1;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "r"(v), "r"(x));
+}
+__device__ __forceinline__ void chunk24(const uint4& v, const uint4& xl, const uint4& xh,
+                                        uint32_t meta, float& a0, float& a1) {
+  uint32_t y = meta & 0xFFFFu;                  // nibble g at bits 4g..4g+3
+  y = (y | (y << 8)) & 0x00FF00FFu;
+  y = (y | (y << 4)) & 0x0F0F0F0Fu;             // nibble g in byte g
+  y = (y | (y << 2)) & 0x33333333u;             // byte g = i0 | i1 << 4
+  const uint32_t s0 = __byte_perm(0x76543210u, 0u, y);
+  const uint32_t s1 = __byte_perm(0x76543210u, 0u, y >> 8);
+  const uint32_t s2 = __byte_perm(0x76543210u, 0u, y >> 16);
+  const uint32_t s3 = __byte_perm(0x76543210u, 0u, y >> 24);
+  fma2_bf16(a0, a1, v.x, __byte_perm(xl.x, xl.y, s0));
+  fma2_bf16(a0, a1, v.y, __byte_perm(xl.z, xl.w, s1));
+  fma2_bf16(a0, a1, v.z, __byte_perm(xh.x, xh.y, s2));
+  fma2_bf16(a0, a1, v.w, __byte_perm(xh.z, xh.w, s3));
+}
+
+// At most 112 registers: 16 warps then leave room on the SM for a CTA of the
+// z kernel, which the apply CTA overlaps (programmatic dependent launch).
+__global__ void __maxnreg__(112) k_apply_24_b1_tma(ApplyArgs a, B1Layout lay) {
   extern __shared__ __align__(16) unsigned char smem[];
-  __shared__ uint32_t sel_lut[16];
   __shared__ int abort_flag;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   unsigned char* const slot0 = smem + (2 * warp) * kUnitSlot;
@@ -492,8 +535,6 @@ __global__ void __launch_bounds__(kB1Threads, 1) k_apply_24_b1_tma(ApplyArgs a, 
   uint64_t* bars = reinterpret_cast<uint64_t*>(
       (reinterpret_cast<uintptr_t>(zs + a.r_pad_max) + 7) & ~uintptr_t(7));
   uint64_t* const mybar = bars + 2 * warp;
-  if (threadIdx.x < 16)
-    sel_lut[threadIdx.x] = 0x1010u + (threadIdx.x & 3u) * 0x22u + (threadIdx.x >> 2) * 0x2200u;
   if (threadIdx.x == 0) {
     abort_flag = 0;
     for (int i = 0; i < 2 * kB1Warps; ++i) tc::mbar_init(&bars[i], 1);
@@ -572,6 +613,9 @@ __global__ void __launch_bounds__(kB1Threads, 1) k_apply_24_b1_tma(ApplyArgs a, 
     }
     __syncthreads();
     const uint4* xs4 = reinterpret_cast<const uint4*>(xs);
+    const int xsw = (lane >> 2) & 1;
+    const uint4* xwin_lo = xs4 + 2 * lane + xsw;
+    const uint4* xwin_hi = xs4 + 2 * lane + 1 - xsw;
     __nv_bfloat16* y = y_of<__nv_bfloat16>(a, p) + int64_t(a.b0) * P.m;
     for (int s0 = l0, seg = 0; s0 < l1; s0 += kSeg, ++seg) {
       const int s1 = min(s0 + kSeg, l1);
@@ -593,30 +637,24 @@ __global__ void __launch_bounds__(kB1Threads, 1) k_apply_24_b1_tma(ApplyArgs a, 
         unit_of(warp + kB1Warps * j, r, sp);
         float acc = 0.f;
         if (ok) {
-          const uint4* vs = reinterpret_cast<const uint4*>(slot0 + sl * kUnitSlot);
+          const uint4* vs = reinterpret_cast<const uint4*>(slot0 + sl * kUnitSlot) + lane;
           const uint4 mw = reinterpret_cast<const uint4*>(slot0 + sl * kUnitSlot + kUnitVBytes)[lane];
           const uint32_t mws[4] = {mw.x, mw.y, mw.z, mw.w};
           const int nch = min(kSupChunks, nq - sp * kSupChunks);
+          // chunk q = 256·sp + 32·t + lane: its x window is 16-byte units 2q, 2q + 1,
+          // stored at 2q + sw and 2q + 1 − sw with sw = (q >> 2) & 1 = (lane >> 2) & 1
+          const uint4* xlo = xwin_lo + sp * (2 * kSupChunks);
+          const uint4* xhi = xwin_hi + sp * (2 * kSupChunks);
           float a0 = 0.f, a1 = 0.f;
+          if (nch == kSupChunks) {
 #pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            const int ql = t * 32 + lane;
-            if (ql < nch) {
-              const int q = sp * kSupChunks + ql;
-              const uint4 v = vs[ql];
-              const int sw = (q >> 2) & 1;
-              const uint4 xl = xs4[(2 * q) ^ sw], xh = xs4[(2 * q + 1) ^ sw];
-              const uint32_t xw[8] = {xl.x, xl.y, xl.z, xl.w, xh.x, xh.y, xh.z, xh.w};
-              const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
-              const uint32_t meta = mws[t >> 1] >> ((t & 1) * 16);
+            for (int t = 0; t < 8; ++t)
+              chunk24(vs[32 * t], xlo[64 * t], xhi[64 * t], mws[t >> 1] >> ((t & 1) * 16), a0, a1);
+          } else {
 #pragma unroll
-              for (int g = 0; g < 4; ++g) {
-                const uint32_t xp =
-                    __byte_perm(xw[2 * g], xw[2 * g + 1], sel_lut[(meta >> (4 * g)) & 0xFu]);
-                a0 = fmaf(bf_lo(vw[g]), bf_lo(xp), a0);
-                a1 = fmaf(bf_hi(vw[g]), bf_hi(xp), a1);
-              }
-            }
+            for (int t = 0; t < 8; ++t)
+              if (t * 32 + lane < nch)
+                chunk24(vs[32 * t], xlo[64 * t], xhi[64 * t], mws[t >> 1] >> ((t & 1) * 16), a0, a1);
           }
           acc = a0 + a1;
         }

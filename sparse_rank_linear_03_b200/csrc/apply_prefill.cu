@@ -598,6 +598,262 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
+// ---- sparse tensor-core prefill on CTA pairs -------------------------------------
+// A cluster of two CTAs shares each MMA (cta_group::2, M = 256): CTA r of the
+// pair stages its own 128 rows of A and half of the X tile (B is split along
+// N), and its TMEM holds the accumulator rows of its A half.  Two such MMAs
+// (pair rows [0, 256) and [256, 512) of the tile) share every X tile, so a
+// pair tile is 512 rows of W × 192 tokens and each SM loads, per K-block,
+// 256 rows of A and 96 tokens of X: ~1.5× the MMA work per byte of the
+// single-CTA 256 × 192 tile, with deeper loads in flight.
+//   Per K-block both CTAs' loads count on the even CTA's `full` barrier; the
+// even CTA's MMA thread waits on it and on `mready` (the 2:4 metadata of both
+// CTAs is in TMEM), issues the MMAs and commits to `empty` in both CTAs.  The
+// metadata warps load their 2 KB of metadata per K-block straight from global
+// memory, ahead of the MMAs, into one of NSLOT slot sets; a slot set is
+// reused once the MMA NSLOT K-blocks back has completed (`empty`).
+constexpr int P2_BN = 192, P2_BNH = P2_BN / 2;  // tokens of a pair tile / staged per CTA
+constexpr int P2_STAGES = 8, P2_NSLOT = 8;
+constexpr int P2_A_HALF = 128 * 64;             // 128 rows × 64 bytes
+constexpr int P2_A = 2 * P2_A_HALF;             // 16 KB: this CTA's rows of both MMAs
+constexpr int P2_B = P2_BNH * 128;              // 12 KB: X, 96 tokens × 64 bf16
+constexpr int P2_B_Z = P2_BNH * 64;             // Z hi / lo: 96 tokens × 32 bf16
+constexpr int P2_STAGE = P2_A + P2_B;
+constexpr int P2_SMEM = P2_STAGES * P2_STAGE + 1024 + 256;
+// TMEM: accumulators [0, 192) and [256, 448); metadata slots of 4 columns,
+// k = 4·set + 2·h + i: 16 in [192, 256), 16 in [448, 512).
+constexpr uint32_t P2_ACC1_COL = 256;
+__device__ __forceinline__ uint32_t p2_meta_col(int set, int h, int i) {
+  const uint32_t k = uint32_t(set * 4 + h * 2 + i);
+  return k < 16 ? 192u + 4u * k : 448u + 4u * (k - 16u);
+}
+static_assert(P2_NSLOT * 4 == 32, "metadata slots");
+static_assert(P2_STAGE % 1024 == 0 && P2_A % 1024 == 0, "tile alignment");
+
+// Barrier 1 over the four metadata warps (128 threads), returning the OR of
+// `v` over them, so that they take every branch together.
+__device__ __forceinline__ int meta_bar_or(int v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.red.or.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(uint32_t(v))
+      : "memory");
+  return int(r);
+}
+
+struct PairMaps {
+  CUtensorMap x;    // X [T][n]         box {64, 96} SW128
+  CUtensorMap sv;   // S values [m][n/2] box {32, 128} SW64
+  CUtensorMap u;    // U [m][r_pad]     box {32, 128} SW64
+  CUtensorMap z;    // Z hi [T][r16]    box {32, 96} SW64
+  CUtensorMap zlo;  // Z lo [T][r16]    box {32, 96} SW64
+};
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+    k_prefill_24sp2(const __grid_constant__ PairMaps maps, const uint2* __restrict__ meta,
+                    __nv_bfloat16* __restrict__ Y, int m, int n, int T, int r16, uint32_t* err) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + P2_STAGES * P2_STAGE);
+  uint64_t* empty = full + P2_STAGES;
+  uint64_t* mready = empty + P2_STAGES;
+  uint64_t* accf = mready + P2_NSLOT;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = tc::cluster_rank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1;
+  const int ntn = (T + P2_BN - 1) / P2_BN;
+  const int mt = pair / ntn, nt = pair % ntn;
+  const int i0 = mt * 512, t0 = nt * P2_BN;
+  const int nkS = n / 64;
+  const int nkL = (r16 + 31) / 32;
+  const int nk = nkS + nkL;
+  const int mtiles128 = (m + 127) / 128;
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int s = 0; s < P2_STAGES; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    for (int j = 0; j < P2_NSLOT; ++j) tc::mbar_init(&mready[j], 2);  // one arrival per CTA
+    tc::mbar_init(accf, 1);
+    tc::fence_mbar_init();
+    tc::prefetch_tmap(&maps.x);
+    tc::prefetch_tmap(&maps.sv);
+    if (r16 > 0) {
+      tc::prefetch_tmap(&maps.u);
+      tc::prefetch_tmap(&maps.z);
+      tc::prefetch_tmap(&maps.zlo);
+    }
+  }
+  if (warp == 1) {
+    tc::tmem_alloc2(tmem_slot, 512);
+    tc::tmem_relinquish2();
+  }
+  tc::tc_fence_before();
+  tc::cluster_sync();  // both CTAs' barriers and TMEM are ready
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  volatile int* abrt = &abort_flag;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t keep = tc::make_policy_evict_last();
+      const uint64_t stream = tc::make_policy_evict_first();
+      const int rowA0 = i0 + 128 * int(rank), rowA1 = rowA0 + 256;
+      const int tB = t0 + P2_BNH * int(rank);
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % P2_STAGES;
+        const uint32_t ph = (kb / P2_STAGES) & 1;
+        if (!wait_or_abort(&empty[s], ph ^ 1, err, abrt)) break;
+        unsigned char* a = smem + s * P2_STAGE;
+        unsigned char* b = a + P2_A;
+        if (kb < nkS) {
+          if (leader) tc::mbar_expect_tx(&full[s], 2 * (P2_A + P2_B));
+          tc::tma_load_2d_pair(a, &maps.sv, kb * 32, rowA0, &full[s], stream);
+          tc::tma_load_2d_pair(a + P2_A_HALF, &maps.sv, kb * 32, rowA1, &full[s], stream);
+          tc::tma_load_2d_pair(b, &maps.x, kb * 64, tB, &full[s], keep);
+        } else {
+          if (kb == nkS) pdl_wait();  // Z is written by the preceding kernel
+          const int kl = kb - nkS;
+          if (leader) tc::mbar_expect_tx(&full[s], 2 * (P2_A + 2 * P2_B_Z));
+          tc::tma_load_2d_pair(a, &maps.u, kl * 32, rowA0, &full[s], stream);
+          tc::tma_load_2d_pair(a + P2_A_HALF, &maps.u, kl * 32, rowA1, &full[s], stream);
+          tc::tma_load_2d_pair(b, &maps.z, kl * 32, tB, &full[s], keep);
+          tc::tma_load_2d_pair(b + P2_B_Z, &maps.zlo, kl * 32, tB, &full[s], keep);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      const uint32_t idesc_sp = tc::idesc_bf16(256, P2_BN) | (1u << 2);
+      const uint32_t idesc_d = tc::idesc_bf16(256, P2_BN);
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % P2_STAGES;
+        const uint32_t ph = (kb / P2_STAGES) & 1;
+        if (!wait_or_abort(&full[s], ph, err, abrt)) break;
+        const int set = kb % P2_NSLOT;
+        if (kb < nkS && !wait_or_abort(&mready[set], (kb / P2_NSLOT) & 1, err, abrt)) break;
+        tc::tc_fence_after();
+        const unsigned char* a = smem + s * P2_STAGE;
+        const unsigned char* b = a + P2_A;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t d = tmem + (h ? P2_ACC1_COL : 0u);
+          const uint64_t ad = tc::desc_sw64(a + h * P2_A_HALF);
+          if (kb < nkS) {
+            const uint64_t bd = tc::desc_sw128(b);
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+              tc::mma_bf16_sp_pair(d, tc::desc_advance(ad, 32 * i), tc::desc_advance(bd, 64 * i),
+                                   tmem + p2_meta_col(set, h, i), idesc_sp,
+                                   (kb > 0 || i > 0) ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {  // Z hi, then Z lo
+              const uint64_t bd = tc::desc_sw64(b + part * P2_B_Z);
+#pragma unroll
+              for (int i = 0; i < 2; ++i)
+                tc::mma_bf16_pair(d, tc::desc_advance(ad, 32 * i), tc::desc_advance(bd, 32 * i),
+                                  idesc_d, 1u);
+            }
+          }
+        }
+        tc::mma_commit_pair(&empty[s]);
+      }
+      tc::mma_commit_pair(accf);
+    }
+  } else {
+    // warps 2..5: metadata into TMEM ahead of the MMAs, then the epilogue
+    const int L = ((warp & 3) << 5) | lane;
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    const uint32_t mready0 = tc::mapa(tc::smem_u32(&mready[0]), 0);
+    const int mtA = i0 / 128 + int(rank);  // 128-row tiles of this CTA: mtA, mtA + 2
+    auto load_meta = [&](int kb, int h) {
+      const int mt128 = mtA + 2 * h;
+      uint2 w = make_uint2(0x44444444u, 0x44444444u);  // rows past m: valid pattern, zero values
+      if (kb < nkS && mt128 < mtiles128) w = __ldg(meta + (int64_t(mt128) * nkS + kb) * 128 + L);
+      return w;
+    };
+    constexpr int D = 4;  // K-blocks of metadata loaded ahead
+    uint2 ring[D][2];
+#pragma unroll
+    for (int d = 0; d < D; ++d) {
+      ring[d][0] = load_meta(d, 0);
+      ring[d][1] = load_meta(d, 1);
+    }
+    bool ok = true;
+    for (int kb0 = 0; kb0 < nkS && ok; kb0 += D) {
+#pragma unroll
+      for (int d = 0; d < D; ++d) {
+        const int kb = kb0 + d;
+        if (kb >= nkS || !ok) break;
+        const int set = kb % P2_NSLOT;
+        // the MMA that last used this slot set has completed (one thread
+        // waits; the four warps decide together whether to go on)
+        int fail = 0;
+        if (kb >= P2_NSLOT && L == 0) {
+          const int kp = kb - P2_NSLOT;
+          fail = !wait_or_abort(&empty[kp % P2_STAGES], (kp / P2_STAGES) & 1, err, abrt);
+        }
+        if (meta_bar_or(fail)) {
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          tc::tmem_st1(tmem + lane_base + p2_meta_col(set, h, 0), ring[d][h].x);
+          tc::tmem_st1(tmem + lane_base + p2_meta_col(set, h, 1), ring[d][h].y);
+        }
+        tc::tmem_st_wait();
+        tc::tc_fence_before();
+        // the four warps' stores are done: one arrival per CTA (cluster-scope
+        // release), not one per thread
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (L == 0) tc::mbar_arrive_cluster(mready0 + uint32_t(set) * 8u);
+        ring[d][0] = load_meta(kb + D, 0);
+        ring[d][1] = load_meta(kb + D, 1);
+      }
+    }
+    if (tc::mbar_wait(accf, 0, err) && !*abrt) {
+      tc::tc_fence_after();
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        const int i = i0 + 256 * h + 128 * int(rank) + L;
+#pragma unroll 1
+        for (int c0 = 0; c0 < P2_BN; c0 += 32) {
+          float v[32];
+          tc::tmem_ld32(tmem + lane_base + (h ? P2_ACC1_COL : 0u) + c0, v);
+          if (i < m) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int t = t0 + c0 + j;
+              if (t < T) __stcs(Y + int64_t(t) * m + i, __float2bfloat16_rn(v[j]));
+            }
+          }
+        }
+      }
+    } else {
+      *abrt = 1;
+    }
+  }
+  tc::tc_fence_before();
+  tc::cluster_sync();  // the pair is done with its TMEM and barriers
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc2(tmem, 512);
+  }
+}
+
 // ---- host: tensor maps through the driver entry point (no libcuda link) -----
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -637,7 +893,18 @@ bool make_map(CUtensorMap* map, CUtensorMapDataType dt, int esize, const void* b
 
 }  // namespace
 
-// Z workspace and Vt come from the handle (Vt built by prefill_pack_run).
+// Z workspace and Vt come from the handle (Vt built when the factors are packed).
+// Pair tiles hold 192 tokens: below a few tiles of tokens the single-CTA
+// kernel wastes less of its tile.
+constexpr int64_t kPairMinTokens = 512;
+// HSL_PREFILL_PAIRS=1 selects the CTA-pair kernel.  It is exact (the parity
+// tests cover it) but measured slower than the single-CTA kernel on the 70B
+// layer (3.2 ms against 1.66 ms for 4096 tokens), so it is not the default.
+bool prefill_pairs_enabled() {
+  const char* e = std::getenv("HSL_PREFILL_PAIRS");
+  return e != nullptr && e[0] == '1';
+}
+
 bool prefill_supported(const Handle& h, const void* X) {
   return h.fmt == HSL_FMT_NM24 && h.dtype == HSL_BF16 && h.n % 64 == 0 &&
          (reinterpret_cast<uintptr_t>(X) % 16) == 0 && encode_fn() != nullptr;
@@ -679,6 +946,44 @@ hsl_status apply_prefill_run(Handle& h, const void* X, void* Y, int64_t T, cudaS
           zm, static_cast<__nv_bfloat16*>(h.zpre.p), int(n), int(T), r16, err0);
       note_launch();
       if (hsl_status e = cuda_fail(cudaGetLastError(), "prefill z launch")) return e;
+    }
+    if (prefill_pairs_enabled() && T >= kPairMinTokens) {
+      // CTA pairs: 512 rows × 192 tokens per pair
+      PairMaps pm;
+      memset(&pm, 0, sizeof(pm));
+      bool okp = make_map(&pm.x, BFs, 2, X, T, n, n, 64, P2_BNH, CU_TENSOR_MAP_SWIZZLE_128B) &&
+                 make_map(&pm.sv, BFs, 2, h.nm_val.p, m, n / 2, n / 2, 32, 128,
+                          CU_TENSOR_MAP_SWIZZLE_64B);
+      if (okp && r16 > 0)
+        okp = make_map(&pm.u, BFs, 2, h.U.p, m, h.r_pad, h.r_pad, 32, 128,
+                       CU_TENSOR_MAP_SWIZZLE_64B) &&
+              make_map(&pm.z, BFs, 2, h.zpre.p, T, r16, r16, 32, P2_BNH, CU_TENSOR_MAP_SWIZZLE_64B) &&
+              make_map(&pm.zlo, BFs, 2, static_cast<__nv_bfloat16*>(h.zpre.p) + T * r16, T, r16,
+                       r16, 32, P2_BNH, CU_TENSOR_MAP_SWIZZLE_64B);
+      if (!okp) {
+        set_message("tensor map encoding failed");
+        return HSL_ERR_CUDA;
+      }
+      if (cudaError_t e = cudaFuncSetAttribute(k_prefill_24sp2,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, P2_SMEM))
+        return cuda_fail(e, "prefill smem attribute");
+      const int64_t pairs = ((m + 511) / 512) * ((T + P2_BN - 1) / P2_BN);
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(unsigned(2 * pairs));
+      cfg.blockDim = dim3(192);
+      cfg.dynamicSmemBytes = P2_SMEM;
+      cfg.stream = s;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].val.programmaticStreamSerializationAllowed = r16 > 0 ? 1 : 0;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      note_launch();
+      return cuda_fail(cudaLaunchKernelEx(&cfg, k_prefill_24sp2, pm,
+                                          static_cast<const uint2*>(h.pmeta_tc.p),
+                                          static_cast<__nv_bfloat16*>(Y), int(m), int(n), int(T),
+                                          r16, err0),
+                       "pair prefill launch");
     }
     if (cudaError_t e = cudaFuncSetAttribute(k_prefill_24sp,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, SP_SMEM))

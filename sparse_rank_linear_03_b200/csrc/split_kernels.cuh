@@ -22,7 +22,6 @@ constexpr int kTileThreads = 256;
 constexpr int kTileBytes = 32768;
 constexpr int kStages = 3;
 constexpr int kTileVPT = kTileBytes / 16 / kTileThreads;  // vectors per thread
-constexpr int kStageOutBytes = 12288;                     // gathered (col, val) of a tile
 
 template <typename KT> struct KeyTraits;
 template <> struct KeyTraits<uint16_t> {
@@ -579,6 +578,38 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* sh_war
   return r;
 }
 
+// Block-wide exclusive scan with two barriers: the warp totals go to one of
+// two buffers (alternate calls use the other), so no third barrier is needed
+// before the buffer is written again.
+__device__ __forceinline__ uint32_t block_excl_scan2(uint32_t v, uint32_t (*sh)[kEmitThreads / 32 + 1],
+                                                     int parity, uint32_t& total) {
+  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+  uint32_t* sw = sh[parity];
+  uint32_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t u = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += u;
+  }
+  if (lane == 31) sw[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    const int nw = kEmitThreads / 32;
+    uint32_t x = lane < nw ? sw[lane] : 0u;
+    uint32_t xi = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t u = __shfl_up_sync(0xffffffffu, xi, o);
+      if (lane >= o) xi += u;
+    }
+    if (lane < nw) sw[lane] = xi - x;
+    if (lane == nw - 1) sw[nw] = xi;
+  }
+  __syncthreads();
+  total = sw[kEmitThreads / 32];
+  return sw[w] + incl - v;
+}
+
 template <typename KT, typename SB>
 __global__ void __launch_bounds__(kEmitThreads) k_split_emit(
     const KT* __restrict__ W, int64_t m, int64_t n, const SelState* __restrict__ st,
@@ -846,8 +877,11 @@ __device__ __forceinline__ void vec_masks<uint32_t>(const uint4& q, uint32_t T, 
 // back with a bulk store from the same buffer.  Thread t owns the vectors
 // [8t, 8t + 8) of its tile and visits them starting at slot t & 7, so at every
 // step the eight threads of a quarter-warp read eight different bank groups.
-// The kept entries of a tile (a contiguous range of S) are gathered in shared
-// memory and written out with coalesced stores.
+// The kept entries of a tile form a contiguous range of S; after one barrier
+// every thread produces outputs i, i + 256, ... of that range (binary search
+// for the owning thread, then its (i − first)-th kept element), so S is
+// written with coalesced stores and the kept elements are zeroed in the staged
+// tile, which the bulk store writes back as the residual.
 
 // Unsigned 32-bit division by an invariant divisor d (1 ≤ d < 2^31): with
 // l = ceil(log2 d) and mult = floor(2^32·(2^l − d)/d) + 1,
@@ -871,37 +905,26 @@ __device__ __forceinline__ uint32_t fdiv(const FastDiv& f, uint32_t x) {
   return (t + ((x - t) >> f.s1)) >> f.s2;
 }
 
-template <typename KT>
-__device__ __forceinline__ void zero_kept(uint4& q, uint32_t sel);
-// bf16: element e's flag goes to the top bit of byte e & 3 of one word (a
-// multiply by 2^7 + 2^14 + 2^21 + 2^28, no carries), and a sign-replicating
-// byte permute widens each flag to the element's two bytes.
-__device__ __forceinline__ uint32_t prmt_sign(uint32_t a, uint32_t sel) {
-  uint32_t r;  // generic prmt: a selector nibble with its top bit set replicates the byte's sign
-  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(r) : "r"(a), "r"(sel));
-  return r;
-}
-template <>
-__device__ __forceinline__ void zero_kept<uint16_t>(uint4& q, uint32_t sel) {
-  const uint32_t f03 = ((sel & 0xFu) * 0x10204080u) & 0x80808080u;
-  const uint32_t f47 = (((sel >> 4) & 0xFu) * 0x10204080u) & 0x80808080u;
-  q.x &= ~prmt_sign(f03, 0x9988u);
-  q.y &= ~prmt_sign(f03, 0xBBAAu);
-  q.z &= ~prmt_sign(f47, 0x9988u);
-  q.w &= ~prmt_sign(f47, 0xBBAAu);
-}
-template <>
-__device__ __forceinline__ void zero_kept<uint32_t>(uint4& q, uint32_t sel) {
-  uint32_t* w = &q.x;
+// Index of the j-th set bit (j counted from 0) of m; m has more than j set bits.
+__device__ __forceinline__ int nth_set_bit64(unsigned long long m, uint32_t j) {
+  uint32_t w = uint32_t(m);
+  int base = 0;
+  uint32_t c = uint32_t(__popc(w));
+  if (j >= c) {
+    j -= c;
+    w = uint32_t(m >> 32);
+    base = 32;
+  }
 #pragma unroll
-  for (int u = 0; u < 4; ++u) w[u] = ((sel >> u) & 1u) ? 0u : w[u];
-}
-
-template <typename KT>
-__device__ __forceinline__ uint32_t vec_elem(const uint4& q, int e) {
-  const uint32_t w0 = (e & (sizeof(KT) == 2 ? 4 : 2)) ? ((e & (sizeof(KT) == 2 ? 2 : 1)) ? q.w : q.z)
-                                                      : ((e & (sizeof(KT) == 2 ? 2 : 1)) ? q.y : q.x);
-  return sizeof(KT) == 2 ? ((w0 >> ((e & 1) * 16)) & 0xFFFFu) : w0;
+  for (int half = 16; half; half >>= 1) {
+    c = uint32_t(__popc(w & ((1u << half) - 1u)));
+    if (j >= c) {
+      j -= c;
+      w >>= half;
+      base += half;
+    }
+  }
+  return base;
 }
 
 template <typename KT, typename SB>
@@ -914,14 +937,13 @@ __global__ void __launch_bounds__(kTileThreads, 2) k_split_emit_tile(
     const unsigned long long* __restrict__ tile_pre) {
   constexpr int EPV = 16 / sizeof(KT);
   constexpr int TE = kTileBytes / sizeof(KT);
-  constexpr int CAP = kStageOutBytes / (4 + sizeof(SB));
   extern __shared__ __align__(16) unsigned char smem[];
   uint4* tiles = reinterpret_cast<uint4*>(smem);
-  int32_t* o_col = reinterpret_cast<int32_t*>(smem + kStages * kTileBytes);
-  SB* o_val = reinterpret_cast<SB*>(o_col + CAP);
+  __shared__ unsigned long long s_keep[kTileThreads];  // kept elements of each thread
+  __shared__ uint32_t s_q[kTileThreads + 1];           // first tile-local S position of each thread
   __shared__ uint64_t bar[kStages];
   __shared__ int64_t s_tile[kStages];
-  __shared__ uint32_t sh_warp[kTileThreads / 32 + 1];
+  __shared__ uint32_t sh_warp[2][kTileThreads / 32 + 1];
   __shared__ uint32_t sh_ex[2];
   __shared__ int s_abort;
   __shared__ uint32_t s_late;  // stages whose wait gave up (bit sg) and its parity (bit 8 + sg)
@@ -983,30 +1005,35 @@ __global__ void __launch_bounds__(kTileThreads, 2) k_split_emit_tile(
       if (s < r0) lo += cnt[kk];
     }
     uint32_t total;
-    const uint32_t ex = block_excl_scan(tot, sh_warp, total);
+    const uint32_t ex = block_excl_scan2(tot, sh_warp, it & 1, total);
+    uint32_t tg, te;  // counts of keys > T and == T in the tiles before this one
     if (pre) {
-      if (t == 0) {
-        const unsigned long long p = tile_pre[tile];
-        sh_ex[0] = uint32_t(p >> 32);
-        sh_ex[1] = uint32_t(p);
+      const unsigned long long p = tile_pre[tile];
+      tg = uint32_t(p >> 32);
+      te = uint32_t(p);
+    } else {
+      if (t < 32) {
+        uint32_t xg, xe;
+        lookback(flags, tile, total >> 16, total & 0xFFFFu, err, xg, xe);
+        if (t == 0) {
+          sh_ex[0] = xg;
+          sh_ex[1] = xe;
+        }
       }
-    } else if (t < 32) {
-      uint32_t xg, xe;
-      lookback(flags, tile, total >> 16, total & 0xFFFFu, err, xg, xe);
-      if (t == 0) {
-        sh_ex[0] = xg;
-        sh_ex[1] = xe;
-      }
+      __syncthreads();
+      tg = sh_ex[0];
+      te = sh_ex[1];
     }
-    __syncthreads();
-    const uint32_t tg = sh_ex[0], te = sh_ex[1];
     const uint32_t P0 = tg + min(need, te);  // first S position of this tile
     const uint32_t ex_gt = tg + (ex >> 16), ex_eq = te + (ex & 0xFFFFu);
     // the tile's columns: x = c0 + offset, row = row0 + x / n
     const int64_t row0 = e0 / n;
     const uint32_t c0 = uint32_t(e0 - row0 * n);
 
-    // phase 2: positions, gathered S entries, residual in place
+    // phase 2: kept-element masks (thread-contiguous, bit e = the thread's
+    // element e in linear order), row starts, and each thread's first
+    // tile-local S position
+    uint64_t keep = 0;
     uint32_t run = lo;
 #pragma unroll
     for (int kk = 0; kk < kTileVPT; ++kk) {
@@ -1016,11 +1043,9 @@ __global__ void __launch_bounds__(kTileThreads, 2) k_split_emit_tile(
       if (v < nv) {
         const uint32_t gm = msk[kk] & 0xFFu, em = msk[kk] >> 8;
         const uint32_t cg = ex_gt + (run >> 16), ce = ex_eq + (run & 0xFFFFu);
-        const uint32_t pos0 = cg + min(need, ce);
         const uint32_t x = c0 + uint32_t(v) * EPV;
         const uint32_t q = fdiv(nd, x);
-        const uint32_t j0 = x - q * uint32_t(n);
-        if (j0 == 0) row_ptr[row0 + q] = int32_t(pos0);
+        if (x == q * uint32_t(n)) row_ptr[row0 + q] = int32_t(cg + min(need, ce));
         // ties kept in this vector: the first `allow` set bits of em
         uint32_t keq = 0;
         if (need > ce && em) {
@@ -1030,29 +1055,36 @@ __global__ void __launch_bounds__(kTileThreads, 2) k_split_emit_tile(
             rest &= rest - 1u;
           }
         }
-        const uint32_t sel = gm | keq;
-        if (sel) {
-          uint4 qv = tv[v];
-          uint32_t p = pos0;
-          for (uint32_t s2 = sel; s2; s2 &= s2 - 1u, ++p) {
-            const int e = __ffs(s2) - 1;
-            const uint32_t bits = vec_elem<KT>(qv, e);
-            const uint32_t loc = p - P0;
-            if (loc < uint32_t(CAP)) {
-              o_col[loc] = int32_t(j0 + e);
-              o_val[loc] = conv_val<SB>(bits, sizeof(KT));
-            } else if (p < k) {
-              col[p] = int32_t(j0 + e);
-              val[p] = conv_val<SB>(bits, sizeof(KT));
-            }
-          }
-          if (R) {
-            zero_kept<KT>(qv, sel);
-            tv[v] = qv;
-          }
-        }
+        keep |= uint64_t(gm | keq) << (s * EPV);
       }
       run += cnt[kk];
+    }
+    const uint32_t kept = (total >> 16) + min(need, te + (total & 0xFFFFu)) - min(need, te);
+    s_keep[t] = keep;
+    s_q[t] = ex_gt + min(need, ex_eq) - P0;
+    if (t == 0) s_q[kTileThreads] = kept;
+    __syncthreads();
+
+    // phase 3: the tile's S entries in order, output i by thread i mod 256
+    // (coalesced stores): find the owning thread u by binary search over the
+    // first positions, then the (i − q_u)-th kept element of u; the element
+    // is zeroed in the staged tile, which becomes the residual
+    KT* te_ = reinterpret_cast<KT*>(tv);
+    for (uint32_t i = t; i < kept; i += kTileThreads) {
+      int u = 0;
+#pragma unroll
+      for (int step = kTileThreads / 2; step; step >>= 1)
+        if (s_q[u + step] <= i) u += step;
+      const int e = nth_set_bit64(s_keep[u], i - s_q[u]);
+      const int idx = u * (kTileVPT * EPV) + e;
+      const uint32_t bits = uint32_t(te_[idx]);
+      const uint32_t x = c0 + uint32_t(idx);
+      const uint32_t p = P0 + i;
+      if (p < k) {
+        col[p] = int32_t(x - fdiv(nd, x) * uint32_t(n));
+        val[p] = conv_val<SB>(bits, sizeof(KT));
+      }
+      if (R) te_[idx] = KT(0);
     }
     if (R) tc::fence_async_smem();
     __syncthreads();
@@ -1063,22 +1095,14 @@ __global__ void __launch_bounds__(kTileThreads, 2) k_split_emit_tile(
       }
       if (tile == ntiles - 1) row_ptr[m] = int32_t(k);
     }
-    // the tile's S entries, gathered above, in coalesced stores
-    const uint32_t kept = (total >> 16) + min(need, te + (total & 0xFFFFu)) - min(need, te);
-    const uint32_t nout = min(kept, uint32_t(CAP));
-    for (uint32_t i = t; i < nout; i += kTileThreads) {
-      if (P0 + i < k) {
-        col[P0 + i] = o_col[i];
-        val[P0 + i] = o_val[i];
-      }
-    }
     if (t == 0) {
       // the stage of the previous tile is free once its store has read it
       // (this tile's store may still be reading its own stage)
       if (R) tc::bulk_wait_read_but_one();
       fetch((it + kStages - 1) % kStages);
     }
-    __syncthreads();
+    // no barrier here: the next tile's scan orders s_tile, and the barrier
+    // before the store above ended every read of s_keep / s_q of this tile
   }
   if (t == 0) {
     tc::bulk_wait_all();

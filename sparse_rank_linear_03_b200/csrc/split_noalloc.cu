@@ -132,7 +132,7 @@ hsl_status run_noalloc(const KT* W, int64_t m, int64_t n, int64_t k, int32_t* ro
   if (vec_ok) {
     constexpr int TE = kTileBytes / int(sizeof(KT));
     const int64_t ntiles = (count + TE - 1) / TE;
-    const size_t smem = size_t(kStages) * kTileBytes + kStageOutBytes;
+    const size_t smem = size_t(kStages) * kTileBytes;
     auto kern = k_split_emit_tile<KT, SB>;
     if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              int(smem)))

@@ -48,7 +48,7 @@ hsl_status emit_launch(Handle& h, const KT* W, int64_t k, KT* R, SelState* st, u
     constexpr int TE = kTileBytes / int(sizeof(KT));
     const int64_t count = h.m * h.n;
     const int64_t ntiles = (count + TE - 1) / TE;
-    const size_t smem = size_t(kStages) * kTileBytes + kStageOutBytes;
+    const size_t smem = size_t(kStages) * kTileBytes;
     auto kern = k_split_emit_tile<KT, SB>;
     if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              int(smem)))

@@ -111,3 +111,16 @@ def test_sparse_mma_matches_expansion_path(hsl, monkeypatch):
     L.check()
     assert oracle.rel_err(f64(host(Ys)), f64(host(Ye))) <= 2 * TOL["bf16"]
     assert oracle.rel_err(f64(host(Ys)), ref_rows(W, U, V, X, np.arange(640))) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("m,n,r,T", [(1100, 256, 40, 700), (512, 128, 0, 2000), (300, 192, 256, 520)])
+def test_cta_pair_kernel_parity(hsl, monkeypatch, m, n, r, T):
+    """The CTA-pair sparse kernel (opt-in) against the oracle: tiles of 512 rows
+    and 192 tokens with ragged rows and tokens, with and without the low-rank term."""
+    L, W, U, V = build(hsl, m, n, r, m + 3 * n + r)
+    X = synth.to_bf16_bits(synth.normal_f32(T, n, T + 1))
+    monkeypatch.setenv("HSL_PREFILL_PAIRS", "1")
+    Y = L.apply(dev(X, "bf16"))
+    monkeypatch.delenv("HSL_PREFILL_PAIRS")
+    L.check()
+    assert oracle.rel_err(f64(host(Y)), ref_rows(W, U, V, X, np.arange(m))) <= TOL["bf16"]
