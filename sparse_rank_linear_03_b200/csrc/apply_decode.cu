@@ -16,10 +16,11 @@
 //                 then griddepcontrol.wait (programmatic dependent launch:
 //                 the S stream overlaps the z kernel), z is staged, and each
 //                 row adds U[i,:]·z and stores y.
-//   k_apply_24_b1_tma  batch 1, bf16 2:4: one CTA of 16 warps per SM; each
-//                 warp pulls (row, super-chunk) units into shared memory with
-//                 1-D bulk copies, two in flight; same partition, z overlap
-//                 and epilogue.
+//   k_apply_24_b1_tma  batch 1, bf16 2:4: one CTA of 16 warps per SM (a
+//                 cooperative launch); the CTAs first compute z among them
+//                 (no second launch), then each warp pulls (row, super-chunk)
+//                 units into shared memory with 1-D bulk copies, two in
+//                 flight; same partition and epilogue.
 #include <algorithm>
 #include <cstdlib>
 #include <cstring>
@@ -45,7 +46,9 @@ struct ApplyArgs {
   int32_t b0, bc;
   int32_t r_pad_max;
   int32_t z_items;  // z work items (rows of Vt) over all layers
+  int32_t z_pieces; // (row, 4096-column piece) items of Vt (in-kernel z)
   uint32_t* err;    // error word (bounded waits that gave up)
+  unsigned long long* zsync;  // CTAs done with z, CTAs done with the call (in-kernel z)
 };
 
 template <typename T>
@@ -549,7 +552,6 @@ __global__ void __maxnreg__(112) k_apply_24_b1_tma(ApplyArgs a, B1Layout lay) {
   const int64_t shi = int64_t(blockIdx.x + 1) * a.slices / gridDim.x;
   int64_t row = a.cta_rows[slo];
   const int64_t row_end = a.cta_rows[shi];
-  if (row >= row_end) return;
   int p = 0;
   {
     int lo = 0, hi = a.count - 1;
@@ -561,6 +563,77 @@ __global__ void __maxnreg__(112) k_apply_24_b1_tma(ApplyArgs a, B1Layout lay) {
   }
   // the abort flag is read by lane 0 and broadcast, so a warp decides as one
   auto aborted = [&]() { return __shfl_sync(0xffffffffu, *abrt, 0) != 0; };
+
+  // z = Vᵀx of every layer of the call in pieces of one row of Vt × 4096
+  // columns, one piece per warp over the whole grid: a warp sums its piece
+  // with a fixed shuffle tree into z_part[q][c] (q = piece of row c), and the
+  // U·z pass adds a row's pieces in order (deterministic).  Each CTA counts
+  // itself in once its warps are done; a CTA waits for the count to reach the
+  // grid only before its first U·z pass.  The launch is cooperative, so all
+  // CTAs are resident and the wait ends (it is bounded all the same).  The
+  // first unit of S is already on its way (issued before the pieces).
+  bool first_issued = false;
+  if (row < row_end) {  // this warp's first S unit (unit `warp` of the first layer)
+    const ApplyProblem& P = a.probs[p];
+    const int l0 = int(row - P.row0), l1 = int(min(row_end, a.prob_row0[p + 1]) - P.row0);
+    const int nq0 = P.n / 16, nsup0 = (nq0 + kSupChunks - 1) / kSupChunks;
+    if (warp < (l1 - l0) * nsup0) {
+      const int r0u = warp / nsup0, sp0 = warp - r0u * nsup0;
+      if (lane == 0) {
+        const int64_t i = int64_t(l0) + r0u;
+        const uint32_t vb = uint32_t(min(kSupChunks, nq0 - sp0 * kSupChunks)) * 16u;
+        tc::fence_async_smem();
+        tc::mbar_expect_tx(mybar, vb + kUnitMBytes);
+        tc::bulk_load_hint(slot0,
+                           static_cast<const unsigned char*>(P.pval) + i * P.n +
+                               int64_t(sp0) * kUnitVBytes,
+                           vb, mybar, policy);
+        tc::bulk_load_hint(slot0 + kUnitVBytes,
+                           reinterpret_cast<const unsigned char*>(P.pmeta) +
+                               i * (int64_t(P.meta_stride) * 2) + sp0 * kUnitMBytes,
+                           kUnitMBytes, mybar, policy);
+      }
+      pending |= 1u;
+      first_issued = true;
+    }
+  }
+  if (a.z_pieces > 0) {
+    const int64_t nw = int64_t(gridDim.x) * kB1Warps;
+    for (int64_t it = int64_t(blockIdx.x) * kB1Warps + warp; it < a.z_pieces; it += nw) {
+      int lo = 0, hi = a.count - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (a.probs[mid].z_piece0 <= it) lo = mid; else hi = mid - 1;
+      }
+      const ApplyProblem& Pz = a.probs[lo];
+      const int nz = Pz.n, Q = (nz + 4095) / 4096;
+      const int local = int(it - Pz.z_piece0), c = local / Q, q = local - c * Q;
+      const __nv_bfloat16* vrow = static_cast<const __nv_bfloat16*>(Pz.Vt) + int64_t(c) * nz;
+      const __nv_bfloat16* xz = x_of<__nv_bfloat16>(a, lo) + int64_t(a.b0) * nz;
+      const int j1 = min(nz, (q + 1) * 4096);
+      float acc = 0.f;
+      if ((reinterpret_cast<uintptr_t>(xz) & 15) == 0) {  // n % 16 == 0: Vt rows are 16-byte aligned
+        for (int j = q * 4096 + lane * 8; j < j1; j += 32 * 8) {
+          float v[8], xv[8];
+          load8<__nv_bfloat16>(vrow + j, v);
+          load8<__nv_bfloat16>(xz + j, xv);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc = fmaf(v[e], xv[e], acc);
+        }
+      } else {
+        for (int j = q * 4096 + lane; j < j1; j += 32)
+          acc = fmaf(ldx<__nv_bfloat16>(vrow + j), ldx<__nv_bfloat16>(xz + j), acc);
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) Pz.z[q * Pz.r_pad + c] = acc;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      __threadfence();
+      atomicAdd(&a.zsync[0], 1ull);
+    }
+  }
   bool waited = false;
   while (row < row_end) {
     const ApplyProblem P = a.probs[p];
@@ -600,7 +673,8 @@ __global__ void __maxnreg__(112) k_apply_24_b1_tma(ApplyArgs a, B1Layout lay) {
       }
       pending |= 1u << sl;
     };
-    if (nu > 0) issue(0);  // lands while x is staged
+    if (nu > 0 && !first_issued) issue(0);  // lands while x is staged
+    first_issued = false;
     const __nv_bfloat16* x = x_of<__nv_bfloat16>(a, p) + int64_t(a.b0) * n;
     __syncthreads();
     if ((reinterpret_cast<uintptr_t>(x) & 15) == 0) {
@@ -669,13 +743,28 @@ __global__ void __maxnreg__(112) k_apply_24_b1_tma(ApplyArgs a, B1Layout lay) {
       const int i = threadIdx.x;
       if (i < s1 - s0)
         for (int q = 0; q < nsup; ++q) yrow += ysp[i * nsup + q];
-      if (!waited) {
-        pdl_wait();
+      if (!waited) {  // every CTA has written its pieces of z
+        if (a.z_pieces > 0 && threadIdx.x == 0) {
+          long long spins = 0;
+          while (ld_acquire_u64(&a.zsync[0]) < gridDim.x) {
+            if (++spins > kSpinLimit) {
+              set_error(a.err, kErrTimeout);
+              break;
+            }
+            __nanosleep(64);
+          }
+        }
         waited = true;
       }
-      if (s0 == l0 && P.r_pad > 0)
-        for (int o = threadIdx.x; o < P.r_pad; o += kB1Threads) zs[o] = __ldcg(P.z + o);
       __syncthreads();
+      if (s0 == l0 && P.r_pad > 0) {  // z of the layer: the sum of its pieces, in order
+        const int Q = (n + 4095) / 4096;
+        for (int o = threadIdx.x; o < P.r_pad; o += kB1Threads) {
+          float zv = 0.f;
+          for (int q = 0; q < Q; ++q) zv += __ldcg(P.z + q * P.r_pad + o);
+          zs[o] = zv;
+        }
+      }
       if (i < s1 - s0) ysp[i] = yrow;
       __syncthreads();
       urows<__nv_bfloat16, 1, kB1Threads>(P, zs, ysp, s0, s1, y, 1);
@@ -687,6 +776,14 @@ __global__ void __maxnreg__(112) k_apply_24_b1_tma(ApplyArgs a, B1Layout lay) {
   // after an abort, copies still in flight land before the CTA exits
   for (int sl = 0; sl < 2; ++sl)
     if ((pending >> sl) & 1u) tc::mbar_wait(mybar + sl, (ph >> sl) & 1u, a.err);
+  // the last CTA out resets the z counters for the next call on the stream
+  __syncthreads();
+  if (a.z_pieces > 0 && threadIdx.x == 0 &&
+      atomicAdd(&a.zsync[1], 1ull) == (unsigned long long)(gridDim.x - 1)) {
+    a.zsync[0] = 0ull;
+    a.zsync[1] = 0ull;
+    __threadfence();
+  }
 }
 
 // Shared memory a CTA of the current device may opt in to.
@@ -717,6 +814,35 @@ size_t apply_smem(const ApplyPlan& plan) {
 
 template <typename T, int BC>
 hsl_status launch_chunk(ApplyPlan& plan, ApplyArgs a, int num_sms, cudaStream_t s) {
+  // every CTA stages the whole x of its layers: keep at least ~64 rows per CTA
+  // so small layers are not dominated by that staging
+  const int64_t row_cap = std::max<int64_t>(1, plan.rows_total / 64);
+  if (BC == 1 && sizeof(T) == 2 && plan.fmt == HSL_FMT_NM24 && plan.vec16 &&
+      decode_b1_bulk_enabled()) {
+    const B1Layout lay = b1_layout(plan.n_max, plan.r_pad_max);
+    // unit indices stay below 2^26, where the unit → (row, super-chunk) split is
+    // exact; z pieces fit the z buffer (at most 16 pieces of 4096 columns)
+    if (lay.total <= max_dyn_smem() && plan.rows_total * lay.nsup < (int64_t(1) << 26) &&
+        plan.n_max <= 16 * 4096) {
+      auto bk = k_apply_24_b1_tma;
+      if (cudaError_t e =
+              cudaFuncSetAttribute(bk, cudaFuncAttributeMaxDynamicSharedMemorySize, lay.total))
+        return cuda_fail(e, "apply smem attribute");
+      // one CTA per SM, all resident (cooperative launch): z is computed inside
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(unsigned(std::min<int64_t>(num_sms, row_cap)));
+      cfg.blockDim = dim3(kB1Threads);
+      cfg.dynamicSmemBytes = size_t(lay.total);
+      cfg.stream = s;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeCooperative;
+      attr[0].val.cooperative = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      note_launch();
+      return cuda_fail(cudaLaunchKernelEx(&cfg, bk, a, lay), "apply launch");
+    }
+  }
   // z = Vᵀ x, normal launch (waits for everything before it on the stream)
   if (plan.z_items > 0) {
     auto zk = k_lowrank_z<T, BC>;
@@ -738,25 +864,6 @@ hsl_status launch_chunk(ApplyPlan& plan, ApplyArgs a, int num_sms, cudaStream_t 
   attr[0].val.programmaticStreamSerializationAllowed = plan.z_items > 0 ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  // every CTA stages the whole x of its layers: keep at least ~64 rows per CTA
-  // so small layers are not dominated by that staging
-  const int64_t row_cap = std::max<int64_t>(1, plan.rows_total / 64);
-  if (BC == 1 && sizeof(T) == 2 && plan.fmt == HSL_FMT_NM24 && plan.vec16 &&
-      decode_b1_bulk_enabled()) {
-    const B1Layout lay = b1_layout(plan.n_max, plan.r_pad_max);
-    // unit indices stay below 2^26, where the unit → (row, super-chunk) split is exact
-    if (lay.total <= max_dyn_smem() && plan.rows_total * lay.nsup < (int64_t(1) << 26)) {
-      auto bk = k_apply_24_b1_tma;
-      if (cudaError_t e =
-              cudaFuncSetAttribute(bk, cudaFuncAttributeMaxDynamicSharedMemorySize, lay.total))
-        return cuda_fail(e, "apply smem attribute");
-      cfg.gridDim = dim3(unsigned(std::min<int64_t>(num_sms, row_cap)));
-      cfg.blockDim = dim3(kB1Threads);
-      cfg.dynamicSmemBytes = size_t(lay.total);
-      note_launch();
-      return cuda_fail(cudaLaunchKernelEx(&cfg, bk, a, lay), "apply launch");
-    }
-  }
   const size_t sm = apply_smem<T, BC>(plan);
   auto ak = plan.fmt == HSL_FMT_CSR ? k_apply_decode<T, BC, true> : k_apply_decode<T, BC, false>;
   if (cudaError_t e = cudaFuncSetAttribute(ak, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm)))
@@ -811,7 +918,9 @@ hsl_status apply_decode_run(ApplyPlan& plan, const void* X, void* Y, const void*
   a.bc = 0;
   a.r_pad_max = plan.r_pad_max;
   a.z_items = plan.z_items;
+  a.z_pieces = plan.z_pieces;
   a.err = plan.err;
+  a.zsync = static_cast<unsigned long long*>(plan.zsync.p);
   if (plan.dtype == HSL_BF16) return run_typed<__nv_bfloat16>(plan, a, batch, num_sms, s);
   return run_typed<float>(plan, a, batch, num_sms, s);
 }

@@ -344,7 +344,7 @@ hsl_status plan_build(ApplyPlan& plan, Handle* const* hs, int count, cudaStream_
   const int eb = dtype_bytes(plan.dtype);
   std::vector<ApplyProblem> probs(count);
   int64_t row0 = 0;
-  int zc = 0;
+  int zc = 0, zp = 0;
   for (int i = 0; i < count; ++i) {
     Handle& h = *hs[i];
     ApplyProblem& P = probs[i];
@@ -367,12 +367,15 @@ hsl_status plan_build(ApplyPlan& plan, Handle* const* hs, int count, cudaStream_
     P.z = static_cast<float*>(h.z.p);
     P.z_item0 = zc;
     zc += h.r_pad;
+    P.z_piece0 = zp;
+    zp += h.r_pad * int32_t((h.n + 4095) / 4096);
     plan.n_max = std::max(plan.n_max, int32_t(h.n));
     plan.vec16 = plan.vec16 && h.n % 16 == 0;
     plan.r_pad_max = std::max(plan.r_pad_max, h.r_pad);
   }
   plan.rows_total = row0;
   plan.z_items = zc;
+  plan.z_pieces = zp;
   if (zc > 0 && plan.zsync.p == nullptr) {
     if (hsl_status e = ensure(plan.zsync, 256, "z barrier")) return e;
     if (cudaError_t ce = cudaMemsetAsync(plan.zsync.p, 0, 256, s)) return cuda_fail(ce, "memset");
