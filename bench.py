@@ -73,6 +73,12 @@ def peaks() -> dict:
     return {"hbm": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
 
 
+# DRAM bytes (read + write) of one launch of the batch-1 2:4 apply kernel on this
+# workload, from one ncu capture of it (dram__bytes_read.sum + dram__bytes_write.sum,
+# the decode70b profile case): 283.21 MB + 3.66 MB against 283.19 MB algorithmic.
+# Re-take it whenever that kernel changes.
+DECODE_TRAFFIC_BYTES = 286_874_880
+
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
@@ -339,7 +345,8 @@ def run_gpu(args, world, rank, local):
         },
         "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1), "peak": pk["hbm"],
                      "unit": "GB/s", "frac": round(dec_gbs / pk["hbm"], 4),
-                     "traffic": None, "kernel": "decode apply (z + fused sparse/U·z)",
+                     "traffic": DECODE_TRAFFIC_BYTES,
+                     "kernel": "batch-1 2:4 apply (z, S stream and U·z in one kernel)",
                      "peak_source": pk["source"]},
         "e2e": {"value": round(e2e_gbs, 1), "unit": "GB/s", "h2d_bytes_per_step": N * 2,
                 "d2h_bytes_per_step": M * 2},

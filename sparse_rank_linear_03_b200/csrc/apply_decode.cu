@@ -46,7 +46,7 @@ struct ApplyArgs {
   int32_t b0, bc;
   int32_t r_pad_max;
   int32_t z_items;  // z work items (rows of Vt) over all layers
-  int32_t z_pieces; // (row, 4096-column piece) items of Vt (in-kernel z)
+  int32_t z_pieces; // (row, column piece) items of Vt (in-kernel z)
   uint32_t* err;    // error word (bounded waits that gave up)
   unsigned long long* zsync;  // CTAs done with z, CTAs done with the call (in-kernel z)
 };
@@ -564,8 +564,8 @@ __global__ void __maxnreg__(112) k_apply_24_b1_tma(ApplyArgs a, B1Layout lay) {
   // the abort flag is read by lane 0 and broadcast, so a warp decides as one
   auto aborted = [&]() { return __shfl_sync(0xffffffffu, *abrt, 0) != 0; };
 
-  // z = Vᵀx of every layer of the call in pieces of one row of Vt × 4096
-  // columns, one piece per warp over the whole grid: a warp sums its piece
+  // z = Vᵀx of every layer of the call in pieces of one row of Vt × ≥ 1024
+  // columns (z_piece_width), one piece per warp over the whole grid: a warp sums its piece
   // with a fixed shuffle tree into z_part[q][c] (q = piece of row c), and the
   // U·z pass adds a row's pieces in order (deterministic).  Each CTA counts
   // itself in once its warps are done; a CTA waits for the count to reach the
@@ -606,22 +606,40 @@ __global__ void __maxnreg__(112) k_apply_24_b1_tma(ApplyArgs a, B1Layout lay) {
         if (a.probs[mid].z_piece0 <= it) lo = mid; else hi = mid - 1;
       }
       const ApplyProblem& Pz = a.probs[lo];
-      const int nz = Pz.n, Q = (nz + 4095) / 4096;
+      const int nz = Pz.n, pw = z_piece_width(nz), Q = (nz + pw - 1) / pw;
       const int local = int(it - Pz.z_piece0), c = local / Q, q = local - c * Q;
       const __nv_bfloat16* vrow = static_cast<const __nv_bfloat16*>(Pz.Vt) + int64_t(c) * nz;
       const __nv_bfloat16* xz = x_of<__nv_bfloat16>(a, lo) + int64_t(a.b0) * nz;
-      const int j1 = min(nz, (q + 1) * 4096);
+      const int j0 = q * pw, j1 = min(nz, j0 + pw);
       float acc = 0.f;
       if ((reinterpret_cast<uintptr_t>(xz) & 15) == 0) {  // n % 16 == 0: Vt rows are 16-byte aligned
-        for (int j = q * 4096 + lane * 8; j < j1; j += 32 * 8) {
-          float v[8], xv[8];
-          load8<__nv_bfloat16>(vrow + j, v);
-          load8<__nv_bfloat16>(xz + j, xv);
+        // at most 8 vectors per lane (pw ≤ 2048), four loads of each operand in flight
 #pragma unroll
-          for (int e = 0; e < 8; ++e) acc = fmaf(v[e], xv[e], acc);
+        for (int half = 0; half < 2; ++half) {
+          uint4 vq[4], xq[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int j = j0 + ((4 * half + u) * 32 + lane) * 8;
+            if (j < j1) {
+              vq[u] = ld_stream16(vrow + j);
+              xq[u] = *reinterpret_cast<const uint4*>(xz + j);
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            if (j0 + ((4 * half + u) * 32 + lane) * 8 < j1) {
+              const uint32_t vw[4] = {vq[u].x, vq[u].y, vq[u].z, vq[u].w};
+              const uint32_t xw[4] = {xq[u].x, xq[u].y, xq[u].z, xq[u].w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                acc = fmaf(bf_lo(vw[e]), bf_lo(xw[e]), acc);
+                acc = fmaf(bf_hi(vw[e]), bf_hi(xw[e]), acc);
+              }
+            }
+          }
         }
       } else {
-        for (int j = q * 4096 + lane; j < j1; j += 32)
+        for (int j = j0 + lane; j < j1; j += 32)
           acc = fmaf(ldx<__nv_bfloat16>(vrow + j), ldx<__nv_bfloat16>(xz + j), acc);
       }
 #pragma unroll
@@ -758,7 +776,7 @@ __global__ void __maxnreg__(112) k_apply_24_b1_tma(ApplyArgs a, B1Layout lay) {
       }
       __syncthreads();
       if (s0 == l0 && P.r_pad > 0) {  // z of the layer: the sum of its pieces, in order
-        const int Q = (n + 4095) / 4096;
+        const int Q = (n + z_piece_width(n) - 1) / z_piece_width(n);
         for (int o = threadIdx.x; o < P.r_pad; o += kB1Threads) {
           float zv = 0.f;
           for (int q = 0; q < Q; ++q) zv += __ldcg(P.z + q * P.r_pad + o);
@@ -821,9 +839,9 @@ hsl_status launch_chunk(ApplyPlan& plan, ApplyArgs a, int num_sms, cudaStream_t 
       decode_b1_bulk_enabled()) {
     const B1Layout lay = b1_layout(plan.n_max, plan.r_pad_max);
     // unit indices stay below 2^26, where the unit → (row, super-chunk) split is
-    // exact; z pieces fit the z buffer (at most 16 pieces of 4096 columns)
+    // exact; z pieces fit the z buffer (at most 16 pieces of at most 2048 columns)
     if (lay.total <= max_dyn_smem() && plan.rows_total * lay.nsup < (int64_t(1) << 26) &&
-        plan.n_max <= 16 * 4096) {
+        plan.n_max <= 16 * 2048) {
       auto bk = k_apply_24_b1_tma;
       if (cudaError_t e =
               cudaFuncSetAttribute(bk, cudaFuncAttributeMaxDynamicSharedMemorySize, lay.total))

@@ -41,9 +41,16 @@ struct ApplyProblem {
   int32_t group;          // CSR: lanes per row (4..32)
   int32_t meta_stride;    // NM24: u16 metadata words per row
   int32_t z_item0;        // this layer's first z work item (one per row of Vt)
-  int32_t z_piece0;       // first (row, 4096-column piece) of Vt of this layer (in-kernel z)
+  int32_t z_piece0;       // first (row, column piece) of Vt of this layer (in-kernel z)
   int64_t row0;           // first row of this layer in the concatenated row space
 };
+
+// Width of the pieces of a row of Vt that the in-kernel z sums (one warp
+// each, at most 8 vectors of 8 per lane): ≥ 1024 columns, at most 16 pieces.
+__host__ __device__ inline int z_piece_width(int n) {
+  const int w = ((n + 15) / 16 + 255) / 256 * 256;
+  return w < 1024 ? 1024 : w;
+}
 
 // Launch plan for one or more layers applied together.
 struct ApplyPlan {
@@ -53,7 +60,7 @@ struct ApplyPlan {
   int32_t n_max = 0, r_pad_max = 0;
   int64_t rows_total = 0;
   int z_items = 0;      // z work items over all layers (0 when r == 0)
-  int z_pieces = 0;     // (row, 4096-column piece) items of Vt over all layers
+  int z_pieces = 0;     // (row, column piece) items of Vt over all layers
   int slices = 0;       // equal-byte row ranges the apply grid divides among CTAs
   bool vec16 = false;   // every layer has n % 16 == 0 (16-byte aligned 2:4 rows)
   uint32_t* err = nullptr;  // error word the apply kernels report to (first member's)

@@ -368,7 +368,7 @@ hsl_status plan_build(ApplyPlan& plan, Handle* const* hs, int count, cudaStream_
     P.z_item0 = zc;
     zc += h.r_pad;
     P.z_piece0 = zp;
-    zp += h.r_pad * int32_t((h.n + 4095) / 4096);
+    zp += h.r_pad * int32_t((h.n + z_piece_width(int(h.n)) - 1) / z_piece_width(int(h.n)));
     plan.n_max = std::max(plan.n_max, int32_t(h.n));
     plan.vec16 = plan.vec16 && h.n % 16 == 0;
     plan.r_pad_max = std::max(plan.r_pad_max, h.r_pad);

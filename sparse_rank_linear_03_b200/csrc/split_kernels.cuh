@@ -225,8 +225,22 @@ __global__ void __launch_bounds__(1024) k_bracket_select(const unsigned* __restr
     key_lo = 0u;       // r_lo beyond the sample: keep every key in the bracket
   }
   const int top = 32767 - t * PER;  // this thread's bins: top, top−1, ..., top−PER+1
+  // the 32 bins [top − 31, top] are one aligned 128-byte run: eight 16-byte loads
+  unsigned hb[PER];
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(shist + (top - PER + 1));
+#pragma unroll
+    for (int u = 0; u < PER / 4; ++u) {
+      const uint4 q = src[u];
+      hb[4 * u] = q.x;
+      hb[4 * u + 1] = q.y;
+      hb[4 * u + 2] = q.z;
+      hb[4 * u + 3] = q.w;
+    }
+  }
   unsigned s = 0;
-  for (int b = 0; b < PER; ++b) s += shist[top - b];
+#pragma unroll
+  for (int b = 0; b < PER; ++b) s += hb[b];
   unsigned incl = s;
   for (int o = 1; o < 32; o <<= 1) {
     const unsigned v = __shfl_up_sync(0xffffffffu, incl, o);
@@ -250,7 +264,7 @@ __global__ void __launch_bounds__(1024) k_bracket_select(const unsigned* __restr
   if (r_hi > 0 && r_hi >= before && r_hi < before + s) {
     unsigned acc = before;
     for (int b = 0; b < PER; ++b) {
-      acc += shist[top - b];
+      acc += hb[PER - 1 - b];  // bin top − b
       if (acc > r_hi) {
         key_hi = uint32_t(top - b);
         break;
@@ -261,7 +275,7 @@ __global__ void __launch_bounds__(1024) k_bracket_select(const unsigned* __restr
   if (r_lo > before && r_lo <= before + s) {
     unsigned acc = before;
     for (int b = 0; b < PER; ++b) {
-      acc += shist[top - b];
+      acc += hb[PER - 1 - b];
       if (acc >= r_lo) {
         key_lo = uint32_t(top - b);
         break;
@@ -415,19 +429,30 @@ __global__ void __launch_bounds__(256) k_tile_counts(const uint32_t* __restrict_
   const int lane = threadIdx.x & 31;
   const int64_t gw = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nw = (int64_t(gridDim.x) * blockDim.x) >> 5;
-  for (int64_t tile = gw; tile < ntiles; tile += nw) {
-    unsigned gt = 0, eq = 0;
-    for (int b = lane; b < kTileBins; b += 32) {
-      const unsigned c = tile_hist[tile * kTileBins + b];
-      gt += lo + uint32_t(b) > T ? c : 0u;
-      eq += lo + uint32_t(b) == T ? c : 0u;
+  constexpr int TW = 4;  // tiles per warp at a time: eight loads in flight per lane
+  for (int64_t tile0 = gw * TW; tile0 < ntiles; tile0 += nw * TW) {
+    unsigned c[TW][2];
+#pragma unroll
+    for (int u = 0; u < TW; ++u)
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        c[u][h] = tile0 + u < ntiles ? tile_hist[(tile0 + u) * kTileBins + lane + 32 * h] : 0u;
+#pragma unroll
+    for (int u = 0; u < TW; ++u) {
+      unsigned gt = 0, eq = 0;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t key = lo + uint32_t(lane + 32 * h);
+        gt += key > T ? c[u][h] : 0u;
+        eq += key == T ? c[u][h] : 0u;
+      }
+      for (int o = 16; o; o >>= 1) {
+        gt += __shfl_xor_sync(0xffffffffu, gt, o);
+        eq += __shfl_xor_sync(0xffffffffu, eq, o);
+      }
+      if (lane == 0 && tile0 + u < ntiles)
+        tile_cnt[tile0 + u] = ((unsigned long long)(tile_above[tile0 + u] + gt) << 32) | eq;
     }
-    for (int o = 16; o; o >>= 1) {
-      gt += __shfl_xor_sync(0xffffffffu, gt, o);
-      eq += __shfl_xor_sync(0xffffffffu, eq, o);
-    }
-    if (lane == 0)
-      tile_cnt[tile] = ((unsigned long long)(tile_above[tile] + gt) << 32) | eq;
   }
 }
 
@@ -441,8 +466,17 @@ __global__ void __launch_bounds__(1024) k_tile_scan(const unsigned long long* __
   const int t = threadIdx.x;
   const int64_t per = (ntiles + 1023) / 1024;
   const int64_t a = min(int64_t(t) * per, ntiles), b = min(a + per, ntiles);
+  constexpr int RB = 16;  // up to 16 tiles per thread are loaded at once and kept
+  unsigned long long reg[RB];
   unsigned long long s = 0;
-  for (int64_t i = a; i < b; ++i) s += tile_cnt[i];
+  if (per <= RB) {
+#pragma unroll
+    for (int u = 0; u < RB; ++u) reg[u] = a + u < b ? tile_cnt[a + u] : 0ull;
+#pragma unroll
+    for (int u = 0; u < RB; ++u) s += reg[u];
+  } else {
+    for (int64_t i = a; i < b; ++i) s += tile_cnt[i];
+  }
   unsigned long long incl = s;
   for (int o = 1; o < 32; o <<= 1) {
     const unsigned long long v = __shfl_up_sync(0xffffffffu, incl, o);
@@ -461,9 +495,17 @@ __global__ void __launch_bounds__(1024) k_tile_scan(const unsigned long long* __
   }
   __syncthreads();
   unsigned long long run = warp_tot[t >> 5] + incl - s;
-  for (int64_t i = a; i < b; ++i) {
-    tile_pre[i] = run;
-    run += tile_cnt[i];
+  if (per <= RB) {
+#pragma unroll
+    for (int u = 0; u < RB; ++u) {
+      if (a + u < b) tile_pre[a + u] = run;
+      run += reg[u];
+    }
+  } else {
+    for (int64_t i = a; i < b; ++i) {
+      tile_pre[i] = run;
+      run += tile_cnt[i];
+    }
   }
 }
 
