@@ -396,7 +396,7 @@ __device__ __forceinline__ void nm24_rows(const ApplyProblem& P, const T* xs, fl
 
 // ---- the persistent apply kernel ---------------------------------------------------
 template <typename T, int BC, bool CSR>
-__global__ void __launch_bounds__(kThreads, 2) k_apply_decode(ApplyArgs a) {
+__global__ void __maxnreg__(112) k_apply_decode(ApplyArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ uint32_t sel_lut[16];  // byte-permute selector of a 2:4 nibble (x[i0], x[i1])
   if (threadIdx.x < 16)
