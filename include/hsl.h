@@ -60,7 +60,7 @@ typedef void* hsl_stream; /* cudaStream_t */
 typedef enum {
   HSL_OK = 0,
   HSL_ERR_INVALID_ARG = 1, /* a NULL/out-of-range argument, host-side check */
-  HSL_ERR_UNSUPPORTED = 2, /* a valid request this build does not cover     */
+  HSL_ERR_UNSUPPORTED = 2, /* a valid request the library does not handle   */
   HSL_ERR_NOT_READY = 3,   /* e.g. hsl_apply before hsl_pack                */
   HSL_ERR_OOM = 4,         /* a device allocation failed                    */
   HSL_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed          */
