@@ -22,6 +22,11 @@ constexpr int kTileThreads = 256;
 constexpr int kTileBytes = 32768;
 constexpr int kStages = 3;
 constexpr int kTileVPT = kTileBytes / 16 / kTileThreads;  // vectors per thread
+// The emit refills, at the end of iteration it, the stage that iteration
+// it + kStages - 1 consumes, and writes that stage's tile id there too: the
+// barriers of the iterations in between make the id visible to every thread.
+// With two stages the next iteration would read the id before any barrier.
+static_assert(kStages >= 3, "the emit's tile ids need three stages");
 
 template <typename KT> struct KeyTraits;
 template <> struct KeyTraits<uint16_t> {
@@ -916,9 +921,9 @@ __device__ __forceinline__ void vec_masks<uint32_t>(const uint4& q, uint32_t T, 
 // W is cut into tiles of kTileBytes (any number of rows or part of one).  A
 // persistent CTA takes tiles in ticket order and keeps kStages of them in
 // flight: a 1-D bulk copy brings each into shared memory; the residual goes
-// back with a bulk store from the same buffer.  Thread t owns the vectors
-// [8t, 8t + 8) of its tile and visits them starting at slot t & 7, so at every
-// step the eight threads of a quarter-warp read eight different bank groups.
+// back with a bulk store from the same buffer.  Thread t owns kTileVPT
+// contiguous vectors of its tile and starts at a slot chosen so that, at every
+// step, the eight threads of a quarter-warp read eight different bank groups.
 // The kept entries of a tile form a contiguous range of S; after one barrier
 // every thread produces outputs i, i + 256, ... of that range (binary search
 // for the owning thread, then its (i − first)-th kept element), so S is
@@ -1018,7 +1023,10 @@ __global__ void __launch_bounds__(kTileThreads, 2) k_split_emit_tile(
   }
   __syncthreads();
 
-  const int r0 = t & (kTileVPT - 1);
+  // first slot of the thread: the eight threads of a quarter-warp read
+  // distinct 16-byte bank groups (a thread's vectors are contiguous)
+  static_assert(kTileVPT <= 8 && 8 % kTileVPT == 0, "slot rotation");
+  const int r0 = (t / (8 / kTileVPT)) & (kTileVPT - 1);
   for (int it = 0;; ++it) {
     const int sg = it % kStages;
     const int64_t tile = s_tile[sg];
