@@ -17,11 +17,15 @@ struct SelState {
   uint32_t pad;
 };
 
-// Emit tiles: W is processed in tiles of kTileBytes by CTAs of kTileThreads.
+// Emit tiles: W is processed in tiles of TB bytes by CTAs of kTileThreads.
+// Tiles whose S prefixes come from the bracket pass's per-tile counts are
+// small, so four CTAs share an SM and hide each other's per-tile latency;
+// tiles that find their prefix by look-back are twice as large, which halves
+// the number of look-backs.
 constexpr int kTileThreads = 256;
-constexpr int kTileBytes = 32768;
+constexpr int kTileBytesPre = 16384;
+constexpr int kTileBytesLB = 32768;
 constexpr int kStages = 3;
-constexpr int kTileVPT = kTileBytes / 16 / kTileThreads;  // vectors per thread
 // The emit refills, at the end of iteration it, the stage that iteration
 // it + kStages - 1 consumes, and writes that stage's tile id there too: the
 // barriers of the iterations in between make the id visible to every thread.
@@ -299,7 +303,7 @@ __global__ void __launch_bounds__(1024) k_bracket_select(const unsigned* __restr
 // Full pass: count keys > hi, histogram keys in [lo, hi] into ghist[key],
 // flag NaN.  bf16 pairs are compared by packed subtraction (see vec_masks).
 // When the bracket spans at most kTileBins keys and tile_hist is given, each
-// warp takes whole emit tiles (kTileBytes of W) and also records, per tile,
+// warp takes whole emit tiles (kTileBytesPre of W) and also records, per tile,
 // the count above the bracket and the tile's bracket histogram; with the
 // threshold known, those give every tile's exact (above T, equal to T) counts,
 // so the emit pass needs no look-back.
@@ -354,7 +358,7 @@ __global__ void __launch_bounds__(1024) k_count_bracket(const uint16_t* __restri
     cnt = 0;
   };
   if (record) {
-    constexpr int VPT = kTileBytes / 16;  // vectors of a tile
+    constexpr int VPT = kTileBytesPre / 16;  // vectors of a tile
     const int64_t ntiles = (nvec + VPT - 1) / VPT;
     const int64_t gw = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nw = (int64_t(gridDim.x) * blockDim.x) >> 5;
@@ -918,10 +922,10 @@ __device__ __forceinline__ void vec_masks<uint32_t>(const uint4& q, uint32_t T, 
 }
 
 // ---- emit over element tiles staged by bulk copies -----------------------------
-// W is cut into tiles of kTileBytes (any number of rows or part of one).  A
+// W is cut into tiles of TB bytes (any number of rows or part of one).  A
 // persistent CTA takes tiles in ticket order and keeps kStages of them in
 // flight: a 1-D bulk copy brings each into shared memory; the residual goes
-// back with a bulk store from the same buffer.  Thread t owns kTileVPT
+// back with a bulk store from the same buffer.  Thread t owns TB / 4096
 // contiguous vectors of its tile and starts at a slot chosen so that, at every
 // step, the eight threads of a quarter-warp read eight different bank groups.
 // The kept entries of a tile form a contiguous range of S; after one barrier
@@ -974,8 +978,8 @@ __device__ __forceinline__ int nth_set_bit64(unsigned long long m, uint32_t j) {
   return base;
 }
 
-template <typename KT, typename SB>
-__global__ void __launch_bounds__(kTileThreads, 2) k_split_emit_tile(
+template <typename KT, typename SB, int TB>
+__global__ void __launch_bounds__(kTileThreads, TB <= 16384 ? 4 : 2) k_split_emit_tile(
     const KT* __restrict__ W, int64_t m, int64_t count, FastDiv nd, int64_t ntiles,
     const SelState* __restrict__ st, unsigned* __restrict__ ticket,
     unsigned long long* __restrict__ flags, int32_t* __restrict__ row_ptr,
@@ -983,7 +987,8 @@ __global__ void __launch_bounds__(kTileThreads, 2) k_split_emit_tile(
     uint32_t* __restrict__ err, const Bracket* __restrict__ br,
     const unsigned long long* __restrict__ tile_pre) {
   constexpr int EPV = 16 / sizeof(KT);
-  constexpr int TE = kTileBytes / sizeof(KT);
+  constexpr int TE = TB / sizeof(KT);
+  constexpr int kTileVPT = TB / 16 / kTileThreads;  // vectors per thread
   extern __shared__ __align__(16) unsigned char smem[];
   uint4* tiles = reinterpret_cast<uint4*>(smem);
   __shared__ unsigned long long s_keep[kTileThreads];  // kept elements of each thread
@@ -1009,7 +1014,7 @@ __global__ void __launch_bounds__(kTileThreads, 2) k_split_emit_tile(
       const int64_t e0 = id * TE;
       const uint32_t bytes = uint32_t((count - e0 < TE ? count - e0 : int64_t(TE)) * int64_t(sizeof(KT)));
       tc::mbar_expect_tx(&bar[sg], bytes);
-      tc::bulk_load_hint(tiles + sg * (kTileBytes / 16), W + e0, bytes, &bar[sg], policy);
+      tc::bulk_load_hint(tiles + sg * (TB / 16), W + e0, bytes, &bar[sg], policy);
     }
     s_tile[sg] = id < ntiles ? id : -1;
   };
@@ -1038,7 +1043,7 @@ __global__ void __launch_bounds__(kTileThreads, 2) k_split_emit_tile(
     }
     const int64_t e0 = tile * TE;
     const int nv = int((count - e0 < TE ? count - e0 : int64_t(TE)) / EPV);
-    uint4* tv = tiles + sg * (kTileBytes / 16);
+    uint4* tv = tiles + sg * (TB / 16);
 
     // phase 1: masks and counts of the thread's vectors, slot order r0, r0+1, ...
     uint32_t msk[kTileVPT], cnt[kTileVPT];

@@ -38,7 +38,7 @@ constexpr int64_t kNoAllocMaxRows = 65536;
 constexpr size_t kNoAllocHist = 32768 * sizeof(unsigned);
 constexpr size_t kNoAllocState = 256;  // SelState at +0, row ticket at +64
 // look-back flags: one per row (per-row emit) or per 32 KB tile of W, m·n < 2^31
-constexpr int64_t kNoAllocFlags = std::max<int64_t>(kNoAllocMaxRows, (int64_t(4) << 31) / kTileBytes);
+constexpr int64_t kNoAllocFlags = std::max<int64_t>(kNoAllocMaxRows, (int64_t(4) << 31) / kTileBytesLB);
 constexpr size_t kNoAllocBytes = kNoAllocHist + kNoAllocState + size_t(kNoAllocFlags) * 8;
 }  // namespace
 }  // namespace hsl
@@ -127,13 +127,13 @@ hsl_status run_noalloc(const KT* W, int64_t m, int64_t n, int64_t k, int32_t* ro
   }
   // the ticket and the look-back flags must start at zero
   if (cudaError_t e = cudaMemsetAsync(ticket, 0, 4, s)) return cuda_fail(e, "memset");
-  const int64_t nflags = std::max<int64_t>(m, (count * int64_t(sizeof(KT)) + kTileBytes - 1) / kTileBytes);
+  const int64_t nflags = std::max<int64_t>(m, (count * int64_t(sizeof(KT)) + kTileBytesLB - 1) / kTileBytesLB);
   if (cudaError_t e = cudaMemsetAsync(flags, 0, size_t(nflags) * 8, s)) return cuda_fail(e, "memset");
   if (vec_ok) {
-    constexpr int TE = kTileBytes / int(sizeof(KT));
+    constexpr int TE = kTileBytesLB / int(sizeof(KT));
     const int64_t ntiles = (count + TE - 1) / TE;
-    const size_t smem = size_t(kStages) * kTileBytes;
-    auto kern = k_split_emit_tile<KT, SB>;
+    const size_t smem = size_t(kStages) * kTileBytesLB;
+    auto kern = k_split_emit_tile<KT, SB, kTileBytesLB>;
     if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              int(smem)))
       return cuda_fail(e, "split emit smem attribute");

@@ -40,28 +40,39 @@
 namespace hsl {
 namespace {
 
+template <typename KT, typename SB, int TB>
+hsl_status emit_tiles(Handle& h, const KT* W, int64_t k, KT* R, SelState* st, unsigned* ticket,
+                      unsigned long long* flags, uint32_t* err, const Bracket* br,
+                      const unsigned long long* tile_pre, cudaStream_t s) {
+  constexpr int TE = TB / int(sizeof(KT));
+  const int64_t count = h.m * h.n;
+  const int64_t ntiles = (count + TE - 1) / TE;
+  const size_t smem = size_t(kStages) * TB;
+  auto kern = k_split_emit_tile<KT, SB, TB>;
+  if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           int(smem)))
+    return cuda_fail(e, "split emit smem attribute");
+  int occ = 0;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kTileThreads, smem);
+  const int64_t grid = std::min<int64_t>(ntiles, int64_t(h.num_sms) * std::max(occ, 1));
+  kern<<<unsigned(std::max<int64_t>(grid, 1)), kTileThreads, smem, s>>>(
+      W, h.m, count, make_fastdiv(uint32_t(h.n)), ntiles, st, ticket, flags,
+      static_cast<int32_t*>(h.row_ptr.p), static_cast<int32_t*>(h.col.p),
+      static_cast<SB*>(h.val.p), R, k, err, br, tile_pre);
+  note_launch();
+  return cuda_fail(cudaGetLastError(), "split emit launch");
+}
+
 template <typename KT, typename SB>
 hsl_status emit_launch(Handle& h, const KT* W, int64_t k, KT* R, SelState* st, unsigned* ticket,
                        unsigned long long* flags, uint32_t* err, bool vec_ok, const Bracket* br,
                        const unsigned long long* tile_pre, cudaStream_t s) {
   if (vec_ok) {
-    constexpr int TE = kTileBytes / int(sizeof(KT));
-    const int64_t count = h.m * h.n;
-    const int64_t ntiles = (count + TE - 1) / TE;
-    const size_t smem = size_t(kStages) * kTileBytes;
-    auto kern = k_split_emit_tile<KT, SB>;
-    if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             int(smem)))
-      return cuda_fail(e, "split emit smem attribute");
-    int occ = 0;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kTileThreads, smem);
-    const int64_t grid = std::min<int64_t>(ntiles, int64_t(h.num_sms) * std::max(occ, 1));
-    kern<<<unsigned(std::max<int64_t>(grid, 1)), kTileThreads, smem, s>>>(
-        W, h.m, count, make_fastdiv(uint32_t(h.n)), ntiles, st, ticket, flags,
-        static_cast<int32_t*>(h.row_ptr.p), static_cast<int32_t*>(h.col.p),
-        static_cast<SB*>(h.val.p), R, k, err, br, tile_pre);
-    note_launch();
-    return cuda_fail(cudaGetLastError(), "split emit launch");
+    // the tile size of the bracket pass's per-tile counts, else look-back tiles
+    return tile_pre ? emit_tiles<KT, SB, kTileBytesPre>(h, W, k, R, st, ticket, flags, err, br,
+                                                        tile_pre, s)
+                    : emit_tiles<KT, SB, kTileBytesLB>(h, W, k, R, st, ticket, flags, err, br,
+                                                       tile_pre, s);
   }
   int occ = 0;
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_split_emit<KT, SB>, kEmitThreads, 0);
@@ -80,8 +91,9 @@ hsl_status run_typed(Handle& h, const KT* W, int64_t k, KT* R, cudaStream_t s) {
   // workspace: hist[32768] | sample hist[32768] | SelState | ticket | Bracket ; flags separately
   const size_t hist_bytes = 32768 * sizeof(unsigned);
   if (hsl_status e = ensure(h.split_ws, 2 * hist_bytes + 256, "split workspace")) return e;
-  // look-back flags: one per row (per-row emit) or per tile
-  const int64_t nflags = std::max<int64_t>(h.m, (count * int64_t(sizeof(KT)) + kTileBytes - 1) / kTileBytes);
+  // look-back flags: one per row (per-row emit) or per tile (at most one per
+  // tile of the smaller size)
+  const int64_t nflags = std::max<int64_t>(h.m, (count * int64_t(sizeof(KT)) + kTileBytesPre - 1) / kTileBytesPre);
   if (hsl_status e = ensure(h.flags, size_t(nflags) * 8, "split look-back flags")) return e;
   char* ws = static_cast<char*>(h.split_ws.p);
   unsigned* hist = reinterpret_cast<unsigned*>(ws);
@@ -132,7 +144,7 @@ hsl_status run_typed(Handle& h, const KT* W, int64_t k, KT* R, cudaStream_t s) {
     cudaFuncSetAttribute(k_count_bracket, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     const uint16_t* W16 = reinterpret_cast<const uint16_t*>(W);
     // per emit tile: count above the bracket, bracket histogram, counts, prefixes
-    const int64_t ntiles = (count * 2 + kTileBytes - 1) / kTileBytes;
+    const int64_t ntiles = (count * 2 + kTileBytesPre - 1) / kTileBytesPre;
     const size_t tb_above = size_t(ntiles) * 4, tb_hist = size_t(ntiles) * kTileBins * 4;
     if (hsl_status e = ensure(h.tiles, tb_above + tb_hist + size_t(ntiles) * 16 + 64, "split tiles"))
       return e;
