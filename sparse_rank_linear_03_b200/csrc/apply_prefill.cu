@@ -941,7 +941,9 @@ hsl_status apply_prefill_run(Handle& h, const void* X, void* Y, int64_t T, cudaS
       return HSL_ERR_CUDA;
     }
     if (r16 > 0) {
-      cudaFuncSetAttribute(k_prefill_z, cudaFuncAttributeMaxDynamicSharedMemorySize, Z_SMEM);
+      if (cudaError_t e = cudaFuncSetAttribute(k_prefill_z,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, Z_SMEM))
+        return cuda_fail(e, "prefill z smem attribute");
       k_prefill_z<<<unsigned((T + 127) / 128), 192, Z_SMEM, s>>>(
           zm, static_cast<__nv_bfloat16*>(h.zpre.p), int(n), int(T), r16, err0);
       note_launch();
@@ -1026,7 +1028,9 @@ hsl_status apply_prefill_run(Handle& h, const void* X, void* Y, int64_t T, cudaS
   }
   uint32_t* err = static_cast<uint32_t*>(h.err.p);
   if (r16 > 0) {
-    cudaFuncSetAttribute(k_prefill_z, cudaFuncAttributeMaxDynamicSharedMemorySize, Z_SMEM);
+    if (cudaError_t e = cudaFuncSetAttribute(k_prefill_z,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, Z_SMEM))
+      return cuda_fail(e, "prefill z smem attribute");
     k_prefill_z<<<unsigned((T + 127) / 128), 192, Z_SMEM, s>>>(
         maps, static_cast<__nv_bfloat16*>(h.zpre.p), int(n), int(T), r16, err);
     note_launch();

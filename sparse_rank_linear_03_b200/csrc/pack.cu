@@ -404,7 +404,8 @@ hsl_status plan_build(ApplyPlan& plan, Handle* const* hs, int count, cudaStream_
   hsl_status st = cuda_fail(cudaGetLastError(), "partition launch");
   // the vectors above are pageable: the copies have completed on return, and
   // the kernel's scratch can be freed once the stream reaches this point
-  cudaStreamSynchronize(s);
+  if (cudaError_t e = cudaStreamSynchronize(s); e != cudaSuccess && st == HSL_OK)
+    st = cuda_fail(e, "plan upload");
   release(cost0);
   plan.host_xy.clear();
   return st;

@@ -108,7 +108,9 @@ hsl_status run_noalloc(const KT* W, int64_t m, int64_t n, int64_t k, int32_t* ro
     const size_t smem = (size_t(1) << bits[p]) * sizeof(unsigned);
     if (bits[p] == 15) {
       auto kern = k_split_hist<KT, 15>;
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+      if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               int(smem)))
+        return cuda_fail(e, "split histogram smem attribute");
       kern<<<d.sms, 1024, smem, s>>>(W, count, st, shifts[p], hist, err, vec_ok ? 1 : 0, skip);
     } else if (bits[p] == 11) {
       k_split_hist<KT, 11><<<d.sms * 2, 1024, smem, s>>>(W, count, st, shifts[p], hist, err,
