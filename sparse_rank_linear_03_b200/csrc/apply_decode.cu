@@ -9,18 +9,19 @@
 //   k_lowrank_z   z = Vᵀ x from V stored transposed: a warp per row of Vt,
 //                 16-byte loads, a fixed shuffle-tree sum (deterministic).
 //                 It triggers the dependent launch at its start.
-//   k_apply_csr   persistent CTAs over row ranges of equal bytes (all layers
-//   k_apply_nm24  of a group concatenated).  x is staged in shared memory as
-//                 [column][token]; S rows are streamed (CSR: G lanes per row;
-//                 2:4: a warp per row) into fp32 sums kept in shared memory;
-//                 then griddepcontrol.wait (programmatic dependent launch:
-//                 the S stream overlaps the z kernel), z is staged, and each
-//                 row adds U[i,:]·z and stores y.
+//   k_apply_decode<T, BC, CSR>  persistent CTAs over row ranges of equal
+//                 bytes (all layers of a group concatenated).  x is staged in
+//                 shared memory as [column][token]; S rows are streamed (CSR:
+//                 G lanes per row; 2:4: a warp per row) into fp32 sums kept in
+//                 shared memory; then griddepcontrol.wait (programmatic
+//                 dependent launch: the S stream overlaps the z kernel), z is
+//                 staged, and each row adds U[i,:]·z and stores y.
 //   k_apply_24_b1_tma  batch 1, bf16 2:4: one CTA of 16 warps per SM (a
-//                 cooperative launch); the CTAs first compute z among them
-//                 (no second launch), then each warp pulls (row, super-chunk)
-//                 units into shared memory with 1-D bulk copies, two in
-//                 flight; same partition and epilogue.
+//                 cooperative launch, no second kernel).  Each warp issues its
+//                 first S unit, then the CTAs compute z among them in pieces;
+//                 each warp pulls (row, super-chunk) units into shared memory
+//                 with 1-D bulk copies, two in flight, and a CTA waits for z
+//                 only before its first U·z pass; same partition and epilogue.
 #include <algorithm>
 #include <cstdlib>
 #include <cstring>

@@ -1,7 +1,9 @@
 // Device code of the magnitude top-k split (see split_topk.cu for the design):
-// radix-digit histogram, digit select, and the two emit kernels (row tickets;
-// blocks of rows held in registers).  Included by the .cu files that launch
-// them; everything here has internal linkage.
+// the sampled bracket (sample histogram, bracket select, count pass, finish,
+// per-tile counts and their scan), the radix-digit histogram and digit
+// select, and the two emit kernels (k_split_emit: one row per ticket;
+// k_split_emit_tile: tiles staged in shared memory by bulk copies).  Included
+// by the .cu files that launch them; everything here has internal linkage.
 #pragma once
 
 #include "common.cuh"

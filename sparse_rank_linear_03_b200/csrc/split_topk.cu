@@ -17,18 +17,21 @@
 //      packed compares and histograms only the keys inside it.  If T falls
 //      outside, the full histogram pass runs (it and its select are launched
 //      always and return at once when the bracket held T).
-//   2. One emit pass over W, persistent CTAs taking blocks of rows (up to 32K
-//      elements, held in registers) in ticket order.  Each block's counts of
-//      keys > T and keys == T are published and the exclusive prefix over
-//      earlier blocks comes from a decoupled look-back, 32 predecessors per
-//      poll (bounded spin; CTAs only wait on blocks whose tickets were taken
-//      earlier, so they are running).  An element's CSR position is
+//   2. One emit pass over W (k_split_emit_tile).  Persistent CTAs take tiles
+//      of W in ticket order and keep three in flight by 1-D bulk copies into
+//      shared memory.  An element's CSR position is
 //      gt_before + min(need, eq_before), need = k − #(key > T): ties are taken
-//      in linear order.  Per 16-byte vector the masks of keys > T / == T come
-//      from one carry-free packed subtraction per threshold (bf16); the kept
-//      elements are walked by their set bits; the residual is the vector with
-//      those elements zeroed (bit copy, +0.0 where kept).  Rows wider than a
-//      register block use a per-row variant of the same scheme.
+//      in linear order.  A tile's (gt, eq) prefix over the tiles before it comes
+//      from the per-tile counts that the bracket pass recorded (16 KB tiles,
+//      four CTAs per SM), or else from a decoupled look-back (32 KB tiles,
+//      32 predecessors per poll, bounded spin; CTAs only wait on tiles whose
+//      tickets were taken earlier, so those tiles' CTAs are running).  Per
+//      16-byte vector, the masks of keys > T and == T come from one carry-free
+//      packed subtraction per threshold (bf16).  A tile's S entries are written
+//      in output order with coalesced stores.  The kept elements are zeroed in
+//      the staged tile, and a bulk store writes it back as the residual (a bit
+//      copy, +0.0 where kept).  When W or R is not 16-byte aligned, a per-row
+//      variant of the same scheme (k_split_emit) runs instead.
 //   HBM traffic: bf16 2 reads of W + 1 write of R + S; fp32 4 reads.
 #include <algorithm>
 #include <cmath>
