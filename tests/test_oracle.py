@@ -134,6 +134,24 @@ def test_split_topk_bruteforce_8x8(dtype, seed):
             assert R[e] == (0 if e in sel else flat[e])
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("shape", [(1, 9), (9, 1), (3, 7), (5, 4), (2, 2)])
+def test_split_topk_bruteforce_shapes(shape, dtype):
+    """Single rows and columns, rows left empty, every k: the CSR rows come from
+    the brute-force selection (empty rows have equal row_ptr entries)."""
+    m, n = shape
+    W = tie_heavy_f32(m, n, 11 + m) if dtype == "f32" else tie_heavy_bf16(m, n, 11 + m)
+    flat = (W.view(np.uint32) if dtype == "f32" else W).reshape(-1)
+    for k in range(0, m * n + 1):
+        s = oracle.split_topk(W, k / (m * n), dtype)
+        assert s["k"] == k
+        sel = brute_selected(flat, dtype, k)
+        per_row = [sum(1 for e in sel if e // n == i) for i in range(m)]
+        assert np.array_equal(np.diff(s["row_ptr"]), per_row)
+        rows = np.repeat(np.arange(m), np.diff(s["row_ptr"]))
+        assert set((rows * n + s["col"]).tolist()) == sel
+
+
 def test_split_topk_nan_rejected():
     W = np.ones((3, 3), dtype=np.float32)
     W[1, 1] = np.nan
