@@ -84,7 +84,9 @@ hsl_status hsl_create(int64_t m, int64_t n, int32_t r, hsl_format fmt,
 
 /* Release the handle and all device memory it owns.  Waits for the device
  * (cudaDeviceSynchronize on the handle's device) before freeing.  NULL is
- * a no-op. */
+ * a no-op.  The handle is the layer object of [HSS] §Implementation and
+ * operational patterns, which holds (S, U, V) in place of the dense weight;
+ * this ends its life. */
 hsl_status hsl_destroy(hsl_handle h);
 
 /* Stage 1: split W into S (kept in the handle) and the residual.
@@ -119,10 +121,11 @@ hsl_status hsl_split_topk(hsl_handle h, const void* W, hsl_dtype w_dtype,
  *             of val_dtype (f32 → bf16 rounds to nearest even).  col/val may
  *             be NULL when k == 0.
  *   residual: device m×n of w_dtype, or NULL.
- *   status:   device uint32 or NULL; cleared, then OR-ed with 1 for a NaN in
- *             W and 2 for a device wait that gave up.
+ *   status:   device uint32, required (NULL → HSL_ERR_INVALID_ARG): it is the
+ *             only channel for device-detected errors.  Cleared, then OR-ed
+ *             with 1 for a NaN in W and 2 for a device wait that gave up.
  * Scratch: one fixed static device array of about 2.2 MB per GPU (held until
- * the process exits).  Limits: m ≤ 65536 and m·n < 2^31, else
+ * the process exits).  Limits: m ≤ 65536, n ≤ 2^31 − 1 and m·n < 2^31, else
  * HSL_ERR_UNSUPPORTED.  The first call on a device looks the array up with
  * that device current (make it before any stream capture).  All calls share
  * the array, so calls that can overlap on the GPU race: serialise them on one
@@ -133,10 +136,14 @@ hsl_status hsl_split_topk_noalloc(const void* W, int64_t m, int64_t n, hsl_dtype
                                   hsl_stream s);
 
 /* Number of stored sparse values (k for CSR, m·n/2 for NM24; 0 before any
- * split/set).  Host-only, no synchronisation (k is known on the host). */
+ * split/set).  Host-only, no synchronisation (k is known on the host).
+ * [HSS] §Two-stage compression, worked example: the count of kept weights
+ * (52,428 for 5 % of a 1024×1024 matrix) that enters the parameter total. */
 hsl_status hsl_get_nnz(hsl_handle h, int64_t* nnz);
 
 /* Export the canonical S (stream-ordered device→device copies).
+ * [HSS] §Two-stage compression, Stage 1: the kept weights are stored as a
+ * sparse matrix in COO/CSR form; [HASSLE] §3 for the N:M form.
  *   CSR:  row_ptr[m+1] int32, col[nnz] int32 (ascending in each row),
  *         val[nnz] of the handle dtype; nm_idx unused (may be NULL).
  *   NM24: val[m][n/2] (the two kept values of each group, ascending column),
@@ -146,13 +153,14 @@ hsl_status hsl_get_sparse(hsl_handle h, int32_t* row_ptr, int32_t* col,
                           void* val, uint8_t* nm_idx, hsl_stream s);
 
 /* Import a canonical CSR S (same layout as hsl_get_sparse), e.g. from a
- * checkpoint.  Columns must be < n; the handle trusts row_ptr to be
+ * checkpoint ([HSS] §Two-stage compression, Stage 1: S in COO/CSR form).  Columns must be < n; the handle trusts row_ptr to be
  * monotone with row_ptr[0] = 0 and row_ptr[m] = nnz.  CSR handles only.
  * Invalidates any earlier hsl_pack. */
 hsl_status hsl_set_sparse_csr(hsl_handle h, int64_t nnz, const int32_t* row_ptr,
                               const int32_t* col, const void* val, hsl_stream s);
 
-/* Import a canonical 2:4 S (layout as hsl_get_sparse).  NM24 handles only.
+/* Import a canonical 2:4 S (layout as hsl_get_sparse; [HASSLE] §3, N:M
+ * structured sparsity).  NM24 handles only.
  * Invalidates any earlier hsl_pack. */
 hsl_status hsl_set_sparse_nm24(hsl_handle h, const void* val, const uint8_t* nm_idx,
                                hsl_stream s);
@@ -181,30 +189,45 @@ hsl_status hsl_apply(hsl_handle h, const void* X, void* Y, int64_t batch, hsl_st
  * The group refers to the members' packed buffers: re-splitting, re-setting,
  * re-packing or destroying a member invalidates it (hsl_group_apply then
  * returns HSL_ERR_NOT_READY for a re-split member; create the group again).
- * Creating a group uploads its plan on s and synchronises s once. */
+ * Creating a group uploads its plan on s and synchronises s once.
+ * [HSS] §Implementation and operational patterns (operating patterns): layers
+ * are compressed and deployed one by one across a model's attention and MLP
+ * projections; a group applies such a set of layers together. */
 typedef struct hsl_group_s* hsl_group;
 hsl_status hsl_group_create(const hsl_handle* hs, int32_t count, hsl_group* out, hsl_stream s);
 
 /* Y[i] = apply(member i, X[i]) for every member; X[i] is [batch][n_i] and
  * Y[i] is [batch][m_i], device pointers.  The pointer tables are host
- * arrays; they are uploaded to the device only when they change. */
+ * arrays; they are uploaded to the device only when they change.
+ * Each member's product is the forward decomposition of hsl_apply ([HSS]
+ * §Implementation and operational patterns; [SQZ] §1). */
 hsl_status hsl_group_apply(hsl_group g, const void* const* X, void* const* Y, int64_t batch,
                            hsl_stream s);
 
-/* Release the group (synchronises its device first).  NULL is a no-op. */
+/* Release the group (synchronises its device first).  NULL is a no-op.
+ * Same passage as hsl_group_create. */
 hsl_status hsl_group_destroy(hsl_group g);
 
 /* Synchronise s and return, then clear, the device-side error of the handle
- * (HSL_ERR_NAN_INPUT, HSL_ERR_TIMEOUT) — HSL_OK if none. */
+ * (HSL_ERR_NAN_INPUT, HSL_ERR_TIMEOUT) — HSL_OK if none.
+ * [HSS] §Risks and mitigations, risk 1: keep the uncompressed weights as a
+ * fallback for a compressed layer that misbehaves; this call is the detection
+ * half of that, as a status. */
 hsl_status hsl_check(hsl_handle h, hsl_stream s);
 
-/* Static text for a status code. */
+/* Static text for a status code (the statuses of hsl_check and of the
+ * host-side checks; [HSS] §Risks and mitigations, risk 1, the same
+ * detection-and-fallback passage). */
 const char* hsl_status_str(hsl_status st);
 
-/* Detail of the last failing call on this thread ("" if none). */
+/* Detail of the last failing call on this thread ("" if none).  Same
+ * passage as hsl_status_str. */
 const char* hsl_last_message(void);
 
-/* Number of kernels libhsl has launched in this process (all devices). */
+/* Number of kernels libhsl has launched in this process (all devices).
+ * [HSS] §Implementation and operational patterns (actionable suggestions):
+ * profile the compressed layers on the target hardware; this count lets a
+ * profile tell the library's own kernels from everything else. */
 uint64_t hsl_launch_count(void);
 
 #ifdef __cplusplus

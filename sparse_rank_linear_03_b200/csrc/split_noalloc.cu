@@ -19,7 +19,10 @@
 //   * its address is looked up once per device, with that device current, by
 //     the first call made on it (cudaGetSymbolAddress); make that first call
 //     before any stream capture;
-//   * sizes beyond the array (m > kNoAllocMaxRows, or m·n ≥ 2^31) are refused.
+//   * sizes beyond the array (m > kNoAllocMaxRows, n > 2^31 - 1, or m·n ≥ 2^31)
+//     are refused;
+//   * the status word is required: it is the only way a caller learns of a
+//     NaN in W or of a device wait that gave up.
 //
 // The kernels are the ones the handle-based split uses (split_kernels.cuh);
 // only the scratch pointers differ.
@@ -186,7 +189,13 @@ extern "C" hsl_status hsl_split_topk_noalloc(const void* W, int64_t m, int64_t n
     set_message("m and n must be >= 1");
     return HSL_ERR_INVALID_ARG;
   }
-  if (m > kNoAllocMaxRows || m * n >= (int64_t(1) << 31)) {
+  if (!status) {
+    set_message("status is NULL: the no-allocation split reports NaN input and device waits "
+                "that gave up only through it");
+    return HSL_ERR_INVALID_ARG;
+  }
+  // n is bounded before m·n is formed, so the product cannot overflow
+  if (m > kNoAllocMaxRows || n > INT32_MAX || m * n >= (int64_t(1) << 31)) {
     set_message("hsl_split_topk_noalloc handles at most " + std::to_string(kNoAllocMaxRows) +
                 " rows and m*n < 2^31 (its scratch is a fixed static array)");
     return HSL_ERR_UNSUPPORTED;
@@ -200,9 +209,7 @@ extern "C" hsl_status hsl_split_topk_noalloc(const void* W, int64_t m, int64_t n
   DeviceScratch d;
   if (hsl_status e = scratch_for_current_device(d)) return e;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (status) {
-    if (cudaError_t e = cudaMemsetAsync(status, 0, 4, s)) return cuda_fail(e, "status clear");
-  }
+  if (cudaError_t e = cudaMemsetAsync(status, 0, 4, s)) return cuda_fail(e, "status clear");
   if (w_dtype == HSL_BF16) {
     const uint16_t* w = static_cast<const uint16_t*>(W);
     uint16_t* r = static_cast<uint16_t*>(residual);
