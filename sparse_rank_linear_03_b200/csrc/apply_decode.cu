@@ -50,6 +50,8 @@ struct ApplyArgs {
   int32_t z_pieces; // (row, column piece) items of Vt (in-kernel z)
   uint32_t* err;    // error word (bounded waits that gave up)
   unsigned long long* zsync;  // CTAs done with z, CTAs done with the call (in-kernel z)
+  long long spin_limit;       // polls of the z-counter wait before it gives up
+  uint32_t zwait_extra;       // added to the z-counter target (0; 1 only under fault injection)
 };
 
 template <typename T>
@@ -765,8 +767,8 @@ __global__ void __maxnreg__(112) k_apply_24_b1_tma(ApplyArgs a, B1Layout lay) {
       if (!waited) {  // every CTA has written its pieces of z
         if (a.z_pieces > 0 && threadIdx.x == 0) {
           long long spins = 0;
-          while (ld_acquire_u64(&a.zsync[0]) < gridDim.x) {
-            if (++spins > kSpinLimit) {
+          while (ld_acquire_u64(&a.zsync[0]) < gridDim.x + a.zwait_extra) {
+            if (++spins > a.spin_limit) {
               set_error(a.err, kErrTimeout);
               break;
             }
@@ -940,6 +942,16 @@ hsl_status apply_decode_run(ApplyPlan& plan, const void* X, void* Y, const void*
   a.z_pieces = plan.z_pieces;
   a.err = plan.err;
   a.zsync = static_cast<unsigned long long*>(plan.zsync.p);
+  a.spin_limit = kSpinLimit;
+  a.zwait_extra = 0;
+  // HSL_FAULT_INJECT=zwait: the batch-1 2:4 kernel's wait for z gets a target no
+  // CTA count reaches and a short limit, so it gives up, records kErrTimeout
+  // and the kernel finishes its normal path (host-side failure testing of the
+  // timeout status; no copy is in flight on that wait)
+  if (fault_injected("zwait")) {
+    a.zwait_extra = 1;
+    a.spin_limit = 1 << 12;
+  }
   if (plan.dtype == HSL_BF16) return run_typed<__nv_bfloat16>(plan, a, batch, num_sms, s);
   return run_typed<float>(plan, a, batch, num_sms, s);
 }

@@ -25,12 +25,14 @@ hsl_status cuda_fail(cudaError_t e, const char* what) {
   return HSL_ERR_CUDA;
 }
 
-// HSL_FAULT_INJECT=alloc makes every device allocation fail (host-side
-// failure testing; no device fault is involved).
-static bool inject_alloc_failure() {
+// HSL_FAULT_INJECT=alloc makes every device allocation fail; =zwait makes the
+// batch-1 2:4 decode's wait for z give up (host-side failure testing; no
+// device fault is involved).
+bool fault_injected(const char* what) {
   const char* v = std::getenv("HSL_FAULT_INJECT");
-  return v && std::strcmp(v, "alloc") == 0;
+  return v && std::strcmp(v, what) == 0;
 }
+static bool inject_alloc_failure() { return fault_injected("alloc"); }
 
 hsl_status ensure(DevBuf& b, size_t bytes, const char* what) {
   if (bytes <= b.bytes && b.p) return HSL_OK;

@@ -16,6 +16,8 @@ extern std::atomic<uint64_t> g_launches;
 inline void note_launch(int n = 1) { g_launches.fetch_add(uint64_t(n), std::memory_order_relaxed); }
 void set_message(const std::string& s);
 hsl_status cuda_fail(cudaError_t e, const char* what);
+// HSL_FAULT_INJECT=<what> (read on every call): host-side failure testing.
+bool fault_injected(const char* what);
 
 // Grow-only device allocation.
 struct DevBuf {

@@ -83,3 +83,23 @@ def test_bulk_fed_and_register_fed_agree(tmp_path, m, n):
     assert a.shape == (1, m)
     fa, fb = oracle.bits_to_f64(a, "bf16"), oracle.bits_to_f64(b, "bf16")
     assert oracle.rel_err(fa, fb) <= 2 ** -8
+
+
+def test_bounded_wait_gives_up_and_reports_timeout(hsl, monkeypatch):
+    """HSL_FAULT_INJECT=zwait gives the batch-1 kernel's wait for z a target no
+    CTA count reaches: the wait gives up after its bounded polls, the kernel
+    finishes, hsl_check reports HSL_ERR_TIMEOUT, and the context stays usable
+    (the next call, without the injection, is correct)."""
+    c = Case(hsl, 3000, 2048, 16, "nm24", "bf16", 0.5, 77)
+    Xb = c.x(1, 78)
+    monkeypatch.setenv("HSL_FAULT_INJECT", "zwait")
+    c.L.apply(dev(Xb, "bf16"))
+    monkeypatch.delenv("HSL_FAULT_INJECT")
+    with pytest.raises(hsl.HslError) as e:
+        c.L.check()
+    assert e.value.name == "HSL_ERR_TIMEOUT"
+    c.L.check()  # the error word was cleared
+    for _ in range(2):
+        Y = c.L.apply(dev(Xb, "bf16"))
+        c.L.check()
+        assert err_of(c, Y, Xb) <= TOL["bf16"]
