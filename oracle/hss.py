@@ -52,7 +52,7 @@ __all__ = [
     "DTYPES", "bits_to_f64", "f32_to_bf16_bits", "topk_count", "magnitude",
     "split_topk", "split_24", "csr_to_dense", "nm24_to_dense",
     "lowrank_svd", "lowrank_randomized", "reconstruct", "apply",
-    "apply_rows", "rel_err", "param_counts", "nm24_count",
+    "apply_rows", "rel_err", "elem_rel_err", "param_counts", "nm24_count",
 ]
 
 DTYPES = ("f32", "bf16")
@@ -303,6 +303,25 @@ def rel_err(Y: np.ndarray, Y_ref: np.ndarray) -> float:
     den = np.abs(R).max(axis=1)
     den = np.where(den > 0, den, 1.0)
     return float((num / den).max())
+
+
+def elem_rel_err(Y: np.ndarray, Y_ref: np.ndarray, floor: float = 1e-3) -> float:
+    """max over tokens b and outputs i of
+    |Y_bi − Y*_bi| / max(|Y*_bi|, floor · max_i |Y*_bi|).
+
+    The element-wise companion of :func:`rel_err` (the target states a
+    relative error without a norm; reading 11 reports both).  The floor keeps
+    outputs that nearly cancel from dividing by ~0.  A token whose reference
+    row is all zero is compared absolutely.
+    """
+    Y = np.atleast_2d(np.asarray(Y, dtype=np.float64))
+    R = np.atleast_2d(np.asarray(Y_ref, dtype=np.float64))
+    if R.size == 0:
+        return 0.0
+    rowmax = np.abs(R).max(axis=1, keepdims=True)
+    den = np.maximum(np.abs(R), floor * rowmax)
+    den = np.where(den > 0, den, 1.0)
+    return float((np.abs(Y - R) / den).max())
 
 
 # --------------------------------------------------------------------------

@@ -408,6 +408,23 @@ def test_rel_err_definition():
     assert oracle.rel_err(np.zeros((0, 3)), np.zeros((0, 3))) == 0.0
 
 
+def test_elem_rel_err_definition():
+    """Hand-computed: row max 10, floor 1e-3 → denominators max(|y*|, 0.01)."""
+    R = np.array([[10.0, -0.001, 2.0, 0.0]])
+    Y = np.array([[10.1, 0.0, 2.0, 0.002]])
+    # 0.1/10, 0.001/0.01, 0/2, 0.002/0.01 → 0.2 from the last column
+    assert oracle.elem_rel_err(Y, R) == pytest.approx(0.2, rel=1e-12)
+    assert oracle.elem_rel_err(Y[:, :3], R[:, :3]) == pytest.approx(0.1, rel=1e-12)
+    # a zero reference row is compared absolutely; empty input is 0
+    assert oracle.elem_rel_err(np.array([[0.5, 0.0]]), np.zeros((1, 2))) == 0.5
+    assert oracle.elem_rel_err(np.zeros((0, 3)), np.zeros((0, 3))) == 0.0
+    # never below the normwise measure (each denominator is at most the row max)
+    rng = np.random.default_rng(3)
+    A = rng.standard_normal((4, 50))
+    B = A + 1e-3 * rng.standard_normal((4, 50))
+    assert oracle.elem_rel_err(B, A) >= oracle.rel_err(B, A)
+
+
 # ---------------------------------------------------------------- planted mistakes
 
 def test_pins_catch_planted_tie_break_bug(monkeypatch):
