@@ -12,6 +12,8 @@ Each case builds its layer once (split + pack), then repeats one operation
   split24_70b   2:4 split of the same W
   attn4096      CSR apply, batch 1, 4096×4096 bf16 at 2 %, r = 128
   stack7b       the 224-matrix CSR group at batch 1 (all 32 layers)
+  stack7b_4     the first 4 layers of it (28 matrices, 178 MB: above L2, small
+                enough for a full ncu capture)
 """
 from __future__ import annotations
 
@@ -66,11 +68,15 @@ def case(name: str):
         X = _bf(synth.normal_f32(1, lay.n, lay.seed + 1))
         Y = torch.empty(1, lay.m, dtype=torch.bfloat16, device="cuda")
         return lambda: L.apply(X, Y), (L,)
-    if name == "stack7b":
+    if name in ("stack7b", "stack7b_4"):
+        # W drawn on the device (6.5 G entries take minutes on the host)
         layers, Xs, Ys = [], [], []
-        for lay in STACK7B.layers:
-            L, W = _layer(lay, STACK7B.r, "csr", STACK7B.frac, "f32")
+        for lay in STACK7B.layers[:28 if name == "stack7b_4" else None]:
+            W = synth.student_t_device(lay.m, lay.n, lay.seed, "cuda")
+            L = hsl.Layer(lay.m, lay.n, STACK7B.r, "csr", "bf16")
+            L.split(W, STACK7B.frac, None)
             del W
+            L.pack(*synth.stand_in_factors_device(lay.m, lay.n, STACK7B.r, lay.seed + 2, "cuda"))
             layers.append(L)
             Xs.append(_bf(synth.normal_f32(1, lay.n, lay.seed + 1)))
             Ys.append(torch.empty(1, lay.m, dtype=torch.bfloat16, device="cuda"))

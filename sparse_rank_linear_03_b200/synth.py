@@ -13,6 +13,10 @@ evaluation data are used):
   weights.  bf16 layers round that float32 once more to bfloat16 (RNE).
 * X ~ N(0, 1) from ``default_rng(seed + 1).standard_normal((B, n))``, rounded
   to the layer's dtype.
+* The 224-matrix 7B stack in the bench draws W on the device instead
+  (:func:`student_t_device`, torch's seeded CUDA generator: t₃ = N / √(χ²₃/3)
+  with χ²₃ the sum of three squared normals), because drawing its 6.5 G
+  entries on the host takes minutes; it is the same distribution.
 * Bench-side stand-in factors: U, V with i.i.d. N(0, s²) entries from
   ``default_rng(seed + 2)`` (s chosen so that (U Vᵀ)ᵢⱼ has standard deviation
   about 0.01).  Throughput does not depend on the factor values; the tests use
@@ -84,3 +88,23 @@ def storage_from_torch(t: torch.Tensor) -> np.ndarray:
     if t.dtype == torch.bfloat16:
         return t.view(torch.int16).numpy().view(np.uint16).copy()
     return t.numpy().copy()
+
+
+def student_t_device(m: int, n: int, seed: int, device, scale: float = 0.02) -> torch.Tensor:
+    """0.02 · t₃ as float32 on `device`, from torch's seeded generator there."""
+    g = torch.Generator(device=device).manual_seed(seed)
+    z = torch.randn(m, n, generator=g, device=device)
+    chi2 = torch.zeros(m, n, device=device)
+    for _ in range(3):
+        chi2.add_(torch.randn(m, n, generator=g, device=device).square_())
+    return (scale * z * torch.rsqrt(chi2 / 3.0)).contiguous()
+
+
+def stand_in_factors_device(m: int, n: int, r: int, seed: int, device, dtype=torch.bfloat16,
+                            target_std: float = 0.01):
+    """Device twin of :func:`stand_in_factors` (same scale, torch's generator)."""
+    g = torch.Generator(device=device).manual_seed(seed)
+    s = (target_std ** 2 / max(r, 1)) ** 0.25 if r else 0.0
+    U = (s * torch.randn(m, r, generator=g, device=device)).to(dtype)
+    V = (s * torch.randn(n, r, generator=g, device=device)).to(dtype)
+    return U.contiguous(), V.contiguous()
