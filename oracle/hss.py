@@ -53,6 +53,7 @@ __all__ = [
     "split_topk", "split_24", "csr_to_dense", "nm24_to_dense",
     "lowrank_svd", "lowrank_randomized", "reconstruct", "apply",
     "apply_rows", "rel_err", "elem_rel_err", "param_counts", "nm24_count",
+    "concentration", "rcm_order", "permute",
 ]
 
 DTYPES = ("f32", "bf16")
@@ -348,3 +349,82 @@ def param_counts(m: int, n: int, frac: float, r: int) -> dict:
         "reduction": (m * n) / total if total else math.inf,
         "residual_footprint_reduction": 1.0 - factor / resid if resid else 0.0,
     }
+
+
+# --------------------------------------------------------------------------
+# Permutation for concentration (a pre-processing step before Stage 1).
+# --------------------------------------------------------------------------
+
+def concentration(W: np.ndarray, dtype: str) -> float:
+    """ρ = Σ_{(i,j) in the diagonal blocks} |W_ij| / Σ_{i,j} |W_ij|.
+
+    [HSS] §Permutation and hierarchical alignment: the concentration ratio of
+    the equation there, with "diagonal" the top-left and bottom-right blocks
+    of the 2×2 block partition (the example names those two quadrants).
+    Readings: the quadrants split at row ⌊m/2⌋ and column ⌊n/2⌋ (top-left =
+    rows < ⌊m/2⌋ and columns < ⌊n/2⌋, bottom-right = the rest of both); an
+    all-zero W has ρ = 0.
+    """
+    A = magnitude(W, dtype)
+    m, n = A.shape
+    mh, nh = m // 2, n // 2
+    total = A.sum()
+    if total == 0:
+        return 0.0
+    diag = A[:mh, :nh].sum() + A[mh:, nh:].sum()
+    return float(diag / total)
+
+
+def rcm_order(m: int, n: int, row_ptr, col) -> tuple[np.ndarray, np.ndarray]:
+    """Reverse Cuthill–McKee order of the rows and columns of a sparse pattern.
+
+    [HSS] §Permutation and hierarchical alignment: RCM reorders rows and
+    columns so that the large entries gather near the diagonal (Cuthill &
+    McKee's bandwidth-reducing ordering, reversed).  Reading for an m×n
+    pattern: the graph is the bipartite row–column graph (vertex i < m is row
+    i, vertex m + j is column j, an edge per stored entry), which needs no
+    symmetric matrix; the order of its m + n vertices gives the row order and
+    the column order.  The steps, in the classic form: take the unvisited
+    vertex of smallest degree (ties: lowest vertex number) as the start of
+    the next component; visit breadth first, appending each vertex's
+    unvisited neighbours by increasing degree (ties: lowest vertex number);
+    reverse the whole order at the end.
+
+    Returns (row_order, col_order): row_order[k] is the original row placed
+    k-th, col_order[k] the original column placed k-th.
+    """
+    rp = np.asarray(row_ptr, dtype=np.int64)
+    cl = np.asarray(col, dtype=np.int64)
+    V = m + n
+    adj = [[] for _ in range(V)]
+    for i in range(m):
+        for j in cl[rp[i]:rp[i + 1]]:
+            adj[i].append(m + int(j))
+            adj[m + int(j)].append(i)
+    deg = [len(a) for a in adj]
+    visited = [False] * V
+    order = []
+    by_degree = sorted(range(V), key=lambda v: (deg[v], v))
+    for start in by_degree:
+        if visited[start]:
+            continue
+        visited[start] = True
+        queue = [start]
+        head = 0
+        while head < len(queue):
+            v = queue[head]
+            head += 1
+            fresh = sorted({u for u in adj[v] if not visited[u]}, key=lambda u: (deg[u], u))
+            for u in fresh:
+                visited[u] = True
+                queue.append(u)
+        order.extend(queue)
+    order.reverse()
+    rows = np.array([v for v in order if v < m], dtype=np.int32)
+    cols = np.array([v - m for v in order if v >= m], dtype=np.int32)
+    return rows, cols
+
+
+def permute(W: np.ndarray, row_order, col_order) -> np.ndarray:
+    """W' with W'[k, l] = W[row_order[k], col_order[l]] (bits copied)."""
+    return np.ascontiguousarray(np.asarray(W)[np.asarray(row_order)][:, np.asarray(col_order)])

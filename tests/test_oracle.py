@@ -467,3 +467,127 @@ def test_pins_catch_dropped_lowrank_term():
     ref = _triple_loop(D.tolist(), U.tolist(), V.tolist(), X.tolist())
     assert np.abs(oracle.apply(D, X) - ref).max() > 1e-6       # S-only is wrong
     assert np.abs(oracle.apply(oracle.reconstruct(D, U, V), X) - ref).max() < 1e-12
+
+
+# ---------------------------------------------------------------- concentration and RCM
+
+def test_concentration_hand_example():
+    """4×4, quadrants split at row 2 and column 2: diagonal blocks hold
+    |1|+|-2|+|3|+|4| + |5|+|6|+|-7|+|8| = 36 of a total 36 + 10 = 46."""
+    W = np.array([[1, -2, 1, 0],
+                  [3, 4, 0, -2],
+                  [0, 3, 5, 6],
+                  [-4, 0, -7, 8]], dtype=np.float32)
+    assert oracle.concentration(W, "f32") == pytest.approx(36 / 46, rel=1e-15)
+
+
+@pytest.mark.parametrize("m,n", [(4, 4), (5, 7), (1, 9), (512, 512), (3, 1)])
+def test_concentration_uniform_magnitude_closed_form(m, n):
+    """Equal |w| everywhere: ρ is the share of entries in the two blocks,
+    (⌊m/2⌋⌊n/2⌋ + ⌈m/2⌉⌈n/2⌉)/(m n), whatever the signs."""
+    rng = np.random.default_rng(m * n)
+    W = np.where(rng.random((m, n)) < 0.5, -0.25, 0.25).astype(np.float32)
+    mh, nh = m // 2, n // 2
+    want = (mh * nh + (m - mh) * (n - nh)) / (m * n)
+    assert oracle.concentration(W, "f32") == pytest.approx(want, rel=1e-15)
+    assert oracle.concentration(synth.to_bf16_bits(W), "bf16") == pytest.approx(want, rel=1e-15)
+
+
+def test_concentration_block_extremes_and_zero():
+    D = np.zeros((6, 8), np.float32)
+    D[:3, :4] = 1.0
+    D[3:, 4:] = -2.0
+    assert oracle.concentration(D, "f32") == 1.0
+    assert oracle.concentration(D[:, ::-1].copy(), "f32") == 0.0     # mass off the diagonal
+    assert oracle.concentration(np.zeros((3, 3), np.float32), "f32") == 0.0
+
+
+def test_permute_definition():
+    W = np.arange(12, dtype=np.float32).reshape(3, 4)
+    ro, co = [2, 0, 1], [3, 1, 0, 2]
+    P = oracle.permute(W, ro, co)
+    for k in range(3):
+        for l in range(4):
+            assert P[k, l] == W[ro[k], co[l]]
+
+
+def _csr_of(mask):
+    m = mask.shape[0]
+    rp = np.zeros(m + 1, np.int64)
+    rp[1:] = np.cumsum(mask.sum(axis=1))
+    return rp, np.nonzero(mask)[1]
+
+
+def test_rcm_returns_permutations():
+    rng = np.random.default_rng(5)
+    mask = rng.random((40, 30)) < 0.08
+    ro, co = oracle.rcm_order(40, 30, *_csr_of(mask))
+    assert sorted(ro.tolist()) == list(range(40)) and sorted(co.tolist()) == list(range(30))
+
+
+def _scipy_rcm_bipartite(mask):
+    from scipy.sparse import bmat, csr_matrix
+    from scipy.sparse.csgraph import reverse_cuthill_mckee
+    S = csr_matrix(mask.astype(np.int8))
+    G = bmat([[None, S], [S.T, None]], format="csr")
+    G.sort_indices()
+    return reverse_cuthill_mckee(G, symmetric_mode=True)
+
+
+def test_rcm_matches_scipy_where_the_start_is_unique():
+    """scipy's reverse_cuthill_mckee on the bipartite graph follows the same
+    steps; its choice among equal-degree start vertices is its sort's, so the
+    comparison uses connected graphs whose smallest degree is held by one
+    vertex (neighbour ties are broken by vertex number on both sides)."""
+    rng = np.random.default_rng(11)
+    checked = 0
+    for trial in range(400):
+        m, n = int(rng.integers(3, 25)), int(rng.integers(3, 25))
+        mask = rng.random((m, n)) < rng.uniform(0.1, 0.5)
+        deg = np.concatenate([mask.sum(1), mask.sum(0)])
+        if deg.min() == 0 or (deg == deg.min()).sum() != 1:
+            continue
+        from scipy.sparse import csr_matrix, bmat
+        from scipy.sparse.csgraph import connected_components
+        G = bmat([[None, csr_matrix(mask)], [csr_matrix(mask).T, None]])
+        if connected_components(G, directed=False)[0] != 1:
+            continue
+        ref = _scipy_rcm_bipartite(mask)
+        ro, co = oracle.rcm_order(m, n, *_csr_of(mask))
+        assert np.array_equal(ro, ref[ref < m]), trial
+        assert np.array_equal(co, ref[ref >= m] - m), trial
+        checked += 1
+    assert checked >= 20
+
+
+def test_rcm_gathers_a_hidden_block_diagonal():
+    """Two dense blocks hidden by random row and column permutations: the
+    RCM order makes each block contiguous again, so ρ of the permuted
+    pattern is 1 (the blocks are the two diagonal quadrants)."""
+    rng = np.random.default_rng(2)
+    B = np.zeros((16, 12), bool)
+    B[:8, :6] = rng.random((8, 6)) < 0.6
+    B[8:, 6:] = rng.random((8, 6)) < 0.6
+    B[0, :6] = B[8, 6:] = True          # every row and column has an entry
+    B[:8, 0] = B[8:, 6] = True
+    pr, pc = rng.permutation(16), rng.permutation(12)
+    H = B[pr][:, pc]
+    ro, co = oracle.rcm_order(16, 12, *_csr_of(H))
+    P = oracle.permute(H.astype(np.float32), ro, co)
+    assert oracle.concentration(P, "f32") == 1.0
+    assert oracle.concentration(H.astype(np.float32), "f32") < 0.8
+
+
+def test_pins_catch_an_unreversed_order():
+    """Cuthill–McKee without the final reversal (a plausible slip) fails the
+    scipy comparison on a graph whose order is not a palindrome."""
+    rng = np.random.default_rng(4)
+    for _ in range(500):
+        mask = rng.random((9, 7)) < 0.35
+        deg = np.concatenate([mask.sum(1), mask.sum(0)])
+        if deg.min() > 0 and (deg == deg.min()).sum() == 1:
+            break
+    ref = _scipy_rcm_bipartite(mask)
+    ro, co = oracle.rcm_order(9, 7, *_csr_of(mask))
+    assert np.array_equal(ro, ref[ref < 9])
+    assert not np.array_equal(ro[::-1], ref[ref < 9])
