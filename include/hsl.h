@@ -208,6 +208,48 @@ hsl_status hsl_group_apply(hsl_group g, const void* const* X, void* const* Y, in
  * Same passage as hsl_group_create. */
 hsl_status hsl_group_destroy(hsl_group g);
 
+/* ---- Permutation for concentration ------------------------------------------
+ * [HSS] §Permutation and hierarchical alignment: reorder the rows and columns
+ * of W (reverse Cuthill–McKee) so that its large entries gather near the
+ * diagonal, measure the gain with the concentration ratio
+ *   ρ = Σ_{diagonal blocks} |W_ij| / Σ |W_ij|,
+ * and keep the order so the layer is applied in the original order. */
+
+/* ρ of W (device, m×n row-major, dtype): the diagonal blocks are the top-left
+ * and bottom-right blocks of the 2×2 partition split at row ⌊m/2⌋ and column
+ * ⌊n/2⌋; an all-zero W gives 0, a NaN in W gives NaN.  Sums in fp64 in a fixed
+ * order (deterministic).  Writes *rho (host) and synchronises s.  Allocates a
+ * small workspace for the call and frees it. */
+hsl_status hsl_concentration(const void* W, int64_t m, int64_t n, hsl_dtype dtype, double* rho,
+                             hsl_stream s);
+
+/* Reverse Cuthill–McKee order of an m×n sparse pattern given as a HOST CSR
+ * (row_ptr[m+1] from 0, col[row_ptr[m]] in [0, n)).  The graph is the
+ * bipartite row–column graph (an edge per stored entry); start each component
+ * at the unvisited vertex of least degree (ties: rows before columns, lower
+ * index first), visit breadth first taking neighbours by increasing degree
+ * (same ties), reverse the whole order.  row_order[k] / col_order[k] (host,
+ * m and n int32) receive the original row / column placed k-th.  Runs on the
+ * host (a one-off graph step); HSL_ERR_INVALID_ARG for a bad pattern. */
+hsl_status hsl_rcm_order(int64_t m, int64_t n, const int32_t* row_ptr, const int32_t* col,
+                         int32_t* row_order, int32_t* col_order);
+
+/* out[k][l] = W[row_order[k]][col_order[l]] (device arrays; bit copies).  The
+ * orders are copied to the host and checked to be permutations first
+ * (HSL_ERR_INVALID_ARG otherwise), which synchronises s. */
+hsl_status hsl_permute(const void* W, int64_t m, int64_t n, hsl_dtype dtype,
+                       const int32_t* row_order, const int32_t* col_order, void* out,
+                       hsl_stream s);
+
+/* Declare that the handle holds the permuted layer W' = W[row_order][:, col_order]
+ * (split, set and packed from W'), so that hsl_apply returns the original
+ * layer's output: x' = x[col_order], y' = Ŵ' x', y[row_order[k]] = y'[k].
+ * Device arrays, copied into the handle after a host-side permutation check
+ * (synchronises s).  NULL for both clears it.  Groups do not take permuted
+ * layers. */
+hsl_status hsl_set_permutation(hsl_handle h, const int32_t* row_order, const int32_t* col_order,
+                               hsl_stream s);
+
 /* Synchronise s and return, then clear, the device-side error of the handle
  * (HSL_ERR_NAN_INPUT, HSL_ERR_TIMEOUT) — HSL_OK if none.
  * [HSS] §Risks and mitigations, risk 1: keep the uncompressed weights as a

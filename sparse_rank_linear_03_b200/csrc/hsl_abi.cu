@@ -98,6 +98,24 @@ struct DeviceGuard {
   }
 };
 
+// A device array of `len` int32 that must hold each of 0..len-1 once: copied to
+// the host and checked there (the permutation calls are one-off set-up steps).
+hsl_status check_order(const int32_t* order_dev, int64_t len, const char* what, cudaStream_t s) {
+  std::vector<int32_t> h(static_cast<size_t>(len));
+  if (cudaError_t e = cudaMemcpyAsync(h.data(), order_dev, size_t(len) * 4, cudaMemcpyDefault, s))
+    return cuda_fail(e, "order copy");
+  if (cudaError_t e = cudaStreamSynchronize(s)) return cuda_fail(e, "order copy");
+  std::vector<char> seen(static_cast<size_t>(len), 0);
+  for (int32_t v : h) {
+    if (v < 0 || v >= len || seen[size_t(v)]) {
+      set_message(std::string(what) + " is not a permutation of 0.." + std::to_string(len - 1));
+      return HSL_ERR_INVALID_ARG;
+    }
+    seen[size_t(v)] = 1;
+  }
+  return HSL_OK;
+}
+
 hsl_status ensure_err_word(Handle& h, cudaStream_t s) {
   if (h.err.p) return HSL_OK;
   if (hsl_status e = ensure(h.err, 256, "error word")) return e;
@@ -107,7 +125,7 @@ hsl_status ensure_err_word(Handle& h, cudaStream_t s) {
 void free_all(Handle& h) {
   DevBuf* bufs[] = {&h.row_ptr, &h.col, &h.val, &h.nm_val, &h.nm_idx, &h.prow, &h.pcol,
                     &h.pval, &h.pmeta, &h.pmeta_tc, &h.U, &h.Vt, &h.z,
-                    &h.err, &h.split_ws, &h.flags, &h.tiles, &h.xstage, &h.ystage, &h.zpre, &h.plan.probs,
+                    &h.err, &h.split_ws, &h.flags, &h.tiles, &h.xstage, &h.ystage, &h.zpre, &h.sk_part, &h.sk_cnt, &h.sk_z, &h.perm_row, &h.perm_col, &h.xperm, &h.yperm, &h.plan.probs,
                     &h.plan.prob_row0, &h.plan.cta_rows, &h.plan.xy_ptrs, &h.plan.zsync};
   for (DevBuf* b : bufs) release(*b);
 }
@@ -375,10 +393,29 @@ hsl_status hsl_apply(hsl_handle h, const void* X, void* Y, int64_t batch, hsl_st
     if (hsl_status e = ensure(H.ystage, size_t(batch) * H.m * eb, "Y staging")) return e;
     Yd = H.ystage.p;
   }
+  // permuted layer: x' = x[col_order], y' = Ŵ' x', y[row_order] = y'
+  void* Yout = Yd;
+  if (H.permuted) {
+    if (hsl_status e = ensure(H.xperm, size_t(batch) * H.n * eb, "permuted X")) return e;
+    if (hsl_status e = ensure(H.yperm, size_t(batch) * H.m * eb, "permuted Y")) return e;
+    if (hsl_status e = gather_cols_run(Xd, batch, H.n, H.dtype,
+                                       static_cast<const int32_t*>(H.perm_col.p), H.xperm.p, s))
+      return e;
+    Xd = H.xperm.p;
+    Yd = H.yperm.p;
+  }
   if (batch >= kPrefillMinBatch && prefill_supported(H, Xd)) {
     if (hsl_status e = apply_prefill_run(H, Xd, Yd, batch, s)) return e;
+  } else if (splitk_supported(H, Xd, batch)) {
+    if (hsl_status e = apply_splitk_run(H, Xd, Yd, batch, s)) return e;
   } else {
     if (hsl_status e = apply_decode_run(H.plan, Xd, Yd, nullptr, batch, H.num_sms, s)) return e;
+  }
+  if (H.permuted) {
+    if (hsl_status e = scatter_rows_run(Yd, batch, H.m, H.dtype,
+                                        static_cast<const int32_t*>(H.perm_row.p), Yout, s))
+      return e;
+    Yd = Yout;
   }
   if (yh)
     return cuda_fail(cudaMemcpyAsync(Y, Yd, size_t(batch) * H.m * eb, cudaMemcpyDeviceToHost, s),
@@ -400,6 +437,7 @@ hsl_status hsl_group_create(const hsl_handle* hs, int32_t count, hsl_group* out,
     if (hs[i]->h.dtype != hs[0]->h.dtype || hs[i]->h.fmt != hs[0]->h.fmt)
       return unsupported("a group needs one format and one dtype");
     if (hs[i]->h.device != hs[0]->h.device) return unsupported("a group lives on one device");
+    if (hs[i]->h.permuted) return unsupported("a group does not take permuted layers");
   }
   hsl_group g = new (std::nothrow) hsl_group_s;
   if (!g) return invalid("host allocation failed");
@@ -463,6 +501,79 @@ hsl_status hsl_group_destroy(hsl_group g) {
     cudaGetLastError();
   }
   delete g;
+  return HSL_OK;
+}
+
+hsl_status hsl_concentration(const void* W, int64_t m, int64_t n, hsl_dtype dtype, double* rho,
+                             hsl_stream stream) {
+  t_msg.clear();
+  if (!W || !rho) return invalid("W/rho is NULL");
+  if (m < 1 || n < 1) return invalid("m and n must be >= 1");
+  if (dtype != HSL_F32 && dtype != HSL_BF16) return invalid("unknown dtype");
+  if (m > INT32_MAX || n > INT32_MAX || m * n >= (int64_t(1) << 40))
+    return unsupported("matrix too large");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int blocks = concentration_blocks(m);
+  DevBuf ws;
+  if (hsl_status e = ensure(ws, size_t(blocks) * 16 + 64, "concentration workspace")) return e;
+  double* out = static_cast<double*>(ws.p);
+  hsl_status st = concentration_run(W, m, n, dtype, out, out + 8, blocks, s);
+  double res[3] = {0.0, 0.0, 0.0};
+  if (st == HSL_OK) {
+    if (cudaError_t e = cudaMemcpyAsync(res, out, sizeof(res), cudaMemcpyDeviceToHost, s))
+      st = cuda_fail(e, "concentration result");
+    else if (cudaError_t e2 = cudaStreamSynchronize(s))
+      st = cuda_fail(e2, "concentration result");
+  }
+  release(ws);
+  if (st == HSL_OK) *rho = res[2];
+  return st;
+}
+
+hsl_status hsl_rcm_order(int64_t m, int64_t n, const int32_t* row_ptr, const int32_t* col,
+                         int32_t* row_order, int32_t* col_order) {
+  t_msg.clear();
+  if (!row_ptr || !row_order || !col_order) return invalid("NULL argument");
+  if (m < 1 || n < 1 || m > INT32_MAX || n > INT32_MAX) return invalid("m and n out of range");
+  if (row_ptr[0] != 0 || row_ptr[m] < 0) return invalid("row_ptr must start at 0");
+  if (row_ptr[m] > 0 && !col) return invalid("col is NULL");
+  return rcm_order(m, n, row_ptr, col, row_order, col_order);
+}
+
+hsl_status hsl_permute(const void* W, int64_t m, int64_t n, hsl_dtype dtype,
+                       const int32_t* row_order, const int32_t* col_order, void* out,
+                       hsl_stream stream) {
+  t_msg.clear();
+  if (!W || !row_order || !col_order || !out) return invalid("NULL argument");
+  if (m < 1 || n < 1 || m > INT32_MAX || n > INT32_MAX) return invalid("m and n out of range");
+  if (dtype != HSL_F32 && dtype != HSL_BF16) return invalid("unknown dtype");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (hsl_status e = check_order(row_order, m, "row_order", s)) return e;
+  if (hsl_status e = check_order(col_order, n, "col_order", s)) return e;
+  return permute_run(W, m, n, dtype, row_order, col_order, out, s);
+}
+
+hsl_status hsl_set_permutation(hsl_handle h, const int32_t* row_order, const int32_t* col_order,
+                               hsl_stream stream) {
+  t_msg.clear();
+  if (!h) return invalid("handle is NULL");
+  Handle& H = h->h;
+  if (!row_order && !col_order) {
+    H.permuted = false;
+    return HSL_OK;
+  }
+  if (!row_order || !col_order) return invalid("give both orders, or neither");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  DeviceGuard g(H.device);
+  if (hsl_status e = check_order(row_order, H.m, "row_order", s)) return e;
+  if (hsl_status e = check_order(col_order, H.n, "col_order", s)) return e;
+  if (hsl_status e = ensure(H.perm_row, size_t(H.m) * 4, "row order")) return e;
+  if (hsl_status e = ensure(H.perm_col, size_t(H.n) * 4, "column order")) return e;
+  if (cudaError_t e = cudaMemcpyAsync(H.perm_row.p, row_order, size_t(H.m) * 4, cudaMemcpyDefault, s))
+    return cuda_fail(e, "row order copy");
+  if (cudaError_t e = cudaMemcpyAsync(H.perm_col.p, col_order, size_t(H.n) * 4, cudaMemcpyDefault, s))
+    return cuda_fail(e, "column order copy");
+  H.permuted = true;
   return HSL_OK;
 }
 

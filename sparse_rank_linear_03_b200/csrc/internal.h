@@ -1,6 +1,7 @@
 // Host-side internals of libhsl: the handle, device buffers, kernel launchers.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -99,6 +100,10 @@ struct Handle {
   DevBuf z, err, split_ws, flags;
   DevBuf tiles;  // per-tile counts of the sampled-bracket split
   DevBuf xstage, ystage, zpre;
+  DevBuf sk_part, sk_cnt, sk_z;  // split-K small-batch apply: partial tiles, tile counters, z
+  // permuted apply: the layer holds W' = W[row_order][:, col_order]
+  DevBuf perm_row, perm_col, xperm, yperm;
+  bool permuted = false;
   ApplyPlan plan;  // the single-layer plan, built by hsl_pack
 };
 
@@ -114,9 +119,32 @@ hsl_status plan_build(ApplyPlan& plan, Handle* const* hs, int count, cudaStream_
 hsl_status apply_decode_run(ApplyPlan& plan, const void* X, void* Y, const void* const* xy_dev,
                             int64_t batch, int num_sms, cudaStream_t s);
 // tensor-core path for large batches (2:4, bf16, n % 64 == 0)
-constexpr int64_t kPrefillMinBatch = 16;
+constexpr int64_t kPrefillMinBatch = 65;
 bool prefill_supported(const Handle& h, const void* X);
 hsl_status apply_prefill_run(Handle& h, const void* X, void* Y, int64_t T, cudaStream_t s);
+// small batches (2..64 tokens) of the same layers: sparse tensor cores with K
+// split across every SM (apply_splitk.cu)
+constexpr int64_t kSplitKMinBatch = 2, kSplitKMaxBatch = 64;
+bool splitk_supported(const Handle& h, const void* X, int64_t T);
+hsl_status apply_splitk_run(Handle& h, const void* X, void* Y, int64_t T, cudaStream_t s);
+// permutation for concentration (permute.cu)
+hsl_status concentration_run(const void* W, int64_t m, int64_t n, hsl_dtype dt, double* out_dev,
+                             double* partial, int blocks, cudaStream_t s);
+int concentration_blocks(int64_t m);
+hsl_status permute_run(const void* W, int64_t m, int64_t n, hsl_dtype dt, const int32_t* row_order,
+                       const int32_t* col_order, void* out, cudaStream_t s);
+hsl_status gather_cols_run(const void* x, int64_t batch, int64_t n, hsl_dtype dt,
+                           const int32_t* order, void* out, cudaStream_t s);
+hsl_status scatter_rows_run(const void* yp, int64_t batch, int64_t m, hsl_dtype dt,
+                            const int32_t* order, void* y, cudaStream_t s);
+hsl_status rcm_order(int64_t m, int64_t n, const int32_t* row_ptr, const int32_t* col,
+                     int32_t* row_order, int32_t* col_order);
+// 2-D row-major TMA map: rows × cols elements, box {box_cols, box_rows}
+// (apply_prefill.cu); false when the driver entry point or the encoding fails.
+bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dt, int esize, const void* base,
+                  int64_t rows, int64_t cols, int64_t row_stride_elems, int box_cols,
+                  int box_rows, CUtensorMapSwizzle sw);
+bool tmap_available();
 
 }  // namespace hsl
 

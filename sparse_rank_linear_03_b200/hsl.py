@@ -27,6 +27,7 @@ EXPORTS = (
     "hsl_set_sparse_csr", "hsl_set_sparse_nm24", "hsl_pack", "hsl_apply",
     "hsl_group_create", "hsl_group_apply", "hsl_group_destroy", "hsl_check",
     "hsl_status_str", "hsl_last_message", "hsl_launch_count", "hsl_split_topk_noalloc",
+    "hsl_concentration", "hsl_rcm_order", "hsl_permute", "hsl_set_permutation",
 )
 
 
@@ -61,6 +62,10 @@ def _load() -> ctypes.CDLL:
         "hsl_last_message": [],
         "hsl_launch_count": [],
         "hsl_split_topk_noalloc": [P, I64, I64, ctypes.c_int, D, P, P, P, ctypes.c_int, P, P, P],
+        "hsl_concentration": [P, I64, I64, ctypes.c_int, ctypes.POINTER(D), P],
+        "hsl_rcm_order": [I64, I64, P, P, P, P],
+        "hsl_permute": [P, I64, I64, ctypes.c_int, P, P, P, P],
+        "hsl_set_permutation": [P, P, P, P],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -104,6 +109,44 @@ def _need(t, numel: int, what: str) -> None:
 def _dtype_of(t, want: str, what: str) -> None:
     if isinstance(t, torch.Tensor) and t.dtype != TORCH_DTYPE[want]:
         raise ValueError(f"{what} is {t.dtype}, the layer stores {want}")
+
+
+def _wdtype(t: torch.Tensor) -> str:
+    return {torch.float32: "f32", torch.bfloat16: "bf16"}[t.dtype]
+
+
+def concentration(W: torch.Tensor, stream=None) -> float:
+    """ρ of a device matrix W (hsl_concentration)."""
+    m, n = W.shape
+    rho = ctypes.c_double()
+    _ok(lib.hsl_concentration(_ptr(W), m, n, DTYPE[_wdtype(W)], ctypes.byref(rho), _stream(stream)),
+        "hsl_concentration")
+    return rho.value
+
+
+def rcm_order(m: int, n: int, row_ptr, col):
+    """RCM row and column orders of a CSR pattern (hsl_rcm_order; host arrays)."""
+    import numpy as np
+    rp = np.ascontiguousarray(np.asarray(row_ptr, dtype=np.int32))
+    cl = np.ascontiguousarray(np.asarray(col, dtype=np.int32))
+    ro = np.empty(m, np.int32)
+    co = np.empty(n, np.int32)
+    _ok(lib.hsl_rcm_order(m, n, rp.ctypes.data, cl.ctypes.data if cl.size else None,
+                          ro.ctypes.data, co.ctypes.data), "hsl_rcm_order")
+    return ro, co
+
+
+def permute(W: torch.Tensor, row_order: torch.Tensor, col_order: torch.Tensor,
+            out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """out[k][l] = W[row_order[k]][col_order[l]] on the device (hsl_permute)."""
+    m, n = W.shape
+    _need(row_order, m, "row_order")
+    _need(col_order, n, "col_order")
+    if out is None:
+        out = torch.empty_like(W)
+    _ok(lib.hsl_permute(_ptr(W), m, n, DTYPE[_wdtype(W)], _ptr(row_order), _ptr(col_order),
+                        _ptr(out), _stream(stream)), "hsl_permute")
+    return out
 
 
 def launch_count() -> int:
@@ -201,6 +244,14 @@ class Layer:
                             pin_memory=(X.device.type == "cpu"))
         _ok(lib.hsl_apply(self._h, _ptr(X), _ptr(Y), batch, _stream(stream)), "hsl_apply")
         return Y
+
+    def set_permutation(self, row_order, col_order, stream=None) -> None:
+        """The layer holds W[row_order][:, col_order]; apply in the original order."""
+        if row_order is not None:
+            _need(row_order, self.m, "row_order")
+            _need(col_order, self.n, "col_order")
+        _ok(lib.hsl_set_permutation(self._h, _ptr(row_order), _ptr(col_order), _stream(stream)),
+            "hsl_set_permutation")
 
     def check(self, stream=None) -> None:
         _ok(lib.hsl_check(self._h, _stream(stream)), "hsl_check")
