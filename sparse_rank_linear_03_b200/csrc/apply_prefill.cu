@@ -893,6 +893,13 @@ bool make_map(CUtensorMap* map, CUtensorMapDataType dt, int esize, const void* b
 
 }  // namespace
 
+bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dt, int esize, const void* base,
+                  int64_t rows, int64_t cols, int64_t row_stride_elems, int box_cols,
+                  int box_rows, CUtensorMapSwizzle sw) {
+  return make_map(map, dt, esize, base, rows, cols, row_stride_elems, box_cols, box_rows, sw);
+}
+bool tmap_available() { return encode_fn() != nullptr; }
+
 // Z workspace and Vt come from the handle (Vt built when the factors are packed).
 // Pair tiles hold 192 tokens: below a few tiles of tokens the single-CTA
 // kernel wastes less of its tile.
