@@ -317,6 +317,41 @@ def test_randomized_matches_exact_on_low_rank():
     assert np.abs(U @ V.T - R).max() < 1e-10 * np.abs(R).max()
 
 
+def test_randomized_matches_exact_truncation_across_a_gap():
+    """Spectrum with a clear gap after r: with power iterations the randomized
+    factors reproduce the exact truncated SVD (Eckart–Young optimum), and keep
+    the √σ balance UᵀU = VᵀV = diag(σ)."""
+    rng = np.random.default_rng(21)
+    m, n, r = 120, 90, 7
+    Ua, _ = np.linalg.qr(rng.standard_normal((m, n)))
+    Va, _ = np.linalg.qr(rng.standard_normal((n, n)))
+    sig = np.concatenate([np.linspace(10, 5, r), np.linspace(1, 0.01, n - r)])
+    R = (Ua * sig) @ Va.T
+    omega = rng.standard_normal((n, r + 6))
+    # subspace error decays like (σ_{r+1}/σ_r)^(2q+1) = 0.2^13 ≈ 1e-9 at q = 6
+    U, V = oracle.lowrank_randomized(R, r, omega, power_iters=6)
+    Ue, Ve = oracle.lowrank_svd(R, r)
+    assert np.abs(U @ V.T - Ue @ Ve.T).max() < 1e-7 * sig[0]
+    assert np.allclose(np.diag(U.T @ U), sig[:r], rtol=1e-9)
+    assert np.allclose(U.T @ U, V.T @ V, atol=1e-9)
+    err = np.linalg.norm(R - U @ V.T, "fro") ** 2
+    assert abs(err - (sig[r:] ** 2).sum()) <= 1e-9 * (sig ** 2).sum()
+
+
+def test_randomized_without_power_iterations_is_worse_but_bounded():
+    """q = 0 on a flat tail: a valid rank-r factorisation whose residual is no
+    better than the optimum (Eckart–Young) and within the HMT bound's order."""
+    rng = np.random.default_rng(22)
+    R = rng.standard_normal((80, 60))
+    r = 5
+    omega = rng.standard_normal((60, r + 10))
+    U, V = oracle.lowrank_randomized(R, r, omega, power_iters=0)
+    s = np.linalg.svd(R, compute_uv=False)
+    err = np.linalg.norm(R - U @ V.T, "fro") ** 2
+    assert err >= (s[r:] ** 2).sum() * (1 - 1e-12)
+    assert err <= 2.0 * (s[r:] ** 2).sum()
+
+
 # ---------------------------------------------------------------- apply
 
 def _triple_loop(S, U, V, X):
