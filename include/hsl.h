@@ -208,6 +208,27 @@ hsl_status hsl_group_apply(hsl_group g, const void* const* X, void* const* Y, in
  * Same passage as hsl_group_create. */
 hsl_status hsl_group_destroy(hsl_group g);
 
+/* Stage 2 on the GPU: the rank-r factors of the residual R (device, m×n of
+ * r_dtype; e.g. the residual hsl_split_topk wrote) as its truncated SVD with
+ * √σ on each side, R ≈ U Vᵀ, U = U_r √Σ_r, V = V_r √Σ_r, computed by the
+ * randomized range finder (Halko–Martinsson–Tropp) with the caller's Gaussian
+ * test matrix:
+ *   omega:       device fp32 [n][k], r ≤ k ≤ min(m, n, 512) (k − r is the
+ *                oversampling);
+ *   power_iters: q ≥ 0 subspace iterations (Y ← R orth(Rᵀ Q));
+ *   U [m][r], V [n][r]: device, handle dtype (pass them to hsl_pack);
+ *   sigma [r]: device fp32, σ_1 ≥ … ≥ σ_r (0 where R has no such direction).
+ * The tall products run on the tensor cores with fp32 operands split into
+ * three bf16 terms (fp32-accurate); orthonormalisation and the small SVD use
+ * fp64 Gram matrices and a Jacobi eigensolver.  Uses the handle's m, n, r and
+ * dtype; allocates its workspace for the call (about 2·m·n·2 bytes for bf16
+ * R) and synchronises s before freeing it.  r = 0 is a no-op.
+ * [HSS] §Two-stage compression, Stage 2 (the residual factored into two
+ * m×r / n×r matrices), and the implementation flow (low-rank factorisation,
+ * O(n³)). */
+hsl_status hsl_factor(hsl_handle h, const void* R, hsl_dtype r_dtype, const float* omega, int32_t k,
+                      int32_t power_iters, void* U, void* V, float* sigma, hsl_stream s);
+
 /* ---- Permutation for concentration ------------------------------------------
  * [HSS] §Permutation and hierarchical alignment: reorder the rows and columns
  * of W (reverse Cuthill–McKee) so that its large entries gather near the

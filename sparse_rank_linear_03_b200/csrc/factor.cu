@@ -1,0 +1,734 @@
+// Stage 2 on the GPU: randomized truncated SVD of the residual, R ≈ U Vᵀ.
+//
+// "Hierarchical Sparse + Low-Rank Compression of LLMs", §Two-stage hierarchical
+// sparse + low-rank compression, Stage 2: the residual left by Stage 1 is
+// factored into an m×r and an n×r matrix (1024×64 twice in the worked
+// example); the implementation flow gives the factorisation an O(n³) cost.
+// The factors are the truncated SVD of R with √σ on each side, computed by the
+// randomized range finder of Halko, Martinsson and Tropp with a caller-given
+// Gaussian test matrix Ω [n×k], k = r + oversampling:
+//   Y = R Ω;  Q = orth(Y);  q times { Z = orth(Rᵀ Q); Q = orth(R Z) };
+//   Bᵀ = Rᵀ Q;  B Bᵀ = W Λ Wᵀ;  σ = √λ;  U = Q W_r √Σ_r,  V = Bᵀ W_r / √Σ_r.
+//
+// Kernels:
+//   k_split_terms  an fp32 (or bf16) matrix as bf16 terms hi + mid + lo
+//                  (hi = bf16(x), mid = bf16(x − hi), lo = bf16(x − hi − mid);
+//                  each difference is exact in fp32), optionally transposed,
+//                  into a zero-padded K-major array.  bf16 input is one term.
+//   k_gemm_tc      C[M×N] = Σ_{a+b<3} A_a[M×K] · B_bᵀ (N ≤ 512): the tall
+//                  products R·Ω, Rᵀ·Q, R·Z on tcgen05 (TMA, 128-byte swizzle,
+//                  fp32 accumulators in TMEM, one or two N halves); the term
+//                  pairs make every product exact and the sums fp32, so the
+//                  product is fp32-accurate although the MMA takes bf16.
+//                  K may be split over CTAs (partials added in split order).
+//   k_gram         G = CᵀC in fp64 over row chunks (partials added in order).
+//   k_jacobi       one CTA: cyclic two-sided Jacobi in fp64 on a k×k
+//                  symmetric matrix (round-robin pairs, rotations of disjoint
+//                  pairs applied together), eigenvalues sorted descending with
+//                  their vectors.  Bounded sweeps.
+//   k_scale_cols   T = W · diag(f(λ)) for the basis changes.
+//   k_small_gemm   C[M×K] · T[K×N] (K, N ≤ 512) in fp32, written row-major
+//                  (fp32 or the layer dtype) or as split bf16 terms transposed
+//                  (the next tall product's B operand).
+// orth(Y) = Y·W₁Λ₁^{-1/2} then once more on the result ("QR by the Gram
+// matrix", twice for orthogonality); eigenvalues below 1e-10 of the largest
+// drop their direction (a zero column), so rank-deficient Y is handled.
+#include <cuda.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <vector>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc.cuh"
+
+namespace hsl {
+namespace {
+
+// ---- split into bf16 terms --------------------------------------------------------
+// out[t][orow][ocol] (row stride ld_out, term stride term_stride) for the
+// element in[row][col] (row stride ld_in); orow/ocol swapped when transposing.
+template <typename TIn>
+__global__ void k_split_terms(const TIn* __restrict__ in, int64_t rows, int64_t cols,
+                              int64_t ld_in, int nterms, int transpose, uint16_t* __restrict__ out,
+                              int64_t ld_out, int64_t term_stride) {
+  __shared__ float tile[32][33];
+  const int64_t r0 = int64_t(blockIdx.y) * 32, c0 = int64_t(blockIdx.x) * 32;
+  for (int dy = threadIdx.y; dy < 32; dy += blockDim.y) {
+    const int64_t r = r0 + dy, c = c0 + threadIdx.x;
+    float v = 0.f;
+    if (r < rows && c < cols) {
+      if constexpr (sizeof(TIn) == 2)
+        v = __uint_as_float(uint32_t(in[r * ld_in + c]) << 16);
+      else
+        v = in[r * ld_in + c];
+    }
+    tile[dy][threadIdx.x] = v;
+  }
+  __syncthreads();
+  for (int dy = threadIdx.y; dy < 32; dy += blockDim.y) {
+    // output element (orow, ocol): consecutive threads write consecutive ocol
+    int64_t orow, ocol;
+    float v;
+    if (transpose) {
+      orow = c0 + dy;
+      ocol = r0 + threadIdx.x;
+      v = tile[threadIdx.x][dy];
+      if (orow >= cols || ocol >= rows) continue;
+    } else {
+      orow = r0 + dy;
+      ocol = c0 + threadIdx.x;
+      v = tile[dy][threadIdx.x];
+      if (orow >= rows || ocol >= cols) continue;
+    }
+    float rest = v;
+    for (int t = 0; t < nterms; ++t) {
+      const __nv_bfloat16 h = __float2bfloat16_rn(rest);
+      out[int64_t(t) * term_stride + orow * ld_out + ocol] = __bfloat16_as_ushort(h);
+      rest = rest - __bfloat162float(h);
+    }
+  }
+}
+
+// ---- tall GEMM on tcgen05 -------------------------------------------------------------
+constexpr int GT_THREADS = 192;
+constexpr int GT_BK = 64;
+constexpr int GT_A = 128 * 128;  // A tile: 128 rows × 64 bf16
+
+struct GemmMaps {
+  CUtensorMap a;  // A terms [nA·M][ldK]  box {64, 128}  SW128
+  CUtensorMap b;  // B terms [nB·N][ldK]  box {64, BH}   SW128
+};
+struct GemmArgs {
+  float* C;          // [M][N] (or partial [split][M][N])
+  uint32_t* err;
+  int M, N, BH, nh;  // BH rows per N half, nh ∈ {1, 2}
+  int nA, nB;        // terms of A and B
+  int nkb, splits;   // K-blocks, K splits
+  int stages, stage_bytes;
+};
+
+__device__ __forceinline__ bool gwait(uint64_t* bar, uint32_t parity, uint32_t* err,
+                                      volatile int* abort_flag) {
+  if (*abort_flag) return false;
+  if (tc::mbar_wait(bar, parity, err)) return true;
+  *abort_flag = 1;
+  return false;
+}
+
+// the term pairs (a, b) with a + b < 3, a < nA, b < nB, in a fixed order
+__device__ __forceinline__ int pair_count(int nA, int nB) {
+  int c = 0;
+  for (int a = 0; a < nA; ++a)
+    for (int b = 0; b < nB; ++b)
+      if (a + b < 3) ++c;
+  return c;
+}
+__device__ __forceinline__ void pair_at(int idx, int nA, int nB, int& pa, int& pb) {
+  for (int a = 0; a < nA; ++a)
+    for (int b = 0; b < nB; ++b)
+      if (a + b < 3) {
+        if (idx == 0) {
+          pa = a;
+          pb = b;
+          return;
+        }
+        --idx;
+      }
+  pa = pb = 0;
+}
+
+__global__ void __launch_bounds__(GT_THREADS, 1)
+    k_gemm_tc(const __grid_constant__ GemmMaps maps, const GemmArgs g) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int ST = g.stages, SB = g.stage_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * SB);
+  uint64_t* empty = full + ST;
+  uint64_t* accf = empty + ST;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int mt = blockIdx.x / g.splits, sp = blockIdx.x % g.splits;
+  const int kb0 = int(int64_t(sp) * g.nkb / g.splits), kb1 = int(int64_t(sp + 1) * g.nkb / g.splits);
+  const int npair = pair_count(g.nA, g.nB);
+  const int steps = (kb1 - kb0) * npair;
+  const int b_bytes = g.BH * 128;
+  const uint32_t ncols = g.nh == 2 ? 512u : (g.BH <= 32 ? 32u : g.BH <= 64 ? 64u : g.BH <= 128 ? 128u : 256u);
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int s = 0; s < ST; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    tc::mbar_init(accf, 1);
+    tc::fence_mbar_init();
+    tc::prefetch_tmap(&maps.a);
+    tc::prefetch_tmap(&maps.b);
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_slot, ncols);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  volatile int* abrt = &abort_flag;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int issued[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      for (int st = 0; st < steps; ++st) {
+        const int s = st % ST;
+        const uint32_t ph = (st / ST) & 1;
+        if (!gwait(&empty[s], ph ^ 1, g.err, abrt)) break;
+        const int kb = kb0 + st / npair;
+        int pa, pb;
+        pair_at(st % npair, g.nA, g.nB, pa, pb);
+        unsigned char* base = smem + s * SB;
+        tc::mbar_expect_tx(&full[s], GT_A + g.nh * b_bytes);
+        tc::tma_load_2d(base, &maps.a, kb * GT_BK, pa * g.M + mt * 128, &full[s]);
+        for (int h = 0; h < g.nh; ++h)
+          tc::tma_load_2d(base + GT_A + h * b_bytes, &maps.b, kb * GT_BK,
+                          pb * (g.nh * g.BH) + h * g.BH, &full[s]);
+        ++issued[s];
+      }
+      for (int s = 0; s < ST; ++s)
+        if (issued[s]) tc::mbar_wait(&full[s], (issued[s] - 1) & 1, g.err);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = tc::idesc_bf16(128, g.BH);
+      for (int st = 0; st < steps; ++st) {
+        const int s = st % ST;
+        const uint32_t ph = (st / ST) & 1;
+        if (!gwait(&full[s], ph, g.err, abrt)) break;
+        tc::tc_fence_after();
+        unsigned char* base = smem + s * SB;
+        const uint64_t ad = tc::desc_sw128(base);
+        for (int h = 0; h < g.nh; ++h) {
+          const uint64_t bd = tc::desc_sw128(base + GT_A + h * b_bytes);
+#pragma unroll
+          for (int k = 0; k < GT_BK / 16; ++k)
+            tc::mma_bf16(tmem + uint32_t(h * 256), tc::desc_advance(ad, k * 32),
+                         tc::desc_advance(bd, k * 32), idesc, (st > 0 || k > 0) ? 1u : 0u);
+        }
+        tc::mma_commit(&empty[s]);
+      }
+      tc::mma_commit(accf);
+    }
+  } else {
+    // epilogue: TMEM lane = row of the tile
+    const int q = warp & 3;
+    const int row = (q << 5) | lane;
+    const int i = mt * 128 + row;
+    const uint32_t lane_base = uint32_t(q * 32) << 16;
+    float* C = g.C + (g.splits > 1 ? int64_t(sp) * g.M * g.N : 0);
+    const bool ok = tc::mbar_wait(accf, 0, g.err) && !*abrt;
+    if (ok && steps > 0) {
+      tc::tc_fence_after();
+      for (int h = 0; h < g.nh; ++h) {
+        for (int c0 = 0; c0 < g.BH; c0 += 32) {
+          float v[32];
+          tc::tmem_ld32(tmem + lane_base + uint32_t(h * 256 + c0), v);
+          if (i < g.M) {
+            float* dst = C + int64_t(i) * g.N + h * g.BH + c0;
+#pragma unroll
+            for (int j = 0; j < 32; j += 4)
+              if (h * g.BH + c0 + j < g.N)
+                *reinterpret_cast<float4*>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+          }
+        }
+      }
+    } else if (i < g.M) {
+      // an empty K range (or a wait that gave up) contributes zeros
+      for (int c = 0; c < g.N; c += 4)
+        *reinterpret_cast<float4*>(C + int64_t(i) * g.N + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, ncols);
+  }
+}
+
+// out = Σ_s part[s] (fixed order)
+template <typename T>
+__global__ void k_sum_parts(const T* __restrict__ part, int splits, int64_t count, T* __restrict__ out) {
+  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < count;
+       e += int64_t(gridDim.x) * blockDim.x) {
+    T acc = part[e];
+    for (int s = 1; s < splits; ++s) acc += part[int64_t(s) * count + e];
+    out[e] = acc;
+  }
+}
+
+// ---- Gram matrix in fp64 -------------------------------------------------------------
+// partial[p][i][j] = Σ_{rows in chunk p} C[row][i]·C[row][j], C [M][N] fp32.
+__global__ void __launch_bounds__(256) k_gram(const float* __restrict__ C, int64_t M, int N,
+                                              int chunks, double* __restrict__ partial) {
+  __shared__ float ta[32][33], tb[32][33];
+  const int ti = blockIdx.x, tj = blockIdx.y, p = blockIdx.z;
+  const int64_t r0 = int64_t(p) * M / chunks, r1 = int64_t(p + 1) * M / chunks;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 × 8
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
+  for (int64_t rb = r0; rb < r1; rb += 32) {
+    for (int dy = ty; dy < 32; dy += 8) {
+      const int64_t r = rb + dy;
+      const int ca = ti * 32 + tx, cb = tj * 32 + tx;
+      ta[dy][tx] = (r < r1 && ca < N) ? C[r * N + ca] : 0.f;
+      tb[dy][tx] = (r < r1 && cb < N) ? C[r * N + cb] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int rr = 0; rr < 32; ++rr) {
+      const double b = tb[rr][tx];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) acc[u] += double(ta[rr][ty + 8 * u]) * b;
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int i = ti * 32 + ty + 8 * u, j = tj * 32 + tx;
+    if (i < N && j < N) partial[(int64_t(p) * N + i) * N + j] = acc[u];
+  }
+}
+
+// ---- symmetric eigensolver (one CTA) -----------------------------------------------------
+constexpr int JT = 1024;
+// A [k][k] fp64 (overwritten), V [k][k] work, evals [k] and vecs [k][k] (columns)
+// sorted by descending eigenvalue.
+__global__ void __launch_bounds__(JT) k_jacobi(double* __restrict__ A, double* __restrict__ V, int k,
+                                               int max_sweeps, double* __restrict__ evals,
+                                               double* __restrict__ vecs) {
+  __shared__ int P[256], Q[256];
+  __shared__ double Cs[256], Sn[256];
+  __shared__ double red[JT / 32];
+  __shared__ int stop;
+  const int K = k + (k & 1);  // even number of players (a dummy when k is odd)
+  const int npair = K / 2;
+  for (int e = threadIdx.x; e < k * k; e += JT) V[e] = (e / k == e % k) ? 1.0 : 0.0;
+  __syncthreads();
+  for (int sweep = 0; sweep < max_sweeps; ++sweep) {
+    // off-diagonal mass against the diagonal: stop when negligible
+    double off = 0.0, dia = 0.0;
+    for (int e = threadIdx.x; e < k * k; e += JT) {
+      const double v = A[e];
+      if (e / k == e % k) dia += v * v; else off += v * v;
+    }
+    for (int o = 16; o; o >>= 1) {
+      off += __shfl_xor_sync(0xffffffffu, off, o);
+      dia += __shfl_xor_sync(0xffffffffu, dia, o);
+    }
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = off;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      double o2 = 0.0;
+      for (int w = 0; w < JT / 32; ++w) o2 += red[w];
+      red[0] = o2;
+    }
+    __syncthreads();
+    const double off_all = red[0];
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = dia;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      double d2 = 0.0;
+      for (int w = 0; w < JT / 32; ++w) d2 += red[w];
+      stop = off_all <= 1e-30 * d2 || off_all == 0.0;
+    }
+    __syncthreads();
+    if (stop) break;
+    for (int round = 0; round < K - 1; ++round) {
+      if (threadIdx.x < npair) {
+        const int i = threadIdx.x;
+        // circle method: player 0 fixed, the others rotate
+        auto player = [&](int j) { return 1 + (j + round) % (K - 1); };
+        int p, q;
+        if (i == 0) {
+          p = 0;
+          q = player(0);
+        } else {
+          p = player(i);
+          q = player(K - 1 - i);
+        }
+        if (p > q) {
+          const int t = p;
+          p = q;
+          q = t;
+        }
+        double c = 1.0, s = 0.0;
+        if (q < k) {
+          const double apq = A[int64_t(p) * k + q];
+          if (apq != 0.0) {
+            const double app = A[int64_t(p) * k + p], aqq = A[int64_t(q) * k + q];
+            const double tau = (aqq - app) / (2.0 * apq);
+            const double t = (tau >= 0.0 ? 1.0 : -1.0) / (fabs(tau) + sqrt(1.0 + tau * tau));
+            c = 1.0 / sqrt(1.0 + t * t);
+            s = t * c;
+          }
+        }
+        P[i] = p;
+        Q[i] = q < k ? q : -1;
+        Cs[i] = c;
+        Sn[i] = s;
+      }
+      __syncthreads();
+      // rows: (p, q) ← (c·row_p − s·row_q, s·row_p + c·row_q)
+      for (int e = threadIdx.x; e < npair * k; e += JT) {
+        const int i = e / k, j = e % k;
+        const int q = Q[i];
+        if (q < 0 || Sn[i] == 0.0) continue;
+        const int p = P[i];
+        const double c = Cs[i], s = Sn[i];
+        const double ap = A[int64_t(p) * k + j], aq = A[int64_t(q) * k + j];
+        A[int64_t(p) * k + j] = c * ap - s * aq;
+        A[int64_t(q) * k + j] = s * ap + c * aq;
+      }
+      __syncthreads();
+      // columns of A and of V
+      for (int e = threadIdx.x; e < npair * k; e += JT) {
+        const int i = e / k, j = e % k;
+        const int q = Q[i];
+        if (q < 0 || Sn[i] == 0.0) continue;
+        const int p = P[i];
+        const double c = Cs[i], s = Sn[i];
+        const double ap = A[int64_t(j) * k + p], aq = A[int64_t(j) * k + q];
+        A[int64_t(j) * k + p] = c * ap - s * aq;
+        A[int64_t(j) * k + q] = s * ap + c * aq;
+        const double vp = V[int64_t(j) * k + p], vq = V[int64_t(j) * k + q];
+        V[int64_t(j) * k + p] = c * vp - s * vq;
+        V[int64_t(j) * k + q] = s * vp + c * vq;
+      }
+      __syncthreads();
+    }
+  }
+  // sort by descending eigenvalue (rank = number ahead; ties by index)
+  for (int i = threadIdx.x; i < k; i += JT) {
+    const double li = A[int64_t(i) * k + i];
+    int rank = 0;
+    for (int j = 0; j < k; ++j) {
+      const double lj = A[int64_t(j) * k + j];
+      if (lj > li || (lj == li && j < i)) ++rank;
+    }
+    evals[rank] = li;
+    for (int r = 0; r < k; ++r) vecs[int64_t(r) * k + rank] = V[int64_t(r) * k + i];
+  }
+}
+
+// T[i][j] = W[i][j]·f(λ_j) for j < ncols (row stride ld_t), with
+// mode 0: f = λ^{-1/2}, 1: f = λ^{1/4} (√σ), 2: f = λ^{-1/4} (1/√σ); an
+// eigenvalue at or below thr_rel·λ_max (λ_max = lam[0]) drops its direction (f = 0).
+__global__ void k_scale_cols(const double* __restrict__ W, const double* __restrict__ lam, int k,
+                             int ncols, int ld_t, int mode, double thr_rel, float* __restrict__ T) {
+  const double thr = thr_rel * fmax(lam[0], 0.0);
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < k * ld_t; e += gridDim.x * blockDim.x) {
+    const int i = e / ld_t, j = e % ld_t;
+    double f = 0.0;
+    if (j < ncols) {
+      const double l = lam[j];
+      if (mode == 0) f = l > thr ? 1.0 / sqrt(l) : 0.0;
+      else if (mode == 1) f = l > thr ? sqrt(sqrt(l)) : 0.0;
+      else f = l > thr ? 1.0 / sqrt(sqrt(l)) : 0.0;
+    }
+    T[e] = float(double(W[int64_t(i) * k + (j < k ? j : 0)]) * f);
+  }
+}
+
+__global__ void k_sigma(const double* __restrict__ lam, int r, double thr_rel, float* __restrict__ sigma) {
+  const double thr = thr_rel * fmax(lam[0], 0.0);
+  for (int j = threadIdx.x; j < r; j += blockDim.x) sigma[j] = lam[j] > thr ? float(sqrt(lam[j])) : 0.f;
+}
+
+// ---- small GEMM: out = C[M][K]·T[K][N] (K, N ≤ 512) -------------------------------------
+// mode 0: fp32 row-major out (row stride ld_out); mode 1: bf16 row-major;
+// mode 2: 3 bf16 terms transposed: out[t][col][row] (row stride ld_out, term stride tstride)
+constexpr int SG = 64;
+__global__ void __launch_bounds__(256) k_small_gemm(const float* __restrict__ C, int64_t M, int K,
+                                                    int ldc, const float* __restrict__ T, int N,
+                                                    int ldt, int mode, void* __restrict__ out,
+                                                    int64_t ld_out, int64_t tstride) {
+  __shared__ float cs[32][SG + 1];  // [k][row]
+  __shared__ float ts[32][SG + 1];  // [k][col]
+  const int64_t row0 = int64_t(blockIdx.x) * SG;
+  const int col0 = blockIdx.y * SG;
+  const int tr = threadIdx.x & 15, tcn = threadIdx.x >> 4;  // 16 × 16 threads, 4×4 outputs
+  float acc[4][4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+  for (int k0 = 0; k0 < K; k0 += 32) {
+    for (int e = threadIdx.x; e < 32 * SG; e += 256) {
+      const int kk = e & 31, rr = e >> 5;
+      const int64_t r = row0 + rr;
+      cs[kk][rr] = (r < M && k0 + kk < K) ? C[r * ldc + k0 + kk] : 0.f;
+      const int cc = e & (SG - 1), k2 = e / SG;
+      ts[k2][cc] = (k0 + k2 < K && col0 + cc < N) ? T[int64_t(k0 + k2) * ldt + col0 + cc] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < 32; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        a[u] = cs[kk][tr + 16 * u];
+        b[u] = ts[kk][tcn + 16 * u];
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(a[u], b[v], acc[u][v]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int64_t r = row0 + tr + 16 * u;
+    if (r >= M) continue;
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const int c = col0 + tcn + 16 * v;
+      if (c >= N) continue;
+      const float x = acc[u][v];
+      if (mode == 0) {
+        static_cast<float*>(out)[r * ld_out + c] = x;
+      } else if (mode == 1) {
+        static_cast<uint16_t*>(out)[r * ld_out + c] = __bfloat16_as_ushort(__float2bfloat16_rn(x));
+      } else {
+        float rest = x;
+        for (int t = 0; t < 3; ++t) {
+          const __nv_bfloat16 h = __float2bfloat16_rn(rest);
+          static_cast<uint16_t*>(out)[t * tstride + int64_t(c) * ld_out + r] = __bfloat16_as_ushort(h);
+          rest -= __bfloat162float(h);
+        }
+      }
+    }
+  }
+}
+
+// ---- host side ------------------------------------------------------------------------------
+
+struct Work {
+  DevBuf bufs[16];
+  ~Work() {
+    for (DevBuf& b : bufs) release(b);
+  }
+};
+
+hsl_status launch_split(const void* in, bool in_bf16, int64_t rows, int64_t cols, int64_t ld_in,
+                        int nterms, bool transpose, uint16_t* out, int64_t ld_out,
+                        int64_t term_stride, cudaStream_t s) {
+  dim3 grid(unsigned((cols + 31) / 32), unsigned((rows + 31) / 32));
+  dim3 block(32, 8);
+  if (in_bf16)
+    k_split_terms<uint16_t><<<grid, block, 0, s>>>(static_cast<const uint16_t*>(in), rows, cols,
+                                                   ld_in, nterms, transpose ? 1 : 0, out, ld_out,
+                                                   term_stride);
+  else
+    k_split_terms<float><<<grid, block, 0, s>>>(static_cast<const float*>(in), rows, cols, ld_in,
+                                                nterms, transpose ? 1 : 0, out, ld_out, term_stride);
+  note_launch();
+  return cuda_fail(cudaGetLastError(), "split terms launch");
+}
+
+// C[M][N] = Σ A_a · B_bᵀ; A terms [nA][M][ld] (term stride M·ld), B terms [nB][N][ld]
+hsl_status gemm_tall(const uint16_t* A, int nA, int64_t M, const uint16_t* B, int nB, int N,
+                     int64_t ld, float* C, float* part, int64_t part_cap, int num_sms,
+                     uint32_t* err, cudaStream_t s) {
+  const int nh = N > 256 ? 2 : 1;
+  const int BH = nh == 2 ? N / 2 : N;
+  const int nkb = int(ld / GT_BK);
+  const int mtiles = int((M + 127) / 128);
+  // split K when the tiles do not fill the SMs (each split keeps ≥ 8 K-blocks)
+  int splits = 1;
+  while (mtiles * (splits + 1) <= num_sms && nkb / (splits + 1) >= 8) ++splits;
+  if (splits > 1 && int64_t(splits) * M * N > part_cap) splits = 1;
+  const int stage_bytes = GT_A + nh * BH * 128;
+  const int stages = std::min(6, (200 * 1024) / stage_bytes);
+  const int smem = stages * stage_bytes + 1024 + 256;
+  GemmMaps maps;
+  memset(&maps, 0, sizeof(maps));
+  const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (!make_tmap_2d(&maps.a, BF, 2, A, int64_t(nA) * M, ld, ld, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&maps.b, BF, 2, B, int64_t(nB) * nh * BH, ld, ld, 64, BH,
+                    CU_TENSOR_MAP_SWIZZLE_128B)) {
+    set_message("tensor map encoding failed (factorisation)");
+    return HSL_ERR_CUDA;
+  }
+  GemmArgs g;
+  g.C = splits > 1 ? part : C;
+  g.err = err;
+  g.M = int(M);
+  g.N = N;
+  g.BH = BH;
+  g.nh = nh;
+  g.nA = nA;
+  g.nB = nB;
+  g.nkb = nkb;
+  g.splits = splits;
+  g.stages = stages;
+  g.stage_bytes = stage_bytes;
+  if (cudaError_t e = cudaFuncSetAttribute(k_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))
+    return cuda_fail(e, "factor gemm smem attribute");
+  k_gemm_tc<<<unsigned(mtiles * splits), GT_THREADS, smem, s>>>(maps, g);
+  note_launch();
+  if (hsl_status e = cuda_fail(cudaGetLastError(), "factor gemm launch")) return e;
+  if (splits > 1) {
+    const int64_t count = M * N;
+    k_sum_parts<float><<<unsigned(std::min<int64_t>((count + 255) / 256, int64_t(num_sms) * 8)), 256, 0,
+                         s>>>(part, splits, count, C);
+    note_launch();
+    return cuda_fail(cudaGetLastError(), "factor gemm reduce launch");
+  }
+  return HSL_OK;
+}
+
+hsl_status gram(const float* C, int64_t M, int N, double* part, int64_t part_cap, double* G,
+                int num_sms, cudaStream_t s) {
+  const int nt = (N + 31) / 32;
+  int chunks = int(std::max<int64_t>(
+      1, std::min<int64_t>({(M + 1023) / 1024, (int64_t(num_sms) * 4 + nt * nt - 1) / (nt * nt),
+                            int64_t(64)})));
+  while (chunks > 1 && int64_t(chunks) * N * N > part_cap) --chunks;
+  k_gram<<<dim3(nt, nt, chunks), 256, 0, s>>>(C, M, N, chunks, part);
+  note_launch();
+  if (hsl_status e = cuda_fail(cudaGetLastError(), "gram launch")) return e;
+  const int64_t count = int64_t(N) * N;
+  k_sum_parts<double><<<unsigned((count + 255) / 256), 256, 0, s>>>(part, chunks, count, G);
+  note_launch();
+  return cuda_fail(cudaGetLastError(), "gram reduce launch");
+}
+
+hsl_status eig(double* G, int k, double* Vw, double* evals, double* vecs, cudaStream_t s) {
+  k_jacobi<<<1, JT, 0, s>>>(G, Vw, k, 40, evals, vecs);
+  note_launch();
+  return cuda_fail(cudaGetLastError(), "eigensolver launch");
+}
+
+hsl_status small_gemm(const float* C, int64_t M, int K, int ldc, const float* T, int N, int ldt,
+                      int mode, void* out, int64_t ld_out, int64_t tstride, cudaStream_t s) {
+  dim3 grid(unsigned((M + SG - 1) / SG), unsigned((N + SG - 1) / SG));
+  k_small_gemm<<<grid, 256, 0, s>>>(C, M, K, ldc, T, N, ldt, mode, out, ld_out, tstride);
+  note_launch();
+  return cuda_fail(cudaGetLastError(), "small gemm launch");
+}
+
+}  // namespace
+
+hsl_status factor_randomized_run(const void* R, int64_t m, int64_t n, hsl_dtype dtype, int r, int k,
+                                 const float* omega, int power_iters, void* U, void* V,
+                                 hsl_dtype out_dtype, float* sigma, uint32_t* err, int num_sms,
+                                 cudaStream_t s) {
+  const int kp = k <= 256 ? int(round_up(k, 16)) : int(round_up(k, 32));
+  const int64_t ldm = round_up(m, 64), ldn = round_up(n, 64);
+  const int nA = dtype == HSL_BF16 ? 1 : 3;
+  const int64_t mx = std::max(m, n);
+  // an eigenvalue of a Gram matrix below this share of the largest is rounding
+  // noise of a direction the data does not have (fp32 data, fp64 sums)
+  const double thr_rel = 1e-10;
+  Work w;
+  enum { RA, RT, OT, QT, ZT, YB, QF, BT, PART, GP, G, VW, EV, EVEC, TT, NB };
+  const size_t sizes[NB] = {
+      size_t(nA) * m * ldn * 2,          // R as K-major A terms
+      size_t(nA) * n * ldm * 2,          // Rᵀ terms
+      size_t(3) * kp * ldn * 2,          // Ωᵀ terms
+      size_t(3) * kp * ldm * 2,          // Qᵀ terms
+      size_t(3) * kp * ldn * 2,          // Zᵀ terms
+      size_t(mx) * kp * 4,               // Y / Z, then the orthonormal basis (fp32)
+      size_t(mx) * kp * 4,               // first-pass basis (fp32)
+      size_t(n) * kp * 4,                // Bᵀ = Rᵀ Q
+      size_t(4) * mx * kp * 4,           // GEMM split partials
+      size_t(64) * kp * kp * 8,          // Gram partials
+      size_t(kp) * kp * 8,               // Gram
+      size_t(kp) * kp * 8,               // eigensolver work
+      size_t(kp) * 8,                    // eigenvalues
+      size_t(kp) * kp * 8,               // eigenvectors
+      size_t(kp) * kp * 4,               // basis change T
+  };
+  for (int b = 0; b < NB; ++b)
+    if (hsl_status e = ensure(w.bufs[b], sizes[b], "factorisation workspace")) return e;
+  auto U16 = [&](int b) { return static_cast<uint16_t*>(w.bufs[b].p); };
+  auto F32 = [&](int b) { return static_cast<float*>(w.bufs[b].p); };
+  auto F64 = [&](int b) { return static_cast<double*>(w.bufs[b].p); };
+  for (int b : {RA, RT, OT, QT, ZT})
+    if (cudaError_t e = cudaMemsetAsync(w.bufs[b].p, 0, sizes[b], s)) return cuda_fail(e, "memset");
+  const bool rb = dtype == HSL_BF16;
+  // R and Rᵀ as bf16 terms (one for bf16 R, three for fp32 R), Ωᵀ as three terms
+  if (hsl_status e = launch_split(R, rb, m, n, n, nA, false, U16(RA), ldn, m * ldn, s)) return e;
+  if (hsl_status e = launch_split(R, rb, m, n, n, nA, true, U16(RT), ldm, n * ldm, s)) return e;
+  if (hsl_status e = launch_split(omega, false, n, k, k, 3, true, U16(OT), ldn, int64_t(kp) * ldn, s))
+    return e;
+  const int64_t part_cap = int64_t(sizes[PART] / 4), gp_cap = int64_t(sizes[GP] / 8);
+
+  // Y [M][kp] in YB → orthonormal basis of its columns in YB (fp32) and as
+  // transposed bf16 terms at `terms` (row stride ld): two passes of
+  // basis = C · W Λ^{-1/2} from the Gram matrix CᵀC = W Λ Wᵀ.
+  auto orth = [&](int64_t M, uint16_t* terms, int64_t ld) -> hsl_status {
+    for (int pass = 0; pass < 2; ++pass) {
+      const float* cur = pass == 0 ? F32(YB) : F32(QF);
+      if (hsl_status e = gram(cur, M, kp, F64(GP), gp_cap, F64(G), num_sms, s)) return e;
+      if (hsl_status e = eig(F64(G), kp, F64(VW), F64(EV), F64(EVEC), s)) return e;
+      k_scale_cols<<<64, 256, 0, s>>>(F64(EVEC), F64(EV), kp, kp, kp, 0, thr_rel, F32(TT));
+      note_launch();
+      if (hsl_status e = cuda_fail(cudaGetLastError(), "basis change launch")) return e;
+      if (pass == 0) {
+        if (hsl_status e = small_gemm(cur, M, kp, kp, F32(TT), kp, kp, 0, F32(QF), kp, 0, s)) return e;
+      } else {
+        if (hsl_status e = small_gemm(cur, M, kp, kp, F32(TT), kp, kp, 0, F32(YB), kp, 0, s)) return e;
+        if (hsl_status e = small_gemm(cur, M, kp, kp, F32(TT), kp, kp, 2, terms, ld, int64_t(kp) * ld, s))
+          return e;
+      }
+    }
+    return HSL_OK;
+  };
+
+  // Y = R Ω, Q = orth(Y)
+  if (hsl_status e = gemm_tall(U16(RA), nA, m, U16(OT), 3, kp, ldn, F32(YB), F32(PART), part_cap,
+                               num_sms, err, s))
+    return e;
+  if (hsl_status e = orth(m, U16(QT), ldm)) return e;
+  for (int it = 0; it < power_iters; ++it) {
+    // Z = orth(Rᵀ Q); Y = R Z; Q = orth(Y)
+    if (hsl_status e = gemm_tall(U16(RT), nA, n, U16(QT), 3, kp, ldm, F32(YB), F32(PART), part_cap,
+                                 num_sms, err, s))
+      return e;
+    if (hsl_status e = orth(n, U16(ZT), ldn)) return e;
+    if (hsl_status e = gemm_tall(U16(RA), nA, m, U16(ZT), 3, kp, ldn, F32(YB), F32(PART), part_cap,
+                                 num_sms, err, s))
+      return e;
+    if (hsl_status e = orth(m, U16(QT), ldm)) return e;
+  }
+  // Bᵀ = Rᵀ Q; B Bᵀ = W Λ Wᵀ; σ = √λ; U = Q W_r √Σ_r; V = Bᵀ W_r / √Σ_r
+  if (hsl_status e = gemm_tall(U16(RT), nA, n, U16(QT), 3, kp, ldm, F32(BT), F32(PART), part_cap,
+                               num_sms, err, s))
+    return e;
+  if (hsl_status e = gram(F32(BT), n, kp, F64(GP), gp_cap, F64(G), num_sms, s)) return e;
+  if (hsl_status e = eig(F64(G), kp, F64(VW), F64(EV), F64(EVEC), s)) return e;
+  // σ below thr_rel^{1/2} of σ_max: no direction (zero factor columns)
+  k_sigma<<<1, 256, 0, s>>>(F64(EV), r, thr_rel, sigma);
+  note_launch();
+  if (hsl_status e = cuda_fail(cudaGetLastError(), "sigma launch")) return e;
+  const int omode = out_dtype == HSL_BF16 ? 1 : 0;
+  k_scale_cols<<<64, 256, 0, s>>>(F64(EVEC), F64(EV), kp, r, r, 1, thr_rel, F32(TT));
+  note_launch();
+  if (hsl_status e = cuda_fail(cudaGetLastError(), "basis change launch")) return e;
+  if (hsl_status e = small_gemm(F32(YB), m, kp, kp, F32(TT), r, r, omode, U, r, 0, s)) return e;
+  k_scale_cols<<<64, 256, 0, s>>>(F64(EVEC), F64(EV), kp, r, r, 2, thr_rel, F32(TT));
+  note_launch();
+  if (hsl_status e = cuda_fail(cudaGetLastError(), "basis change launch")) return e;
+  if (hsl_status e = small_gemm(F32(BT), n, kp, kp, F32(TT), r, r, omode, V, r, 0, s)) return e;
+  // the workspace is freed when `w` goes out of scope: wait for the kernels first
+  return cuda_fail(cudaStreamSynchronize(s), "factorisation");
+}
+
+}  // namespace hsl

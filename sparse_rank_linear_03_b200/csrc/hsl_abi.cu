@@ -504,6 +504,25 @@ hsl_status hsl_group_destroy(hsl_group g) {
   return HSL_OK;
 }
 
+hsl_status hsl_factor(hsl_handle h, const void* R, hsl_dtype r_dtype, const float* omega, int32_t k,
+                      int32_t power_iters, void* U, void* V, float* sigma, hsl_stream stream) {
+  t_msg.clear();
+  if (!h) return invalid("handle is NULL");
+  Handle& H = h->h;
+  if (!R || !omega) return invalid("R/omega is NULL");
+  if (r_dtype != HSL_F32 && r_dtype != HSL_BF16) return invalid("unknown R dtype");
+  if (H.r == 0) return HSL_OK;
+  if (!U || !V || !sigma) return invalid("U/V/sigma is NULL");
+  if (k < H.r || k > 512) return unsupported("need r <= k <= 512 columns in omega");
+  if (k > std::min(H.m, H.n)) return unsupported("need k <= min(m, n)");
+  if (power_iters < 0 || power_iters > 64) return invalid("power_iters out of [0, 64]");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  DeviceGuard g(H.device);
+  if (hsl_status e = ensure_err_word(H, s)) return e;
+  return factor_randomized_run(R, H.m, H.n, r_dtype, H.r, k, omega, power_iters, U, V, H.dtype,
+                               sigma, static_cast<uint32_t*>(H.err.p), H.num_sms, s);
+}
+
 hsl_status hsl_concentration(const void* W, int64_t m, int64_t n, hsl_dtype dtype, double* rho,
                              hsl_stream stream) {
   t_msg.clear();

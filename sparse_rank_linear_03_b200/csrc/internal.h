@@ -127,6 +127,11 @@ hsl_status apply_prefill_run(Handle& h, const void* X, void* Y, int64_t T, cudaS
 constexpr int64_t kSplitKMinBatch = 2, kSplitKMaxBatch = 64;
 bool splitk_supported(const Handle& h, const void* X, int64_t T);
 hsl_status apply_splitk_run(Handle& h, const void* X, void* Y, int64_t T, cudaStream_t s);
+// Stage 2: randomized truncated SVD of the residual (factor.cu)
+hsl_status factor_randomized_run(const void* R, int64_t m, int64_t n, hsl_dtype dtype, int r, int k,
+                                 const float* omega, int power_iters, void* U, void* V,
+                                 hsl_dtype out_dtype, float* sigma, uint32_t* err, int num_sms,
+                                 cudaStream_t s);
 // permutation for concentration (permute.cu)
 hsl_status concentration_run(const void* W, int64_t m, int64_t n, hsl_dtype dt, double* out_dev,
                              double* partial, int blocks, cudaStream_t s);

@@ -27,7 +27,7 @@ EXPORTS = (
     "hsl_set_sparse_csr", "hsl_set_sparse_nm24", "hsl_pack", "hsl_apply",
     "hsl_group_create", "hsl_group_apply", "hsl_group_destroy", "hsl_check",
     "hsl_status_str", "hsl_last_message", "hsl_launch_count", "hsl_split_topk_noalloc",
-    "hsl_concentration", "hsl_rcm_order", "hsl_permute", "hsl_set_permutation",
+    "hsl_concentration", "hsl_rcm_order", "hsl_permute", "hsl_set_permutation", "hsl_factor",
 )
 
 
@@ -66,6 +66,7 @@ def _load() -> ctypes.CDLL:
         "hsl_rcm_order": [I64, I64, P, P, P, P],
         "hsl_permute": [P, I64, I64, ctypes.c_int, P, P, P, P],
         "hsl_set_permutation": [P, P, P, P],
+        "hsl_factor": [P, P, ctypes.c_int, P, I32, I32, P, P, P, P],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -244,6 +245,21 @@ class Layer:
                             pin_memory=(X.device.type == "cpu"))
         _ok(lib.hsl_apply(self._h, _ptr(X), _ptr(Y), batch, _stream(stream)), "hsl_apply")
         return Y
+
+    def factor(self, R: torch.Tensor, omega: torch.Tensor, power_iters: int = 2, stream=None):
+        """Stage 2: U [m][r], V [n][r] (layer dtype) and σ [r] of the residual R
+        by the randomized truncated SVD with test matrix omega [n][k] (fp32)."""
+        _need(R, self.m * self.n, "R")
+        if omega.dtype != torch.float32 or omega.dim() != 2 or omega.shape[0] != self.n:
+            raise ValueError("omega must be fp32 [n][k]")
+        dev = R.device
+        U = torch.empty(self.m, self.r, dtype=TORCH_DTYPE[self.dtype], device=dev)
+        V = torch.empty(self.n, self.r, dtype=TORCH_DTYPE[self.dtype], device=dev)
+        sig = torch.empty(self.r, dtype=torch.float32, device=dev)
+        _ok(lib.hsl_factor(self._h, _ptr(R), DTYPE[_wdtype(R)], _ptr(omega), int(omega.shape[1]),
+                           int(power_iters), _ptr(U), _ptr(V), _ptr(sig), _stream(stream)),
+            "hsl_factor")
+        return U, V, sig
 
     def set_permutation(self, row_order, col_order, stream=None) -> None:
         """The layer holds W[row_order][:, col_order]; apply in the original order."""
