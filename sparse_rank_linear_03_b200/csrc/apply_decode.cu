@@ -232,42 +232,102 @@ __device__ __forceinline__ void urows(const ApplyProblem& P, const float* zs, co
 }
 
 // ---- sparse row sums -------------------------------------------------------------
+// G lanes share a row (8 entries per lane per step); a warp pass covers RG row
+// groups per lane, and every step issues the column and value loads of all of a
+// lane's rows before any arithmetic, so each lane keeps RG 16-byte pairs in
+// flight (the bandwidth needs ~44 KB in flight per SM; one pair per lane gave
+// 16 KB).  Raw words are held until use, converted only in the FMA loop.
+template <typename T>
+struct RawVals;
+template <>
+struct RawVals<__nv_bfloat16> {
+  uint4 q;
+  __device__ __forceinline__ void load(const __nv_bfloat16* p) { q = ld_stream16(p); }
+  __device__ __forceinline__ float at(int t) const {
+    const uint32_t w = t < 2 ? q.x : t < 4 ? q.y : t < 6 ? q.z : q.w;
+    return (t & 1) ? bf_hi(w) : bf_lo(w);
+  }
+};
+template <>
+struct RawVals<float> {
+  uint4 a, b;
+  __device__ __forceinline__ void load(const float* p) {
+    a = ld_stream16(p);
+    b = ld_stream16(p + 4);
+  }
+  __device__ __forceinline__ float at(int t) const {
+    const uint4& h = t < 4 ? a : b;
+    const int u = t & 3;
+    return __uint_as_float(u == 0 ? h.x : u == 1 ? h.y : u == 2 ? h.z : h.w);
+  }
+};
+
 template <typename T, int BC>
 __device__ __forceinline__ void csr_rows(const ApplyProblem& P, const T* xs, float* ysp, int s0,
                                          int s1) {
+  constexpr int RG = BC <= 2 ? 4 : (BC <= 4 ? 2 : 1);
   const int G = P.group;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int gl = lane & (G - 1);
   const int rpw = 32 / G;
   const T* pval = static_cast<const T*>(P.pval);
-  for (int ib = s0 + warp * rpw; ib < s1; ib += (kThreads / 32) * rpw) {
-    const int i = ib + lane / G;
-    float acc[BC];
+  for (int ib = s0 + warp * rpw * RG; ib < s1; ib += (kThreads / 32) * rpw * RG) {
+    int32_t e[RG], e1[RG];
 #pragma unroll
-    for (int b = 0; b < BC; ++b) acc[b] = 0.f;
-    if (i < s1) {
-      const int32_t e1 = P.prow[i + 1];
-      for (int32_t e = P.prow[i] + 8 * gl; e < e1; e += 8 * G) {
-        const uint4 cv = ld_stream16(P.pcol + e);
-        float v[8];
-        load8<T>(pval + e, v);
-        const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
+    for (int g = 0; g < RG; ++g) {
+      const int i = ib + g * rpw + lane / G;
+      e[g] = 0;
+      e1[g] = 0;
+      if (i < s1) {
+        e[g] = P.prow[i] + 8 * gl;
+        e1[g] = P.prow[i + 1];
+      }
+    }
+    float acc[RG][BC];
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          const int c = int((cw[t >> 1] >> ((t & 1) * 16)) & 0xFFFFu);
-          float xv[BC];
-          xcol<T, BC>(xs, c, xv);
+    for (int g = 0; g < RG; ++g)
 #pragma unroll
-          for (int b = 0; b < BC; ++b) acc[b] = fmaf(v[t], xv[b], acc[b]);
+      for (int b = 0; b < BC; ++b) acc[g][b] = 0.f;
+    for (;;) {
+      bool any = false;
+      uint4 cv[RG];
+      RawVals<T> rv[RG];
+#pragma unroll
+      for (int g = 0; g < RG; ++g) {
+        if (e[g] < e1[g]) {
+          cv[g] = ld_stream16(P.pcol + e[g]);
+          rv[g].load(pval + e[g]);
+          any = true;
+        }
+      }
+      if (!any) break;
+#pragma unroll
+      for (int g = 0; g < RG; ++g) {
+        if (e[g] < e1[g]) {
+          const uint32_t cw[4] = {cv[g].x, cv[g].y, cv[g].z, cv[g].w};
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const int c = int((cw[t >> 1] >> ((t & 1) * 16)) & 0xFFFFu);
+            float xv[BC];
+            xcol<T, BC>(xs, c, xv);
+            const float v = rv[g].at(t);
+#pragma unroll
+            for (int b = 0; b < BC; ++b) acc[g][b] = fmaf(v, xv[b], acc[g][b]);
+          }
+          e[g] += 8 * G;
         }
       }
     }
-    for (int o = G >> 1; o; o >>= 1)
 #pragma unroll
-      for (int b = 0; b < BC; ++b) acc[b] += __shfl_xor_sync(0xffffffffu, acc[b], o);
-    if (gl == 0 && i < s1)
+    for (int g = 0; g < RG; ++g) {
+      for (int o = G >> 1; o; o >>= 1)
 #pragma unroll
-      for (int b = 0; b < BC; ++b) ysp[(i - s0) * BC + b] = acc[b];
+        for (int b = 0; b < BC; ++b) acc[g][b] += __shfl_xor_sync(0xffffffffu, acc[g][b], o);
+      const int i = ib + g * rpw + lane / G;
+      if (gl == 0 && i < s1)
+#pragma unroll
+        for (int b = 0; b < BC; ++b) ysp[(i - s0) * BC + b] = acc[g][b];
+    }
   }
 }
 
