@@ -912,6 +912,30 @@ bool prefill_pairs_enabled() {
   return e != nullptr && e[0] == '1';
 }
 
+// Z = X·V as a bf16 (hi, lo) pair into h.zpre ([2][T][r16]); the kernel
+// triggers programmatic dependent launch at its start.
+hsl_status prefill_z_run(Handle& h, const void* X, int64_t T, cudaStream_t s) {
+  const int r16 = int(round_up(h.r, 16));
+  if (r16 == 0) return HSL_OK;
+  if (r16 > 256) return HSL_ERR_UNSUPPORTED;
+  if (hsl_status e = ensure(h.zpre, size_t(T) * r16 * 2 * 2, "prefill Z (hi, lo)")) return e;
+  PrefillMaps zm;
+  memset(&zm, 0, sizeof(zm));
+  const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (!make_map(&zm.xz, BF, 2, X, T, h.n, h.n, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&zm.vt, BF, 2, h.Vt.p, r16, h.n, h.n, 64, r16, CU_TENSOR_MAP_SWIZZLE_128B)) {
+    set_message("tensor map encoding failed");
+    return HSL_ERR_CUDA;
+  }
+  if (cudaError_t e = cudaFuncSetAttribute(k_prefill_z, cudaFuncAttributeMaxDynamicSharedMemorySize, Z_SMEM))
+    return cuda_fail(e, "prefill z smem attribute");
+  k_prefill_z<<<unsigned((T + 127) / 128), 192, Z_SMEM, s>>>(
+      zm, static_cast<__nv_bfloat16*>(h.zpre.p), int(h.n), int(T), r16,
+      static_cast<uint32_t*>(h.err.p));
+  note_launch();
+  return cuda_fail(cudaGetLastError(), "prefill z launch");
+}
+
 bool prefill_supported(const Handle& h, const void* X) {
   return h.fmt == HSL_FMT_NM24 && h.dtype == HSL_BF16 && h.n % 64 == 0 &&
          (reinterpret_cast<uintptr_t>(X) % 16) == 0 && encode_fn() != nullptr;

@@ -360,6 +360,14 @@ hsl_status hsl_pack(hsl_handle h, const void* U, const void* V, hsl_stream strea
   if (hsl_status e = pack_factors_run(H, U, V, s)) return e;
   Handle* one = &H;
   if (hsl_status e = plan_build(H.plan, &one, 1, s)) return e;
+  H.csr_ascending = false;
+  if (H.fmt == HSL_FMT_CSR) {  // the plan upload has synchronised s
+    uint32_t unordered = 1;
+    if (cudaError_t e = cudaMemcpy(&unordered, static_cast<uint32_t*>(H.err.p) + 1, 4,
+                                   cudaMemcpyDeviceToHost))
+      return cuda_fail(e, "column order flag read");
+    H.csr_ascending = unordered == 0;
+  }
   H.packed = true;
   return HSL_OK;
 }
@@ -406,6 +414,8 @@ hsl_status hsl_apply(hsl_handle h, const void* X, void* Y, int64_t batch, hsl_st
   }
   if (batch >= kPrefillMinBatch && prefill_supported(H, Xd)) {
     if (hsl_status e = apply_prefill_run(H, Xd, Yd, batch, s)) return e;
+  } else if (batch >= kPrefillMinBatch && prefill_csr_supported(H, Xd)) {
+    if (hsl_status e = apply_prefill_csr_run(H, Xd, Yd, batch, s)) return e;
   } else if (splitk_supported(H, Xd, batch)) {
     if (hsl_status e = apply_splitk_run(H, Xd, Yd, batch, s)) return e;
   } else {

@@ -93,6 +93,7 @@ struct Handle {
   // packed layouts
   DevBuf prow, pcol, pval, pmeta, pmeta_tc, U, Vt;
   int32_t group = 8, meta_stride = 0;
+  bool csr_ascending = false;  // every packed row has strictly ascending columns
   int64_t pack_cap = 0;
   bool packed = false;
 
@@ -122,6 +123,11 @@ hsl_status apply_decode_run(ApplyPlan& plan, const void* X, void* Y, const void*
 constexpr int64_t kPrefillMinBatch = 65;
 bool prefill_supported(const Handle& h, const void* X);
 hsl_status apply_prefill_run(Handle& h, const void* X, void* Y, int64_t T, cudaStream_t s);
+hsl_status prefill_z_run(Handle& h, const void* X, int64_t T, cudaStream_t s);
+// CSR layers at large batches: each 64-column block of S densified into shared
+// memory for dense tcgen05 MMAs (apply_prefill_csr.cu)
+bool prefill_csr_supported(const Handle& h, const void* X);
+hsl_status apply_prefill_csr_run(Handle& h, const void* X, void* Y, int64_t T, cudaStream_t s);
 // small batches (2..64 tokens) of the same layers: sparse tensor cores with K
 // split across every SM (apply_splitk.cu)
 constexpr int64_t kSplitKMinBatch = 2, kSplitKMaxBatch = 64;

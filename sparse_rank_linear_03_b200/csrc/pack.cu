@@ -86,9 +86,10 @@ __global__ void __launch_bounds__(256) k_csr_fill(const int32_t* __restrict__ ro
                                                   const SB* __restrict__ val,
                                                   const int32_t* __restrict__ prow, int64_t m,
                                                   int64_t nnz, int32_t n, uint16_t* __restrict__ pcol,
-                                                  SB* __restrict__ pval, uint32_t* err) {
+                                                  SB* __restrict__ pval, uint32_t* err,
+                                                  uint32_t* order_flag) {
   const int lane = threadIdx.x & 31;
-  bool bad = false;
+  bool bad = false, unordered = false;
   for (int64_t i = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; i < m;
        i += (int64_t(gridDim.x) * blockDim.x) >> 5) {
     bool badrow = false;
@@ -104,9 +105,12 @@ __global__ void __launch_bounds__(256) k_csr_fill(const int32_t* __restrict__ ro
       }
       pcol[d0 + e] = in ? uint16_t(c) : uint16_t(n);
       pval[d0 + e] = in ? val[s0 + e] : SB(0);
+      // the large-batch CSR path needs strictly ascending columns in a row
+      if (in && e > 0 && c <= col[s0 + e - 1]) unordered = true;
     }
   }
   if (bad) set_error(err, kErrBadIndex);
+  if (unordered) atomicOr(order_flag, 1u);
 }
 
 __global__ void k_nm24_meta(const uint8_t* __restrict__ idx, int64_t m, int64_t n,
@@ -260,6 +264,8 @@ hsl_status pack_sparse_run(Handle& h, cudaStream_t s) {
   const int eb = dtype_bytes(h.dtype);
   if (h.fmt == HSL_FMT_CSR) {
     const int64_t cap = round_up(h.nnz + 7 * h.m + 8, 8);  // multiple of 8: every row start stays 16-byte aligned
+    if (cudaError_t e = cudaMemsetAsync(static_cast<uint32_t*>(h.err.p) + 1, 0, 4, s))
+      return cuda_fail(e, "column order flag clear");
     if (hsl_status e = ensure(h.prow, size_t(h.m + 1) * 4, "packed row starts")) return e;
     if (hsl_status e = ensure(h.pcol, size_t(cap) * 2, "packed columns")) return e;
     if (hsl_status e = ensure(h.pval, size_t(cap) * eb, "packed values")) return e;
@@ -273,13 +279,13 @@ hsl_status pack_sparse_run(Handle& h, cudaStream_t s) {
           static_cast<const int32_t*>(h.row_ptr.p), static_cast<const int32_t*>(h.col.p),
           static_cast<const uint16_t*>(h.val.p), static_cast<const int32_t*>(h.prow.p), h.m,
           h.nnz, int32_t(h.n), static_cast<uint16_t*>(h.pcol.p), static_cast<uint16_t*>(h.pval.p),
-          static_cast<uint32_t*>(h.err.p));
+          static_cast<uint32_t*>(h.err.p), static_cast<uint32_t*>(h.err.p) + 1);
     else
       k_csr_fill<uint32_t><<<unsigned(std::max<int64_t>(grid, 1)), 256, 0, s>>>(
           static_cast<const int32_t*>(h.row_ptr.p), static_cast<const int32_t*>(h.col.p),
           static_cast<const uint32_t*>(h.val.p), static_cast<const int32_t*>(h.prow.p), h.m,
           h.nnz, int32_t(h.n), static_cast<uint16_t*>(h.pcol.p), static_cast<uint32_t*>(h.pval.p),
-          static_cast<uint32_t*>(h.err.p));
+          static_cast<uint32_t*>(h.err.p), static_cast<uint32_t*>(h.err.p) + 1);
     note_launch();
     // lanes per row: about two 8-entry vectors per lane on an average row
     const double avg_vec = double(h.nnz) / double(std::max<int64_t>(h.m, 1)) / 8.0;

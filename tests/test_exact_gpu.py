@@ -179,17 +179,19 @@ def csr_rows(ref, rows, n, dtype):
     return csr_dense_rows(ref["row_ptr"], ref["col"], oracle.bits_to_f64(ref["val"], dtype), rows, n)
 
 
-@pytest.mark.parametrize("T", [1, 4, 16])
+@pytest.mark.parametrize("T", [1, 4, 16, 2048])
 def test_exact_csr_attn4096(hsl, T):
-    """4096², 2 % top-k, r = 128 at batch 1/4/16 (the CSR decode kernel)."""
+    """4096², 2 % top-k, r = 128 at batch 1/4/16 (the CSR decode kernel) and
+    2048 tokens (the tensor-core path that decompresses S block by block)."""
     m = n = 4096
     L, ref, U, V = build_csr(hsl, m, n, 128, 0.02, 551)
     X = tokens(T, n, 552 + T, "bf16")
     Y = L.apply(dev(X, "bf16"))
     L.check()
-    rows = sample_rows(m, 2000, 553)
-    assert_exact(got_bits(Y, rows, "bf16"),
-                 expected_bits(csr_rows(ref, rows, n, "bf16"), U, V, X, rows, "bf16"))
+    rows = sample_rows(m, 2000 if T <= 16 else 256, 553)
+    tok = np.arange(T) if T <= 16 else np.sort(np.random.default_rng(T).choice(T, 256, replace=False))
+    assert_exact(got_bits(Y, rows, "bf16")[tok],
+                 expected_bits(csr_rows(ref, rows, n, "bf16"), U, V, X[tok], rows, "bf16"))
 
 
 def test_exact_csr_7b_layer_group(hsl):
