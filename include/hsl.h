@@ -167,10 +167,28 @@ hsl_status hsl_set_sparse_nm24(hsl_handle h, const void* val, const uint8_t* nm_
 
 /* Build the device layouts hsl_apply streams: S repacked (CSR: rows padded
  * to 8 values with 16-bit column indices, [HSS] §Implementation (mixed
- * precision: narrow indices); NM24: metadata interleaved per warp lane),
+ * precision: narrow indices; the width is chosen by hsl_set_index_bits);
+ * NM24: metadata interleaved per warp lane),
  * and copies of U [m][r] and V [n][r] (row-major, handle dtype, device).
- * Needs S (split or set) first, else HSL_ERR_NOT_READY.  CSR needs n < 65535. */
+ * Needs S (split or set) first, else HSL_ERR_NOT_READY. */
 hsl_status hsl_pack(hsl_handle h, const void* U, const void* V, hsl_stream s);
+
+/* Column-index width of the packed CSR S, used from the next hsl_pack on:
+ *   16 — 16-bit columns (needs n < 65535); the default when n < 65535;
+ *   32 — 32-bit columns (any n); the default when n ≥ 65535;
+ *    8 — one delta byte per entry (column minus the previous entry's) plus a
+ *        16-bit column base per 8-entry vector: 1.25 bytes per entry against
+ *        2, so 3.25 instead of 4 streamed bytes per bf16 entry at decode.
+ *        A gap of more than 255 columns inside a row takes filler entries
+ *        (value 0, one per 255 columns); needs n < 65535 and each row's
+ *        columns in ascending order (else hsl_pack returns HSL_ERR_UNSUPPORTED);
+ *    0 — back to the default.
+ * Large batches on the tensor cores use 16-bit columns; with another width
+ * they run on the decode kernel.  CSR handles only; invalidates hsl_pack.
+ * [HSS] §Implementation and operational patterns (from theory to production),
+ * mixed precision: sparse indices as INT32 or in narrower integers (INT16,
+ * INT8) to cut the memory of S further. */
+hsl_status hsl_set_index_bits(hsl_handle h, int32_t bits);
 
 /* Y = X Ŵᵀ, i.e. y = S x + U (Vᵀ x) for each of the batch rows of X.
  *   X: [batch][n], Y: [batch][m], handle dtype, row-major.  X and Y may be

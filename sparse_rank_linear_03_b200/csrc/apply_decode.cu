@@ -262,7 +262,56 @@ struct RawVals<float> {
   }
 };
 
-template <typename T, int BC>
+// The 8 column indices of a packed vector, for each column width: 16-bit
+// (one 16-byte load), 32-bit (two), or 8-bit deltas (an 8-byte load plus the
+// vector's 16-bit base: column 0 is the base, column t adds delta t).
+template <int IDX>
+struct RawCols;
+template <>
+struct RawCols<16> {
+  uint4 q;
+  __device__ __forceinline__ void load(const ApplyProblem& P, int32_t e) {
+    q = ld_stream16(static_cast<const uint16_t*>(P.pcol) + e);
+  }
+  __device__ __forceinline__ void cols(int (&c)[8]) const {
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int t = 0; t < 8; ++t) c[t] = int((w[t >> 1] >> ((t & 1) * 16)) & 0xFFFFu);
+  }
+};
+template <>
+struct RawCols<32> {
+  uint4 a, b;
+  __device__ __forceinline__ void load(const ApplyProblem& P, int32_t e) {
+    const uint32_t* p = static_cast<const uint32_t*>(P.pcol) + e;
+    a = ld_stream16(p);
+    b = ld_stream16(p + 4);
+  }
+  __device__ __forceinline__ void cols(int (&c)[8]) const {
+    c[0] = int(a.x); c[1] = int(a.y); c[2] = int(a.z); c[3] = int(a.w);
+    c[4] = int(b.x); c[5] = int(b.y); c[6] = int(b.z); c[7] = int(b.w);
+  }
+};
+template <>
+struct RawCols<8> {
+  uint2 d;
+  uint32_t base;
+  __device__ __forceinline__ void load(const ApplyProblem& P, int32_t e) {
+    d = ld_stream8(static_cast<const uint8_t*>(P.pcol) + e);
+    base = P.pbase[e >> 3];
+  }
+  __device__ __forceinline__ void cols(int (&c)[8]) const {
+    int v = int(base);
+    c[0] = v;
+#pragma unroll
+    for (int t = 1; t < 8; ++t) {
+      v += int(((t < 4 ? d.x : d.y) >> (8 * (t & 3))) & 0xFFu);
+      c[t] = v;
+    }
+  }
+};
+
+template <typename T, int BC, int IDX>
 __device__ __forceinline__ void csr_rows(const ApplyProblem& P, const T* xs, float* ysp, int s0,
                                          int s1) {
   constexpr int RG = BC <= 2 ? 4 : (BC <= 4 ? 2 : 1);
@@ -290,12 +339,12 @@ __device__ __forceinline__ void csr_rows(const ApplyProblem& P, const T* xs, flo
       for (int b = 0; b < BC; ++b) acc[g][b] = 0.f;
     for (;;) {
       bool any = false;
-      uint4 cv[RG];
+      RawCols<IDX> cv[RG];
       RawVals<T> rv[RG];
 #pragma unroll
       for (int g = 0; g < RG; ++g) {
         if (e[g] < e1[g]) {
-          cv[g] = ld_stream16(P.pcol + e[g]);
+          cv[g].load(P, e[g]);
           rv[g].load(pval + e[g]);
           any = true;
         }
@@ -304,10 +353,11 @@ __device__ __forceinline__ void csr_rows(const ApplyProblem& P, const T* xs, flo
 #pragma unroll
       for (int g = 0; g < RG; ++g) {
         if (e[g] < e1[g]) {
-          const uint32_t cw[4] = {cv[g].x, cv[g].y, cv[g].z, cv[g].w};
+          int cidx[8];
+          cv[g].cols(cidx);
 #pragma unroll
           for (int t = 0; t < 8; ++t) {
-            const int c = int((cw[t >> 1] >> ((t & 1) * 16)) & 0xFFFFu);
+            const int c = cidx[t];
             float xv[BC];
             xcol<T, BC>(xs, c, xv);
             const float v = rv[g].at(t);
@@ -458,7 +508,7 @@ __device__ __forceinline__ void nm24_rows(const ApplyProblem& P, const T* xs, fl
 }
 
 // ---- the persistent apply kernel ---------------------------------------------------
-template <typename T, int BC, bool CSR>
+template <typename T, int BC, bool CSR, int IDX>
 __global__ void __maxnreg__(112) k_apply_decode(ApplyArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ uint32_t sel_lut[16];  // byte-permute selector of a 2:4 nibble (x[i0], x[i1])
@@ -502,7 +552,7 @@ __global__ void __maxnreg__(112) k_apply_decode(ApplyArgs a) {
     T* y = y_of<T>(a, p) + int64_t(a.b0) * P.m;
     for (int s0 = l0; s0 < l1; s0 += kSeg) {
       const int s1 = min(s0 + kSeg, l1);
-      if (CSR) csr_rows<T, BC>(P, xs, ysp, s0, s1);
+      if (CSR) csr_rows<T, BC, IDX>(P, xs, ysp, s0, s1);
       else if (fast24)
         nm24_rows_b1(P, reinterpret_cast<const __nv_bfloat16*>(xs), sel_lut, ysp, s0, s1);
       else nm24_rows<T, BC>(P, xs, ysp, s0, s1);
@@ -946,7 +996,14 @@ hsl_status launch_chunk(ApplyPlan& plan, ApplyArgs a, int num_sms, cudaStream_t 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const size_t sm = apply_smem<T, BC>(plan);
-  auto ak = plan.fmt == HSL_FMT_CSR ? k_apply_decode<T, BC, true> : k_apply_decode<T, BC, false>;
+  if (sm > size_t(std::max(max_dyn_smem(), 0))) {
+    set_message("the staged x of this layer does not fit in shared memory");
+    return HSL_ERR_UNSUPPORTED;
+  }
+  auto ak = plan.fmt != HSL_FMT_CSR ? k_apply_decode<T, BC, false, 16>
+            : plan.idx_bits == 8    ? k_apply_decode<T, BC, true, 8>
+            : plan.idx_bits == 32   ? k_apply_decode<T, BC, true, 32>
+                                    : k_apply_decode<T, BC, true, 16>;
   if (cudaError_t e = cudaFuncSetAttribute(ak, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm)))
     return cuda_fail(e, "apply smem attribute");
   int occ = 0;

@@ -125,7 +125,7 @@ hsl_status ensure_err_word(Handle& h, cudaStream_t s) {
 void free_all(Handle& h) {
   DevBuf* bufs[] = {&h.row_ptr, &h.col, &h.val, &h.nm_val, &h.nm_idx, &h.prow, &h.pcol,
                     &h.pval, &h.pmeta, &h.pmeta_tc, &h.U, &h.Vt, &h.z,
-                    &h.err, &h.split_ws, &h.flags, &h.tiles, &h.xstage, &h.ystage, &h.zpre, &h.sk_part, &h.sk_cnt, &h.sk_z, &h.perm_row, &h.perm_col, &h.xperm, &h.yperm, &h.plan.probs,
+                    &h.err, &h.split_ws, &h.flags, &h.tiles, &h.xstage, &h.ystage, &h.zpre, &h.sk_part, &h.sk_cnt, &h.sk_z, &h.perm_row, &h.perm_col, &h.xperm, &h.yperm, &h.pbase, &h.d8_lens, &h.plan.probs,
                     &h.plan.prob_row0, &h.plan.cta_rows, &h.plan.xy_ptrs, &h.plan.zsync};
   for (DevBuf* b : bufs) release(*b);
 }
@@ -351,7 +351,8 @@ hsl_status hsl_pack(hsl_handle h, const void* U, const void* V, hsl_stream strea
     set_message("no sparse part yet (split or set first)");
     return HSL_ERR_NOT_READY;
   }
-  if (H.fmt == HSL_FMT_CSR && H.n >= 65535) return unsupported("packed CSR needs n < 65535");
+  if (H.fmt == HSL_FMT_CSR && (H.index_bits == 16 || H.index_bits == 8) && H.n >= 65535)
+    return unsupported("8- and 16-bit packed CSR columns need n < 65535");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   DeviceGuard g(H.device);
   H.packed = false;
@@ -366,9 +367,22 @@ hsl_status hsl_pack(hsl_handle h, const void* U, const void* V, hsl_stream strea
     if (cudaError_t e = cudaMemcpy(&unordered, static_cast<uint32_t*>(H.err.p) + 1, 4,
                                    cudaMemcpyDeviceToHost))
       return cuda_fail(e, "column order flag read");
-    H.csr_ascending = unordered == 0;
+    H.csr_ascending = unordered == 0 && H.idx_bits == 16;
   }
   H.packed = true;
+  return HSL_OK;
+}
+
+hsl_status hsl_set_index_bits(hsl_handle h, int32_t bits) {
+  t_msg.clear();
+  if (!h) return invalid("handle is NULL");
+  Handle& H = h->h;
+  if (bits != 0 && bits != 8 && bits != 16 && bits != 32) return invalid("bits must be 0, 8, 16 or 32");
+  if (H.fmt != HSL_FMT_CSR) return unsupported("column widths apply to CSR handles");
+  if ((bits == 8 || bits == 16) && H.n >= 65535)
+    return unsupported("8- and 16-bit packed CSR columns need n < 65535");
+  H.index_bits = bits;
+  H.packed = false;
   return HSL_OK;
 }
 

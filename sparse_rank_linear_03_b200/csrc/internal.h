@@ -34,7 +34,9 @@ inline int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
 // ---- the apply problem descriptor (device-resident, one per layer) --------
 struct ApplyProblem {
   const int32_t* prow;    // CSR: packed row starts (elements, multiples of 8), m+1
-  const uint16_t* pcol;   // CSR: packed 16-bit columns (pad = n)
+  const void* pcol;       // CSR: packed columns (pad = n): u16, u32, or u8 deltas
+  const uint16_t* pbase;  // CSR, 8-bit columns: column of each 8-entry vector's first entry
+  int32_t idx_bits;       // CSR: 8, 16 or 32
   const void* pval;       // CSR: packed values; NM24: values [m][n/2]
   const uint16_t* pmeta;  // NM24: metadata, interleaved per lane (see pack.cu)
   const void* U;          // [m][r_pad]
@@ -66,6 +68,7 @@ struct ApplyPlan {
   int z_pieces = 0;     // (row, column piece) items of Vt over all layers
   int slices = 0;       // equal-byte row ranges the apply grid divides among CTAs
   bool vec16 = false;   // every layer has n % 16 == 0 (16-byte aligned 2:4 rows)
+  int32_t idx_bits = 16;  // CSR column width of every member
   uint32_t* err = nullptr;  // error word the apply kernels report to (first member's)
   DevBuf probs;         // ApplyProblem[count]
   DevBuf prob_row0;     // int64[count+1]
@@ -94,6 +97,9 @@ struct Handle {
   DevBuf prow, pcol, pval, pmeta, pmeta_tc, U, Vt;
   int32_t group = 8, meta_stride = 0;
   bool csr_ascending = false;  // every packed row has strictly ascending columns
+  int32_t index_bits = 0;       // requested column width (0: 16, or 32 when n ≥ 65535)
+  int32_t idx_bits = 16;        // column width of the current pack
+  DevBuf pbase, d8_lens;        // 8-bit columns: vector bases, row lengths with fillers
   int64_t pack_cap = 0;
   bool packed = false;
 

@@ -37,9 +37,12 @@ __device__ __forceinline__ int32_t row_len_checked(const int32_t* row_ptr, int64
   return b - a;
 }
 
+// lens (optional): the row lengths to pad, in place of row_ptr's differences
+// (the 8-bit layout adds filler entries to rows).
 __global__ void __launch_bounds__(1024) k_csr_prow(const int32_t* __restrict__ row_ptr, int64_t m,
                                                    int64_t nnz, int64_t cap,
-                                                   int32_t* __restrict__ prow, uint32_t* err) {
+                                                   int32_t* __restrict__ prow, uint32_t* err,
+                                                   const int32_t* __restrict__ lens) {
   __shared__ int64_t wsum[32];
   const int t = threadIdx.x, nt = blockDim.x;
   const int64_t per = (m + nt - 1) / nt;
@@ -47,7 +50,11 @@ __global__ void __launch_bounds__(1024) k_csr_prow(const int32_t* __restrict__ r
   const int64_t hi = lo + per < m ? lo + per : m;
   bool bad = false;
   int64_t s = 0;
-  for (int64_t i = lo; i < hi; ++i) s += pad8(row_len_checked(row_ptr, i, nnz, bad));
+  auto len_of = [&](int64_t i) {
+    const int32_t l = row_len_checked(row_ptr, i, nnz, bad);
+    return lens ? lens[i] : l;
+  };
+  for (int64_t i = lo; i < hi; ++i) s += pad8(len_of(i));
   int64_t incl = s;
   for (int o = 1; o < 32; o <<= 1) {
     const int64_t v = __shfl_up_sync(0xffffffffu, incl, o);
@@ -68,7 +75,7 @@ __global__ void __launch_bounds__(1024) k_csr_prow(const int32_t* __restrict__ r
   int64_t off = wsum[t >> 5] + incl - s;
   for (int64_t i = lo; i < hi; ++i) {
     prow[i] = int32_t(off < cap ? off : cap);
-    off += pad8(row_len_checked(row_ptr, i, nnz, bad));
+    off += pad8(len_of(i));
   }
   if (hi == m && lo < hi) {
     if (off > cap) bad = true;
@@ -79,17 +86,19 @@ __global__ void __launch_bounds__(1024) k_csr_prow(const int32_t* __restrict__ r
   if (bad) set_error(err, kErrBadIndex);
 }
 
-// Warp per row: copy columns (int32 → u16) and values; pad with (n, 0).
-template <typename SB>
+// Warp per row: copy columns (int32 → the packed column type) and values;
+// pad with (n, 0).  order_flag bit 0: a row's columns are not strictly
+// ascending; bit 1: a row's columns decrease somewhere.
+template <typename SB, typename CT>
 __global__ void __launch_bounds__(256) k_csr_fill(const int32_t* __restrict__ row_ptr,
                                                   const int32_t* __restrict__ col,
                                                   const SB* __restrict__ val,
                                                   const int32_t* __restrict__ prow, int64_t m,
-                                                  int64_t nnz, int32_t n, uint16_t* __restrict__ pcol,
+                                                  int64_t nnz, int32_t n, CT* __restrict__ pcol,
                                                   SB* __restrict__ pval, uint32_t* err,
                                                   uint32_t* order_flag) {
   const int lane = threadIdx.x & 31;
-  bool bad = false, unordered = false;
+  bool bad = false, unordered = false, descending = false;
   for (int64_t i = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; i < m;
        i += (int64_t(gridDim.x) * blockDim.x) >> 5) {
     bool badrow = false;
@@ -103,14 +112,89 @@ __global__ void __launch_bounds__(256) k_csr_fill(const int32_t* __restrict__ ro
         bad = true;
         in = false;
       }
-      pcol[d0 + e] = in ? uint16_t(c) : uint16_t(n);
+      pcol[d0 + e] = in ? CT(c) : CT(n);
       pval[d0 + e] = in ? val[s0 + e] : SB(0);
       // the large-batch CSR path needs strictly ascending columns in a row
       if (in && e > 0 && c <= col[s0 + e - 1]) unordered = true;
+      if (in && e > 0 && c < col[s0 + e - 1]) descending = true;
     }
   }
   if (bad) set_error(err, kErrBadIndex);
-  if (unordered) atomicOr(order_flag, 1u);
+  if (unordered || descending) atomicOr(order_flag, (unordered ? 1u : 0u) | (descending ? 2u : 0u));
+}
+
+// 8-bit layout: a filler entry (value 0) goes before every entry whose column
+// is more than 255 past the previous one, once per 255 columns of the gap.
+__device__ __forceinline__ int32_t d8_fillers(int32_t gap) { return gap > 255 ? (gap - 1) / 255 : 0; }
+
+// Thread per row: the row length in the 8-bit layout (entries + fillers).
+// Rows whose columns decrease are flagged (order_flag bit 1) and counted as
+// they are; the pack then refuses the layout.
+__global__ void k_csr_d8_len(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col,
+                             int64_t m, int64_t nnz, int32_t n, int32_t* __restrict__ lens,
+                             uint32_t* order_flag) {
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < m;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    bool bad = false;
+    const int32_t len = row_len_checked(row_ptr, i, nnz, bad);
+    const int32_t s0 = bad ? 0 : row_ptr[i];
+    int32_t extra = 0, prev = -1;
+    bool first = true;
+    for (int32_t e = 0; e < len; ++e) {
+      const int32_t c = col[s0 + e];
+      if (c < 0 || c >= n) continue;  // dropped by the fill as well
+      if (!first) {
+        if (c < prev) atomicOr(order_flag, 2u);
+        else extra += d8_fillers(c - prev);
+      }
+      prev = c;
+      first = false;
+    }
+    lens[i] = len + extra;
+  }
+}
+
+// Thread per row: values, one delta byte per entry (column minus the previous
+// entry's; 0 for the first entry of an 8-entry vector, whose column is the
+// vector's 16-bit base), fillers (value 0, delta 255) and padding (value 0,
+// delta 0) up to the padded length.
+template <typename SB>
+__global__ void k_csr_d8_fill(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col,
+                              const SB* __restrict__ val, const int32_t* __restrict__ prow,
+                              int64_t m, int64_t nnz, int32_t n, uint8_t* __restrict__ pdelta,
+                              uint16_t* __restrict__ pbase, SB* __restrict__ pval, uint32_t* err) {
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < m;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    bool bad = false;
+    const int32_t len = row_len_checked(row_ptr, i, nnz, bad);
+    const int32_t s0 = bad ? 0 : row_ptr[i];
+    const int32_t d0 = prow[i], d1 = prow[i + 1];
+    int32_t pos = d0, prev = 0;
+    auto put = [&](int32_t c, SB v) {
+      if (pos >= d1) return;  // never past the row's packed slots
+      const bool vstart = ((pos - d0) & 7) == 0;
+      pdelta[pos] = vstart ? uint8_t(0) : uint8_t(c - prev);
+      if (vstart) pbase[pos >> 3] = uint16_t(c);
+      pval[pos] = v;
+      prev = c;
+      ++pos;
+    };
+    bool first = true, badcol = false;
+    for (int32_t e = 0; e < len; ++e) {
+      const int32_t c = col[s0 + e];
+      if (c < 0 || c >= n) {
+        badcol = true;
+        continue;
+      }
+      if (!first && c >= prev)
+        for (int32_t f = d8_fillers(c - prev); f > 0; --f) put(prev + 255, SB(0));
+      put(c, val[s0 + e]);
+      first = false;
+    }
+    const int32_t last = first ? 0 : prev;
+    while (pos < d1) put(last, SB(0));
+    if (badcol) set_error(err, kErrBadIndex);
+  }
 }
 
 __global__ void k_nm24_meta(const uint8_t* __restrict__ idx, int64_t m, int64_t n,
@@ -217,7 +301,10 @@ __global__ void __launch_bounds__(1024) k_partition(const ApplyProblem* __restri
                                                     int64_t* __restrict__ cta_rows) {
   auto row_cost = [&](const ApplyProblem& P, int64_t i) -> int64_t {
     const int64_t u = int64_t(P.r_pad) * eb + 8;
-    if (fmt_csr) return int64_t(P.prow[i]) * (eb + 2) + i * u;
+    // per packed entry, in quarter bytes: the value and its column (8-bit
+    // deltas carry a 16-bit base per 8 entries)
+    const int64_t q = 4 * eb + (P.idx_bits == 8 ? 5 : P.idx_bits == 16 ? 8 : 16);
+    if (fmt_csr) return int64_t(P.prow[i]) * q / 4 + i * u;
     return i * (int64_t(P.n / 2) * eb + P.n / 8 + u);
   };
   if (threadIdx.x == 0) {
@@ -263,30 +350,89 @@ constexpr int kSlicesPerSM = 24;
 hsl_status pack_sparse_run(Handle& h, cudaStream_t s) {
   const int eb = dtype_bytes(h.dtype);
   if (h.fmt == HSL_FMT_CSR) {
-    const int64_t cap = round_up(h.nnz + 7 * h.m + 8, 8);  // multiple of 8: every row start stays 16-byte aligned
-    if (cudaError_t e = cudaMemsetAsync(static_cast<uint32_t*>(h.err.p) + 1, 0, 4, s))
+    const int bits = h.index_bits ? h.index_bits : (h.n < 65535 ? 16 : 32);
+    uint32_t* order_flag = static_cast<uint32_t*>(h.err.p) + 1;
+    if (cudaError_t e = cudaMemsetAsync(order_flag, 0, 4, s))
       return cuda_fail(e, "column order flag clear");
     if (hsl_status e = ensure(h.prow, size_t(h.m + 1) * 4, "packed row starts")) return e;
-    if (hsl_status e = ensure(h.pcol, size_t(cap) * 2, "packed columns")) return e;
-    if (hsl_status e = ensure(h.pval, size_t(cap) * eb, "packed values")) return e;
-    h.pack_cap = cap;
-    k_csr_prow<<<1, 1024, 0, s>>>(static_cast<const int32_t*>(h.row_ptr.p), h.m, h.nnz, cap,
-                                  static_cast<int32_t*>(h.prow.p), static_cast<uint32_t*>(h.err.p));
-    note_launch();
     const int64_t grid = std::min<int64_t>((h.m * 32 + 255) / 256, int64_t(h.num_sms) * 8);
-    if (eb == 2)
-      k_csr_fill<uint16_t><<<unsigned(std::max<int64_t>(grid, 1)), 256, 0, s>>>(
-          static_cast<const int32_t*>(h.row_ptr.p), static_cast<const int32_t*>(h.col.p),
-          static_cast<const uint16_t*>(h.val.p), static_cast<const int32_t*>(h.prow.p), h.m,
-          h.nnz, int32_t(h.n), static_cast<uint16_t*>(h.pcol.p), static_cast<uint16_t*>(h.pval.p),
-          static_cast<uint32_t*>(h.err.p), static_cast<uint32_t*>(h.err.p) + 1);
-    else
-      k_csr_fill<uint32_t><<<unsigned(std::max<int64_t>(grid, 1)), 256, 0, s>>>(
-          static_cast<const int32_t*>(h.row_ptr.p), static_cast<const int32_t*>(h.col.p),
-          static_cast<const uint32_t*>(h.val.p), static_cast<const int32_t*>(h.prow.p), h.m,
-          h.nnz, int32_t(h.n), static_cast<uint16_t*>(h.pcol.p), static_cast<uint32_t*>(h.pval.p),
-          static_cast<uint32_t*>(h.err.p), static_cast<uint32_t*>(h.err.p) + 1);
-    note_launch();
+    const unsigned tgrid = unsigned(std::max<int64_t>(1, std::min<int64_t>((h.m + 255) / 256,
+                                                                          int64_t(h.num_sms) * 8)));
+    if (bits == 8) {
+      // row lengths with fillers, their padded starts, then the sizes
+      if (hsl_status e = ensure(h.d8_lens, size_t(h.m) * 4, "8-bit row lengths")) return e;
+      k_csr_d8_len<<<tgrid, 256, 0, s>>>(static_cast<const int32_t*>(h.row_ptr.p),
+                                         static_cast<const int32_t*>(h.col.p), h.m, h.nnz,
+                                         int32_t(h.n), static_cast<int32_t*>(h.d8_lens.p), order_flag);
+      k_csr_prow<<<1, 1024, 0, s>>>(static_cast<const int32_t*>(h.row_ptr.p), h.m, h.nnz,
+                                    int64_t(INT32_MAX) & ~int64_t(7), static_cast<int32_t*>(h.prow.p),
+                                    static_cast<uint32_t*>(h.err.p),
+                                    static_cast<const int32_t*>(h.d8_lens.p));
+      note_launch(2);
+      int32_t total = 0;
+      uint32_t flags = 0;
+      if (cudaError_t e = cudaMemcpyAsync(&total, static_cast<int32_t*>(h.prow.p) + h.m, 4,
+                                          cudaMemcpyDeviceToHost, s))
+        return cuda_fail(e, "8-bit pack size");
+      if (cudaError_t e = cudaMemcpyAsync(&flags, order_flag, 4, cudaMemcpyDeviceToHost, s))
+        return cuda_fail(e, "8-bit pack size");
+      if (cudaError_t e = cudaStreamSynchronize(s)) return cuda_fail(e, "8-bit pack size");
+      if (flags & 2u) {
+        set_message("8-bit delta columns need the columns of every row in ascending order");
+        return HSL_ERR_UNSUPPORTED;
+      }
+      const int64_t cap = round_up(int64_t(total) + 8, 8);
+      if (hsl_status e = ensure(h.pcol, size_t(cap), "packed column deltas")) return e;
+      if (hsl_status e = ensure(h.pbase, size_t(cap / 8) * 2, "packed vector bases")) return e;
+      if (hsl_status e = ensure(h.pval, size_t(cap) * eb, "packed values")) return e;
+      h.pack_cap = cap;
+      if (eb == 2)
+        k_csr_d8_fill<uint16_t><<<tgrid, 256, 0, s>>>(
+            static_cast<const int32_t*>(h.row_ptr.p), static_cast<const int32_t*>(h.col.p),
+            static_cast<const uint16_t*>(h.val.p), static_cast<const int32_t*>(h.prow.p), h.m, h.nnz,
+            int32_t(h.n), static_cast<uint8_t*>(h.pcol.p), static_cast<uint16_t*>(h.pbase.p),
+            static_cast<uint16_t*>(h.pval.p), static_cast<uint32_t*>(h.err.p));
+      else
+        k_csr_d8_fill<uint32_t><<<tgrid, 256, 0, s>>>(
+            static_cast<const int32_t*>(h.row_ptr.p), static_cast<const int32_t*>(h.col.p),
+            static_cast<const uint32_t*>(h.val.p), static_cast<const int32_t*>(h.prow.p), h.m, h.nnz,
+            int32_t(h.n), static_cast<uint8_t*>(h.pcol.p), static_cast<uint16_t*>(h.pbase.p),
+            static_cast<uint32_t*>(h.pval.p), static_cast<uint32_t*>(h.err.p));
+      note_launch();
+    } else {
+      const int64_t cap = round_up(h.nnz + 7 * h.m + 8, 8);  // multiple of 8: every row start stays 16-byte aligned
+      const int cb = bits / 8;
+      if (hsl_status e = ensure(h.pcol, size_t(cap) * cb, "packed columns")) return e;
+      if (hsl_status e = ensure(h.pval, size_t(cap) * eb, "packed values")) return e;
+      h.pack_cap = cap;
+      k_csr_prow<<<1, 1024, 0, s>>>(static_cast<const int32_t*>(h.row_ptr.p), h.m, h.nnz, cap,
+                                    static_cast<int32_t*>(h.prow.p), static_cast<uint32_t*>(h.err.p),
+                                    nullptr);
+      note_launch();
+      const unsigned g = unsigned(std::max<int64_t>(grid, 1));
+      const int32_t* rp = static_cast<const int32_t*>(h.row_ptr.p);
+      const int32_t* cl = static_cast<const int32_t*>(h.col.p);
+      const int32_t* pr = static_cast<const int32_t*>(h.prow.p);
+      uint32_t* err = static_cast<uint32_t*>(h.err.p);
+      if (eb == 2 && cb == 2)
+        k_csr_fill<uint16_t, uint16_t><<<g, 256, 0, s>>>(rp, cl, static_cast<const uint16_t*>(h.val.p),
+            pr, h.m, h.nnz, int32_t(h.n), static_cast<uint16_t*>(h.pcol.p),
+            static_cast<uint16_t*>(h.pval.p), err, order_flag);
+      else if (eb == 2)
+        k_csr_fill<uint16_t, uint32_t><<<g, 256, 0, s>>>(rp, cl, static_cast<const uint16_t*>(h.val.p),
+            pr, h.m, h.nnz, int32_t(h.n), static_cast<uint32_t*>(h.pcol.p),
+            static_cast<uint16_t*>(h.pval.p), err, order_flag);
+      else if (cb == 2)
+        k_csr_fill<uint32_t, uint16_t><<<g, 256, 0, s>>>(rp, cl, static_cast<const uint32_t*>(h.val.p),
+            pr, h.m, h.nnz, int32_t(h.n), static_cast<uint16_t*>(h.pcol.p),
+            static_cast<uint32_t*>(h.pval.p), err, order_flag);
+      else
+        k_csr_fill<uint32_t, uint32_t><<<g, 256, 0, s>>>(rp, cl, static_cast<const uint32_t*>(h.val.p),
+            pr, h.m, h.nnz, int32_t(h.n), static_cast<uint32_t*>(h.pcol.p),
+            static_cast<uint32_t*>(h.pval.p), err, order_flag);
+      note_launch();
+    }
+    h.idx_bits = bits;
     // lanes per row: about two 8-entry vectors per lane on an average row
     const double avg_vec = double(h.nnz) / double(std::max<int64_t>(h.m, 1)) / 8.0;
     int g = 4;
@@ -347,6 +493,12 @@ hsl_status plan_build(ApplyPlan& plan, Handle* const* hs, int count, cudaStream_
   plan.r_pad_max = 0;
   plan.vec16 = true;
   plan.err = static_cast<uint32_t*>(hs[0]->err.p);
+  plan.idx_bits = hs[0]->idx_bits;
+  for (int i = 0; i < count; ++i)
+    if (plan.fmt == HSL_FMT_CSR && hs[i]->idx_bits != plan.idx_bits) {
+      set_message("a group needs one CSR column width");
+      return HSL_ERR_UNSUPPORTED;
+    }
   const int eb = dtype_bytes(plan.dtype);
   std::vector<ApplyProblem> probs(count);
   int64_t row0 = 0;
@@ -355,7 +507,9 @@ hsl_status plan_build(ApplyPlan& plan, Handle* const* hs, int count, cudaStream_
     Handle& h = *hs[i];
     ApplyProblem& P = probs[i];
     P.prow = static_cast<const int32_t*>(h.prow.p);
-    P.pcol = static_cast<const uint16_t*>(h.pcol.p);
+    P.pcol = h.pcol.p;
+    P.pbase = static_cast<const uint16_t*>(h.pbase.p);
+    P.idx_bits = h.idx_bits;
     P.pval = h.fmt == HSL_FMT_CSR ? h.pval.p : h.nm_val.p;
     P.pmeta = static_cast<const uint16_t*>(h.pmeta.p);
     P.U = h.U.p;

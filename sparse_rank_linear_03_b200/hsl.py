@@ -28,6 +28,7 @@ EXPORTS = (
     "hsl_group_create", "hsl_group_apply", "hsl_group_destroy", "hsl_check",
     "hsl_status_str", "hsl_last_message", "hsl_launch_count", "hsl_split_topk_noalloc",
     "hsl_concentration", "hsl_rcm_order", "hsl_permute", "hsl_set_permutation", "hsl_factor",
+    "hsl_set_index_bits",
 )
 
 
@@ -67,6 +68,7 @@ def _load() -> ctypes.CDLL:
         "hsl_permute": [P, I64, I64, ctypes.c_int, P, P, P, P],
         "hsl_set_permutation": [P, P, P, P],
         "hsl_factor": [P, P, ctypes.c_int, P, I32, I32, P, P, P, P],
+        "hsl_set_index_bits": [P, I32],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -224,6 +226,10 @@ class Layer:
         _dtype_of(val, self.dtype, "val")
         _ok(lib.hsl_set_sparse_nm24(self._h, _ptr(val), _ptr(idx), _stream(stream)),
             "hsl_set_sparse_nm24")
+
+    def set_index_bits(self, bits: int) -> None:
+        """Column width of the packed CSR S (8, 16, 32; 0 = default) from the next pack."""
+        _ok(lib.hsl_set_index_bits(self._h, int(bits)), "hsl_set_index_bits")
 
     # -- pack + apply -------------------------------------------------------
     def pack(self, U, V, stream=None) -> None:

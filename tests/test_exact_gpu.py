@@ -222,3 +222,23 @@ def test_exact_csr_square1024_f32(hsl, T):
     rows = np.arange(m)
     assert_exact(got_bits(Y, rows, "f32"),
                  expected_bits(csr_rows(ref, rows, n, "f32"), U, V, X, rows, "f32"))
+
+
+@pytest.mark.parametrize("bits", [8, 32])
+def test_exact_csr_other_column_widths(hsl, bits):
+    """The 4096² layer with 8-bit delta or 32-bit columns, batch 1 and 4."""
+    m = n = 4096
+    W = weights(m, n, 591, "bf16", csr=True)
+    U, V = factors(m, n, 128, 601, "bf16")
+    L = hsl.Layer(m, n, 128, "csr", "bf16")
+    L.set_index_bits(bits)
+    L.split(dev(W, "bf16"), 0.02, None)
+    L.pack(dev(U, "bf16"), dev(V, "bf16"))
+    ref = oracle.split_topk(W, 0.02, "bf16")
+    rows = sample_rows(m, 2000, 592)
+    for T in (1, 4):
+        X = tokens(T, n, 593 + T, "bf16")
+        Y = L.apply(dev(X, "bf16"))
+        L.check()
+        assert_exact(got_bits(Y, rows, "bf16"),
+                     expected_bits(csr_rows(ref, rows, n, "bf16"), U, V, X, rows, "bf16"))
