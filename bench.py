@@ -340,6 +340,42 @@ def oracle_split_rate(m, n, fmt, dtype, frac, seed, target_s):
     return by / dt, f"{nr} of {m} rows, split of the block alone, {dt:.2f} s"
 
 
+def oracle_factor_rate(m, n, r, k, q, seed, target_s):
+    """The oracle's randomized truncated SVD (float64) on a row block of a
+    Student-t matrix; returns (FLOP/s over 2·rows·n·k·(2q + 2), sample text)."""
+    import oracle
+    from sparse_rank_linear_03_b200 import synth
+    omega = np.random.default_rng(seed + 5).standard_normal((n, k))
+
+    def run(nrows):
+        R = synth.student_t_f32(nrows, n, seed).astype(np.float64)
+        t0 = time.perf_counter()
+        oracle.lowrank_randomized(R, min(r, nrows), omega[:, :min(k, nrows)], power_iters=q)
+        return time.perf_counter() - t0
+
+    nr = max(k + 1, 256)
+    dt = run(nr)
+    nr = int(min(m, max(nr, nr * target_s / max(dt, 1e-3))))
+    dt = run(nr)
+    return 2.0 * nr * n * k * (2 * q + 2) / dt, f"{nr} of {m} rows, r = {r}, k = {k}, q = {q}: {dt:.2f} s"
+
+
+def oracle_rho_rate(m, n, seed, target_s):
+    import oracle
+    from sparse_rank_linear_03_b200 import synth
+
+    def run(nrows):
+        W = synth.to_bf16_bits(synth.student_t_f32(nrows, n, seed))
+        t0 = time.perf_counter()
+        oracle.concentration(W, "bf16")
+        return time.perf_counter() - t0
+
+    dt = run(64)
+    nr = int(min(m, max(64, 64 * target_s / max(dt, 1e-3))))
+    dt = run(nr)
+    return nr * n * 2 / dt, f"{nr} of {m} rows (bf16): {dt:.2f} s"
+
+
 # ------------------------------------------------------------------ per-workload GPU leg
 
 def time_calls(fn, stream, reps=20, flush=None):
@@ -431,6 +467,19 @@ def measure_configs(dev, pk, oracle_seconds: float, with_oracle: bool) -> dict:
             recs[f"apply_b{b}"] = with_cpu(rec, cpu(oracle_layer_rate, lay.m, lay.n, wl.r, "csr",
                                                     wl.dtype, wl.frac, b, lay.seed,
                                                     oracle_seconds / 4), "GB/s")
+        if wl is ATTN4096:
+            # 2048 tokens: S decompressed block by block for the dense MMA
+            T = 2048
+            X, Y = xy(wl, lay, T)
+            ms = time_calls(lambda: L.apply(X, Y), stream, flush=flush)
+            dense = 2 * T * lay.m * lay.n + 2 * T * 2 * wl.r * (lay.m + lay.n)
+            rec = dict(_rate(dense, ms, pk["bf16"], "TFLOP/s"), flops_executed=dense,
+                       peak="bf16 burst",
+                       algorithmic_TFLOP_s=round(apply_flops(L.nnz(), lay.m, lay.n, wl.r, T)
+                                                 / (ms * 1e-3) / 1e12, 2))
+            recs[f"apply_T{T}"] = with_cpu(rec, cpu(oracle_layer_rate, lay.m, lay.n, wl.r, "csr",
+                                                    wl.dtype, wl.frac, T, lay.seed,
+                                                    oracle_seconds / 4), "TFLOP/s")
         web = 4 if wl.split_dtype == "f32" else 2
         ms = time_calls(lambda: L.split(W, wl.frac, None), stream, flush=flush)
         by = topk_split_bytes(lay.m, lay.n, L.nnz(), web, eb) - lay.m * lay.n * web  # no R
@@ -474,31 +523,82 @@ def measure_configs(dev, pk, oracle_seconds: float, with_oracle: bool) -> dict:
     # the 7B stack: 224 CSR matrices (3 %, r = 128) applied as one group at batch 1.
     # W is drawn on the device (same Student-t recipe; 6.5 G entries take minutes on the host).
     wl = STACK7B
-    layers, Xs, Ys, total = [], [], [], 0
+    layers, Xs, Ys, total, nnz_all = [], [], [], 0, 0
     for lay in wl.layers:
         Wd = synth.student_t_device(lay.m, lay.n, lay.seed, dev)
         L = hsl.Layer(lay.m, lay.n, wl.r, "csr", "bf16")
         L.split(Wd, wl.frac, None)
         U, V = synth.stand_in_factors_device(lay.m, lay.n, wl.r, lay.seed + 2, dev)
         L.pack(U, V)
-        del Wd, U, V
-        layers.append(L)
+        del Wd
+        layers.append((L, U, V))
         Xs.append(torch.randn(1, lay.n, generator=torch.Generator(device=dev).manual_seed(lay.seed + 1),
                               device=dev).to(torch.bfloat16))
         Ys.append(torch.empty(1, lay.m, dtype=torch.bfloat16, device=dev))
         total += csr_apply_bytes(L.nnz(), lay.m, lay.n, wl.r, 1, 2)
-    g = hsl.Group(layers)
-    ms = time_calls(lambda: g.apply(Xs, Ys), stream)
-    rec = dict(_rate(total, ms, pk["hbm"], "GB/s"), bytes=total, matrices=len(layers),
-               timing="back to back (1.43 GB > L2)")
+        nnz_all += L.nnz()
     gate = wl.layers[4]
-    out[wl.name] = {"group_apply_b1": with_cpu(
-        rec, cpu(oracle_layer_rate, gate.m, gate.n, wl.r, "csr", "bf16", wl.frac, 1, gate.seed,
-                 oracle_seconds / 4), "GB/s")}
-    g.close()
-    for L in layers:
+    recs = {}
+    for bits in (16, 8):
+        if bits != 16:
+            for L, U, V in layers:
+                L.set_index_bits(bits)
+                L.pack(U, V)
+        g = hsl.Group([L for L, _, _ in layers])
+        ms = time_calls(lambda: g.apply(Xs, Ys), stream)
+        # 8-bit columns: 1.25 index bytes per entry instead of 2
+        by = total if bits == 16 else total - nnz_all * 2 + nnz_all * 5 // 4
+        rec = dict(_rate(by, ms, pk["hbm"], "GB/s"), bytes=by, matrices=len(layers),
+                   column_bits=bits, timing="back to back (> L2)")
+        recs["group_apply_b1" if bits == 16 else "group_apply_b1_cols8"] = with_cpu(
+            rec, cpu(oracle_layer_rate, gate.m, gate.n, wl.r, "csr", "bf16", wl.frac, 1, gate.seed,
+                     oracle_seconds / 4) if bits == 16 else None, "GB/s")
+        g.close()
+    out[wl.name] = recs
+    for L, _, _ in layers:
         L.close()
+    del layers
     torch.cuda.synchronize()
+    return out
+
+
+def measure_stage2_and_permutation(W, R24, dev, pk, oracle_seconds: float, with_oracle: bool) -> dict:
+    """Stage 2 (randomized truncated SVD of the 70B layer's 2:4 residual, r = 256,
+    k = 266, two power iterations) and the concentration ratio and permuted copy
+    of its W, each timed with CUDA events (median of 5 after 2 warm-up calls)."""
+    import torch
+    from sparse_rank_linear_03_b200 import hsl
+    stream = torch.cuda.current_stream()
+    out = {}
+    k, q = R_RANK + 10, 2
+    L = hsl.Layer(M, N, R_RANK, "nm24", "bf16")
+    omega = torch.randn(N, k, generator=torch.Generator(device=dev).manual_seed(SEED + 7), device=dev)
+    ms = time_calls(lambda: L.factor(R24, omega, q), stream, reps=5)
+    fl = 2.0 * M * N * k * (2 * q + 2)
+    rec = dict(_rate(fl, ms, pk["bf16"], "TFLOP/s"), flops=fl, peak="bf16 burst",
+               note="algorithmic FLOPs of the 2q+2 tall products; each runs as three bf16 "
+                    "products (fp32-accurate), plus Gram matrices and Jacobi eigensolves")
+    if with_oracle:
+        v, sample = oracle_factor_rate(M, N, R_RANK, k, q, SEED, oracle_seconds)
+        rec["cpu_oracle"] = {"value": round(v / 1e12, 6), "unit": "TFLOP/s", "sample": sample}
+    out["factor_r256_k266_q2"] = rec
+    L.close()
+    ms = time_calls(lambda: hsl.concentration(W), stream, reps=5)
+    by = M * N * 2
+    rec = dict(_rate(by, ms, pk["hbm"], "GB/s"), bytes=by,
+               note="includes the result's device-to-host copy and stream synchronisation")
+    if with_oracle:
+        v, sample = oracle_rho_rate(M, N, SEED, oracle_seconds / 2)
+        rec["cpu_oracle"] = {"value": round(v / 1e9, 6), "unit": "GB/s", "sample": sample}
+    out["concentration"] = rec
+    g = torch.Generator(device=dev).manual_seed(SEED + 8)
+    ro = torch.randperm(M, generator=g, device=dev).to(torch.int32)
+    co = torch.randperm(N, generator=g, device=dev).to(torch.int32)
+    dst = torch.empty_like(W)
+    ms = time_calls(lambda: hsl.permute(W, ro, co, dst), stream, reps=5)
+    by = 2 * M * N * 2
+    out["permute"] = dict(_rate(by, ms, pk["hbm"], "GB/s"), bytes=by,
+                          note="includes the host-side check of both orders")
     return out
 
 
@@ -669,6 +769,8 @@ def run_gpu(args, world, rank, local):
                    "reasons": clocks["reasons"]},
     }
     if world == 1 and not args.no_configs:
+        result["stage2_and_permutation"] = measure_stage2_and_permutation(
+            W, R_24, dev, pk, args.cpu_seconds / 2, not args.no_cpu_baseline)
         del W, R_csr, R_24, Xp, Yp
         csr.close()
         nm.close()
