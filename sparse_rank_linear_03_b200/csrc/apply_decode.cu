@@ -590,6 +590,11 @@ constexpr int kSupChunks = 256;                  // chunks of a super-chunk
 constexpr int kUnitVBytes = kSupChunks * 16;     // values of a full unit
 constexpr int kUnitMBytes = kSupChunks * 2;      // metadata of a unit
 constexpr int kUnitSlot = kUnitVBytes + kUnitMBytes;
+// Rows per segment of the bulk-copy kernel.  A segment's U·z pass (U rows by
+// plain loads) runs while every warp's first S unit of the next segment is
+// already in flight, so short segments overlap the factor term with the S
+// stream; a multiple of 16 (= kB1Warps) keeps every warp's units in step.
+constexpr int kSegB1 = 64;
 
 struct B1Layout {
   int32_t xs;     // bytes of the staged x
@@ -601,7 +606,7 @@ B1Layout b1_layout(int n_max, int r_pad_max) {
   B1Layout L;
   L.xs = int32_t(round_up(int64_t(n_max) * 2, 16));
   L.nsup = int32_t(((n_max + 15) / 16 + kSupChunks - 1) / kSupChunks);
-  L.total = int32_t(int64_t(2 * kB1Warps) * kUnitSlot + L.xs + int64_t(kSeg) * L.nsup * 4 +
+  L.total = int32_t(int64_t(2 * kB1Warps) * kUnitSlot + L.xs + int64_t(kSegB1) * L.nsup * 4 +
                     int64_t(r_pad_max) * 4 + 2 * kB1Warps * 8 + 16);
   return L;
 }
@@ -646,8 +651,8 @@ __global__ void __maxnreg__(112) k_apply_24_b1_tma(ApplyArgs a, B1Layout lay) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   unsigned char* const slot0 = smem + (2 * warp) * kUnitSlot;
   __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(smem + 2 * kB1Warps * kUnitSlot);
-  float* ysp = reinterpret_cast<float*>(smem + 2 * kB1Warps * kUnitSlot + lay.xs);  // [kSeg][nsup]
-  float* zs = ysp + kSeg * lay.nsup;
+  float* ysp = reinterpret_cast<float*>(smem + 2 * kB1Warps * kUnitSlot + lay.xs);  // [kSegB1][nsup]
+  float* zs = ysp + kSegB1 * lay.nsup;
   uint64_t* bars = reinterpret_cast<uint64_t*>(
       (reinterpret_cast<uintptr_t>(zs + a.r_pad_max) + 7) & ~uintptr_t(7));
   uint64_t* const mybar = bars + 2 * warp;
@@ -777,7 +782,7 @@ __global__ void __maxnreg__(112) k_apply_24_b1_tma(ApplyArgs a, B1Layout lay) {
     const uint32_t nsup_magic = nsup > 1 ? 0xFFFFFFFFu / uint32_t(nsup) + 1u : 0u;
     const int units = (l1 - l0) * nsup;
     const int nu = warp < units ? (units - warp + kB1Warps - 1) / kB1Warps : 0;
-    const int useg = kSeg * nsup / kB1Warps;  // units of a warp in one segment
+    const int useg = kSegB1 * nsup / kB1Warps;  // units of a warp in one segment
     const uint32_t mstride = uint32_t(P.meta_stride) * 2u;
     const unsigned char* pval = static_cast<const unsigned char*>(P.pval);
     const unsigned char* pmeta = reinterpret_cast<const unsigned char*>(P.pmeta);
@@ -822,8 +827,8 @@ __global__ void __maxnreg__(112) k_apply_24_b1_tma(ApplyArgs a, B1Layout lay) {
     const uint4* xwin_lo = xs4 + 2 * lane + xsw;
     const uint4* xwin_hi = xs4 + 2 * lane + 1 - xsw;
     __nv_bfloat16* y = y_of<__nv_bfloat16>(a, p) + int64_t(a.b0) * P.m;
-    for (int s0 = l0, seg = 0; s0 < l1; s0 += kSeg, ++seg) {
-      const int s1 = min(s0 + kSeg, l1);
+    for (int s0 = l0, seg = 0; s0 < l1; s0 += kSegB1, ++seg) {
+      const int s1 = min(s0 + kSegB1, l1);
       const int jend = min(nu, (seg + 1) * useg);
       for (int j = seg * useg; j < jend; ++j) {
         const int sl = j & 1;
