@@ -922,6 +922,251 @@ __global__ void __maxnreg__(112) k_apply_24_b1_tma(ApplyArgs a, B1Layout lay) {
   }
 }
 
+// ---- batch-1 CSR, entries fed by bulk copies ----------------------------------------
+// The packed entries of a CTA's rows in one layer are contiguous, so the CTA
+// streams them as chunks of kCsrChunk entries (values, columns and, for 8-bit
+// columns, vector bases), 1-D bulk copies into a ring of shared-memory slots:
+// SLOTS − 1 chunks are requested ahead, so about two stay in flight while the
+// warps compute, without holding registers.  A row is taken when its last chunk
+// has landed; rows are at most kCsrChunk − 64 entries (longer rows read global
+// memory directly), so its first chunk is still in the ring.  Warp 0 finds the
+// rows that a chunk completes with ballots over the row starts staged in shared
+// memory; each row is one warp's (lane l takes vectors l, l + 32, …, a fixed
+// shuffle tree sums them).  S sums collect in a segment of kCsrSeg rows, whose
+// U·z pass (after z is ready, programmatic dependent launch) writes y.  Chunks
+// are aligned to 64 entries (the copies read up to 63 entries either side of a
+// CTA's range, inside the packed arrays' slack).
+constexpr int kCsrThreads = 512;
+constexpr int kCsrWarps = kCsrThreads / 32;
+constexpr int kCsrChunk = 4096;
+constexpr int kCsrSeg = 1024;
+constexpr int kCsrProw = 8192;  // rows per staged window of row starts
+constexpr int kCsrMaxSlots = 6;
+
+struct CsrLayout {
+  int32_t slots;
+  int32_t vbytes, cbytes, bbytes;  // per chunk: values, columns, vector bases
+  int32_t slot;                    // bytes of a slot
+  int32_t xs;                      // bytes of the staged x (n_max + 1 values)
+  int32_t total;                   // dynamic shared memory
+};
+
+CsrLayout csr_layout(int eb, int idx_bits, int n_max, int r_pad_max, int smem_max) {
+  CsrLayout L;
+  L.vbytes = kCsrChunk * eb;
+  L.cbytes = idx_bits == 8 ? kCsrChunk : kCsrChunk * (idx_bits / 8);
+  L.bbytes = idx_bits == 8 ? kCsrChunk / 8 * 2 : 0;
+  L.slot = L.vbytes + L.cbytes + L.bbytes;
+  L.xs = int32_t(round_up(int64_t(n_max + 1) * eb, 16));
+  const int fixed = L.xs + (kCsrProw + 1) * 4 + kCsrSeg * 4 + r_pad_max * 4 + kCsrMaxSlots * 8 + 64;
+  L.slots = std::min(kCsrMaxSlots, (smem_max - fixed) / L.slot);
+  L.total = L.slots * L.slot + fixed;
+  return L;
+}
+
+template <typename T, int IDX>
+__device__ __forceinline__ float csr_vec_dot(const T* xs, const unsigned char* vals,
+                                             const unsigned char* cols, const uint16_t* bases,
+                                             int off) {
+  // values of entries [off, off + 8) of the slot (or of global memory)
+  RawVals<T> rv;
+  if constexpr (sizeof(T) == 2) {
+    rv.q = *reinterpret_cast<const uint4*>(vals + size_t(off) * 2);
+  } else {
+    rv.a = *reinterpret_cast<const uint4*>(vals + size_t(off) * 4);
+    rv.b = *reinterpret_cast<const uint4*>(vals + size_t(off) * 4 + 16);
+  }
+  int c[8];
+  if constexpr (IDX == 16) {
+    const uint4 q = *reinterpret_cast<const uint4*>(cols + size_t(off) * 2);
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int t = 0; t < 8; ++t) c[t] = int((w[t >> 1] >> ((t & 1) * 16)) & 0xFFFFu);
+  } else if constexpr (IDX == 32) {
+    const uint4 qa = *reinterpret_cast<const uint4*>(cols + size_t(off) * 4);
+    const uint4 qb = *reinterpret_cast<const uint4*>(cols + size_t(off) * 4 + 16);
+    c[0] = int(qa.x); c[1] = int(qa.y); c[2] = int(qa.z); c[3] = int(qa.w);
+    c[4] = int(qb.x); c[5] = int(qb.y); c[6] = int(qb.z); c[7] = int(qb.w);
+  } else {
+    const uint2 d = *reinterpret_cast<const uint2*>(cols + off);
+    int v = int(bases[off >> 3]);
+    c[0] = v;
+#pragma unroll
+    for (int t = 1; t < 8; ++t) {
+      v += int(((t < 4 ? d.x : d.y) >> (8 * (t & 3))) & 0xFFu);
+      c[t] = v;
+    }
+  }
+  float acc = 0.f;
+#pragma unroll
+  for (int t = 0; t < 8; ++t) acc = fmaf(rv.at(t), VT<T>::f(xs[c[t]]), acc);
+  return acc;
+}
+
+template <typename T, int IDX>
+__global__ void __launch_bounds__(kCsrThreads, 1) k_apply_csr_b1(ApplyArgs a, CsrLayout lay) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ int sh_end, abort_flag;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int SL = lay.slots;
+  T* xs = reinterpret_cast<T*>(smem + SL * lay.slot);
+  int32_t* prow_s = reinterpret_cast<int32_t*>(smem + SL * lay.slot + lay.xs);
+  float* ysp = reinterpret_cast<float*>(prow_s + kCsrProw + 1);
+  float* zs = ysp + kCsrSeg;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(
+      (reinterpret_cast<uintptr_t>(zs + a.r_pad_max) + 7) & ~uintptr_t(7));
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int i = 0; i < SL; ++i) tc::mbar_init(&bars[i], 1);
+    tc::fence_mbar_init();
+  }
+  __syncthreads();
+  volatile int* abrt = &abort_flag;
+  uint32_t ph = 0u, pending = 0u;  // per slot: parity of the next wait, a copy in flight
+  const uint64_t policy = tc::make_policy_evict_first();
+
+  const int64_t slo = int64_t(blockIdx.x) * a.slices / gridDim.x;
+  const int64_t shi = int64_t(blockIdx.x + 1) * a.slices / gridDim.x;
+  int64_t row = a.cta_rows[slo];
+  const int64_t row_end = a.cta_rows[shi];
+  int p = 0;
+  {
+    int lo = 0, hi = a.count - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (a.prob_row0[mid] <= row) lo = mid; else hi = mid - 1;
+    }
+    p = lo;
+  }
+  bool waited = false;
+  while (row < row_end) {
+    const ApplyProblem P = a.probs[p];
+    const int64_t p_end = a.prob_row0[p + 1];
+    const int lp0 = int(row - P.row0);
+    const int lp1 = int(min(row_end, p_end) - P.row0);
+    const T* x = x_of<T>(a, p);
+    T* y = y_of<T>(a, p);
+    const int n = P.n;
+    __syncthreads();  // the previous layer is done with xs and zs
+    for (int c = threadIdx.x; c < n; c += kCsrThreads) xs[c] = x[c];
+    if (threadIdx.x == 0) xs[n] = VT<T>::from_f(0.f);
+    bool z_staged = false;
+    // sub-parts of at most kCsrProw rows: their row starts fit the staged window
+    for (int w0 = lp0; w0 < lp1; w0 += kCsrProw) {
+      const int w1 = min(lp1, w0 + kCsrProw);
+      __syncthreads();
+      for (int i = threadIdx.x; i <= w1 - w0; i += kCsrThreads) prow_s[i] = P.prow[w0 + i];
+      __syncthreads();
+      const int64_t E0 = prow_s[0], E1 = prow_s[w1 - w0];
+      const int64_t A0 = E0 & ~int64_t(63), A1 = (E1 + 63) & ~int64_t(63);
+      const int nch = int((A1 - A0 + kCsrChunk - 1) / kCsrChunk);
+      const unsigned char* gv = static_cast<const unsigned char*>(P.pval);
+      const unsigned char* gc = static_cast<const unsigned char*>(P.pcol);
+      const unsigned char* gb = reinterpret_cast<const unsigned char*>(P.pbase);
+      const int eb = int(sizeof(T));
+      const int cbn = IDX == 8 ? 1 : IDX / 8;
+      auto issue = [&](int c) {  // thread 0: chunk c into its slot
+        if (*abrt) return;
+        const int sl = c % SL;
+        const int64_t st = A0 + int64_t(c) * kCsrChunk;
+        const int cnt = int(A1 - st < int64_t(kCsrChunk) ? A1 - st : int64_t(kCsrChunk));
+        unsigned char* dst = smem + sl * lay.slot;
+        const uint32_t vb = uint32_t(cnt * eb), cb = uint32_t(cnt * cbn);
+        const uint32_t bb = IDX == 8 ? uint32_t(cnt / 8 * 2) : 0u;
+        tc::fence_async_smem();
+        tc::mbar_expect_tx(&bars[sl], vb + cb + bb);
+        tc::bulk_load_hint(dst, gv + st * eb, vb, &bars[sl], policy);
+        tc::bulk_load_hint(dst + lay.vbytes, gc + st * cbn, cb, &bars[sl], policy);
+        if (IDX == 8) tc::bulk_load_hint(dst + lay.vbytes + lay.cbytes, gb + st / 8 * 2, bb, &bars[sl], policy);
+        pending |= 1u << sl;
+      };
+      if (threadIdx.x == 0)
+        for (int c = 0; c < min(nch, SL - 1); ++c) issue(c);
+      int cur = w0, seg0 = w0;
+      for (int c = 0; c < nch || cur < w1; ++c) {
+        if (c < nch) {
+          const int sl = c % SL;
+          if (!*abrt) {
+            const bool ok = tc::mbar_wait(&bars[sl], (ph >> sl) & 1u, a.err);
+            if (!ok) *abrt = 1;
+          }
+          ph ^= 1u << sl;
+          if (threadIdx.x == 0) pending &= ~(1u << sl);
+        }
+        const int64_t bound = c + 1 < nch ? A0 + int64_t(c + 1) * kCsrChunk : INT64_MAX;
+        // the rows this chunk completes, kCsrSeg at most per pass
+        for (;;) {
+          __syncthreads();
+          if (warp == 0) {
+            int r = cur;
+            const int cap = min(w1, seg0 + kCsrSeg);
+            for (;;) {
+              const int q = r + lane;
+              const bool ok = q < cap && int64_t(prow_s[q + 1 - w0]) <= bound;
+              const unsigned b = __ballot_sync(0xffffffffu, ok);
+              const int cnt = __popc(b);
+              r += cnt;
+              if (cnt < 32) break;
+            }
+            if (lane == 0) sh_end = r;
+          }
+          __syncthreads();
+          const int rend = sh_end;
+          if (!*abrt) {
+            for (int r = cur + warp; r < rend; r += kCsrWarps) {
+              const int e0 = prow_s[r - w0], e1 = prow_s[r + 1 - w0];
+              float acc = 0.f;
+              if (e1 - e0 <= kCsrChunk - 64) {
+                for (int e = e0 + 8 * lane; e < e1; e += 256) {
+                  const int64_t pos = int64_t(e) - A0;
+                  const int sl = int((pos / kCsrChunk) % SL), off = int(pos % kCsrChunk);
+                  const unsigned char* base = smem + sl * lay.slot;
+                  acc += csr_vec_dot<T, IDX>(xs, base, base + lay.vbytes,
+                                             reinterpret_cast<const uint16_t*>(base + lay.vbytes + lay.cbytes),
+                                             off);
+                }
+              } else {  // a long row: straight from global memory
+                for (int e = e0 + 8 * lane; e < e1; e += 256)
+                  acc += csr_vec_dot<T, IDX>(xs, gv, gc, P.pbase, e);
+              }
+#pragma unroll
+              for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+              if (lane == 0) ysp[r - seg0] = acc;
+            }
+          }
+          cur = rend;
+          if (cur - seg0 == kCsrSeg || (cur == w1 && cur > seg0)) {
+            // the segment's U·z pass (z from the preceding kernel)
+            if (!waited) {
+              pdl_wait();
+              waited = true;
+            }
+            __syncthreads();
+            if (!z_staged && P.r_pad > 0) {
+              for (int o = threadIdx.x; o < P.r_pad; o += kCsrThreads) zs[o] = __ldcg(P.z + o);
+              z_staged = true;
+            }
+            __syncthreads();
+            urows<T, 1, kCsrThreads>(P, zs, ysp, seg0, cur, y, 1);
+            seg0 = cur;
+            continue;  // the chunk may complete more rows
+          }
+          break;
+        }
+        __syncthreads();  // every warp is done with chunk c - 1
+        if (threadIdx.x == 0 && c + SL - 1 < nch) issue(c + SL - 1);
+        if (c >= nch) break;
+      }
+    }
+    row = P.row0 + lp1;
+    ++p;
+  }
+  // after an abort, copies still in flight land before the CTA exits
+  if (threadIdx.x == 0)
+    for (int sl = 0; sl < SL; ++sl)
+      if ((pending >> sl) & 1u) tc::mbar_wait(&bars[sl], (ph >> sl) & 1u, a.err);
+}
+
 // Shared memory a CTA of the current device may opt in to.
 int max_dyn_smem() {
   int dev = 0, v = 0;
@@ -940,6 +1185,13 @@ bool decode_b1_bulk_enabled() {
     return !(e && std::strcmp(e, "regs") == 0);
   }();
   return on;
+}
+
+// HSL_DECODE_CSR=regs (read on every call) keeps batch-1 CSR on the
+// register-fed kernel (a cross-check of the bulk-copy fed one).
+bool decode_csr_bulk_enabled() {
+  const char* e = std::getenv("HSL_DECODE_CSR");
+  return !(e && std::strcmp(e, "regs") == 0);
 }
 
 template <typename T, int BC>
@@ -979,6 +1231,11 @@ hsl_status launch_chunk(ApplyPlan& plan, ApplyArgs a, int num_sms, cudaStream_t 
       return cuda_fail(cudaLaunchKernelEx(&cfg, bk, a, lay), "apply launch");
     }
   }
+  // batch-1 CSR: the bulk-copy fed kernel when its ring fits shared memory
+  const bool csr_bulk = BC == 1 && plan.fmt == HSL_FMT_CSR && decode_csr_bulk_enabled();
+  CsrLayout clay{};
+  if (csr_bulk) clay = csr_layout(int(sizeof(T)), plan.idx_bits, plan.n_max, plan.r_pad_max, max_dyn_smem());
+  const bool use_csr_bulk = csr_bulk && clay.slots >= 3;
   // z = Vᵀ x, normal launch (waits for everything before it on the stream)
   if (plan.z_items > 0) {
     auto zk = k_lowrank_z<T, BC>;
@@ -1000,6 +1257,18 @@ hsl_status launch_chunk(ApplyPlan& plan, ApplyArgs a, int num_sms, cudaStream_t 
   attr[0].val.programmaticStreamSerializationAllowed = plan.z_items > 0 ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (use_csr_bulk) {
+    auto ck = plan.idx_bits == 8    ? k_apply_csr_b1<T, 8>
+              : plan.idx_bits == 32 ? k_apply_csr_b1<T, 32>
+                                    : k_apply_csr_b1<T, 16>;
+    if (cudaError_t e = cudaFuncSetAttribute(ck, cudaFuncAttributeMaxDynamicSharedMemorySize, clay.total))
+      return cuda_fail(e, "apply smem attribute");
+    cfg.blockDim = dim3(kCsrThreads);
+    cfg.gridDim = dim3(unsigned(std::min<int64_t>(num_sms, row_cap)));
+    cfg.dynamicSmemBytes = size_t(clay.total);
+    note_launch();
+    return cuda_fail(cudaLaunchKernelEx(&cfg, ck, a, clay), "apply launch");
+  }
   const size_t sm = apply_smem<T, BC>(plan);
   if (sm > size_t(std::max(max_dyn_smem(), 0))) {
     set_message("the staged x of this layer does not fit in shared memory");

@@ -381,7 +381,8 @@ hsl_status pack_sparse_run(Handle& h, cudaStream_t s) {
         set_message("8-bit delta columns need the columns of every row in ascending order");
         return HSL_ERR_UNSUPPORTED;
       }
-      const int64_t cap = round_up(int64_t(total) + 8, 8);
+      // slack past the last row: the bulk-fed decode copies whole 64-entry blocks
+      const int64_t cap = round_up(int64_t(total) + 64, 64);
       if (hsl_status e = ensure(h.pcol, size_t(cap), "packed column deltas")) return e;
       if (hsl_status e = ensure(h.pbase, size_t(cap / 8) * 2, "packed vector bases")) return e;
       if (hsl_status e = ensure(h.pval, size_t(cap) * eb, "packed values")) return e;
@@ -400,7 +401,9 @@ hsl_status pack_sparse_run(Handle& h, cudaStream_t s) {
             static_cast<uint32_t*>(h.pval.p), static_cast<uint32_t*>(h.err.p));
       note_launch();
     } else {
-      const int64_t cap = round_up(h.nnz + 7 * h.m + 8, 8);  // multiple of 8: every row start stays 16-byte aligned
+      // every row start a multiple of 8 (16-byte aligned vectors); slack past the
+      // last row, as the bulk-fed decode copies whole 64-entry blocks
+      const int64_t cap = round_up(h.nnz + 7 * h.m + 64, 64);
       const int cb = bits / 8;
       if (hsl_status e = ensure(h.pcol, size_t(cap) * cb, "packed columns")) return e;
       if (hsl_status e = ensure(h.pval, size_t(cap) * eb, "packed values")) return e;

@@ -228,3 +228,64 @@ def test_bad_imported_column_reported(hsl):
     with pytest.raises(hsl.HslError) as e:
         L.check()
     assert e.value.name == "HSL_ERR_INVALID_ARG"
+
+
+# ---------------------------------------------------------------- batch-1 CSR, bulk-copy fed
+
+def _import_csr(hsl, m, n, rp, col, vals, dtype="bf16", r=0, seed=0):
+    L = hsl.Layer(m, n, r, "csr", dtype)
+    L.set_sparse_csr(torch.from_numpy(np.asarray(rp, np.int32)).cuda(),
+                     torch.from_numpy(np.asarray(col, np.int32)).cuda(), dev(vals, dtype))
+    rng = np.random.default_rng(seed)
+    U = synth.as_storage((0.05 * rng.standard_normal((m, r))).astype(np.float32), dtype)
+    V = synth.as_storage((0.05 * rng.standard_normal((n, r))).astype(np.float32), dtype)
+    L.pack(dev(U, dtype), dev(V, dtype))
+    return L, U, V
+
+
+def test_csr_batch1_long_rows_and_empty_rows(hsl):
+    """Rows longer than a streamed chunk (read from global memory), rows with
+    no entries, and ordinary rows between them."""
+    m, n = 300, 8192
+    rng = np.random.default_rng(12)
+    lens = rng.integers(0, 60, size=m)
+    lens[::7] = 0
+    lens[5], lens[150], lens[299] = 5000, 8192, 4033
+    rp = np.zeros(m + 1, np.int64)
+    rp[1:] = np.cumsum(lens)
+    col = np.concatenate([np.sort(rng.choice(n, size=l, replace=False)) for l in lens]).astype(np.int32)
+    vals = synth.to_bf16_bits(rng.standard_normal(int(rp[-1])).astype(np.float32))
+    L, U, V = _import_csr(hsl, m, n, rp, col, vals, r=8, seed=3)
+    X = synth.to_bf16_bits(synth.normal_f32(1, n, 4))
+    Y = L.apply(dev(X, "bf16"))
+    L.check()
+    Sd = oracle.csr_to_dense(m, n, rp, col, f64(vals, "bf16"))
+    ref = oracle.apply(oracle.reconstruct(Sd, f64(U, "bf16"), f64(V, "bf16")), f64(X, "bf16"))
+    assert oracle.rel_err(f64(host(Y), "bf16"), ref) <= TOL["bf16"]
+    assert oracle.elem_rel_err(f64(host(Y), "bf16"), ref) <= ELEM_TOL["bf16"]
+
+
+def test_csr_batch1_many_rows_per_cta(hsl):
+    """1.3 M rows of 16 columns: each CTA's range is longer than the window of
+    row starts it stages, so it runs in several sub-parts."""
+    m, n = 1_300_000, 16
+    c = Case(hsl, m, n, 4, "csr", "f32", 0.1, 13)
+    Xb = c.x(1, 14)
+    rows = np.sort(np.random.default_rng(15).choice(m, 4000, replace=False))
+    rows[-1] = m - 1
+    assert err_of(c, c.L.apply(dev(Xb, "f32")), Xb, rows) <= TOL["f32"]
+
+
+@pytest.mark.parametrize("bits", [8, 16, 32])
+def test_csr_batch1_bulk_and_register_kernels_agree(hsl, monkeypatch, bits):
+    """The bulk-copy fed and the register-fed batch-1 CSR kernels sum each row
+    in different orders; they agree to bf16 output rounding."""
+    c = Case(hsl, 3000, 2048, 16, "csr", "bf16", 0.03, 16)
+    c.L.set_index_bits(bits)
+    c.L.pack(dev(c.U, "bf16"), dev(c.V, "bf16"))
+    X = dev(c.x(1, 17), "bf16")
+    a = f64(host(c.L.apply(X)), "bf16")
+    monkeypatch.setenv("HSL_DECODE_CSR", "regs")
+    b = f64(host(c.L.apply(X)), "bf16")
+    monkeypatch.delenv("HSL_DECODE_CSR")
+    assert oracle.rel_err(a, b) <= 2 ** -7
