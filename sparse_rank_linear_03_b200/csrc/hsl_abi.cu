@@ -100,7 +100,7 @@ struct DeviceGuard {
 
 // A device array of `len` int32 that must hold each of 0..len-1 once: copied to
 // the host and checked there (the permutation calls are one-off set-up steps).
-hsl_status check_order(const int32_t* order_dev, int64_t len, const char* what, cudaStream_t s) {
+hsl_status check_order(const int32_t* order_dev, int64_t len, const char* what, cudaStream_t s) try {
   std::vector<int32_t> h(static_cast<size_t>(len));
   if (cudaError_t e = cudaMemcpyAsync(h.data(), order_dev, size_t(len) * 4, cudaMemcpyDefault, s))
     return cuda_fail(e, "order copy");
@@ -114,6 +114,9 @@ hsl_status check_order(const int32_t* order_dev, int64_t len, const char* what, 
     seen[size_t(v)] = 1;
   }
   return HSL_OK;
+} catch (const std::bad_alloc&) {
+  set_message("host allocation failed while checking an order");
+  return HSL_ERR_OOM;
 }
 
 hsl_status ensure_err_word(Handle& h, cudaStream_t s) {
@@ -578,9 +581,20 @@ hsl_status hsl_rcm_order(int64_t m, int64_t n, const int32_t* row_ptr, const int
   t_msg.clear();
   if (!row_ptr || !row_order || !col_order) return invalid("NULL argument");
   if (m < 1 || n < 1 || m > INT32_MAX || n > INT32_MAX) return invalid("m and n out of range");
-  if (row_ptr[0] != 0 || row_ptr[m] < 0) return invalid("row_ptr must start at 0");
+  if (row_ptr[0] != 0) return invalid("row_ptr must start at 0");
+  for (int64_t i = 0; i < m; ++i)
+    if (row_ptr[i + 1] < row_ptr[i]) return invalid("row_ptr is not monotone");
+  if (int64_t(row_ptr[m]) > m * n) return invalid("row_ptr[m] exceeds m*n");
   if (row_ptr[m] > 0 && !col) return invalid("col is NULL");
-  return rcm_order(m, n, row_ptr, col, row_order, col_order);
+  try {
+    return rcm_order(m, n, row_ptr, col, row_order, col_order);
+  } catch (const std::bad_alloc&) {
+    set_message("host allocation failed in the RCM order");
+    return HSL_ERR_OOM;
+  } catch (...) {
+    set_message("RCM order failed");
+    return HSL_ERR_INVALID_ARG;
+  }
 }
 
 hsl_status hsl_permute(const void* W, int64_t m, int64_t n, hsl_dtype dtype,
