@@ -423,8 +423,7 @@ struct SpMaps {
 
 __global__ void __launch_bounds__(192, 1)
     k_prefill_24sp(const __grid_constant__ SpMaps maps, const uint2* __restrict__ meta,
-                   __nv_bfloat16* __restrict__ Y, int m, int n, int T, int r16, uint32_t* err,
-                   int raster) {
+                   __nv_bfloat16* __restrict__ Y, int m, int n, int T, int r16, uint32_t* err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -440,21 +439,7 @@ __global__ void __launch_bounds__(192, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntn = (T + SP_BN - 1) / SP_BN;
-  // tile order: with raster = G > 0, CTAs in launch order sweep G row panels of
-  // S across every token tile before the next G panels (a working set of G
-  // panels and all of X); raster = 0 takes a panel's token tiles in a row
-  int mt, nt;
-  if (raster > 0) {
-    const int mtn = (m + 255) / 256;
-    const int per_group = raster * ntn;
-    const int g = blockIdx.x / per_group, idx = blockIdx.x % per_group;
-    const int gsize = min(raster, mtn - g * raster);
-    mt = g * raster + idx % gsize;
-    nt = idx / gsize;
-  } else {
-    mt = blockIdx.x / ntn;
-    nt = blockIdx.x % ntn;
-  }
+  const int mt = blockIdx.x / ntn, nt = blockIdx.x % ntn;
   const int i0 = mt * 256, t0 = nt * SP_BN;
   const int nkS = n / 64;
   const int nkL = (r16 + 31) / 32;
@@ -922,14 +907,6 @@ constexpr int64_t kPairMinTokens = 512;
 // HSL_PREFILL_PAIRS=1 selects the CTA-pair kernel.  It is exact (the parity
 // tests cover it) but measured slower than the single-CTA kernel on the 70B
 // layer (3.2 ms against 1.66 ms for 4096 tokens), so it is not the default.
-// HSL_PREFILL_RASTER=G (read on every call): row panels per group of the tile
-// order; 0 (the default) keeps a panel's token tiles together.
-int prefill_raster() {
-  const char* e = std::getenv("HSL_PREFILL_RASTER");
-  const int g = e ? std::atoi(e) : 0;
-  return g > 0 ? g : 0;
-}
-
 bool prefill_pairs_enabled() {
   const char* e = std::getenv("HSL_PREFILL_PAIRS");
   return e != nullptr && e[0] == '1';
@@ -1059,7 +1036,7 @@ hsl_status apply_prefill_run(Handle& h, const void* X, void* Y, int64_t T, cudaS
     return cuda_fail(cudaLaunchKernelEx(&cfg, k_prefill_24sp, sm,
                                         static_cast<const uint2*>(h.pmeta_tc.p),
                                         static_cast<__nv_bfloat16*>(Y), int(m), int(n), int(T),
-                                        r16, err0, prefill_raster()),
+                                        r16, err0),
                      "sparse prefill launch");
   }
   PrefillMaps maps;

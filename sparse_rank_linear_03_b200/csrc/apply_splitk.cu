@@ -17,7 +17,8 @@
 //   k_apply_24_splitk<TP>  per unit: TMA of the 128×32 compressed values
 //                (64-byte swizzle) and the X block [TP tokens × 64] (128-byte
 //                swizzle, tokens past T zero-filled), 1 KB of TMEM-ordered
-//                metadata by bulk copy; two tcgen05.mma.sp of K = 32 into a
+//                metadata by bulk copy, spread to one 16-byte row per TMEM
+//                lane and copied into TMEM by tcgen05.cp; two tcgen05.mma.sp of K = 32 into a
 //                128×TP fp32 accumulator in TMEM.  A CTA's range covers the end
 //                of one tile and the start of the next (or a whole tile), so it
 //                keeps two accumulators and hands each finished tile segment to
@@ -31,7 +32,8 @@
 //   call.  Nobody waits on anybody: no spin on another CTA.
 //
 // Warp roles (320 threads): warp 0 lane 0 issues the copies; warp 1 owns TMEM
-// and lane 0 issues the MMAs; warps 2-5 copy each unit's metadata into TMEM;
+// and lane 0 copies each unit's metadata into TMEM (tcgen05.cp, ordered before
+// its MMAs) and issues the MMAs; warps 2-5 lay the metadata out for that copy;
 // warps 6-9 run the epilogues (TMEM lane quarter = warp % 4).  Every wait is
 // bounded; a wait that gives up sets the error word, and the CTA still drains
 // its copies, takes part in the tile counters and frees TMEM.
@@ -49,13 +51,14 @@ namespace {
 
 constexpr int SK_THREADS = 320;
 constexpr int SK_A = 128 * 64;      // compressed values of a unit: 128 rows × 64 bytes
-constexpr int SK_M = 128 * 8;       // TMEM-ordered metadata of a unit
+constexpr int SK_M = 128 * 8;       // TMEM-ordered metadata of a unit (compact)
+constexpr int SK_MX = 2 * 128 * 16; // the same, one 16-byte row per TMEM lane and MMA
 constexpr uint32_t SK_TMEM_COLS = 256;
 // accumulator b at TMEM column 64·b
 __host__ __device__ constexpr uint32_t sk_acc_col(int b) { return 64u * uint32_t(b); }
 
-__host__ __device__ constexpr int sk_stages(int tp) { return tp <= 32 ? 8 : 6; }
-__host__ __device__ constexpr int sk_stage_bytes(int tp) { return SK_A + tp * 128 + SK_M; }
+__host__ __device__ constexpr int sk_stages(int tp) { return tp <= 16 ? 6 : tp <= 32 ? 5 : 4; }
+__host__ __device__ constexpr int sk_stage_bytes(int tp) { return SK_A + tp * 128 + SK_M + SK_MX; }
 __host__ __device__ constexpr int sk_smem(int tp) {
   return sk_stages(tp) * sk_stage_bytes(tp) + 1024 + 256;
 }
@@ -115,34 +118,46 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
 __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 // ---- z = Vᵀ x ------------------------------------------------------------------
-// One warp per (row c of Vt, 8 tokens): 16-byte loads of the row and of the
-// tokens, fp32 sums, a fixed shuffle tree.  n % 64 == 0 and 16-byte aligned X.
-constexpr int kSkZThreads = 128;
+// Work items (row c of Vt, 8 tokens) are cut into pieces of 256 columns, a warp
+// per piece (16-byte loads of the row and of the 8 tokens, fixed shuffle
+// trees), so thousands of warps share the V stream.  Each piece's 8 sums go to
+// its own slot; the warp that finishes an item last (a counter per item)
+// adds the item's pieces in piece order and writes z, then resets the counter:
+// the result does not depend on timing, and no warp waits for another.
+constexpr int kSkZThreads = 256;
+constexpr int kSkZPiece = 256;  // columns per piece
 __global__ void __launch_bounds__(kSkZThreads) k_splitk_z(const __nv_bfloat16* __restrict__ Vt,
                                                           const __nv_bfloat16* __restrict__ X,
                                                           float* __restrict__ z, int n, int T,
-                                                          int r, int r_pad) {
+                                                          int r, int r_pad, float* __restrict__ zpart,
+                                                          unsigned* __restrict__ zcnt) {
   pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int tb_count = (T + 7) / 8;
+  const int Q = (n + kSkZPiece - 1) / kSkZPiece;
   const long long items = (long long)r * tb_count;
+  const long long total = items * Q;
   const long long nw = (long long)gridDim.x * (kSkZThreads / 32);
-  for (long long it = ((long long)blockIdx.x * kSkZThreads + threadIdx.x) >> 5; it < items;
-       it += nw) {
-    const int c = int(it / tb_count), tb = int(it % tb_count);
+  for (long long it = ((long long)blockIdx.x * kSkZThreads + threadIdx.x) >> 5; it < total; it += nw) {
+    const long long item = it / Q;
+    const int q = int(it - item * Q);
+    const int c = int(item / tb_count), tb = int(item % tb_count);
     const int t0 = tb * 8;
-    const __nv_bfloat16* vrow = Vt + (long long)c * n;
+    const int j = q * kSkZPiece + lane * 8;
     float acc[8];
 #pragma unroll
     for (int b = 0; b < 8; ++b) acc[b] = 0.f;
-    for (int j = lane * 8; j < n; j += 256) {
-      const uint4 v = ld_stream16(vrow + j);
+    if (j < n) {
+      const uint4 v = ld_stream16(Vt + (long long)c * n + j);
       const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+      uint4 xq[8];
+#pragma unroll
+      for (int b = 0; b < 8; ++b)
+        if (t0 + b < T) xq[b] = *reinterpret_cast<const uint4*>(X + (long long)(t0 + b) * n + j);
 #pragma unroll
       for (int b = 0; b < 8; ++b) {
         if (t0 + b < T) {
-          const uint4 xq = *reinterpret_cast<const uint4*>(X + (long long)(t0 + b) * n + j);
-          const uint32_t xw[4] = {xq.x, xq.y, xq.z, xq.w};
+          const uint32_t xw[4] = {xq[b].x, xq[b].y, xq[b].z, xq[b].w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             acc[b] = fmaf(bf_lo(vw[e]), bf_lo(xw[e]), acc[b]);
@@ -152,10 +167,30 @@ __global__ void __launch_bounds__(kSkZThreads) k_splitk_z(const __nv_bfloat16* _
       }
     }
 #pragma unroll
-    for (int b = 0; b < 8; ++b) {
+    for (int b = 0; b < 8; ++b)
 #pragma unroll
       for (int o = 16; o; o >>= 1) acc[b] += __shfl_xor_sync(0xffffffffu, acc[b], o);
-      if (lane == 0 && t0 + b < T) z[(long long)(t0 + b) * r_pad + c] = acc[b];
+    float* slot = zpart + (item * Q + q) * 8;
+    if (lane < 8) {
+      float mine = acc[0];
+#pragma unroll
+      for (int b = 1; b < 8; ++b)
+        if (lane == b) mine = acc[b];
+      slot[lane] = mine;
+    }
+    __threadfence();
+    __syncwarp();
+    unsigned last = 0;
+    if (lane == 0) last = atomicAdd(&zcnt[item], 1u) == unsigned(Q - 1);
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (last) {
+      __threadfence();
+      if (lane < 8 && t0 + lane < T) {
+        float zv = 0.f;
+        for (int qq = 0; qq < Q; ++qq) zv += __ldcg(zpart + (item * Q + qq) * 8 + lane);
+        z[(long long)(t0 + lane) * r_pad + c] = zv;
+      }
+      if (lane == 0) zcnt[item] = 0u;  // ready for the next call
     }
   }
 }
@@ -257,6 +292,10 @@ __global__ void __launch_bounds__(SK_THREADS, 2)
         const uint64_t ad = tc::desc_sw64(st);
         const uint64_t bd = tc::desc_sw128(st + SK_A);
         const uint32_t d = tmem + sk_acc_col(seg & 1);
+        // the unit's metadata into its TMEM slots, ahead of the MMAs that read it
+        const unsigned char* mx = st + SK_A + B_BYTES + SK_M;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) tc::tmem_cp_128x128b(tmem + sk_meta_col(s, i), tc::desc_rows16(mx + i * 2048));
 #pragma unroll
         for (int i = 0; i < 2; ++i)
           tc::mma_bf16_sp(d, tc::desc_advance(ad, 32 * i), tc::desc_advance(bd, 64 * i),
@@ -266,19 +305,20 @@ __global__ void __launch_bounds__(SK_THREADS, 2)
       }
     }
   } else if (warp < 6) {
-    // metadata of each unit into its stage's TMEM slots (TMEM lane = L)
+    // metadata of each unit, expanded to one 16-byte row per TMEM lane and MMA
+    // (the layout tcgen05.cp copies); the MMA thread moves it into TMEM
     const int L = ((warp & 3) << 5) | lane;
-    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     for (long long u = u0; u < u1; ++u) {
       const int k = int(u - u0), s = k % ST;
       const uint32_t ph = (k / ST) & 1;
-      // the stage's bytes have landed, so its previous MMAs are done with the slots
+      // the stage's bytes have landed, so the MMAs of its previous use are done
       if (!wait_or_abort(&full[s], ph, a.err, abrt)) break;
-      const uint2 w = *reinterpret_cast<const uint2*>(smem + s * STAGE + SK_A + B_BYTES + L * 8);
-      tc::tmem_st1(tmem + lane_base + sk_meta_col(s, 0), w.x);
-      tc::tmem_st1(tmem + lane_base + sk_meta_col(s, 1), w.y);
-      tc::tmem_st_wait();
-      tc::tc_fence_before();
+      unsigned char* st = smem + s * STAGE;
+      const uint2 w = *reinterpret_cast<const uint2*>(st + SK_A + B_BYTES + L * 8);
+      unsigned char* mx = st + SK_A + B_BYTES + SK_M;
+      *reinterpret_cast<uint4*>(mx + L * 16) = make_uint4(w.x, 0u, 0u, 0u);
+      *reinterpret_cast<uint4*>(mx + 2048 + L * 16) = make_uint4(w.y, 0u, 0u, 0u);
+      tc::fence_async_smem();
       tc::mbar_arrive(&mfull[s]);
     }
   } else {
@@ -394,6 +434,10 @@ hsl_status launch_tp(Handle& h, const void* X, void* Y, int64_t T, cudaStream_t 
   const int smem = sk_smem(TP);
   if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))
     return cuda_fail(e, "split-K smem attribute");
+  // two CTAs per SM need the largest shared-memory carveout
+  if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                           int(cudaSharedmemCarveoutMaxShared)))
+    return cuda_fail(e, "split-K carveout attribute");
   int occ = 0;
   if (cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, SK_THREADS, smem))
     return cuda_fail(e, "split-K occupancy");
@@ -410,8 +454,22 @@ hsl_status launch_tp(Handle& h, const void* X, void* Y, int64_t T, cudaStream_t 
       return cuda_fail(e, "split-K counter init");
   }
   const int r_pad = int(h.r_pad);
+  const long long zitems = (long long)h.r * ((T + 7) / 8);
+  const int zQ = int((n + kSkZPiece - 1) / kSkZPiece);
   if (h.r > 0) {
-    if (hsl_status e = ensure(h.sk_z, size_t(T) * r_pad * 4, "split-K z")) return e;
+    // per-item counters first (a fixed place, zero at rest: kept across calls),
+    // then z, then the pieces' partial sums
+    const size_t cb = size_t(round_up(int64_t(h.r) * 8 * 4, 256));  // items for T up to 64
+    const size_t zb = size_t(round_up(int64_t(T) * r_pad * 4, 256));
+    const size_t pb = size_t(zitems) * zQ * 8 * 4;
+    const bool fresh = !h.sk_z.p || h.sk_z.bytes < cb + zb + pb;
+    if (hsl_status e = ensure(h.sk_z, cb + zb + pb, "split-K z")) return e;
+    if (fresh) {
+      if (cudaError_t e = cudaMemsetAsync(h.sk_z.p, 0, cb, s)) return cuda_fail(e, "split-K z counters");
+    }
+    h.sk_zcnt_off = 0;
+    h.sk_zout_off = cb;
+    h.sk_zpart_off = cb + zb;
   }
 
   SkMaps maps;
@@ -426,7 +484,7 @@ hsl_status launch_tp(Handle& h, const void* X, void* Y, int64_t T, cudaStream_t 
   SkArgs a;
   a.meta = static_cast<const uint2*>(h.pmeta_tc.p);
   a.U = static_cast<const __nv_bfloat16*>(h.U.p);
-  a.z = static_cast<const float*>(h.sk_z.p);
+  a.z = reinterpret_cast<const float*>(static_cast<const char*>(h.sk_z.p) + h.sk_zout_off);
   a.part = static_cast<float*>(h.sk_part.p);
   a.cnt = static_cast<unsigned*>(h.sk_cnt.p);
   a.Y = static_cast<__nv_bfloat16*>(Y);
@@ -441,12 +499,14 @@ hsl_status launch_tp(Handle& h, const void* X, void* Y, int64_t T, cudaStream_t 
   a.units = units;
 
   if (h.r > 0) {
-    const long long items = (long long)h.r * ((T + 7) / 8);
-    const long long zgrid = std::min<long long>((items * 32 + kSkZThreads - 1) / kSkZThreads,
+    const long long warps = zitems * zQ;
+    const long long zgrid = std::min<long long>((warps * 32 + kSkZThreads - 1) / kSkZThreads,
                                                 (long long)h.num_sms * 8);
+    char* zb = static_cast<char*>(h.sk_z.p);
     k_splitk_z<<<unsigned(zgrid), kSkZThreads, 0, s>>>(
         static_cast<const __nv_bfloat16*>(h.Vt.p), static_cast<const __nv_bfloat16*>(X),
-        static_cast<float*>(h.sk_z.p), int(n), int(T), h.r, r_pad);
+        reinterpret_cast<float*>(zb + h.sk_zout_off), int(n), int(T), h.r, r_pad,
+        reinterpret_cast<float*>(zb + h.sk_zpart_off), reinterpret_cast<unsigned*>(zb + h.sk_zcnt_off));
     note_launch();
     if (hsl_status e = cuda_fail(cudaGetLastError(), "split-K z launch")) return e;
   }

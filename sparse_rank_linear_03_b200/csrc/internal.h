@@ -108,6 +108,7 @@ struct Handle {
   DevBuf tiles;  // per-tile counts of the sampled-bracket split
   DevBuf xstage, ystage, zpre;
   DevBuf sk_part, sk_cnt, sk_z;  // split-K small-batch apply: partial tiles, tile counters, z
+  size_t sk_zcnt_off = 0, sk_zout_off = 0, sk_zpart_off = 0;  // in sk_z: counters, z, z pieces
   // permuted apply: the layer holds W' = W[row_order][:, col_order]
   DevBuf perm_row, perm_col, xperm, yperm;
   bool permuted = false;

@@ -180,6 +180,23 @@ __device__ __forceinline__ void tmem_st2(uint32_t taddr, uint32_t a, uint32_t b)
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
+// Copy a 128-row × 16-byte matrix from shared memory into TMEM lanes 0..127,
+// columns [taddr, taddr + 4): lane L gets bytes 16L..16L+15 of the source.
+// Issued by one thread; ordered before the tcgen05.mma that thread issues after it.
+__device__ __forceinline__ void tmem_cp_128x128b(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+// Shared-memory descriptor of a 128-row × 16-byte matrix with rows 16 bytes
+// apart and no swizzle: 8-row core matrices of 128 bytes, 128 bytes apart.
+__device__ __forceinline__ uint64_t desc_rows16(const void* smem_tile) {
+  const uint64_t addr = smem_u32(smem_tile);
+  uint64_t d = 0;
+  d |= (addr >> 4) & 0x3FFFull;          // start address
+  d |= uint64_t(128 >> 4) << 16;         // leading byte offset (one core matrix along K)
+  d |= uint64_t(128 >> 4) << 32;         // stride byte offset: the next 8 rows
+  d |= uint64_t(1) << 46;                // descriptor version (sm_100)
+  return d;                              // layout type 0: no swizzle
+}
 // Arrive on an mbarrier once all MMAs issued so far by this thread complete.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile(
