@@ -233,7 +233,7 @@ hsl_status hsl_group_destroy(hsl_group g);
  * test matrix:
  *   omega:       device fp32 [n][k], r ≤ k ≤ min(m, n, 512) (k − r is the
  *                oversampling);
- *   power_iters: q ≥ 0 subspace iterations (Y ← R orth(Rᵀ Q));
+ *   power_iters: q ≥ 0 subspace iterations (Y ← R Rᵀ Q, then Q = orth(Y));
  *   U [m][r], V [n][r]: device, handle dtype (pass them to hsl_pack);
  *   sigma [r]: device fp32, σ_1 ≥ … ≥ σ_r (0 where R has no such direction).
  * The tall products run on the tensor cores with fp32 operands split into

@@ -7,7 +7,7 @@
 // The factors are the truncated SVD of R with √σ on each side, computed by the
 // randomized range finder of Halko, Martinsson and Tropp with a caller-given
 // Gaussian test matrix Ω [n×k], k = r + oversampling:
-//   Y = R Ω;  Q = orth(Y);  q times { Z = orth(Rᵀ Q); Q = orth(R Z) };
+//   Y = R Ω;  Q = orth(Y);  q times { Z = Rᵀ Q; Q = orth(R Z) };
 //   Bᵀ = Rᵀ Q;  B Bᵀ = W Λ Wᵀ;  σ = √λ;  U = Q W_r √Σ_r,  V = Bᵀ W_r / √Σ_r.
 //
 // Kernels:
@@ -304,7 +304,7 @@ __global__ void __launch_bounds__(256) k_gram(const float* __restrict__ C, int64
 }
 
 // ---- symmetric eigensolver (one CTA) -----------------------------------------------------
-constexpr int JT = 1024;
+constexpr int JT = 512;
 // A [k][k] fp64 (overwritten), V [k][k] work, evals [k] and vecs [k][k] (columns)
 // sorted by descending eigenvalue.
 __global__ void __launch_bounds__(JT) k_jacobi(double* __restrict__ A, double* __restrict__ V, int k,
@@ -344,7 +344,8 @@ __global__ void __launch_bounds__(JT) k_jacobi(double* __restrict__ A, double* _
     if (threadIdx.x == 0) {
       double d2 = 0.0;
       for (int w = 0; w < JT / 32; ++w) d2 += red[w];
-      stop = off_all <= 1e-30 * d2 || off_all == 0.0;
+      // off-diagonal mass below (1e-13)² of the diagonal: converged to fp64 rounding
+      stop = off_all <= 1e-26 * d2 || off_all == 0.0;
     }
     __syncthreads();
     if (stop) break;
@@ -383,31 +384,75 @@ __global__ void __launch_bounds__(JT) k_jacobi(double* __restrict__ A, double* _
         Sn[i] = s;
       }
       __syncthreads();
+      // Rotations of disjoint pairs touch disjoint rows (then columns), so every
+      // element pair a thread updates is independent: a thread loads a batch of
+      // JB pairs before storing any, keeping JB loads of L2 latency in flight.
+      constexpr int JB = 4;
+      const int work = npair * k;
       // rows: (p, q) ← (c·row_p − s·row_q, s·row_p + c·row_q)
-      for (int e = threadIdx.x; e < npair * k; e += JT) {
-        const int i = e / k, j = e % k;
-        const int q = Q[i];
-        if (q < 0 || Sn[i] == 0.0) continue;
-        const int p = P[i];
-        const double c = Cs[i], s = Sn[i];
-        const double ap = A[int64_t(p) * k + j], aq = A[int64_t(q) * k + j];
-        A[int64_t(p) * k + j] = c * ap - s * aq;
-        A[int64_t(q) * k + j] = s * ap + c * aq;
+      for (int e0 = threadIdx.x; e0 < work; e0 += JT * JB) {
+        double ap[JB], aq[JB];
+        int64_t ip[JB], iq[JB];
+        bool act[JB];
+#pragma unroll
+        for (int b = 0; b < JB; ++b) {
+          const int e = e0 + b * JT;
+          act[b] = false;
+          if (e < work) {
+            const int i = e / k, j = e % k;
+            if (Q[i] >= 0 && Sn[i] != 0.0) {
+              act[b] = true;
+              ip[b] = int64_t(P[i]) * k + j;
+              iq[b] = int64_t(Q[i]) * k + j;
+              ap[b] = A[ip[b]];
+              aq[b] = A[iq[b]];
+            }
+          }
+        }
+#pragma unroll
+        for (int b = 0; b < JB; ++b) {
+          if (act[b]) {
+            const int i = (e0 + b * JT) / k;
+            const double c = Cs[i], sn = Sn[i];
+            A[ip[b]] = c * ap[b] - sn * aq[b];
+            A[iq[b]] = sn * ap[b] + c * aq[b];
+          }
+        }
       }
       __syncthreads();
       // columns of A and of V
-      for (int e = threadIdx.x; e < npair * k; e += JT) {
-        const int i = e / k, j = e % k;
-        const int q = Q[i];
-        if (q < 0 || Sn[i] == 0.0) continue;
-        const int p = P[i];
-        const double c = Cs[i], s = Sn[i];
-        const double ap = A[int64_t(j) * k + p], aq = A[int64_t(j) * k + q];
-        A[int64_t(j) * k + p] = c * ap - s * aq;
-        A[int64_t(j) * k + q] = s * ap + c * aq;
-        const double vp = V[int64_t(j) * k + p], vq = V[int64_t(j) * k + q];
-        V[int64_t(j) * k + p] = c * vp - s * vq;
-        V[int64_t(j) * k + q] = s * vp + c * vq;
+      for (int e0 = threadIdx.x; e0 < work; e0 += JT * JB) {
+        double ap[JB], aq[JB], vp[JB], vq[JB];
+        int64_t ip[JB], iq[JB];
+        bool act[JB];
+#pragma unroll
+        for (int b = 0; b < JB; ++b) {
+          const int e = e0 + b * JT;
+          act[b] = false;
+          if (e < work) {
+            const int i = e / k, j = e % k;
+            if (Q[i] >= 0 && Sn[i] != 0.0) {
+              act[b] = true;
+              ip[b] = int64_t(j) * k + P[i];
+              iq[b] = int64_t(j) * k + Q[i];
+              ap[b] = A[ip[b]];
+              aq[b] = A[iq[b]];
+              vp[b] = V[ip[b]];
+              vq[b] = V[iq[b]];
+            }
+          }
+        }
+#pragma unroll
+        for (int b = 0; b < JB; ++b) {
+          if (act[b]) {
+            const int i = (e0 + b * JT) / k;
+            const double c = Cs[i], sn = Sn[i];
+            A[ip[b]] = c * ap[b] - sn * aq[b];
+            A[iq[b]] = sn * ap[b] + c * aq[b];
+            V[ip[b]] = c * vp[b] - sn * vq[b];
+            V[iq[b]] = sn * vp[b] + c * vq[b];
+          }
+        }
       }
       __syncthreads();
     }
@@ -698,11 +743,16 @@ hsl_status factor_randomized_run(const void* R, int64_t m, int64_t n, hsl_dtype 
     return e;
   if (hsl_status e = orth(m, U16(QT), ldm)) return e;
   for (int it = 0; it < power_iters; ++it) {
-    // Z = orth(Rᵀ Q); Y = R Z; Q = orth(Y)
+    // Z = Rᵀ Q; Y = R Z; Q = orth(Y)
     if (hsl_status e = gemm_tall(U16(RT), nA, n, U16(QT), 3, kp, ldm, F32(YB), F32(PART), part_cap,
                                  num_sms, err, s))
       return e;
-    if (hsl_status e = orth(n, U16(ZT), ldn)) return e;
+    // Z = Rᵀ Q as three bf16 terms, transposed, for the next product: span(R Z)
+    // is span(R Rᵀ Q) whether or not Z is orthonormalised first, and Q (whose
+    // columns are orthonormal) keeps Z well scaled, so Z is used as it is
+    if (hsl_status e = launch_split(F32(YB), false, n, kp, kp, 3, true, U16(ZT), ldn,
+                                    int64_t(kp) * ldn, s))
+      return e;
     if (hsl_status e = gemm_tall(U16(RA), nA, m, U16(ZT), 3, kp, ldn, F32(YB), F32(PART), part_cap,
                                  num_sms, err, s))
       return e;

@@ -4,6 +4,7 @@
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <string>
 #include <vector>
@@ -560,9 +561,16 @@ hsl_status hsl_concentration(const void* W, int64_t m, int64_t n, hsl_dtype dtyp
     return unsupported("matrix too large");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int blocks = concentration_blocks(m);
-  DevBuf ws;
-  if (hsl_status e = ensure(ws, size_t(blocks) * 16 + 64, "concentration workspace")) return e;
-  double* out = static_cast<double*>(ws.p);
+  // a small workspace per device, kept for later calls (calls on one device
+  // are serialised by the lock: each waits for its result before returning)
+  static std::mutex mu;
+  static DevBuf ws[64];
+  int dev = 0;
+  if (cudaError_t e = cudaGetDevice(&dev)) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return unsupported("device ordinal out of range");
+  std::lock_guard<std::mutex> lock(mu);
+  if (hsl_status e = ensure(ws[dev], size_t(blocks) * 16 + 64, "concentration workspace")) return e;
+  double* out = static_cast<double*>(ws[dev].p);
   hsl_status st = concentration_run(W, m, n, dtype, out, out + 8, blocks, s);
   double res[3] = {0.0, 0.0, 0.0};
   if (st == HSL_OK) {
@@ -571,7 +579,6 @@ hsl_status hsl_concentration(const void* W, int64_t m, int64_t n, hsl_dtype dtyp
     else if (cudaError_t e2 = cudaStreamSynchronize(s))
       st = cuda_fail(e2, "concentration result");
   }
-  release(ws);
   if (st == HSL_OK) *rho = res[2];
   return st;
 }

@@ -107,18 +107,33 @@ __global__ void k_concentration_final(const double* __restrict__ partial, int bl
   }
 }
 
+// A CTA per row of W': the source row is read whole (coalesced) into shared
+// memory when it fits (staged), then gathered from there by the column order;
+// wider rows gather straight from global memory.
 template <typename KT>
 __global__ void k_permute(const KT* __restrict__ W, int64_t m, int64_t n,
                           const int32_t* __restrict__ row_order, const int32_t* __restrict__ col_order,
-                          KT* __restrict__ out) {
+                          KT* __restrict__ out, int staged) {
+  extern __shared__ __align__(16) unsigned char prow_smem[];
+  KT* rowbuf = reinterpret_cast<KT*>(prow_smem);
   for (int64_t k = blockIdx.x; k < m; k += gridDim.x) {
     const int32_t r = row_order[k];
     if (r < 0 || r >= m) continue;  // orders are checked on the host; never read out of bounds
     const KT* src = W + int64_t(r) * n;
     KT* dst = out + k * n;
-    for (int64_t l = threadIdx.x; l < n; l += blockDim.x) {
-      const int32_t c = col_order[l];
-      if (c >= 0 && c < n) dst[l] = src[c];
+    if (staged) {
+      __syncthreads();
+      for (int64_t l = threadIdx.x; l < n; l += blockDim.x) rowbuf[l] = src[l];
+      __syncthreads();
+      for (int64_t l = threadIdx.x; l < n; l += blockDim.x) {
+        const int32_t c = col_order[l];
+        if (c >= 0 && c < n) dst[l] = rowbuf[c];
+      }
+    } else {
+      for (int64_t l = threadIdx.x; l < n; l += blockDim.x) {
+        const int32_t c = col_order[l];
+        if (c >= 0 && c < n) dst[l] = src[c];
+      }
     }
   }
 }
@@ -182,13 +197,16 @@ int concentration_blocks(int64_t m) {
 
 hsl_status permute_run(const void* W, int64_t m, int64_t n, hsl_dtype dt, const int32_t* row_order,
                        const int32_t* col_order, void* out, cudaStream_t s) {
-  const unsigned grid = unsigned(std::max<int64_t>(1, std::min<int64_t>(m, int64_t(device_sms()) * 16)));
+  const unsigned grid = unsigned(std::max<int64_t>(1, std::min<int64_t>(m, int64_t(device_sms()) * 8)));
+  const size_t row_bytes = size_t(n) * dtype_bytes(dt);
+  const int staged = row_bytes <= 48 * 1024 ? 1 : 0;
+  const size_t sm = staged ? row_bytes : 0;
   if (dt == HSL_BF16)
-    k_permute<uint16_t><<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(W), m, n, row_order,
-                                            col_order, static_cast<uint16_t*>(out));
+    k_permute<uint16_t><<<grid, 512, sm, s>>>(static_cast<const uint16_t*>(W), m, n, row_order,
+                                             col_order, static_cast<uint16_t*>(out), staged);
   else
-    k_permute<uint32_t><<<grid, 256, 0, s>>>(static_cast<const uint32_t*>(W), m, n, row_order,
-                                            col_order, static_cast<uint32_t*>(out));
+    k_permute<uint32_t><<<grid, 512, sm, s>>>(static_cast<const uint32_t*>(W), m, n, row_order,
+                                             col_order, static_cast<uint32_t*>(out), staged);
   note_launch();
   return cuda_fail(cudaGetLastError(), "permute launch");
 }
