@@ -11,6 +11,8 @@ Each case builds its layer once (split + pack), then repeats one operation
   topk70b       top-k split at 5 % of the 28672×8192 bf16 W
   split24_70b   2:4 split of the same W
   attn4096      CSR apply, batch 1, 4096×4096 bf16 at 2 %, r = 128
+  attn4096_t2048  the same layer with 2048 tokens (S decompressed for the dense MMA)
+  factor70b     Stage 2 on the 70B layer's 2:4 residual (r = 256, k = 266, q = 2)
   stack7b       the 224-matrix CSR group at batch 1 (all 32 layers)
   stack7b_4     the first 4 layers of it (28 matrices, 178 MB: above L2, small
                 enough for a full ncu capture)
@@ -62,12 +64,22 @@ def case(name: str):
             return lambda: L.split(W, MLP70B.topk_frac_extra, R), (L,)
         L = hsl.Layer(lay.m, lay.n, 0, "nm24", "bf16")
         return lambda: L.split(W, 0.5, R), (L,)
-    if name == "attn4096":
+    if name in ("attn4096", "attn4096_t2048"):
         lay = ATTN4096.layers[0]
         L, _ = _layer(lay, ATTN4096.r, "csr", ATTN4096.frac, "f32")
-        X = _bf(synth.normal_f32(1, lay.n, lay.seed + 1))
-        Y = torch.empty(1, lay.m, dtype=torch.bfloat16, device="cuda")
+        b = 1 if name == "attn4096" else 2048
+        X = _bf(synth.normal_f32(b, lay.n, lay.seed + 1))
+        Y = torch.empty(b, lay.m, dtype=torch.bfloat16, device="cuda")
         return lambda: L.apply(X, Y), (L,)
+    if name == "factor70b":
+        lay = MLP70B.layers[0]
+        W = _bf(synth.student_t_f32(lay.m, lay.n, lay.seed))
+        L = hsl.Layer(lay.m, lay.n, MLP70B.r, "nm24", "bf16")
+        R = torch.empty_like(W)
+        L.split(W, 0.5, R)
+        del W
+        omega = torch.randn(lay.n, MLP70B.r + 10, device="cuda")
+        return lambda: L.factor(R, omega, 2), (L, R)
     if name in ("stack7b", "stack7b_4"):
         # W drawn on the device (6.5 G entries take minutes on the host)
         layers, Xs, Ys = [], [], []
