@@ -145,3 +145,83 @@ def test_binding_raises_typed_errors():
     with pytest.raises(hsl.HslError) as e:
         hsl.Layer(0, 4, 1)
     assert e.value.name == "HSL_ERR_INVALID_ARG"
+
+
+# ---------------------------------------------------------------- the later entry points
+
+def test_index_bits_checks():
+    st, h = _create(8, 8, 2, 0, 1)
+    assert st == OK
+    assert lib.hsl_set_index_bits(h, 12) == INVALID
+    for bits in (0, 8, 16, 32):
+        assert lib.hsl_set_index_bits(h, bits) == OK
+    lib.hsl_destroy(h)
+    st, h = _create(8, 8, 2, 1, 1)       # 2:4 handle
+    assert lib.hsl_set_index_bits(h, 8) == UNSUPPORTED
+    lib.hsl_destroy(h)
+    st, h = _create(4, 70000, 2, 0, 1)   # n ≥ 65535: only 32-bit columns
+    assert lib.hsl_set_index_bits(h, 16) == UNSUPPORTED
+    assert lib.hsl_set_index_bits(h, 8) == UNSUPPORTED
+    assert lib.hsl_set_index_bits(h, 32) == OK
+    lib.hsl_destroy(h)
+
+
+def test_factor_checks_before_any_device_work():
+    st, h = _create(64, 32, 8, 0, 0)
+    p = ctypes.c_void_p(16)
+    assert lib.hsl_factor(h, None, 0, p, 16, 1, p, p, p, None) == INVALID
+    assert lib.hsl_factor(h, p, 0, p, 4, 1, p, p, p, None) == UNSUPPORTED       # k < r
+    assert lib.hsl_factor(h, p, 0, p, 40, 1, p, p, p, None) == UNSUPPORTED      # k > min(m, n)
+    assert lib.hsl_factor(h, p, 0, p, 16, -1, p, p, p, None) == INVALID
+    assert lib.hsl_factor(h, p, 0, p, 16, 1, None, p, p, None) == INVALID
+    lib.hsl_destroy(h)
+
+
+def test_permutation_calls_check_arguments_on_the_host():
+    rho = ctypes.c_double()
+    assert lib.hsl_concentration(None, 4, 4, 0, ctypes.byref(rho), None) == INVALID
+    assert lib.hsl_concentration(ctypes.c_void_p(16), 0, 4, 0, ctypes.byref(rho), None) == INVALID
+    p = ctypes.c_void_p(16)
+    assert lib.hsl_permute(p, 4, 4, 5, p, p, p, None) == INVALID
+    assert lib.hsl_set_permutation(None, p, p, None) == INVALID
+    st, h = _create(8, 8, 2, 0, 0)
+    assert lib.hsl_set_permutation(h, p, None, None) == INVALID   # one order without the other
+    assert lib.hsl_set_permutation(h, None, None, None) == OK     # clearing needs no device
+    lib.hsl_destroy(h)
+
+
+def _rcm(m, n, rp, col):
+    import numpy as np
+    rp = np.ascontiguousarray(rp, dtype=np.int32)
+    col = np.ascontiguousarray(col, dtype=np.int32)
+    ro = np.empty(m, np.int32)
+    co = np.empty(n, np.int32)
+    st = lib.hsl_rcm_order(m, n, rp.ctypes.data, col.ctypes.data if col.size else None,
+                           ro.ctypes.data, co.ctypes.data)
+    return st, ro, co
+
+
+def test_rcm_order_is_the_oracles_on_random_patterns():
+    """The RCM order is a host-side graph step of the library: identical to the
+    oracle's on random patterns, empty rows and columns included."""
+    import numpy as np
+    import oracle
+    rng = np.random.default_rng(0)
+    for _ in range(60):
+        m, n = int(rng.integers(1, 70)), int(rng.integers(1, 70))
+        mask = rng.random((m, n)) < rng.uniform(0.0, 0.2)
+        rp = np.zeros(m + 1, np.int64)
+        rp[1:] = np.cumsum(mask.sum(1))
+        col = np.nonzero(mask)[1]
+        st, ro, co = _rcm(m, n, rp, col)
+        assert st == OK
+        wr, wc = oracle.rcm_order(m, n, rp, col)
+        assert np.array_equal(ro, wr) and np.array_equal(co, wc)
+
+
+def test_rcm_order_rejects_bad_patterns():
+    import numpy as np
+    assert _rcm(3, 4, [1, 1, 2, 2], [0, 1])[0] == INVALID          # row_ptr[0] != 0
+    assert _rcm(3, 4, [0, 2, 1, 2], [0, 1])[0] == INVALID          # not monotone
+    assert _rcm(2, 4, [0, 1, 2], [0, 9])[0] == INVALID             # column outside [0, n)
+    assert _rcm(2, 2, [0, 1, 9], np.zeros(9, np.int32))[0] == INVALID  # more entries than m·n
