@@ -6,20 +6,23 @@
 // layer factored in memory and decompress on the fly where latency matters;
 // the same section notes that large batches gain less from sparsity, being
 // compute-bound.  At thousands of tokens the CUDA-core CSR kernel would stream
-// S once per 16 tokens; here every CTA owns a Yᵀ tile of 128 rows × 256 tokens
-// and runs the dense 5th-generation MMA over S's rows block by block:
+// S once per 16 tokens; here every CTA owns a Yᵀ tile of 256 rows × 256 tokens
+// (two 128-row TMEM accumulators sharing every X block, which halves the X
+// bytes per FLOP of a 128-row tile) and runs the dense 5th-generation MMA over
+// S's rows block by block:
 //
 //   warp 0 lane 0   TMA of the X block [256 tokens × 64] (128-byte swizzle);
 //                   for the low-rank tail, TMA of U [128 × 64] and of Z hi or
 //                   Z lo [256 × 64] (Z = X·V from k_prefill_z, a bf16 pair).
-//   warps 2-5       one row of the tile per thread: zero the row of the A tile
+//   warps 2-9       one row of the tile per thread: zero the row of the A tile
 //                   (128-byte swizzle) and drop in the row's entries whose
 //                   column falls in the block, from a register cursor over the
 //                   packed row (16-bit columns, ascending, the next 8 entries
 //                   prefetched), then hand the tile to the MMA warp.
-//   warp 1 lane 0   tcgen05.mma (M = 128, N = 256, K = 16 × 4 per block) into
-//                   one fp32 TMEM accumulator: S·Xᵀ, then U·Z_hiᵀ + U·Z_loᵀ.
-//   warps 2-5       epilogue: tcgen05.ld, round to bf16, Y[t][i].
+//   warp 1 lane 0   tcgen05.mma (M = 128, N = 256, K = 16 × 4 per block, per
+//                   half) into two fp32 TMEM accumulators: S·Xᵀ, then
+//                   U·Z_hiᵀ + U·Z_loᵀ.
+//   warps 2-9       epilogue: tcgen05.ld, round to bf16, Y[t][i].
 // The work executed is the dense product (2·T·m·n) plus the low-rank term;
 // the decompression costs shared-memory stores only.  Every wait is bounded.
 #include <cuda.h>
@@ -34,11 +37,14 @@
 namespace hsl {
 namespace {
 
-constexpr int PC_BN = 256, PC_BK = 64, PC_STAGES = 4;
-constexpr int PC_A = 128 * 128;        // 16 KB: 128 rows × 64 bf16
+constexpr int PC_BM = 256, PC_BN = 256, PC_BK = 64, PC_STAGES = 3;
+constexpr int PC_THREADS = 320;        // 10 warps: copies, MMA, 8 × decompression + epilogue
+constexpr int PC_AH = 128 * 128;       // 16 KB: 128 rows × 64 bf16 (one accumulator's rows)
+constexpr int PC_A = 2 * PC_AH;        // both halves of the 256-row tile
 constexpr int PC_B = PC_BN * 128;      // 32 KB: 256 tokens × 64 bf16
 constexpr int PC_STAGE = PC_A + PC_B;
 constexpr int PC_SMEM = PC_STAGES * PC_STAGE + 1024 + 256;
+constexpr uint32_t PC_ACC1 = 256;      // TMEM column of the second accumulator
 
 struct PcMaps {
   CUtensorMap x;    // X [T][n]         box {64, 256} SW128
@@ -55,7 +61,7 @@ __device__ __forceinline__ bool pc_wait(uint64_t* bar, uint32_t parity, uint32_t
   return false;
 }
 
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(PC_THREADS, 1)
     k_prefill_csr(const __grid_constant__ PcMaps maps, const int32_t* __restrict__ prow,
                   const uint16_t* __restrict__ pcol, const uint16_t* __restrict__ pval,
                   __nv_bfloat16* __restrict__ Y, int m, int n, int T, int r16, uint32_t* err) {
@@ -72,7 +78,7 @@ __global__ void __launch_bounds__(192, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntn = (T + PC_BN - 1) / PC_BN;
   const int mt = blockIdx.x / ntn, nt = blockIdx.x % ntn;
-  const int i0 = mt * 128, t0 = nt * PC_BN;
+  const int i0 = mt * PC_BM, t0 = nt * PC_BN;
   const int nkS = (n + PC_BK - 1) / PC_BK;
   const int nkL = r16 > 0 ? 2 * ((r16 + PC_BK - 1) / PC_BK) : 0;
   const int nk = nkS + nkL;
@@ -81,7 +87,7 @@ __global__ void __launch_bounds__(192, 1)
     abort_flag = 0;
     for (int s = 0; s < PC_STAGES; ++s) {
       tc::mbar_init(&full[s], 1);
-      tc::mbar_init(&dense[s], 128);
+      tc::mbar_init(&dense[s], 256);
       tc::mbar_init(&empty[s], 1);
     }
     tc::mbar_init(accf, 1);
@@ -94,7 +100,7 @@ __global__ void __launch_bounds__(192, 1)
     }
   }
   if (warp == 1) {
-    tc::tmem_alloc(tmem_slot, PC_BN);
+    tc::tmem_alloc(tmem_slot, 512);
     tc::tmem_relinquish();
   }
   tc::tc_fence_before();
@@ -107,7 +113,7 @@ __global__ void __launch_bounds__(192, 1)
     if (lane == 0) {
       const uint64_t keep = tc::make_policy_evict_last();
       const uint64_t stream = tc::make_policy_evict_first();
-      int issued[PC_STAGES] = {0, 0, 0, 0};
+      int issued[PC_STAGES] = {0, 0, 0};
       for (int kb = 0; kb < nk; ++kb) {
         const int s = kb % PC_STAGES;
         const uint32_t ph = (kb / PC_STAGES) & 1;
@@ -122,6 +128,7 @@ __global__ void __launch_bounds__(192, 1)
           const int lr = kb - nkS, rb = lr >> 1;
           tc::mbar_expect_tx(&full[s], PC_A + PC_B);
           tc::tma_load_2d_hint(a, &maps.u, rb * PC_BK, i0, &full[s], stream);
+          tc::tma_load_2d_hint(a + PC_AH, &maps.u, rb * PC_BK, i0 + 128, &full[s], stream);
           tc::tma_load_2d_hint(b, (lr & 1) ? &maps.zlo : &maps.zhi, rb * PC_BK, t0, &full[s], keep);
         }
         ++issued[s];
@@ -139,20 +146,27 @@ __global__ void __launch_bounds__(192, 1)
         if (kb < nkS && !pc_wait(&dense[s], ph, err, abrt)) break;
         tc::tc_fence_after();
         unsigned char* a = smem + s * PC_STAGE;
-        const uint64_t ad = tc::desc_sw128(a);
         const uint64_t bd = tc::desc_sw128(a + PC_A);
 #pragma unroll
-        for (int k = 0; k < PC_BK / 16; ++k)
-          tc::mma_bf16(tmem, tc::desc_advance(ad, k * 32), tc::desc_advance(bd, k * 32), idesc,
-                       (kb > 0 || k > 0) ? 1u : 0u);
+        for (int h = 0; h < 2; ++h) {
+          const uint64_t ad = tc::desc_sw128(a + h * PC_AH);
+#pragma unroll
+          for (int k = 0; k < PC_BK / 16; ++k)
+            tc::mma_bf16(tmem + (h ? PC_ACC1 : 0u), tc::desc_advance(ad, k * 32),
+                         tc::desc_advance(bd, k * 32), idesc, (kb > 0 || k > 0) ? 1u : 0u);
+        }
         tc::mma_commit(&empty[s]);
       }
       tc::mma_commit(accf);
     }
   } else {
-    // decompression: thread L owns row i0 + L of the tile (= TMEM lane L)
+    // decompression: thread R owns row i0 + R of the tile; rows 0..127 belong to
+    // the first accumulator, 128..255 to the second (TMEM lane R mod 128; warp
+    // w may reach TMEM lanes 32·(w mod 4) onwards)
+    const int half = warp >= 6 ? 1 : 0;
     const int L = ((warp & 3) << 5) | lane;
-    const int i = i0 + L;
+    const int R = half * 128 + L;
+    const int i = i0 + R;
     int32_t e = 0, e_end = 0;
     if (i < m) {
       e = prow[i];
@@ -174,7 +188,7 @@ __global__ void __launch_bounds__(192, 1)
       const uint32_t ph = (kb / PC_STAGES) & 1;
       // the MMAs of this stage's previous use have read its A tile
       if (!pc_wait(&empty[s], ph ^ 1, err, abrt)) break;
-      unsigned char* arow = smem + s * PC_STAGE + (L >> 3) * 1024 + (L & 7) * 128;
+      unsigned char* arow = smem + s * PC_STAGE + half * PC_AH + (L >> 3) * 1024 + (L & 7) * 128;
 #pragma unroll
       for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(arow + c * 16) = make_uint4(0, 0, 0, 0);
       const int k0 = kb * PC_BK, kend = k0 + PC_BK;
@@ -211,7 +225,7 @@ __global__ void __launch_bounds__(192, 1)
     // epilogue
     if (tc::mbar_wait(accf, 0, err) && !*abrt) {
       tc::tc_fence_after();
-      const uint32_t tbase = tmem + (uint32_t((warp & 3) * 32) << 16);
+      const uint32_t tbase = tmem + (uint32_t((warp & 3) * 32) << 16) + (half ? PC_ACC1 : 0u);
 #pragma unroll 1
       for (int c0 = 0; c0 < PC_BN; c0 += 32) {
         float v[32];
@@ -232,7 +246,7 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   if (warp == 1) {
     tc::tc_fence_after();
-    tc::tmem_dealloc(tmem, PC_BN);
+    tc::tmem_dealloc(tmem, 512);
   }
 }
 
@@ -265,10 +279,10 @@ hsl_status apply_prefill_csr_run(Handle& h, const void* X, void* Y, int64_t T, c
   if (cudaError_t e = cudaFuncSetAttribute(k_prefill_csr, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            PC_SMEM))
     return cuda_fail(e, "CSR prefill smem attribute");
-  const int64_t tiles = ((m + 127) / 128) * ((T + PC_BN - 1) / PC_BN);
+  const int64_t tiles = ((m + PC_BM - 1) / PC_BM) * ((T + PC_BN - 1) / PC_BN);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(tiles));
-  cfg.blockDim = dim3(192);
+  cfg.blockDim = dim3(PC_THREADS);
   cfg.dynamicSmemBytes = PC_SMEM;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
