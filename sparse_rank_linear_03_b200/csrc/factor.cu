@@ -22,17 +22,23 @@
 //                  product is fp32-accurate although the MMA takes bf16.
 //                  K may be split over CTAs (partials added in split order).
 //   k_gram         G = CᵀC in fp64 over row chunks (partials added in order).
-//   k_jacobi       one CTA: cyclic two-sided Jacobi in fp64 on a k×k
-//                  symmetric matrix (round-robin pairs, rotations of disjoint
-//                  pairs applied together), eigenvalues sorted descending with
-//                  their vectors.  Bounded sweeps.
+//   k_chol_orth    one CTA: Cholesky of G with diagonal pivoting, stopped at
+//                  the first negligible pivot, then T = Π R⁻¹ (fp64), so C·T
+//                  is an orthonormal basis of span(C).
+//   k_jacobi_coop  cyclic two-sided Jacobi in fp64 on a k×k symmetric matrix,
+//                  a cooperative grid with one CTA per rotation pair of a
+//                  round (circle method), grid barriers between the row and
+//                  column passes; eigenvalues sorted descending with their
+//                  vectors.  Bounded sweeps and bounded barriers.
 //   k_scale_cols   T = W · diag(f(λ)) for the basis changes.
 //   k_small_gemm   C[M×K] · T[K×N] (K, N ≤ 512) in fp32, written row-major
 //                  (fp32 or the layer dtype) or as split bf16 terms transposed
 //                  (the next tall product's B operand).
-// orth(Y) = Y·W₁Λ₁^{-1/2} then once more on the result ("QR by the Gram
-// matrix", twice for orthogonality); eigenvalues below 1e-10 of the largest
-// drop their direction (a zero column), so rank-deficient Y is handled.
+// orth(Y) = Y·Π R⁻¹ from the pivoted Cholesky factor of YᵀY, then once more
+// on the result (Cholesky QR twice, for orthogonality); pivots below 1e-10 of
+// the largest diagonal end the factor, their directions become zero columns,
+// so rank-deficient Y is handled.  Only the final B Bᵀ needs eigenvectors
+// (Jacobi).
 #include <cuda.h>
 
 #include <algorithm>
@@ -303,170 +309,258 @@ __global__ void __launch_bounds__(256) k_gram(const float* __restrict__ C, int64
   }
 }
 
-// ---- symmetric eigensolver (one CTA) -----------------------------------------------------
-constexpr int JT = 512;
-// A [k][k] fp64 (overwritten), V [k][k] work, evals [k] and vecs [k][k] (columns)
-// sorted by descending eigenvalue.
-__global__ void __launch_bounds__(JT) k_jacobi(double* __restrict__ A, double* __restrict__ V, int k,
-                                               int max_sweeps, double* __restrict__ evals,
-                                               double* __restrict__ vecs) {
-  __shared__ int P[256], Q[256];
-  __shared__ double Cs[256], Sn[256];
-  __shared__ double red[JT / 32];
-  __shared__ int stop;
-  const int K = k + (k & 1);  // even number of players (a dummy when k is odd)
-  const int npair = K / 2;
-  for (int e = threadIdx.x; e < k * k; e += JT) V[e] = (e / k == e % k) ? 1.0 : 0.0;
+// ---- orthonormal basis by pivoted Cholesky of the Gram matrix (one CTA) -----------------
+// G = CᵀC [k][k] fp64.  Diagonal pivoting (largest remaining pivot first, ties to
+// the lower position) gives Πᵀ G Π = RᵀR with R upper triangular; the
+// factorisation stops at the first pivot at or below thr_rel · max diag(G) (the
+// columns of C past it are, to rounding, combinations of the earlier ones).
+// Then T = Π R⁻¹ on the kept rank (zero columns after it), so C·T has
+// orthonormal columns spanning span(C).  R is kept column-major (Rc[i][t] =
+// R[t][i]) so every dot product reads contiguous memory; Ri likewise for R⁻¹.
+constexpr int CT = 1024;
+constexpr int kMaxK = 512;
+__global__ void __launch_bounds__(CT) k_chol_orth(const double* __restrict__ G, int k, double thr_rel,
+                                                  double* __restrict__ Rc, double* __restrict__ Ri,
+                                                  float* __restrict__ T) {
+  __shared__ double d[kMaxK];
+  __shared__ int perm[kMaxK];
+  __shared__ double rv[CT / 32];
+  __shared__ int ri[CT / 32];
+  __shared__ int piv;
+  __shared__ double pval, dmax0;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int NW = CT / 32;
+  for (int i = tid; i < k; i += CT) {
+    d[i] = G[int64_t(i) * k + i];
+    perm[i] = i;
+  }
+  for (int e = tid; e < k * k; e += CT) {
+    Rc[e] = 0.0;
+    Ri[e] = 0.0;
+  }
   __syncthreads();
-  for (int sweep = 0; sweep < max_sweeps; ++sweep) {
-    // off-diagonal mass against the diagonal: stop when negligible
-    double off = 0.0, dia = 0.0;
-    for (int e = threadIdx.x; e < k * k; e += JT) {
-      const double v = A[e];
-      if (e / k == e % k) dia += v * v; else off += v * v;
-    }
+  // (value, position) maximum over positions [j0, k): ties to the lower position
+  auto argmax = [&](int j0) {
+    double bv = -1.0;
+    int bi = k;
+    for (int i = j0 + tid; i < k; i += CT)
+      if (d[i] > bv) { bv = d[i]; bi = i; }
     for (int o = 16; o; o >>= 1) {
-      off += __shfl_xor_sync(0xffffffffu, off, o);
-      dia += __shfl_xor_sync(0xffffffffu, dia, o);
+      const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
     }
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = off;
+    if (lane == 0) { rv[warp] = bv; ri[warp] = bi; }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      double o2 = 0.0;
-      for (int w = 0; w < JT / 32; ++w) o2 += red[w];
-      red[0] = o2;
-    }
-    __syncthreads();
-    const double off_all = red[0];
-    __syncthreads();
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = dia;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      double d2 = 0.0;
-      for (int w = 0; w < JT / 32; ++w) d2 += red[w];
-      // off-diagonal mass below (1e-13)² of the diagonal: converged to fp64 rounding
-      stop = off_all <= 1e-26 * d2 || off_all == 0.0;
+    if (tid == 0) {
+      double v = rv[0];
+      int p = ri[0];
+      for (int w = 1; w < NW; ++w)
+        if (rv[w] > v || (rv[w] == v && ri[w] < p)) { v = rv[w]; p = ri[w]; }
+      piv = p;
+      pval = v;
     }
     __syncthreads();
-    if (stop) break;
+  };
+  argmax(0);
+  if (tid == 0) dmax0 = pval > 0.0 ? pval : 0.0;
+  __syncthreads();
+  int rank = k;
+  for (int j = 0; j < k; ++j) {
+    if (j > 0) argmax(j);
+    const int p = piv;
+    const double dp = pval;
+    if (p >= k || !(dp > thr_rel * dmax0) || !(dp > 0.0)) {  // uniform: all read the same values
+      rank = j;
+      break;
+    }
+    if (p != j) {
+      for (int t = tid; t < j; t += CT) {
+        const double a = Rc[int64_t(j) * k + t];
+        Rc[int64_t(j) * k + t] = Rc[int64_t(p) * k + t];
+        Rc[int64_t(p) * k + t] = a;
+      }
+      if (tid == 0) {
+        const double dt = d[j];
+        d[j] = d[p];
+        d[p] = dt;
+        const int pt = perm[j];
+        perm[j] = perm[p];
+        perm[p] = pt;
+      }
+    }
+    __syncthreads();
+    const double rjj = sqrt(d[j]);
+    const int gj = perm[j];
+    // row j of R at the positions after j: a warp per position, fixed-order sums
+    for (int i = j + 1 + warp; i < k; i += NW) {
+      double s = 0.0;
+      for (int t = lane; t < j; t += 32) s = fma(Rc[int64_t(j) * k + t], Rc[int64_t(i) * k + t], s);
+      for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if (lane == 0) {
+        const double v = (G[int64_t(gj) * k + perm[i]] - s) / rjj;
+        Rc[int64_t(i) * k + j] = v;
+        d[i] -= v * v;
+      }
+    }
+    if (tid == 0) Rc[int64_t(j) * k + j] = rjj;
+    __syncthreads();
+  }
+  // R⁻¹ on the kept rank, a warp per column c (back substitution, bottom up):
+  // Ri[c][i] = −(Σ_{l=i+1..c} R[i][l]·Ri[c][l]) / R[i][i],  Ri[c][c] = 1 / R[c][c]
+  for (int c = warp; c < rank; c += NW) {
+    if (lane == 0) Ri[int64_t(c) * k + c] = 1.0 / Rc[int64_t(c) * k + c];
+    __syncwarp();
+    for (int i = c - 1; i >= 0; --i) {
+      double s = 0.0;
+      for (int l = i + 1 + lane; l <= c; l += 32)
+        s = fma(Rc[int64_t(l) * k + i], Ri[int64_t(c) * k + l], s);
+      for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if (lane == 0) Ri[int64_t(c) * k + i] = -s / Rc[int64_t(i) * k + i];
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  // T[perm[i]][c] = R⁻¹[i][c] for c < rank (upper triangle), zero elsewhere
+  for (int e = tid; e < k * k; e += CT) {
+    const int i = e / k, c = e % k;
+    T[int64_t(perm[i]) * k + c] = (c < rank && i <= c) ? float(Ri[int64_t(c) * k + i]) : 0.f;
+  }
+}
+
+// ---- symmetric eigensolver (cooperative grid, one CTA per rotation pair) -------------------
+// Cyclic two-sided Jacobi in fp64 on A [k][k] (overwritten), V [k][k] work;
+// eigenvalues sorted descending into evals [k], their vectors into the
+// columns of vecs [k][k].  A round of the circle method pairs every index
+// with one other (a dummy when k is odd): CTA b owns pair b, computes its
+// rotation from the round's A, rotates rows p and q, and after a grid barrier
+// columns p and q of A and V.  Disjoint pairs touch disjoint rows (columns),
+// so the order of the updates inside a pass does not matter and the result is
+// the same on every run.  A rotation is skipped when |a_pq| is negligible
+// against √|a_pp·a_qq| (relative 1e-16) or against the largest diagonal entry
+// (relative 1e-18); the sweeps stop after one with no rotation (at most
+// max_sweeps).  The grid barrier is a counter and a generation word in `sync`
+// (zeroed by the host before each launch); a wait that runs out of polls sets the abort word
+// and kErrTimeout, and from then on every barrier returns at once, so the
+// kernel still ends.
+constexpr int JC = 256;
+// sync: [0] arrivals, [1] generation, [2] abort, [3] [4] sweep flags
+__device__ __forceinline__ void grid_sync(unsigned* sync, unsigned nb, uint32_t* err) {
+  __syncthreads();
+  if (threadIdx.x == 0 && atomicAdd(&sync[2], 0u) == 0u) {
+    const unsigned g = atomicAdd(&sync[1], 0u);
+    __threadfence();
+    if (atomicAdd(&sync[0], 1u) == nb - 1) {
+      atomicExch(&sync[0], 0u);
+      __threadfence();
+      atomicAdd(&sync[1], 1u);
+    } else {
+      long long i = 0;
+      while (atomicAdd(&sync[1], 0u) == g && atomicAdd(&sync[2], 0u) == 0u) {
+        if (++i > kSpinLimit) {
+          atomicExch(&sync[2], 1u);
+          set_error(err, kErrTimeout);
+          break;
+        }
+      }
+    }
+    __threadfence();
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(JC) k_jacobi_coop(double* __restrict__ A, double* __restrict__ V, int k,
+                                                    int max_sweeps, double* __restrict__ evals,
+                                                    double* __restrict__ vecs, unsigned* sync,
+                                                    uint32_t* err) {
+  __shared__ double cs_s, sn_s, red[JC / 32];
+  __shared__ int p_s, q_s, cnt_s;
+  const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const unsigned G = gridDim.x;
+  const int K = k + (k & 1);
+  for (int64_t e = int64_t(b) * JC + tid; e < int64_t(k) * k; e += int64_t(G) * JC)
+    V[e] = (e / k == e % k) ? 1.0 : 0.0;
+  // scale of the absolute skip test: the largest |diagonal entry| (same in every CTA)
+  double dm = 0.0;
+  for (int i = tid; i < k; i += JC) dm = fmax(dm, fabs(A[int64_t(i) * k + i]));
+  for (int o = 16; o; o >>= 1) dm = fmax(dm, __shfl_xor_sync(0xffffffffu, dm, o));
+  if (lane == 0) red[warp] = dm;
+  __syncthreads();
+  double dmax = 0.0;
+  for (int w = 0; w < JC / 32; ++w) dmax = fmax(dmax, red[w]);
+  const double abs_tol = 1e-18 * dmax;
+  grid_sync(sync, G, err);
+  for (int sweep = 0; sweep < max_sweeps; ++sweep) {
+    bool rotated = false;
     for (int round = 0; round < K - 1; ++round) {
-      if (threadIdx.x < npair) {
-        const int i = threadIdx.x;
-        // circle method: player 0 fixed, the others rotate
+      if (tid == 0) {
         auto player = [&](int j) { return 1 + (j + round) % (K - 1); };
-        int p, q;
-        if (i == 0) {
-          p = 0;
-          q = player(0);
-        } else {
-          p = player(i);
-          q = player(K - 1 - i);
-        }
-        if (p > q) {
-          const int t = p;
-          p = q;
-          q = t;
-        }
-        double c = 1.0, s = 0.0;
+        int p = b == 0 ? 0 : player(b), q = b == 0 ? player(0) : player(K - 1 - b);
+        if (p > q) { const int t = p; p = q; q = t; }
+        double c = 1.0, sn = 0.0;
         if (q < k) {
           const double apq = A[int64_t(p) * k + q];
-          if (apq != 0.0) {
-            const double app = A[int64_t(p) * k + p], aqq = A[int64_t(q) * k + q];
+          const double app = A[int64_t(p) * k + p], aqq = A[int64_t(q) * k + q];
+          if (fabs(apq) > abs_tol && fabs(apq) > 1e-16 * sqrt(fabs(app * aqq))) {
             const double tau = (aqq - app) / (2.0 * apq);
             const double t = (tau >= 0.0 ? 1.0 : -1.0) / (fabs(tau) + sqrt(1.0 + tau * tau));
             c = 1.0 / sqrt(1.0 + t * t);
-            s = t * c;
+            sn = t * c;
+            rotated = true;
           }
         }
-        P[i] = p;
-        Q[i] = q < k ? q : -1;
-        Cs[i] = c;
-        Sn[i] = s;
+        p_s = p;
+        q_s = q;
+        cs_s = c;
+        sn_s = sn;
       }
       __syncthreads();
-      // Rotations of disjoint pairs touch disjoint rows (then columns), so every
-      // element pair a thread updates is independent: a thread loads a batch of
-      // JB pairs before storing any, keeping JB loads of L2 latency in flight.
-      constexpr int JB = 4;
-      const int work = npair * k;
-      // rows: (p, q) ← (c·row_p − s·row_q, s·row_p + c·row_q)
-      for (int e0 = threadIdx.x; e0 < work; e0 += JT * JB) {
-        double ap[JB], aq[JB];
-        int64_t ip[JB], iq[JB];
-        bool act[JB];
-#pragma unroll
-        for (int b = 0; b < JB; ++b) {
-          const int e = e0 + b * JT;
-          act[b] = false;
-          if (e < work) {
-            const int i = e / k, j = e % k;
-            if (Q[i] >= 0 && Sn[i] != 0.0) {
-              act[b] = true;
-              ip[b] = int64_t(P[i]) * k + j;
-              iq[b] = int64_t(Q[i]) * k + j;
-              ap[b] = A[ip[b]];
-              aq[b] = A[iq[b]];
-            }
-          }
+      const int p = p_s, q = q_s;
+      const double c = cs_s, sn = sn_s;
+      if (sn != 0.0)  // rows p, q: (p, q) ← (c·row_p − s·row_q, s·row_p + c·row_q)
+        for (int j = tid; j < k; j += JC) {
+          const double ap = A[int64_t(p) * k + j], aq = A[int64_t(q) * k + j];
+          A[int64_t(p) * k + j] = c * ap - sn * aq;
+          A[int64_t(q) * k + j] = sn * ap + c * aq;
         }
-#pragma unroll
-        for (int b = 0; b < JB; ++b) {
-          if (act[b]) {
-            const int i = (e0 + b * JT) / k;
-            const double c = Cs[i], sn = Sn[i];
-            A[ip[b]] = c * ap[b] - sn * aq[b];
-            A[iq[b]] = sn * ap[b] + c * aq[b];
-          }
+      grid_sync(sync, G, err);
+      if (sn != 0.0)  // columns p, q of A and of V
+        for (int j = tid; j < k; j += JC) {
+          const double ap = A[int64_t(j) * k + p], aq = A[int64_t(j) * k + q];
+          A[int64_t(j) * k + p] = c * ap - sn * aq;
+          A[int64_t(j) * k + q] = sn * ap + c * aq;
+          const double vp = V[int64_t(j) * k + p], vq = V[int64_t(j) * k + q];
+          V[int64_t(j) * k + p] = c * vp - sn * vq;
+          V[int64_t(j) * k + q] = sn * vp + c * vq;
         }
-      }
-      __syncthreads();
-      // columns of A and of V
-      for (int e0 = threadIdx.x; e0 < work; e0 += JT * JB) {
-        double ap[JB], aq[JB], vp[JB], vq[JB];
-        int64_t ip[JB], iq[JB];
-        bool act[JB];
-#pragma unroll
-        for (int b = 0; b < JB; ++b) {
-          const int e = e0 + b * JT;
-          act[b] = false;
-          if (e < work) {
-            const int i = e / k, j = e % k;
-            if (Q[i] >= 0 && Sn[i] != 0.0) {
-              act[b] = true;
-              ip[b] = int64_t(j) * k + P[i];
-              iq[b] = int64_t(j) * k + Q[i];
-              ap[b] = A[ip[b]];
-              aq[b] = A[iq[b]];
-              vp[b] = V[ip[b]];
-              vq[b] = V[iq[b]];
-            }
-          }
-        }
-#pragma unroll
-        for (int b = 0; b < JB; ++b) {
-          if (act[b]) {
-            const int i = (e0 + b * JT) / k;
-            const double c = Cs[i], sn = Sn[i];
-            A[ip[b]] = c * ap[b] - sn * aq[b];
-            A[iq[b]] = sn * ap[b] + c * aq[b];
-            V[ip[b]] = c * vp[b] - sn * vq[b];
-            V[iq[b]] = sn * vp[b] + c * vq[b];
-          }
-        }
-      }
-      __syncthreads();
+      grid_sync(sync, G, err);
     }
+    // a sweep without any rotation ends the iteration (flags alternate by sweep)
+    if (tid == 0 && rotated) atomicOr(&sync[3 + (sweep & 1)], 1u);
+    grid_sync(sync, G, err);
+    const bool stop = atomicAdd(&sync[3 + (sweep & 1)], 0u) == 0u;
+    // the other flag was last read before this sweep's barriers: clear it for the next sweep
+    if (tid == 0 && b == 0) atomicExch(&sync[3 + ((sweep + 1) & 1)], 0u);
+    grid_sync(sync, G, err);
+    if (stop) break;
   }
-  // sort by descending eigenvalue (rank = number ahead; ties by index)
-  for (int i = threadIdx.x; i < k; i += JT) {
+  // sort by descending eigenvalue (rank = entries ahead; ties by index); CTA b
+  // places the columns i ≡ b (mod G)
+  for (int i = b; i < k; i += G) {
     const double li = A[int64_t(i) * k + i];
-    int rank = 0;
-    for (int j = 0; j < k; ++j) {
+    if (tid == 0) cnt_s = 0;
+    __syncthreads();
+    int ahead = 0;
+    for (int j = tid; j < k; j += JC) {
       const double lj = A[int64_t(j) * k + j];
-      if (lj > li || (lj == li && j < i)) ++rank;
+      if (lj > li || (lj == li && j < i)) ++ahead;
     }
-    evals[rank] = li;
-    for (int r = 0; r < k; ++r) vecs[int64_t(r) * k + rank] = V[int64_t(r) * k + i];
+    atomicAdd(&cnt_s, ahead);
+    __syncthreads();
+    const int rank = cnt_s;
+    if (tid == 0) evals[rank] = li;
+    for (int r = tid; r < k; r += JC) vecs[int64_t(r) * k + rank] = V[int64_t(r) * k + i];
+    __syncthreads();
   }
 }
 
@@ -654,10 +748,18 @@ hsl_status gram(const float* C, int64_t M, int N, double* part, int64_t part_cap
   return cuda_fail(cudaGetLastError(), "gram reduce launch");
 }
 
-hsl_status eig(double* G, int k, double* Vw, double* evals, double* vecs, cudaStream_t s) {
-  k_jacobi<<<1, JT, 0, s>>>(G, Vw, k, 40, evals, vecs);
+hsl_status eig(double* G, int k, double* Vw, double* evals, double* vecs, unsigned* sync,
+               uint32_t* err, cudaStream_t s) {
+  if (cudaError_t e = cudaMemsetAsync(sync, 0, 8 * sizeof(unsigned), s))
+    return cuda_fail(e, "eigensolver barrier reset");
+  // one CTA per rotation pair, all resident at once (cooperative launch)
+  const unsigned grid = unsigned((k + (k & 1)) / 2);
+  int max_sweeps = 40;
+  void* args[] = {&G, &Vw, &k, &max_sweeps, &evals, &vecs, &sync, &err};
   note_launch();
-  return cuda_fail(cudaGetLastError(), "eigensolver launch");
+  return cuda_fail(cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(k_jacobi_coop), dim3(grid),
+                                               dim3(JC), args, 0, s),
+                   "eigensolver launch");
 }
 
 hsl_status small_gemm(const float* C, int64_t M, int K, int ldc, const float* T, int N, int ldt,
@@ -682,7 +784,7 @@ hsl_status factor_randomized_run(const void* R, int64_t m, int64_t n, hsl_dtype 
   // noise of a direction the data does not have (fp32 data, fp64 sums)
   const double thr_rel = 1e-10;
   Work w;
-  enum { RA, RT, OT, QT, ZT, YB, QF, BT, PART, GP, G, VW, EV, EVEC, TT, NB };
+  enum { RA, RT, OT, QT, ZT, YB, QF, BT, PART, GP, G, VW, EV, EVEC, TT, SY, NB };
   const size_t sizes[NB] = {
       size_t(nA) * m * ldn * 2,          // R as K-major A terms
       size_t(nA) * n * ldm * 2,          // Rᵀ terms
@@ -699,6 +801,7 @@ hsl_status factor_randomized_run(const void* R, int64_t m, int64_t n, hsl_dtype 
       size_t(kp) * 8,                    // eigenvalues
       size_t(kp) * kp * 8,               // eigenvectors
       size_t(kp) * kp * 4,               // basis change T
+      size_t(64),                        // eigensolver grid barrier
   };
   for (int b = 0; b < NB; ++b)
     if (hsl_status e = ensure(w.bufs[b], sizes[b], "factorisation workspace")) return e;
@@ -722,10 +825,9 @@ hsl_status factor_randomized_run(const void* R, int64_t m, int64_t n, hsl_dtype 
     for (int pass = 0; pass < 2; ++pass) {
       const float* cur = pass == 0 ? F32(YB) : F32(QF);
       if (hsl_status e = gram(cur, M, kp, F64(GP), gp_cap, F64(G), num_sms, s)) return e;
-      if (hsl_status e = eig(F64(G), kp, F64(VW), F64(EV), F64(EVEC), s)) return e;
-      k_scale_cols<<<64, 256, 0, s>>>(F64(EVEC), F64(EV), kp, kp, kp, 0, thr_rel, F32(TT));
+      k_chol_orth<<<1, CT, 0, s>>>(F64(G), kp, thr_rel, F64(VW), F64(EVEC), F32(TT));
       note_launch();
-      if (hsl_status e = cuda_fail(cudaGetLastError(), "basis change launch")) return e;
+      if (hsl_status e = cuda_fail(cudaGetLastError(), "pivoted Cholesky launch")) return e;
       if (pass == 0) {
         if (hsl_status e = small_gemm(cur, M, kp, kp, F32(TT), kp, kp, 0, F32(QF), kp, 0, s)) return e;
       } else {
@@ -763,7 +865,9 @@ hsl_status factor_randomized_run(const void* R, int64_t m, int64_t n, hsl_dtype 
                                num_sms, err, s))
     return e;
   if (hsl_status e = gram(F32(BT), n, kp, F64(GP), gp_cap, F64(G), num_sms, s)) return e;
-  if (hsl_status e = eig(F64(G), kp, F64(VW), F64(EV), F64(EVEC), s)) return e;
+  if (hsl_status e = eig(F64(G), kp, F64(VW), F64(EV), F64(EVEC),
+                         static_cast<unsigned*>(w.bufs[SY].p), err, s))
+    return e;
   // σ below thr_rel^{1/2} of σ_max: no direction (zero factor columns)
   k_sigma<<<1, 256, 0, s>>>(F64(EV), r, thr_rel, sigma);
   note_launch();
