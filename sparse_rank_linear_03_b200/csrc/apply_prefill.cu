@@ -387,9 +387,12 @@ __global__ void __launch_bounds__(192, 1)
 // ---- sparse tensor-core prefill -------------------------------------------------
 // Yᵀ tile [256 rows of W × 192 tokens]: two 128-row accumulators in TMEM share
 // every X tile (half the X traffic of one 128-row tile per flop).  K-blocks of
-// 64 logical columns: A = the compressed 2:4 values (TMA, 64-byte swizzle,
-// 32 values per row), B = X (TMA, 128-byte swizzle), two tcgen05.mma.sp of
-// K = 32 per half.  The metadata of a K-block is copied into TMEM by four warps
+// 64 logical columns: A = the compressed 2:4 values of all 256 rows in one TMA
+// (64-byte swizzle, 32 values per row, 16 KB: a copy instruction costs a
+// near-fixed time, so two 8 KB copies took about twice as long), B = X (TMA,
+// 128-byte swizzle), two tcgen05.mma.sp of K = 32 per half.  Two threads issue
+// the copies of a stage, both arriving on its barrier: warp 0 the A tile,
+// warp 6 the B tile and the metadata, so their copy instructions overlap.  The metadata of a K-block is copied into TMEM by four warps
 // (tcgen05.st) from a layout built at pack time, one 8-byte word pair per TMEM
 // lane; each MMA's metadata column is 4-column aligned (a requirement of the
 // sparse MMA's metadata address).  The low-rank tail runs dense MMAs on
@@ -415,13 +418,14 @@ static_assert(SP_STAGES * 4 <= 32, "metadata slots");
 
 struct SpMaps {
   CUtensorMap x;   // X [T][n]       box {64, 192} SW128
-  CUtensorMap sv;  // S values [m][n/2] box {32, 128} SW64
-  CUtensorMap u;   // U [m][r_pad]   box {32, 128} SW64
+  CUtensorMap sv;  // S values [m][n/2] box {32, 256} SW64
+  CUtensorMap u;   // U [m][r_pad]   box {32, 256} SW64
   CUtensorMap z;   // Z hi [T][r16]  box {32, 192} SW64
   CUtensorMap zlo; // Z lo [T][r16]  box {32, 192} SW64
 };
 
-__global__ void __launch_bounds__(192, 1)
+constexpr int SP_THREADS = 224;  // warps: 0 A copies, 1 MMA, 2-5 metadata + epilogue, 6 B copies
+__global__ void __launch_bounds__(SP_THREADS, 1)
     k_prefill_24sp(const __grid_constant__ SpMaps maps, const uint2* __restrict__ meta,
                    __nv_bfloat16* __restrict__ Y, int m, int n, int T, int r16, uint32_t* err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -449,7 +453,7 @@ __global__ void __launch_bounds__(192, 1)
   if (threadIdx.x == 0) {
     abort_flag = 0;
     for (int s = 0; s < SP_STAGES; ++s) {
-      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&full[s], 2);  // the A issuer and the B issuer
       tc::mbar_init(&mfull[s], 128);
       tc::mbar_init(&empty[s], 1);
     }
@@ -472,24 +476,29 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem = *tmem_slot;
   volatile int* abrt = &abort_flag;
 
-  if (warp == 0) {
+  if (warp == 0 || warp == 6) {
+    // warp 0: the A tile (S values, then U); warp 6: the B tile (X, then Z hi
+    // and lo) and the metadata
     if (lane == 0) {
+      const bool bs = warp == 6;
       const uint64_t keep = tc::make_policy_evict_last();
       const uint64_t stream = tc::make_policy_evict_first();
-      int issued[SP_STAGES] = {0, 0, 0, 0, 0};
-      for (int kb = 0; kb < nk; ++kb) {
+      int kb = 0;
+      for (; kb < nk; ++kb) {
         const int s = kb % SP_STAGES;
         const uint32_t ph = (kb / SP_STAGES) & 1;
         if (!wait_or_abort(&empty[s], ph ^ 1, err, abrt)) break;
         unsigned char* a = sA + s * SP_A;
         unsigned char* b = sB + s * SP_B;
-        if (kb < nkS) {
-          // the metadata of both halves rides on the same barrier (1 KB each)
+        if (!bs) {
+          tc::mbar_expect_tx(&full[s], SP_A);
+          if (kb < nkS) tc::tma_load_2d_hint(a, &maps.sv, kb * 32, i0, &full[s], stream);
+          else tc::tma_load_2d_hint(a, &maps.u, (kb - nkS) * 32, i0, &full[s], stream);
+        } else if (kb < nkS) {
+          // the metadata of both halves (1 KB each)
           const int mt0 = i0 / 128;
           const int nmeta = (mt0 < mtiles128) + (mt0 + 1 < mtiles128);
-          tc::mbar_expect_tx(&full[s], SP_A + SP_B + nmeta * 1024);
-          tc::tma_load_2d_hint(a, &maps.sv, kb * 32, i0, &full[s], stream);
-          tc::tma_load_2d_hint(a + SP_A_HALF, &maps.sv, kb * 32, i0 + 128, &full[s], stream);
+          tc::mbar_expect_tx(&full[s], SP_B + nmeta * 1024);
           tc::tma_load_2d_hint(b, &maps.x, kb * 64, t0, &full[s], keep);
           for (int h = 0; h < 2; ++h)
             if (mt0 + h < mtiles128)
@@ -498,16 +507,15 @@ __global__ void __launch_bounds__(192, 1)
         } else {
           if (kb == nkS) pdl_wait();  // Z is written by the preceding kernel
           const int kl = kb - nkS;
-          tc::mbar_expect_tx(&full[s], SP_A + 2 * SP_B_Z);
-          tc::tma_load_2d_hint(a, &maps.u, kl * 32, i0, &full[s], stream);
-          tc::tma_load_2d_hint(a + SP_A_HALF, &maps.u, kl * 32, i0 + 128, &full[s], stream);
+          tc::mbar_expect_tx(&full[s], 2 * SP_B_Z);
           tc::tma_load_2d_hint(b, &maps.z, kl * 32, t0, &full[s], keep);
           tc::tma_load_2d_hint(b + SP_B_Z, &maps.zlo, kl * 32, t0, &full[s], keep);
         }
-        ++issued[s];
       }
-      for (int s = 0; s < SP_STAGES; ++s)
-        if (issued[s]) tc::mbar_wait(&full[s], (issued[s] - 1) & 1, err);
+      // drain: the last stages this thread issued have landed (the other
+      // issuer's copies complete the same phases)
+      for (int j = kb > SP_STAGES ? kb - SP_STAGES : 0; j < kb; ++j)
+        tc::mbar_wait(&full[j % SP_STAGES], (j / SP_STAGES) & 1, err);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -547,7 +555,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       tc::mma_commit(accf);
     }
-  } else {
+  } else if (warp < 6) {
     // warps 2..5: metadata into TMEM, then the epilogue.  TMEM lane = L.
     const int L = ((warp & 3) << 5) | lane;
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
@@ -955,10 +963,10 @@ hsl_status apply_prefill_run(Handle& h, const void* X, void* Y, int64_t T, cudaS
     memset(&sm, 0, sizeof(sm));
     const auto BFs = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     bool ok = make_map(&sm.x, BFs, 2, X, T, n, n, 64, SP_BN, CU_TENSOR_MAP_SWIZZLE_128B) &&
-              make_map(&sm.sv, BFs, 2, h.nm_val.p, m, n / 2, n / 2, 32, 128,
+              make_map(&sm.sv, BFs, 2, h.nm_val.p, m, n / 2, n / 2, 32, 256,
                        CU_TENSOR_MAP_SWIZZLE_64B);
     if (ok && r16 > 0)
-      ok = make_map(&sm.u, BFs, 2, h.U.p, m, h.r_pad, h.r_pad, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B) &&
+      ok = make_map(&sm.u, BFs, 2, h.U.p, m, h.r_pad, h.r_pad, 32, 256, CU_TENSOR_MAP_SWIZZLE_64B) &&
            make_map(&sm.z, BFs, 2, h.zpre.p, T, r16, r16, 32, SP_BN, CU_TENSOR_MAP_SWIZZLE_64B) &&
            make_map(&sm.zlo, BFs, 2, static_cast<__nv_bfloat16*>(h.zpre.p) + T * r16, T, r16, r16,
                     32, SP_BN, CU_TENSOR_MAP_SWIZZLE_64B);
@@ -1024,7 +1032,7 @@ hsl_status apply_prefill_run(Handle& h, const void* X, void* Y, int64_t T, cudaS
     const int64_t tiles = ((m + 255) / 256) * ((T + SP_BN - 1) / SP_BN);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(unsigned(tiles));
-    cfg.blockDim = dim3(192);
+    cfg.blockDim = dim3(SP_THREADS);
     cfg.dynamicSmemBytes = SP_SMEM;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];

@@ -9,17 +9,20 @@
 // as in the prefill kernel.  What differs is how the work is cut: a layer has
 // only m/128 row tiles (86 for 11008 rows), far fewer than the SMs × CTAs per
 // SM, so the (row tile, 64-column K-block) units of the whole layer are dealt
-// out in equal contiguous ranges to a persistent grid of two CTAs per SM.
+// out in equal contiguous ranges to a persistent grid of one CTA per SM.
 //
 //   k_splitk_z   z = Vᵀ x for the T tokens in fp32 (a warp per (row of Vt,
 //                8 tokens), fixed shuffle-tree sums); triggers the dependent
 //                launch at its start.
-//   k_apply_24_splitk<TP>  per unit: TMA of the 128×32 compressed values
-//                (64-byte swizzle) and the X block [TP tokens × 64] (128-byte
-//                swizzle, tokens past T zero-filled), 1 KB of TMEM-ordered
-//                metadata by bulk copy, spread to one 16-byte row per TMEM
-//                lane and copied into TMEM by tcgen05.cp; two tcgen05.mma.sp of K = 32 into a
-//                128×TP fp32 accumulator in TMEM.  A CTA's range covers the end
+//   k_apply_24_splitk<TP>  a unit is a 128-row tile × two 64-column K-blocks:
+//                one 16 KB TMA of the 128×64 compressed values (128-byte
+//                swizzle; a copy instruction costs a near-fixed time, so
+//                16 KB per instruction streams about twice as fast as 8 KB),
+//                the two X blocks [TP tokens × 64] (128-byte swizzle, tokens
+//                past T zero-filled) and 2 KB of TMEM-ordered metadata by
+//                bulk copy, spread to one 16-byte row per TMEM lane and
+//                copied into TMEM by tcgen05.cp; four tcgen05.mma.sp of
+//                K = 32 into a 128×TP fp32 accumulator in TMEM.  A CTA's range covers the end
 //                of one tile and the start of the next (or a whole tile), so it
 //                keeps two accumulators and hands each finished tile segment to
 //                its epilogue warps.
@@ -31,10 +34,12 @@
 //   the result is deterministic.  That CTA resets the counter for the next
 //   call.  Nobody waits on anybody: no spin on another CTA.
 //
-// Warp roles (320 threads): warp 0 lane 0 issues the copies; warp 1 owns TMEM
-// and lane 0 copies each unit's metadata into TMEM (tcgen05.cp, ordered before
-// its MMAs) and issues the MMAs; warps 2-5 lay the metadata out for that copy;
-// warps 6-9 run the epilogues (TMEM lane quarter = warp % 4).  Every wait is
+// Warp roles (352 threads): warp 0 lane 0 issues the S copies and warp 10
+// lane 0 the X and metadata copies (two issuers, both arriving on the stage's
+// barrier, so their copy instructions overlap); warp 1 owns TMEM and lane 0
+// copies each unit's metadata into TMEM (tcgen05.cp, ordered before its MMAs)
+// and issues the MMAs; warps 2-5 lay the metadata out for that copy; warps
+// 6-9 run the epilogues (TMEM lane quarter = warp % 4).  Every wait is
 // bounded; a wait that gives up sets the error word, and the CTA still drains
 // its copies, takes part in the tile counters and frees TMEM.
 #include <cuda.h>
@@ -49,24 +54,24 @@
 namespace hsl {
 namespace {
 
-constexpr int SK_THREADS = 320;
-constexpr int SK_A = 128 * 64;      // compressed values of a unit: 128 rows × 64 bytes
-constexpr int SK_M = 128 * 8;       // TMEM-ordered metadata of a unit (compact)
-constexpr int SK_MX = 2 * 128 * 16; // the same, one 16-byte row per TMEM lane and MMA
+constexpr int SK_THREADS = 352;    // 11 warps (roles below)
+constexpr int SK_A = 128 * 128;     // compressed values of a unit: 128 rows × 128 bytes (2 K-blocks)
+constexpr int SK_M = 2 * 128 * 8;   // TMEM-ordered metadata of the unit's 2 K-blocks (compact)
+constexpr int SK_MX = 4 * 128 * 16; // the same, one 16-byte row per TMEM lane and MMA (4 MMAs)
 constexpr uint32_t SK_TMEM_COLS = 256;
 // accumulator b at TMEM column 64·b
 __host__ __device__ constexpr uint32_t sk_acc_col(int b) { return 64u * uint32_t(b); }
 
-__host__ __device__ constexpr int sk_stages(int tp) { return tp <= 16 ? 6 : tp <= 32 ? 5 : 4; }
-__host__ __device__ constexpr int sk_stage_bytes(int tp) { return SK_A + tp * 128 + SK_M + SK_MX; }
+__host__ __device__ constexpr int sk_stages(int tp) { return tp <= 32 ? 6 : 4; }
+__host__ __device__ constexpr int sk_stage_bytes(int tp) { return SK_A + 2 * tp * 128 + SK_M + SK_MX; }
 __host__ __device__ constexpr int sk_smem(int tp) {
   return sk_stages(tp) * sk_stage_bytes(tp) + 1024 + 256;
 }
 // metadata slot of (stage, MMA i): 4-column aligned, after both accumulators
-__device__ __forceinline__ uint32_t sk_meta_col(int s, int i) { return 128u + 8u * s + 4u * i; }
+__device__ __forceinline__ uint32_t sk_meta_col(int s, int i) { return 128u + 16u * s + 4u * i; }
 
 struct SkMaps {
-  CUtensorMap sv;  // S values [m][n/2]  box {32, 128} SW64
+  CUtensorMap sv;  // S values [m][n/2]  box {64, 128} SW128 (two K-blocks of 64 columns)
   CUtensorMap x;   // X [T][n]           box {64, TP}  SW128
 };
 
@@ -78,7 +83,7 @@ struct SkArgs {
   unsigned* cnt;            // [tiles]
   __nv_bfloat16* Y;         // [T][m]
   uint32_t* err;
-  int m, n, T, r, r_pad, nkb, tiles;
+  int m, n, T, r, r_pad, nkb, tiles;  // nkb: units per tile (pairs of 64-column K-blocks)
   long long units;          // tiles · nkb
 };
 
@@ -197,7 +202,7 @@ __global__ void __launch_bounds__(kSkZThreads) k_splitk_z(const __nv_bfloat16* _
 
 // ---- the split-K kernel ------------------------------------------------------------
 template <int TP>
-__global__ void __launch_bounds__(SK_THREADS, 2)
+__global__ void __launch_bounds__(SK_THREADS, 1)
     k_apply_24_splitk(const __grid_constant__ SkMaps maps, const SkArgs a) {
   constexpr int ST = sk_stages(TP);
   constexpr int STAGE = sk_stage_bytes(TP);
@@ -223,7 +228,7 @@ __global__ void __launch_bounds__(SK_THREADS, 2)
   if (threadIdx.x == 0) {
     abort_flag = 0;
     for (int s = 0; s < ST; ++s) {
-      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&full[s], 2);  // the S issuer and the X/metadata issuer
       tc::mbar_init(&mfull[s], 128);
       tc::mbar_init(&empty[s], 1);
     }
@@ -245,29 +250,34 @@ __global__ void __launch_bounds__(SK_THREADS, 2)
   const uint32_t tmem = *tmem_slot;
   volatile int* abrt = &abort_flag;
 
-  if (warp == 0) {
+  if (warp == 0 || warp == 10) {
+    // warp 0: the unit's S values; warp 10: its two X blocks and metadata
     if (lane == 0) {
+      const bool xs = warp == 10;
       const uint64_t keep = tc::make_policy_evict_last();
       const uint64_t stream = tc::make_policy_evict_first();
-      int issued[ST];
-#pragma unroll
-      for (int s = 0; s < ST; ++s) issued[s] = 0;
-      for (long long u = u0; u < u1; ++u) {
-        const int k = int(u - u0), s = k % ST;
+      int k = 0;
+      for (long long u = u0; u < u1; ++u, ++k) {
+        const int s = k % ST;
         const uint32_t ph = (k / ST) & 1;
         if (!wait_or_abort(&empty[s], ph ^ 1, a.err, abrt)) break;
-        const int tile = int(u / nkb), kb = int(u % nkb);
+        const int tile = int(u / nkb), kp = int(u % nkb);
         unsigned char* st = smem + s * STAGE;
-        tc::mbar_expect_tx(&full[s], SK_A + B_BYTES + SK_M);
-        tc::tma_load_2d_hint(st, &maps.sv, kb * 32, tile * 128, &full[s], stream);
-        tc::tma_load_2d_hint(st + SK_A, &maps.x, kb * 64, 0, &full[s], keep);
-        tc::bulk_load(st + SK_A + B_BYTES, a.meta + ((long long)tile * nkb + kb) * 128, SK_M,
-                      &full[s]);
-        ++issued[s];
+        if (!xs) {
+          tc::mbar_expect_tx(&full[s], SK_A);
+          tc::tma_load_2d_hint(st, &maps.sv, kp * 64, tile * 128, &full[s], stream);
+        } else {
+          tc::mbar_expect_tx(&full[s], 2 * B_BYTES + SK_M);
+          tc::tma_load_2d_hint(st + SK_A, &maps.x, kp * 128, 0, &full[s], keep);
+          tc::tma_load_2d_hint(st + SK_A + B_BYTES, &maps.x, kp * 128 + 64, 0, &full[s], keep);
+          // the metadata of K-blocks 2·kp and 2·kp + 1 lie next to each other
+          tc::bulk_load(st + SK_A + 2 * B_BYTES, a.meta + ((long long)tile * nkb + kp) * 256, SK_M,
+                        &full[s]);
+        }
       }
-      // drain: every copy this thread started has landed before the CTA exits
-      for (int s = 0; s < ST; ++s)
-        if (issued[s]) tc::mbar_wait(&full[s], (issued[s] - 1) & 1, a.err);
+      // drain: the stages of the last (up to ST) units this thread issued have landed
+      // (the other issuer's copies complete the same phases)
+      for (int j = k > ST ? k - ST : 0; j < k; ++j) tc::mbar_wait(&full[j % ST], (j / ST) & 1, a.err);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -289,17 +299,20 @@ __global__ void __launch_bounds__(SK_THREADS, 2)
         if (!wait_or_abort(&mfull[s], ph, a.err, abrt)) break;
         tc::tc_fence_after();
         const unsigned char* st = smem + s * STAGE;
-        const uint64_t ad = tc::desc_sw64(st);
-        const uint64_t bd = tc::desc_sw128(st + SK_A);
+        const uint64_t ad = tc::desc_sw128(st);
         const uint32_t d = tmem + sk_acc_col(seg & 1);
         // the unit's metadata into its TMEM slots, ahead of the MMAs that read it
-        const unsigned char* mx = st + SK_A + B_BYTES + SK_M;
+        const unsigned char* mx = st + SK_A + 2 * B_BYTES + SK_M;
 #pragma unroll
-        for (int i = 0; i < 2; ++i) tc::tmem_cp_128x128b(tmem + sk_meta_col(s, i), tc::desc_rows16(mx + i * 2048));
+        for (int i = 0; i < 4; ++i) tc::tmem_cp_128x128b(tmem + sk_meta_col(s, i), tc::desc_rows16(mx + i * 2048));
+        // MMA i: K-block i / 2 (its X block), 32 logical columns (i % 2) of it;
+        // the values advance 32 bytes per MMA within their 128-byte rows
 #pragma unroll
-        for (int i = 0; i < 2; ++i)
-          tc::mma_bf16_sp(d, tc::desc_advance(ad, 32 * i), tc::desc_advance(bd, 64 * i),
+        for (int i = 0; i < 4; ++i) {
+          const uint64_t bd = tc::desc_sw128(st + SK_A + (i >> 1) * B_BYTES);
+          tc::mma_bf16_sp(d, tc::desc_advance(ad, 32 * i), tc::desc_advance(bd, 64 * (i & 1)),
                           tmem + sk_meta_col(s, i), idesc_sp, (!first || i > 0) ? 1u : 0u);
+        }
         tc::mma_commit(&empty[s]);
         if (last) tc::mma_commit(&accfull[seg & 1]);
       }
@@ -314,10 +327,13 @@ __global__ void __launch_bounds__(SK_THREADS, 2)
       // the stage's bytes have landed, so the MMAs of its previous use are done
       if (!wait_or_abort(&full[s], ph, a.err, abrt)) break;
       unsigned char* st = smem + s * STAGE;
-      const uint2 w = *reinterpret_cast<const uint2*>(st + SK_A + B_BYTES + L * 8);
-      unsigned char* mx = st + SK_A + B_BYTES + SK_M;
-      *reinterpret_cast<uint4*>(mx + L * 16) = make_uint4(w.x, 0u, 0u, 0u);
-      *reinterpret_cast<uint4*>(mx + 2048 + L * 16) = make_uint4(w.y, 0u, 0u, 0u);
+      unsigned char* mx = st + SK_A + 2 * B_BYTES + SK_M;
+#pragma unroll
+      for (int kb = 0; kb < 2; ++kb) {
+        const uint2 w = *reinterpret_cast<const uint2*>(st + SK_A + 2 * B_BYTES + kb * 1024 + L * 8);
+        *reinterpret_cast<uint4*>(mx + (2 * kb) * 2048 + L * 16) = make_uint4(w.x, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(mx + (2 * kb + 1) * 2048 + L * 16) = make_uint4(w.y, 0u, 0u, 0u);
+      }
       tc::fence_async_smem();
       tc::mbar_arrive(&mfull[s]);
     }
@@ -427,23 +443,15 @@ __global__ void __launch_bounds__(SK_THREADS, 2)
 template <int TP>
 hsl_status launch_tp(Handle& h, const void* X, void* Y, int64_t T, cudaStream_t s) {
   const int64_t m = h.m, n = h.n;
-  const int nkb = int(n / 64);
+  const int nkb = int(n / 128);  // units per tile: pairs of 64-column K-blocks
   const int tiles = int((m + 127) / 128);
   const long long units = (long long)tiles * nkb;
   auto kern = k_apply_24_splitk<TP>;
   const int smem = sk_smem(TP);
   if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))
     return cuda_fail(e, "split-K smem attribute");
-  // two CTAs per SM need the largest shared-memory carveout
-  if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                           int(cudaSharedmemCarveoutMaxShared)))
-    return cuda_fail(e, "split-K carveout attribute");
-  int occ = 0;
-  if (cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, SK_THREADS, smem))
-    return cuda_fail(e, "split-K occupancy");
-  // at most two CTAs per SM: their TMEM (256 columns each) must fit the SM's 512
-  occ = std::max(1, std::min(occ, 2));
-  const int grid = int(std::min<long long>((long long)occ * h.num_sms, units));
+  // one CTA per SM (its stage ring takes most of the shared memory)
+  const int grid = int(std::min<long long>(h.num_sms, units));
 
   // workspace: partial slots (tile + CTA index), tile counters (zero at rest), z
   const size_t part_bytes = size_t(tiles + grid) * TP * 128 * 4;
@@ -475,8 +483,8 @@ hsl_status launch_tp(Handle& h, const void* X, void* Y, int64_t T, cudaStream_t 
   SkMaps maps;
   memset(&maps, 0, sizeof(maps));
   const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  if (!make_tmap_2d(&maps.sv, BF, 2, h.nm_val.p, m, n / 2, n / 2, 32, 128,
-                    CU_TENSOR_MAP_SWIZZLE_64B) ||
+  if (!make_tmap_2d(&maps.sv, BF, 2, h.nm_val.p, m, n / 2, n / 2, 64, 128,
+                    CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap_2d(&maps.x, BF, 2, X, T, n, n, 64, TP, CU_TENSOR_MAP_SWIZZLE_128B)) {
     set_message("tensor map encoding failed");
     return HSL_ERR_CUDA;
@@ -527,7 +535,7 @@ hsl_status launch_tp(Handle& h, const void* X, void* Y, int64_t T, cudaStream_t 
 }  // namespace
 
 bool splitk_supported(const Handle& h, const void* X, int64_t T) {
-  return h.fmt == HSL_FMT_NM24 && h.dtype == HSL_BF16 && h.n % 64 == 0 && h.pmeta_tc.p &&
+  return h.fmt == HSL_FMT_NM24 && h.dtype == HSL_BF16 && h.n % 128 == 0 && h.pmeta_tc.p &&
          T >= kSplitKMinBatch && T <= kSplitKMaxBatch && h.r <= 256 &&
          (reinterpret_cast<uintptr_t>(X) % 16) == 0 && tmap_available();
 }

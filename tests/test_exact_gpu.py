@@ -144,6 +144,16 @@ def test_exact_2to4_11008(hsl, T):
     check_24(hsl, L, W, U, V, T, 522 + T, sample_rows(m, 1500 if T <= 16 else 256, 523), tok=tok)
 
 
+@pytest.mark.parametrize("T", [2, 8, 33, 64, 700])
+def test_exact_2to4_ragged_rows(hsl, T):
+    """1100 rows (a partial last row tile) × 1024: the split-K kernel at 2-64
+    tokens (units of two K-blocks dealt over all SMs) and the default prefill
+    kernel at 700 tokens, every output compared bit for bit."""
+    m, n, r = 1100, 1024, 40
+    L, W, U, V = build_24(hsl, m, n, r, 535)
+    check_24(hsl, L, W, U, V, T, 536 + T, np.arange(m))
+
+
 @pytest.mark.parametrize("env", ["HSL_PREFILL_EXPAND", "HSL_PREFILL_PAIRS"])
 def test_exact_2to4_alternate_prefill_kernels(hsl, monkeypatch, env):
     """The expansion kernel and the CTA-pair kernel, exact on a ragged shape."""
