@@ -74,7 +74,10 @@ def as_storage(x_f32: np.ndarray, dtype: str) -> np.ndarray:
 def torch_from_storage(bits: np.ndarray, dtype: str, device="cpu") -> torch.Tensor:
     """Wrap storage bits as a torch tensor of the matching dtype."""
     if dtype == "f32":
-        t = torch.from_numpy(np.ascontiguousarray(bits, dtype=np.float32))
+        a = np.ascontiguousarray(bits)
+        # uint32 storage bits are reinterpreted, float arrays taken as values
+        a = a.view(np.float32) if a.dtype in (np.uint32, np.int32) else a.astype(np.float32, copy=False)
+        t = torch.from_numpy(a)
     else:
         t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
     return t.to(device)

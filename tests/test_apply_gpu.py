@@ -230,7 +230,17 @@ def test_bad_imported_column_reported(hsl):
     assert e.value.name == "HSL_ERR_INVALID_ARG"
 
 
-# ---------------------------------------------------------------- batch-1 CSR, bulk-copy fed
+# ---------------------------------------------------------------- batch-1 CSR, both kernels
+
+@pytest.fixture(params=["regs", "bulk"])
+def csr_kernel(request, monkeypatch):
+    """The register-fed (default) and the bulk-copy fed batch-1 CSR kernels."""
+    if request.param == "bulk":
+        monkeypatch.setenv("HSL_DECODE_CSR", "bulk")
+    else:
+        monkeypatch.delenv("HSL_DECODE_CSR", raising=False)
+    return request.param
+
 
 def _import_csr(hsl, m, n, rp, col, vals, dtype="bf16", r=0, seed=0):
     L = hsl.Layer(m, n, r, "csr", dtype)
@@ -243,7 +253,7 @@ def _import_csr(hsl, m, n, rp, col, vals, dtype="bf16", r=0, seed=0):
     return L, U, V
 
 
-def test_csr_batch1_long_rows_and_empty_rows(hsl):
+def test_csr_batch1_long_rows_and_empty_rows(hsl, csr_kernel):
     """Rows longer than a streamed chunk (read from global memory), rows with
     no entries, and ordinary rows between them."""
     m, n = 300, 8192
@@ -265,7 +275,7 @@ def test_csr_batch1_long_rows_and_empty_rows(hsl):
     assert oracle.elem_rel_err(f64(host(Y), "bf16"), ref) <= ELEM_TOL["bf16"]
 
 
-def test_csr_batch1_many_rows_per_cta(hsl):
+def test_csr_batch1_many_rows_per_cta(hsl, csr_kernel):
     """1.3 M rows of 16 columns: each CTA's range is longer than the window of
     row starts it stages, so it runs in several sub-parts."""
     m, n = 1_300_000, 16
@@ -284,8 +294,17 @@ def test_csr_batch1_bulk_and_register_kernels_agree(hsl, monkeypatch, bits):
     c.L.set_index_bits(bits)
     c.L.pack(dev(c.U, "bf16"), dev(c.V, "bf16"))
     X = dev(c.x(1, 17), "bf16")
+    monkeypatch.setenv("HSL_DECODE_CSR", "bulk")
     a = f64(host(c.L.apply(X)), "bf16")
-    monkeypatch.setenv("HSL_DECODE_CSR", "regs")
-    b = f64(host(c.L.apply(X)), "bf16")
     monkeypatch.delenv("HSL_DECODE_CSR")
+    b = f64(host(c.L.apply(X)), "bf16")
     assert oracle.rel_err(a, b) <= 2 ** -7
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_csr_batch17_last_token_alone(hsl, csr_kernel, dtype):
+    """17 tokens: a pass of 16, then the 17th alone through the batch-1 kernel,
+    which must read and write that token's rows (offset 16), not the first."""
+    c = Case(hsl, 513, 1000, 3, "csr", dtype, 0.07, 513 * 31 + 1000)
+    Xb = c.x(17, 5)
+    assert err_of(c, c.L.apply(dev(Xb, dtype)), Xb) <= TOL[dtype]

@@ -93,7 +93,7 @@ def test_factor_square1024_worked_example_residual(hsl):
     """The worked example's residual: 1024² f32 W minus its top 5 %, rank 64,
     k = 74, two power iterations (the oracle's own defaults)."""
     W = synth.student_t_f32(1024, 1024, 0)
-    R = oracle.split_topk(W, 0.05, "f32")["R"]
+    R = oracle.split_topk(W, 0.05, "f32")["R"].view(np.float32)   # storage bits as values
     om = omega_of(1024, 74, 35)
     Ug, Vg, sg = gpu_factor(hsl, R, "f32", 64, om, 2)
     R64 = R.astype(np.float64)

@@ -5,8 +5,10 @@ compared element by element with the oracle's reconstruction Ŵ = S + U Vᵀ.
 With one unit vector per token, S·e_t is a single stored value and z = Vᵀ e_t
 is a row of V (exact in bf16, so the tensor-core path's hi/lo pair is exact
 too); the only rounding is the fp32 sum of U·z and the output's conversion to
-the layer dtype.  Bound per element: half an output ulp of |Ŵ_ij| plus the fp32
-sum's error, r·2⁻²⁴·Σ_c|U_ic V_jc|."""
+the layer dtype.  Bound per element: half an output ulp of |Ŵ_ij| (2⁻⁸·|Ŵ_ij|
+for bf16, 2⁻²⁴·|Ŵ_ij| for f32) plus the fp32 sum's error, taken as one fp32 ulp
+per addition, r·2⁻²³·Σ_c|U_ic V_jc| (a tensor-core adder may truncate rather
+than round).  A wrong index or a dropped group costs a whole |S_ij| and fails."""
 import numpy as np
 import pytest
 import torch
@@ -34,8 +36,8 @@ def check(Y, S64, U, V, dtype):
     U64, V64 = f(U), f(V)
     W_hat = oracle.reconstruct(S64, U64, V64)
     got = f(host(Y)).T                             # Y = Ŵᵀ
-    ulp = 2.0 ** -8 if dtype == "bf16" else 2.0 ** -23
-    bound = 0.5 * ulp * np.abs(W_hat) + U64.shape[1] * 2.0 ** -24 * (np.abs(U64) @ np.abs(V64).T) + 1e-30
+    ulp = 2.0 ** -7 if dtype == "bf16" else 2.0 ** -23   # spacing at 1.0 (8 / 24 significant bits)
+    bound = 0.5 * ulp * np.abs(W_hat) + U64.shape[1] * 2.0 ** -23 * (np.abs(U64) @ np.abs(V64).T) + 1e-30
     bad = np.argwhere(np.abs(got - W_hat) > bound)
     assert bad.size == 0, f"{len(bad)} entries of Ŵ off, first at {tuple(bad[0])}"
 
@@ -78,11 +80,11 @@ def test_identity_reconstructs_w_hat_square1024_f32(hsl):
     m = n = 1024
     W = synth.student_t_f32(m, n, 0)
     ref = oracle.split_topk(W, 0.05, "f32")
-    U, V = factors(ref["R"].astype(np.float64), 64, "f32", exact=True)
+    U, V = factors(oracle.bits_to_f64(ref["R"], "f32"), 64, "f32", exact=True)
     L = hsl.Layer(m, n, 64, "csr", "f32")
     L.split(dev(W, "f32"), 0.05, None)
     L.pack(dev(U, "f32"), dev(V, "f32"))
     Y = L.apply(dev(identity(n, "f32"), "f32"))
     L.check()
-    S = csr_dense_rows(ref["row_ptr"], ref["col"], ref["val"].astype(np.float64), np.arange(m), n)
+    S = csr_dense_rows(ref["row_ptr"], ref["col"], oracle.bits_to_f64(ref["val"], "f32"), np.arange(m), n)
     check(Y, S, U, V, "f32")
