@@ -52,6 +52,7 @@ struct ApplyArgs {
   unsigned long long* zsync;  // CTAs done with z, CTAs done with the call (in-kernel z)
   long long spin_limit;       // polls of the z-counter wait before it gives up
   uint32_t zwait_extra;       // added to the z-counter target (0; 1 only under fault injection)
+  int32_t n_max;              // widest layer (the staged x)
 };
 
 template <typename T>
@@ -189,10 +190,9 @@ __device__ __forceinline__ void xcol(const T* xs, int c, float (&xv)[BC]) {
 // y[row] = ysp[row] + U[row,:]·z for rows [s0, s1) of layer P.  GU lanes
 // share a row (8 elements each); a warp takes R row groups per pass and issues
 // all their U loads before using any, so the pass costs one load latency.
-template <typename T, int BC, int NT = kThreads>
+template <typename T, int BC, int NT = kThreads, int R = (BC <= 2 ? 4 : 1)>
 __device__ __forceinline__ void urows(const ApplyProblem& P, const float* zs, const float* ysp,
-                                      int s0, int s1, T* y, int bc) {
-  constexpr int R = BC <= 2 ? 4 : 1;
+                                      int s0, int s1, T* y, int bc, const T* Us = nullptr) {
   const int rp = P.r_pad;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int GU = 1;
@@ -205,7 +205,21 @@ __device__ __forceinline__ void urows(const ApplyProblem& P, const float* zs, co
 #pragma unroll
     for (int q = 0; q < R; ++q) {
       const int i = ib + q * rpw + lane / GU;
-      if (i < s1 && gl * 8 < rp) load8<T>(U + int64_t(i) * rp + gl * 8, u[q]);
+      if (i < s1 && gl * 8 < rp) {
+        if (Us != nullptr) {  // the segment's U rows, staged in shared memory
+          const T* ur = Us + int64_t(i - s0) * rp + gl * 8;
+          if constexpr (sizeof(T) == 2) {
+            const uint4 q4 = *reinterpret_cast<const uint4*>(ur);
+            u[q][0] = bf_lo(q4.x); u[q][1] = bf_hi(q4.x); u[q][2] = bf_lo(q4.y); u[q][3] = bf_hi(q4.y);
+            u[q][4] = bf_lo(q4.z); u[q][5] = bf_hi(q4.z); u[q][6] = bf_lo(q4.w); u[q][7] = bf_hi(q4.w);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) u[q][e] = VT<T>::f(ur[e]);
+          }
+        } else {
+          load8<T>(U + int64_t(i) * rp + gl * 8, u[q]);
+        }
+      }
     }
 #pragma unroll
     for (int q = 0; q < R; ++q) {
@@ -381,6 +395,104 @@ __device__ __forceinline__ void csr_rows(const ApplyProblem& P, const T* xs, flo
   }
 }
 
+// Batch-1 CSR rows, vector-parallel.  The segment's packed vectors (8 entries
+// each; rows are padded to whole vectors, so a vector belongs to one row) are
+// dealt to the warps in runs of whole rows with about equal vector counts.  A
+// warp streams its run 32 vectors per step, lane l taking vector v0 + 32·u + l,
+// with the column and value loads of kVecU steps issued before any arithmetic:
+// every load is a coalesced 16-byte vector whatever the row lengths.  A lane
+// finds its vector's row by walking the staged row starts; the vectors of a row
+// are summed by a segmented shuffle reduction in lane order, and a row that
+// runs past the end of a step carries its partial into the next.  Each row is
+// owned by one warp, so its sum has a fixed order and is written once.
+template <typename T, int IDX>
+__device__ __forceinline__ void csr_rows_vec(const ApplyProblem& P, const T* xs, float* ysp,
+                                             const int32_t* prow_s, int s0, int s1) {
+  constexpr int NW = kThreads / 32;
+  constexpr int kVecU = 2;  // steps whose loads are in flight together (more warps per SM instead)
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nrows = s1 - s0;
+  const int32_t V0 = prow_s[0] >> 3, V1 = prow_s[nrows] >> 3;
+  // rows [ra, rb) of this warp: the first row starting at or after its share
+  auto first_row_at = [&](int32_t vt) {
+    int lo = 0, hi = nrows;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if ((prow_s[mid] >> 3) < vt) lo = mid + 1; else hi = mid;
+    }
+    return lo;
+  };
+  const int ra = warp == 0 ? 0 : first_row_at(V0 + int32_t(int64_t(V1 - V0) * warp / NW));
+  const int rb = warp == NW - 1 ? nrows : first_row_at(V0 + int32_t(int64_t(V1 - V0) * (warp + 1) / NW));
+  for (int i = ra + lane; i < rb; i += 32) ysp[i] = 0.f;  // rows without entries
+  __syncwarp();
+  if (ra >= rb) return;
+  const int32_t va = prow_s[ra] >> 3, ve = prow_s[rb] >> 3;
+  const T* pval = static_cast<const T*>(P.pval);
+  int cur = ra;             // this lane's row walk (its vectors only move forward)
+  int carry_row = -1;       // a row continued from the previous step (warp-uniform)
+  float carry = 0.f;
+  for (int32_t vb = va; vb < ve; vb += 32 * kVecU) {
+    RawCols<IDX> cv[kVecU];
+    RawVals<T> rv[kVecU];
+#pragma unroll
+    for (int u = 0; u < kVecU; ++u) {
+      const int32_t v = vb + 32 * u + lane;
+      if (v < ve) {
+        cv[u].load(P, v * 8);
+        rv[u].load(pval + int64_t(v) * 8);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kVecU; ++u) {
+      const int32_t v = vb + 32 * u + lane;
+      if (vb + 32 * u >= ve) break;  // warp-uniform
+      float p = 0.f;
+      int row = 0x7fffffff;  // lanes past the end form a run of their own
+      if (v < ve) {
+        while (prow_s[cur + 1] <= v * 8) ++cur;
+        row = cur;
+        int c[8];
+        cv[u].cols(c);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) p = fmaf(rv[u].at(t), VT<T>::f(xs[c[t]]), p);
+      }
+      // suffix sums within runs of equal rows (runs are contiguous in lanes)
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float q = __shfl_down_sync(0xffffffffu, p, o);
+        const int rq = __shfl_down_sync(0xffffffffu, row, o);
+        if (lane + o < 32 && rq == row) p += q;
+      }
+      const int prev = __shfl_up_sync(0xffffffffu, row, 1);
+      const bool head = lane == 0 || prev != row;
+      const int row0 = __shfl_sync(0xffffffffu, row, 0);
+      if (carry_row >= 0) {
+        if (row0 == carry_row) {
+          if (lane == 0) p += carry;
+        } else if (lane == 0) {
+          ysp[carry_row] = carry;  // the carried row ended with the last step
+        }
+      }
+      // the run holding lane 31 may go on in the next step: carry it
+      const int row31 = __shfl_sync(0xffffffffu, row, 31);
+      const bool more = vb + 32 * (u + 1) < ve;
+      const unsigned tail = __ballot_sync(0xffffffffu, row == row31);
+      const int htail = __ffs(tail) - 1;
+      const float ptail = __shfl_sync(0xffffffffu, p, htail);
+      if (more) {
+        carry_row = row31;
+        carry = ptail;
+        if (head && row != row31) ysp[row] = p;
+      } else {
+        carry_row = -1;
+        if (head && row != 0x7fffffff) ysp[row] = p;
+      }
+    }
+  }
+  if (carry_row >= 0 && lane == 0) ysp[carry_row] = carry;
+}
+
 // Batch-1 bf16 2:4 rows.  A warp takes a row; lane l handles value chunks
 // q = (8·s + t)·32 + l (8 values = 4 groups each) and, per super-chunk s,
 // issues its metadata load and all eight 16-byte value loads before using any.
@@ -508,8 +620,8 @@ __device__ __forceinline__ void nm24_rows(const ApplyProblem& P, const T* xs, fl
 }
 
 // ---- the persistent apply kernel ---------------------------------------------------
-template <typename T, int BC, bool CSR, int IDX>
-__global__ void __maxnreg__(112) k_apply_decode(ApplyArgs a) {
+template <typename T, int BC, bool CSR, int IDX, bool VEC>
+__device__ __forceinline__ void apply_decode_body(const ApplyArgs& a) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ uint32_t sel_lut[16];  // byte-permute selector of a 2:4 nibble (x[i0], x[i1])
   if (threadIdx.x < 16)
@@ -517,6 +629,8 @@ __global__ void __maxnreg__(112) k_apply_decode(ApplyArgs a) {
   float* zs = reinterpret_cast<float*>(smem);                 // [BC][r_pad_max]
   float* ysp = zs + BC * a.r_pad_max;                          // [kSeg][BC]
   T* xs = reinterpret_cast<T*>(ysp + kSeg * BC);               // [(n+1)][BC]
+  int32_t* prow_s = reinterpret_cast<int32_t*>(                 // [kSeg + 1]
+      reinterpret_cast<unsigned char*>(xs) + ((size_t(a.n_max + 1) * BC * sizeof(T) + 15) & ~size_t(15)));
 
   const int64_t slo = int64_t(blockIdx.x) * a.slices / gridDim.x;
   const int64_t shi = int64_t(blockIdx.x + 1) * a.slices / gridDim.x;
@@ -552,7 +666,11 @@ __global__ void __maxnreg__(112) k_apply_decode(ApplyArgs a) {
     T* y = y_of<T>(a, p) + int64_t(a.b0) * P.m;
     for (int s0 = l0; s0 < l1; s0 += kSeg) {
       const int s1 = min(s0 + kSeg, l1);
-      if (CSR) csr_rows<T, BC, IDX>(P, xs, ysp, s0, s1);
+      if (CSR && BC == 1 && VEC) {
+        for (int i = threadIdx.x; i <= s1 - s0; i += kThreads) prow_s[i] = P.prow[s0 + i];
+        __syncthreads();
+        csr_rows_vec<T, IDX>(P, xs, ysp, prow_s, s0, s1);
+      } else if (CSR) csr_rows<T, BC, IDX>(P, xs, ysp, s0, s1);
       else if (fast24)
         nm24_rows_b1(P, reinterpret_cast<const __nv_bfloat16*>(xs), sel_lut, ysp, s0, s1);
       else nm24_rows<T, BC>(P, xs, ysp, s0, s1);
@@ -566,12 +684,26 @@ __global__ void __maxnreg__(112) k_apply_decode(ApplyArgs a) {
         for (int o = a.bc * P.r_pad + threadIdx.x; o < BC * P.r_pad; o += kThreads) zs[o] = 0.f;
       }
       __syncthreads();
-      urows<T, BC>(P, zs, ysp, s0, s1, y, a.bc);
+      // (the 80-register vector-parallel kernel keeps two row groups of U in flight)
+      urows<T, BC, kThreads, VEC ? 2 : (BC <= 2 ? 4 : 1)>(P, zs, ysp, s0, s1, y, a.bc);
       __syncthreads();
     }
     row = P.row0 + l1;
     ++p;
   }
+}
+
+// At most 112 registers, so an apply CTA fits beside a z CTA (programmatic
+// dependent launch).
+template <typename T, int BC, bool CSR, int IDX>
+__global__ void __maxnreg__(112) k_apply_decode(ApplyArgs a) {
+  apply_decode_body<T, BC, CSR, IDX, false>(a);
+}
+// Batch-1 CSR with vector-parallel rows: at most 64 registers, four CTAs
+// (32 warps) per SM, so more loads are in flight to hide their latency.
+template <typename T, int IDX>
+__global__ void __maxnreg__(80) k_apply_csr_vec(ApplyArgs a) {
+  apply_decode_body<T, 1, true, IDX, true>(a);
 }
 
 // ---- batch-1 bf16 2:4, rows fed by bulk copies ---------------------------------
@@ -599,15 +731,18 @@ constexpr int kSegB1 = 64;
 struct B1Layout {
   int32_t xs;     // bytes of the staged x
   int32_t nsup;   // super-chunks of the widest row
+  int32_t us;     // byte offset of a segment's U rows (bulk copied), from the slots' end
   int32_t total;  // dynamic shared memory of the launch
 };
 
+// [unit slots][x][row partials][z][a segment's U rows][mbarriers]
 B1Layout b1_layout(int n_max, int r_pad_max) {
   B1Layout L;
   L.xs = int32_t(round_up(int64_t(n_max) * 2, 16));
   L.nsup = int32_t(((n_max + 15) / 16 + kSupChunks - 1) / kSupChunks);
-  L.total = int32_t(int64_t(2 * kB1Warps) * kUnitSlot + L.xs + int64_t(kSegB1) * L.nsup * 4 +
-                    int64_t(r_pad_max) * 4 + 2 * kB1Warps * 8 + 16);
+  L.us = int32_t(round_up(int64_t(L.xs) + int64_t(kSegB1) * L.nsup * 4 + int64_t(r_pad_max) * 4, 16));
+  L.total = int32_t(int64_t(2 * kB1Warps) * kUnitSlot + L.us + int64_t(kSegB1) * r_pad_max * 2 +
+                    (2 * kB1Warps + 1) * 8 + 16);
   return L;
 }
 
@@ -653,14 +788,18 @@ __global__ void __maxnreg__(112) k_apply_24_b1_tma(ApplyArgs a, B1Layout lay) {
   __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(smem + 2 * kB1Warps * kUnitSlot);
   float* ysp = reinterpret_cast<float*>(smem + 2 * kB1Warps * kUnitSlot + lay.xs);  // [kSegB1][nsup]
   float* zs = ysp + kSegB1 * lay.nsup;
+  __nv_bfloat16* us = reinterpret_cast<__nv_bfloat16*>(smem + 2 * kB1Warps * kUnitSlot + lay.us);
   uint64_t* bars = reinterpret_cast<uint64_t*>(
-      (reinterpret_cast<uintptr_t>(zs + a.r_pad_max) + 7) & ~uintptr_t(7));
+      (reinterpret_cast<uintptr_t>(us + kSegB1 * a.r_pad_max) + 7) & ~uintptr_t(7));
   uint64_t* const mybar = bars + 2 * warp;
+  uint64_t* const ubar = bars + 2 * kB1Warps;  // a segment's U rows
   if (threadIdx.x == 0) {
     abort_flag = 0;
-    for (int i = 0; i < 2 * kB1Warps; ++i) tc::mbar_init(&bars[i], 1);
+    for (int i = 0; i <= 2 * kB1Warps; ++i) tc::mbar_init(&bars[i], 1);
     tc::fence_mbar_init();
   }
+  uint32_t uph = 0u;
+  bool upending = false;  // thread 0: a U copy in flight
   __syncthreads();
   volatile int* abrt = &abort_flag;
   uint32_t ph = 0u, pending = 0u;  // per-slot bits: mbarrier parity, copy in flight
@@ -829,6 +968,15 @@ __global__ void __maxnreg__(112) k_apply_24_b1_tma(ApplyArgs a, B1Layout lay) {
     __nv_bfloat16* y = y_of<__nv_bfloat16>(a, p) + int64_t(a.b0) * P.m;
     for (int s0 = l0, seg = 0; s0 < l1; s0 += kSegB1, ++seg) {
       const int s1 = min(s0 + kSegB1, l1);
+      // the segment's U rows: one bulk copy, landing while the S units stream
+      if (threadIdx.x == 0 && P.r_pad > 0 && !*abrt) {
+        const uint32_t ub = uint32_t(s1 - s0) * uint32_t(P.r_pad) * 2u;
+        tc::fence_async_smem();
+        tc::mbar_expect_tx(ubar, ub);
+        tc::bulk_load_hint(us, static_cast<const __nv_bfloat16*>(P.U) + int64_t(s0) * P.r_pad, ub,
+                           ubar, policy);
+        upending = true;
+      }
       const int jend = min(nu, (seg + 1) * useg);
       for (int j = seg * useg; j < jend; ++j) {
         const int sl = j & 1;
@@ -902,8 +1050,13 @@ __global__ void __maxnreg__(112) k_apply_24_b1_tma(ApplyArgs a, B1Layout lay) {
         }
       }
       if (i < s1 - s0) ysp[i] = yrow;
+      if (threadIdx.x == 0 && upending) {
+        if (!tc::mbar_wait(ubar, uph, a.err)) *abrt = 1;
+        uph ^= 1u;
+        upending = false;
+      }
       __syncthreads();
-      urows<__nv_bfloat16, 1, kB1Threads>(P, zs, ysp, s0, s1, y, 1);
+      urows<__nv_bfloat16, 1, kB1Threads>(P, zs, ysp, s0, s1, y, 1, us);
       __syncthreads();
     }
     row = P.row0 + l1;
@@ -912,6 +1065,7 @@ __global__ void __maxnreg__(112) k_apply_24_b1_tma(ApplyArgs a, B1Layout lay) {
   // after an abort, copies still in flight land before the CTA exits
   for (int sl = 0; sl < 2; ++sl)
     if ((pending >> sl) & 1u) tc::mbar_wait(mybar + sl, (ph >> sl) & 1u, a.err);
+  if (threadIdx.x == 0 && upending) tc::mbar_wait(ubar, uph, a.err);
   // the last CTA out resets the z counters for the next call on the stream
   __syncthreads();
   if (a.z_pieces > 0 && threadIdx.x == 0 &&
@@ -1044,9 +1198,9 @@ __global__ void __launch_bounds__(kCsrThreads, 1) k_apply_csr_b1(ApplyArgs a, Cs
     const int64_t p_end = a.prob_row0[p + 1];
     const int lp0 = int(row - P.row0);
     const int lp1 = int(min(row_end, p_end) - P.row0);
-    const T* x = x_of<T>(a, p);
-    T* y = y_of<T>(a, p);
     const int n = P.n;
+    const T* x = x_of<T>(a, p) + int64_t(a.b0) * n;   // this launch's token
+    T* y = y_of<T>(a, p) + int64_t(a.b0) * P.m;
     __syncthreads();  // the previous layer is done with xs and zs
     for (int c = threadIdx.x; c < n; c += kCsrThreads) xs[c] = x[c];
     if (threadIdx.x == 0) xs[n] = VT<T>::from_f(0.f);
@@ -1187,17 +1341,26 @@ bool decode_b1_bulk_enabled() {
   return on;
 }
 
-// HSL_DECODE_CSR=regs (read on every call) keeps batch-1 CSR on the
-// register-fed kernel (a cross-check of the bulk-copy fed one).
+// HSL_DECODE_CSR=bulk (read on every call) moves batch-1 CSR onto the
+// bulk-copy fed kernel.  It is not the default: on four layers of the 7B stack
+// it took 122 µs against 66 µs for the register-fed kernel (issue-bound on
+// shared-memory reads and chunk barriers).
+// HSL_DECODE_CSR=rows (read on every call) keeps batch-1 CSR rows on lane
+// groups per row instead of the vector-parallel walk (a cross-check).
+bool csr_vec_enabled() {
+  const char* e = std::getenv("HSL_DECODE_CSR");
+  return !(e && std::strcmp(e, "rows") == 0);
+}
+
 bool decode_csr_bulk_enabled() {
   const char* e = std::getenv("HSL_DECODE_CSR");
-  return !(e && std::strcmp(e, "regs") == 0);
+  return e && std::strcmp(e, "bulk") == 0;
 }
 
 template <typename T, int BC>
 size_t apply_smem(const ApplyPlan& plan) {
   return size_t(BC) * plan.r_pad_max * 4 + size_t(kSeg) * BC * 4 +
-         round_up(size_t(plan.n_max + 1) * BC * sizeof(T), 16);
+         round_up(size_t(plan.n_max + 1) * BC * sizeof(T), 16) + round_up(size_t(kSeg + 1) * 4, 16);
 }
 
 template <typename T, int BC>
@@ -1274,10 +1437,12 @@ hsl_status launch_chunk(ApplyPlan& plan, ApplyArgs a, int num_sms, cudaStream_t 
     set_message("the staged x of this layer does not fit in shared memory");
     return HSL_ERR_UNSUPPORTED;
   }
+  // batch-1 CSR rows vector-parallel unless HSL_DECODE_CSR=rows
+  const bool vec = BC == 1 && csr_vec_enabled();
   auto ak = plan.fmt != HSL_FMT_CSR ? k_apply_decode<T, BC, false, 16>
-            : plan.idx_bits == 8    ? k_apply_decode<T, BC, true, 8>
-            : plan.idx_bits == 32   ? k_apply_decode<T, BC, true, 32>
-                                    : k_apply_decode<T, BC, true, 16>;
+            : plan.idx_bits == 8    ? (vec ? k_apply_csr_vec<T, 8> : k_apply_decode<T, BC, true, 8>)
+            : plan.idx_bits == 32   ? (vec ? k_apply_csr_vec<T, 32> : k_apply_decode<T, BC, true, 32>)
+                                    : (vec ? k_apply_csr_vec<T, 16> : k_apply_decode<T, BC, true, 16>);
   if (cudaError_t e = cudaFuncSetAttribute(ak, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm)))
     return cuda_fail(e, "apply smem attribute");
   int occ = 0;
@@ -1335,6 +1500,7 @@ hsl_status apply_decode_run(ApplyPlan& plan, const void* X, void* Y, const void*
   a.zsync = static_cast<unsigned long long*>(plan.zsync.p);
   a.spin_limit = kSpinLimit;
   a.zwait_extra = 0;
+  a.n_max = plan.n_max;
   // HSL_FAULT_INJECT=zwait: the batch-1 2:4 kernel's wait for z gets a target no
   // CTA count reaches and a short limit, so it gives up, records kErrTimeout
   // and the kernel finishes its normal path (host-side failure testing of the
