@@ -378,10 +378,15 @@ def oracle_rho_rate(m, n, seed, target_s):
 
 # ------------------------------------------------------------------ per-workload GPU leg
 
+HOLD_CYCLES = 400_000  # ~0.2 ms of device spin before each timed call
+
+
 def time_calls(fn, stream, reps=20, flush=None):
     """Median CUDA-event time (ms) of `reps` calls on `stream` after 3 warm-up
     calls; with `flush` (a buffer larger than L2) written before each call,
-    outside its events."""
+    outside its events.  A short device spin precedes the start event, so the
+    host has queued the call's launches before it records: the interval holds
+    the call's kernels, not the host's time to enqueue them."""
     import torch
     for _ in range(3):
         fn()
@@ -389,6 +394,7 @@ def time_calls(fn, stream, reps=20, flush=None):
     for _ in range(reps):
         if flush is not None:
             flush.fill_(1)
+        torch.cuda._sleep(HOLD_CYCLES)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         fn()

@@ -175,6 +175,7 @@ __global__ void __launch_bounds__(192, 1)
       for (int s = 0; s < STAGES; ++s)
         if (issued[s]) tc::mbar_wait(&full[s], (issued[s] - 1) & 1, err);
     }
+    __syncwarp();  // lanes 1-31 wait here for lane 0: the warp meets the CTA barrier converged
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = tc::idesc_bf16(BM, BN);
@@ -195,6 +196,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       tc::mma_commit(accf);
     }
+    __syncwarp();  // lanes 1-31 wait here for lane 0: the warp meets the CTA barrier converged
   } else {
     // warps 2..5: expansion of S, then the epilogue.  Row = TMEM lane.
     const int row = ((warp & 3) << 5) | lane;
@@ -321,6 +323,7 @@ __global__ void __launch_bounds__(192, 1)
       for (int s = 0; s < ZSTAGES; ++s)
         if (issued[s]) tc::mbar_wait(&full[s], (issued[s] - 1) & 1, err);
     }
+    __syncwarp();  // lanes 1-31 wait here for lane 0: the warp meets the CTA barrier converged
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = tc::idesc_bf16(128, r16);
@@ -339,6 +342,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       tc::mma_commit(accf);
     }
+    __syncwarp();  // lanes 1-31 wait here for lane 0: the warp meets the CTA barrier converged
   } else {
     const int row = ((warp & 3) << 5) | lane;  // token within the tile
     if (tc::mbar_wait(accf, 0, err) && !*abrt) {
@@ -517,6 +521,7 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
       for (int j = kb > SP_STAGES ? kb - SP_STAGES : 0; j < kb; ++j)
         tc::mbar_wait(&full[j % SP_STAGES], (j / SP_STAGES) & 1, err);
     }
+    __syncwarp();  // lanes 1-31 wait here for lane 0: the warp meets the CTA barrier converged
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc_sp = tc::idesc_bf16(128, SP_BN) | (1u << 2);
@@ -555,6 +560,7 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
       }
       tc::mma_commit(accf);
     }
+    __syncwarp();  // lanes 1-31 wait here for lane 0: the warp meets the CTA barrier converged
   } else if (warp < 6) {
     // warps 2..5: metadata into TMEM, then the epilogue.  TMEM lane = L.
     const int L = ((warp & 3) << 5) | lane;
@@ -741,6 +747,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         }
       }
     }
+    __syncwarp();  // lanes 1-31 wait here for lane 0: the warp meets the CTA barrier converged
   } else if (warp == 1) {
     if (lane == 0 && leader) {
       const uint32_t idesc_sp = tc::idesc_bf16(256, P2_BN) | (1u << 2);
@@ -780,6 +787,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       }
       tc::mma_commit_pair(accf);
     }
+    __syncwarp();  // lanes 1-31 wait here for lane 0: the warp meets the CTA barrier converged
   } else {
     // warps 2..5: metadata into TMEM ahead of the MMAs, then the epilogue
     const int L = ((warp & 3) << 5) | lane;

@@ -136,6 +136,7 @@ __global__ void __launch_bounds__(PC_THREADS, 1)
       for (int s = 0; s < PC_STAGES; ++s)
         if (issued[s]) tc::mbar_wait(&full[s], (issued[s] - 1) & 1, err);
     }
+    __syncwarp();  // lanes 1-31 wait here for lane 0: the warp meets the CTA barrier converged
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = tc::idesc_bf16(128, PC_BN);
@@ -159,6 +160,7 @@ __global__ void __launch_bounds__(PC_THREADS, 1)
       }
       tc::mma_commit(accf);
     }
+    __syncwarp();  // lanes 1-31 wait here for lane 0: the warp meets the CTA barrier converged
   } else {
     // decompression: thread R owns row i0 + R of the tile; rows 0..127 belong to
     // the first accumulator, 128..255 to the second (TMEM lane R mod 128; warp

@@ -256,12 +256,14 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
       const bool xs = warp == 10;
       const uint64_t keep = tc::make_policy_evict_last();
       const uint64_t stream = tc::make_policy_evict_first();
-      int k = 0;
-      for (long long u = u0; u < u1; ++u, ++k) {
-        const int s = k % ST;
-        const uint32_t ph = (k / ST) & 1;
+      // (tile, K-block pair) of the unit advanced incrementally: a single
+      // thread's 64-bit division would cost hundreds of cycles per unit
+      int tile = int(u0 / nkb), kp = int(u0 % nkb);
+      const int nu = int(u1 - u0);
+      int k = 0, s = 0;
+      uint32_t ph = 0;
+      for (; k < nu; ++k) {
         if (!wait_or_abort(&empty[s], ph ^ 1, a.err, abrt)) break;
-        const int tile = int(u / nkb), kp = int(u % nkb);
         unsigned char* st = smem + s * STAGE;
         if (!xs) {
           tc::mbar_expect_tx(&full[s], SK_A);
@@ -274,21 +276,25 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
           tc::bulk_load(st + SK_A + 2 * B_BYTES, a.meta + ((long long)tile * nkb + kp) * 256, SK_M,
                         &full[s]);
         }
+        if (++kp == nkb) { kp = 0; ++tile; }
+        if (++s == ST) { s = 0; ph ^= 1u; }
       }
       // drain: the stages of the last (up to ST) units this thread issued have landed
       // (the other issuer's copies complete the same phases)
       for (int j = k > ST ? k - ST : 0; j < k; ++j) tc::mbar_wait(&full[j % ST], (j / ST) & 1, a.err);
     }
+    __syncwarp();  // lanes 1-31 wait here for lane 0: the warp meets the CTA barrier converged
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc_sp = tc::idesc_bf16(128, TP) | (1u << 2);
       int seg = -1;
-      for (long long u = u0; u < u1; ++u) {
-        const int k = int(u - u0), s = k % ST;
-        const uint32_t ph = (k / ST) & 1;
-        const int kb = int(u % nkb);
-        const bool first = (u == u0) || kb == 0;
-        const bool last = (u + 1 == u1) || kb == nkb - 1;
+      const int nu = int(u1 - u0);
+      int kb = int(u0 % nkb), s = 0;
+      uint32_t ph = 0;
+      for (int k = 0; k < nu; ++k, kb = (kb + 1 == nkb ? 0 : kb + 1), s = (s + 1 == ST ? 0 : s + 1),
+               ph ^= (s == 0 ? 1u : 0u)) {
+        const bool first = k == 0 || kb == 0;
+        const bool last = k + 1 == nu || kb == nkb - 1;
         if (first) {
           ++seg;
           // the accumulator of two segments back must have been read out
@@ -317,6 +323,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
         if (last) tc::mma_commit(&accfull[seg & 1]);
       }
     }
+    __syncwarp();  // lanes 1-31 wait here for lane 0: the warp meets the CTA barrier converged
   } else if (warp < 6) {
     // metadata of each unit, expanded to one 16-byte row per TMEM lane and MMA
     // (the layout tcgen05.cp copies); the MMA thread moves it into TMEM

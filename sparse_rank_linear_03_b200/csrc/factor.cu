@@ -208,6 +208,7 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
       for (int s = 0; s < ST; ++s)
         if (issued[s]) tc::mbar_wait(&full[s], (issued[s] - 1) & 1, g.err);
     }
+    __syncwarp();  // lanes 1-31 wait here for lane 0: the warp meets the CTA barrier converged
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = tc::idesc_bf16(128, g.BH);
@@ -229,6 +230,7 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
       }
       tc::mma_commit(accf);
     }
+    __syncwarp();  // lanes 1-31 wait here for lane 0: the warp meets the CTA barrier converged
   } else {
     // epilogue: TMEM lane = row of the tile
     const int q = warp & 3;
