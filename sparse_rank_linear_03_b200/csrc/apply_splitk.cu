@@ -62,10 +62,13 @@ constexpr uint32_t SK_TMEM_COLS = 256;
 // accumulator b at TMEM column 64·b
 __host__ __device__ constexpr uint32_t sk_acc_col(int b) { return 64u * uint32_t(b); }
 
-__host__ __device__ constexpr int sk_stages(int tp) { return tp <= 32 ? 6 : 4; }
+// stages per token padding: the ring and z (TP rows × up to 256 fp32, staged
+// once for the U·z sums of the tiles the CTA finishes) share the shared memory
+__host__ __device__ constexpr int sk_stages(int tp) { return tp <= 16 ? 6 : tp <= 32 ? 5 : tp <= 48 ? 4 : 3; }
 __host__ __device__ constexpr int sk_stage_bytes(int tp) { return SK_A + 2 * tp * 128 + SK_M + SK_MX; }
+__host__ __device__ constexpr int sk_zbytes(int tp) { return tp * 256 * 4; }
 __host__ __device__ constexpr int sk_smem(int tp) {
-  return sk_stages(tp) * sk_stage_bytes(tp) + 1024 + 256;
+  return sk_stages(tp) * sk_stage_bytes(tp) + sk_zbytes(tp) + 1024 + 256;
 }
 // metadata slot of (stage, MMA i): 4-column aligned, after both accumulators
 __device__ __forceinline__ uint32_t sk_meta_col(int s, int i) { return 128u + 16u * s + 4u * i; }
@@ -210,7 +213,8 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * STAGE);
+  float* zs = reinterpret_cast<float*>(smem + ST * STAGE);  // [TP][r_pad], staged once
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * STAGE + sk_zbytes(TP));
   uint64_t* mfull = full + ST;
   uint64_t* empty = mfull + ST;
   uint64_t* accfull = empty + ST;   // [2]
@@ -359,6 +363,13 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
       const int c_first = cta_of(tile_u0, a.units, grid);
       const int c_last = cta_of(tile_u1 - 1, a.units, grid);
       const int nseg = c_last - c_first + 1;
+      // this row's U into L2 while the segment's MMAs run (the CTA that finishes
+      // the tile reads it after the partial sums; from DRAM each of its loads
+      // would cost a full memory latency)
+      if (a.r > 0 && tile * 128 + L < a.m) {
+        const char* up = reinterpret_cast<const char*>(a.U + (long long)(tile * 128 + L) * a.r_pad);
+        for (int b = 0; b < a.r_pad * 2; b += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(up + b));
+      }
       float v[TP];
       const bool ok = wait_or_abort(&accfull[seg & 1], (seg >> 1) & 1, a.err, abrt);
       if (ok) {
@@ -400,24 +411,37 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
           if (tid == 0) a.cnt[tile] = 0u;  // ready for the next call
         }
       }
+      if (finish && a.r > 0 && !z_ready) {
+        // z into shared memory, once: the sums below read it for every row
+        pdl_wait();  // z is written by the preceding kernel
+        for (int e = tid; e < TP * a.r_pad / 4; e += 128)
+          reinterpret_cast<float4*>(zs)[e] = __ldcg(reinterpret_cast<const float4*>(a.z) + e);
+        epi_sync();
+        z_ready = true;
+      }
       if (finish && i < a.m) {
         if (a.r > 0) {
-          if (!z_ready) {
-            pdl_wait();  // z is written by the preceding kernel
-            z_ready = true;
-          }
-          // + U[i,:]·z[t,:], added to the tile's sum in factor-column order (fp32)
+          // + U[i,:]·z[t,:], added to the tile's sum in factor-column order (fp32).
+          // Two 16-byte pieces of the U row are loaded before either is used; z
+          // has TP rows (rows past T hold whatever the last call left; their
+          // sums are never stored), so its reads need no guard.
           const __nv_bfloat16* urow = a.U + (long long)i * a.r_pad;
-          for (int c = 0; c < a.r_pad; c += 8) {
-            const uint4 uq = *reinterpret_cast<const uint4*>(urow + c);
-            const float uf[8] = {bf_lo(uq.x), bf_hi(uq.x), bf_lo(uq.y), bf_hi(uq.y),
-                                 bf_lo(uq.z), bf_hi(uq.z), bf_lo(uq.w), bf_hi(uq.w)};
+          for (int c0 = 0; c0 < a.r_pad; c0 += 16) {
+            uint4 uq[2];
 #pragma unroll
-            for (int t = 0; t < TP; ++t) {
-              if (t < a.T) {
-                const float4 z0 = *reinterpret_cast<const float4*>(a.z + (long long)t * a.r_pad + c);
-                const float4 z1 =
-                    *reinterpret_cast<const float4*>(a.z + (long long)t * a.r_pad + c + 4);
+            for (int j = 0; j < 2; ++j)
+              uq[j] = c0 + 8 * j < a.r_pad ? *reinterpret_cast<const uint4*>(urow + c0 + 8 * j)
+                                          : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const int c = c0 + 8 * j;
+              if (c >= a.r_pad) break;
+              const float uf[8] = {bf_lo(uq[j].x), bf_hi(uq[j].x), bf_lo(uq[j].y), bf_hi(uq[j].y),
+                                   bf_lo(uq[j].z), bf_hi(uq[j].z), bf_lo(uq[j].w), bf_hi(uq[j].w)};
+#pragma unroll
+              for (int t = 0; t < TP; ++t) {
+                const float4 z0 = *reinterpret_cast<const float4*>(zs + t * a.r_pad + c);
+                const float4 z1 = *reinterpret_cast<const float4*>(zs + t * a.r_pad + c + 4);
                 float acc = v[t];
                 acc = fmaf(uf[0], z0.x, acc);
                 acc = fmaf(uf[1], z0.y, acc);
@@ -475,7 +499,7 @@ hsl_status launch_tp(Handle& h, const void* X, void* Y, int64_t T, cudaStream_t 
     // per-item counters first (a fixed place, zero at rest: kept across calls),
     // then z, then the pieces' partial sums
     const size_t cb = size_t(round_up(int64_t(h.r) * 8 * 4, 256));  // items for T up to 64
-    const size_t zb = size_t(round_up(int64_t(T) * r_pad * 4, 256));
+    const size_t zb = size_t(round_up(int64_t(TP) * r_pad * 4, 256));  // TP rows: the epilogue reads all
     const size_t pb = size_t(zitems) * zQ * 8 * 4;
     const bool fresh = !h.sk_z.p || h.sk_z.bytes < cb + zb + pb;
     if (hsl_status e = ensure(h.sk_z, cb + zb + pb, "split-K z")) return e;
