@@ -189,10 +189,12 @@ __device__ __forceinline__ void xcol(const T* xs, int c, float (&xv)[BC]) {
 
 // y[row] = ysp[row] + U[row,:]·z for rows [s0, s1) of layer P.  GU lanes
 // share a row (8 elements each); a warp takes R row groups per pass and issues
-// all their U loads before using any, so the pass costs one load latency.
+// all their U loads before using any, so the pass costs one load latency.  For
+// up to 4 tokens a lane reads its 8 z values once into registers (read per row
+// from shared memory they are 8-way bank conflicts, lanes 32 bytes apart).
 template <typename T, int BC, int NT = kThreads, int R = (BC <= 2 ? 4 : 1)>
 __device__ __forceinline__ void urows(const ApplyProblem& P, const float* zs, const float* ysp,
-                                      int s0, int s1, T* y, int bc, const T* Us = nullptr) {
+                                      int s0, int s1, T* y, int bc) {
   const int rp = P.r_pad;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int GU = 1;
@@ -200,25 +202,27 @@ __device__ __forceinline__ void urows(const ApplyProblem& P, const float* zs, co
   const int rpw = 32 / GU;        // rows per warp pass
   const int gl = lane % GU;
   const T* U = static_cast<const T*>(P.U);
+  constexpr bool kZReg = BC <= 4;
+  float zr[kZReg ? BC : 1][8];
+  if constexpr (kZReg) {
+#pragma unroll
+    for (int b = 0; b < BC; ++b) {
+      float4 z0 = make_float4(0.f, 0.f, 0.f, 0.f), z1 = z0;
+      if (gl * 8 < rp) {
+        z0 = *reinterpret_cast<const float4*>(zs + b * rp + gl * 8);
+        z1 = *reinterpret_cast<const float4*>(zs + b * rp + gl * 8 + 4);
+      }
+      zr[b][0] = z0.x; zr[b][1] = z0.y; zr[b][2] = z0.z; zr[b][3] = z0.w;
+      zr[b][4] = z1.x; zr[b][5] = z1.y; zr[b][6] = z1.z; zr[b][7] = z1.w;
+    }
+  }
   for (int ib = s0 + warp * rpw * R; ib < s1; ib += (NT / 32) * rpw * R) {
     float u[R][8];
 #pragma unroll
     for (int q = 0; q < R; ++q) {
       const int i = ib + q * rpw + lane / GU;
       if (i < s1 && gl * 8 < rp) {
-        if (Us != nullptr) {  // the segment's U rows, staged in shared memory
-          const T* ur = Us + int64_t(i - s0) * rp + gl * 8;
-          if constexpr (sizeof(T) == 2) {
-            const uint4 q4 = *reinterpret_cast<const uint4*>(ur);
-            u[q][0] = bf_lo(q4.x); u[q][1] = bf_hi(q4.x); u[q][2] = bf_lo(q4.y); u[q][3] = bf_hi(q4.y);
-            u[q][4] = bf_lo(q4.z); u[q][5] = bf_hi(q4.z); u[q][6] = bf_lo(q4.w); u[q][7] = bf_hi(q4.w);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) u[q][e] = VT<T>::f(ur[e]);
-          }
-        } else {
-          load8<T>(U + int64_t(i) * rp + gl * 8, u[q]);
-        }
+        load8<T>(U + int64_t(i) * rp + gl * 8, u[q]);
       }
     }
 #pragma unroll
@@ -231,7 +235,8 @@ __device__ __forceinline__ void urows(const ApplyProblem& P, const float* zs, co
 #pragma unroll
         for (int b = 0; b < BC; ++b)
 #pragma unroll
-          for (int e = 0; e < 8; ++e) acc[b] = fmaf(u[q][e], zs[b * rp + gl * 8 + e], acc[b]);
+          for (int e = 0; e < 8; ++e)
+            acc[b] = fmaf(u[q][e], kZReg ? zr[kZReg ? b : 0][e] : zs[b * rp + gl * 8 + e], acc[b]);
       }
       for (int o = GU >> 1; o; o >>= 1)
 #pragma unroll
@@ -722,27 +727,26 @@ constexpr int kSupChunks = 256;                  // chunks of a super-chunk
 constexpr int kUnitVBytes = kSupChunks * 16;     // values of a full unit
 constexpr int kUnitMBytes = kSupChunks * 2;      // metadata of a unit
 constexpr int kUnitSlot = kUnitVBytes + kUnitMBytes;
-// Rows per segment of the bulk-copy kernel.  A segment's U·z pass (U rows by
-// plain loads) runs while every warp's first S unit of the next segment is
-// already in flight, so short segments overlap the factor term with the S
-// stream; a multiple of 16 (= kB1Warps) keeps every warp's units in step.
-constexpr int kSegB1 = 64;
+// Most rows per segment of the bulk-copy kernel.  At a segment's end the S
+// stream pauses (only every warp's first unit of the next segment is in
+// flight) while the row partials are summed and the U·z pass runs; measured
+// on the 70B layer each such boundary costs about 5 µs, so a CTA's rows are cut
+// into as few segments as the row-partial buffer allows, of equal length.
+constexpr int kSegB1 = 128;
 
 struct B1Layout {
   int32_t xs;     // bytes of the staged x
   int32_t nsup;   // super-chunks of the widest row
-  int32_t us;     // byte offset of a segment's U rows (bulk copied), from the slots' end
   int32_t total;  // dynamic shared memory of the launch
 };
 
-// [unit slots][x][row partials][z][a segment's U rows][mbarriers]
+// [unit slots][x][row partials][z][mbarriers]
 B1Layout b1_layout(int n_max, int r_pad_max) {
   B1Layout L;
   L.xs = int32_t(round_up(int64_t(n_max) * 2, 16));
   L.nsup = int32_t(((n_max + 15) / 16 + kSupChunks - 1) / kSupChunks);
-  L.us = int32_t(round_up(int64_t(L.xs) + int64_t(kSegB1) * L.nsup * 4 + int64_t(r_pad_max) * 4, 16));
-  L.total = int32_t(int64_t(2 * kB1Warps) * kUnitSlot + L.us + int64_t(kSegB1) * r_pad_max * 2 +
-                    (2 * kB1Warps + 1) * 8 + 16);
+  L.total = int32_t(int64_t(2 * kB1Warps) * kUnitSlot + L.xs + int64_t(kSegB1) * L.nsup * 4 +
+                    int64_t(r_pad_max) * 4 + 2 * kB1Warps * 8 + 16);
   return L;
 }
 
@@ -778,28 +782,87 @@ __device__ __forceinline__ void chunk24(const uint4& v, const uint4& xl, const u
   fma2_bf16(a0, a1, v.w, __byte_perm(xh.z, xh.w, s3));
 }
 
+// The z pieces of one warp of the batch-1 2:4 kernel (see the kernel), then the
+// warp counts itself in; the CTA's last warp counts the CTA in on the grid's
+// counter.  Out of line: it runs once per warp, and inlined into the unit loop
+// it would raise that loop's register pressure.
+__device__ __noinline__ void b1_z_pieces(const ApplyArgs& a, int warp, int lane, int* zwarps) {
+  const int64_t nw = int64_t(gridDim.x) * kB1Warps;
+  for (int64_t it = int64_t(blockIdx.x) * kB1Warps + warp; it < a.z_pieces; it += nw) {
+    int lo = 0, hi = a.count - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (a.probs[mid].z_piece0 <= it) lo = mid; else hi = mid - 1;
+    }
+    const ApplyProblem& Pz = a.probs[lo];
+    const int nz = Pz.n, pw = z_piece_width(nz), Q = (nz + pw - 1) / pw;
+    const int local = int(it - Pz.z_piece0), c = local / Q, q = local - c * Q;
+    const __nv_bfloat16* vrow = static_cast<const __nv_bfloat16*>(Pz.Vt) + int64_t(c) * nz;
+    const __nv_bfloat16* xz = x_of<__nv_bfloat16>(a, lo) + int64_t(a.b0) * nz;
+    const int j0 = q * pw, j1 = min(nz, j0 + pw);
+    float acc = 0.f;
+    if ((reinterpret_cast<uintptr_t>(xz) & 15) == 0) {  // n % 16 == 0: Vt rows are 16-byte aligned
+      // at most 8 vectors per lane (pw ≤ 2048), four loads of each operand in flight
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint4 vq[4], xq[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int j = j0 + ((4 * half + u) * 32 + lane) * 8;
+          if (j < j1) {
+            vq[u] = ld_stream16(vrow + j);
+            xq[u] = *reinterpret_cast<const uint4*>(xz + j);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (j0 + ((4 * half + u) * 32 + lane) * 8 < j1) {
+            const uint32_t vw[4] = {vq[u].x, vq[u].y, vq[u].z, vq[u].w};
+            const uint32_t xw[4] = {xq[u].x, xq[u].y, xq[u].z, xq[u].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              acc = fmaf(bf_lo(vw[e]), bf_lo(xw[e]), acc);
+              acc = fmaf(bf_hi(vw[e]), bf_hi(xw[e]), acc);
+            }
+          }
+        }
+      }
+    } else {
+      for (int j = j0 + lane; j < j1; j += 32)
+        acc = fmaf(ldx<__nv_bfloat16>(vrow + j), ldx<__nv_bfloat16>(xz + j), acc);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) Pz.z[q * Pz.r_pad + c] = acc;
+  }
+  __threadfence();  // this warp's pieces are visible before it counts itself in
+  __syncwarp();
+  if (lane == 0 && atomicAdd(zwarps, 1) == kB1Warps - 1) {
+    __threadfence();
+    atomicAdd(&a.zsync[0], 1ull);
+  }
+}
+
 // At most 112 registers: 16 warps then leave room on the SM for a CTA of the
 // z kernel, which the apply CTA overlaps (programmatic dependent launch).
 __global__ void __maxnreg__(112) k_apply_24_b1_tma(ApplyArgs a, B1Layout lay) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ int abort_flag;
+  __shared__ int zwarps;  // warps of this CTA done with their z pieces
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   unsigned char* const slot0 = smem + (2 * warp) * kUnitSlot;
   __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(smem + 2 * kB1Warps * kUnitSlot);
   float* ysp = reinterpret_cast<float*>(smem + 2 * kB1Warps * kUnitSlot + lay.xs);  // [kSegB1][nsup]
   float* zs = ysp + kSegB1 * lay.nsup;
-  __nv_bfloat16* us = reinterpret_cast<__nv_bfloat16*>(smem + 2 * kB1Warps * kUnitSlot + lay.us);
   uint64_t* bars = reinterpret_cast<uint64_t*>(
-      (reinterpret_cast<uintptr_t>(us + kSegB1 * a.r_pad_max) + 7) & ~uintptr_t(7));
+      (reinterpret_cast<uintptr_t>(zs + a.r_pad_max) + 7) & ~uintptr_t(7));
   uint64_t* const mybar = bars + 2 * warp;
-  uint64_t* const ubar = bars + 2 * kB1Warps;  // a segment's U rows
   if (threadIdx.x == 0) {
     abort_flag = 0;
-    for (int i = 0; i <= 2 * kB1Warps; ++i) tc::mbar_init(&bars[i], 1);
+    zwarps = 0;
+    for (int i = 0; i < 2 * kB1Warps; ++i) tc::mbar_init(&bars[i], 1);
     tc::fence_mbar_init();
   }
-  uint32_t uph = 0u;
-  bool upending = false;  // thread 0: a U copy in flight
   __syncthreads();
   volatile int* abrt = &abort_flag;
   uint32_t ph = 0u, pending = 0u;  // per-slot bits: mbarrier parity, copy in flight
@@ -824,91 +887,18 @@ __global__ void __maxnreg__(112) k_apply_24_b1_tma(ApplyArgs a, B1Layout lay) {
   // z = Vᵀx of every layer of the call in pieces of one row of Vt × ≥ 1024
   // columns (z_piece_width), one piece per warp over the whole grid: a warp sums its piece
   // with a fixed shuffle tree into z_part[q][c] (q = piece of row c), and the
-  // U·z pass adds a row's pieces in order (deterministic).  Each CTA counts
-  // itself in once its warps are done; a CTA waits for the count to reach the
-  // grid only before its first U·z pass.  The launch is cooperative, so all
-  // CTAs are resident and the wait ends (it is bounded all the same).  The
-  // first unit of S is already on its way (issued before the pieces).
-  bool first_issued = false;
-  if (row < row_end) {  // this warp's first S unit (unit `warp` of the first layer)
-    const ApplyProblem& P = a.probs[p];
-    const int l0 = int(row - P.row0), l1 = int(min(row_end, a.prob_row0[p + 1]) - P.row0);
-    const int nq0 = P.n / 16, nsup0 = (nq0 + kSupChunks - 1) / kSupChunks;
-    if (warp < (l1 - l0) * nsup0) {
-      const int r0u = warp / nsup0, sp0 = warp - r0u * nsup0;
-      if (lane == 0) {
-        const int64_t i = int64_t(l0) + r0u;
-        const uint32_t vb = uint32_t(min(kSupChunks, nq0 - sp0 * kSupChunks)) * 16u;
-        tc::fence_async_smem();
-        tc::mbar_expect_tx(mybar, vb + kUnitMBytes);
-        tc::bulk_load_hint(slot0,
-                           static_cast<const unsigned char*>(P.pval) + i * P.n +
-                               int64_t(sp0) * kUnitVBytes,
-                           vb, mybar, policy);
-        tc::bulk_load_hint(slot0 + kUnitVBytes,
-                           reinterpret_cast<const unsigned char*>(P.pmeta) +
-                               i * (int64_t(P.meta_stride) * 2) + sp0 * kUnitMBytes,
-                           kUnitMBytes, mybar, policy);
-      }
-      pending |= 1u;
-      first_issued = true;
-    }
-  }
-  if (a.z_pieces > 0) {
-    const int64_t nw = int64_t(gridDim.x) * kB1Warps;
-    for (int64_t it = int64_t(blockIdx.x) * kB1Warps + warp; it < a.z_pieces; it += nw) {
-      int lo = 0, hi = a.count - 1;
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (a.probs[mid].z_piece0 <= it) lo = mid; else hi = mid - 1;
-      }
-      const ApplyProblem& Pz = a.probs[lo];
-      const int nz = Pz.n, pw = z_piece_width(nz), Q = (nz + pw - 1) / pw;
-      const int local = int(it - Pz.z_piece0), c = local / Q, q = local - c * Q;
-      const __nv_bfloat16* vrow = static_cast<const __nv_bfloat16*>(Pz.Vt) + int64_t(c) * nz;
-      const __nv_bfloat16* xz = x_of<__nv_bfloat16>(a, lo) + int64_t(a.b0) * nz;
-      const int j0 = q * pw, j1 = min(nz, j0 + pw);
-      float acc = 0.f;
-      if ((reinterpret_cast<uintptr_t>(xz) & 15) == 0) {  // n % 16 == 0: Vt rows are 16-byte aligned
-        // at most 8 vectors per lane (pw ≤ 2048), four loads of each operand in flight
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint4 vq[4], xq[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int j = j0 + ((4 * half + u) * 32 + lane) * 8;
-            if (j < j1) {
-              vq[u] = ld_stream16(vrow + j);
-              xq[u] = *reinterpret_cast<const uint4*>(xz + j);
-            }
-          }
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            if (j0 + ((4 * half + u) * 32 + lane) * 8 < j1) {
-              const uint32_t vw[4] = {vq[u].x, vq[u].y, vq[u].z, vq[u].w};
-              const uint32_t xw[4] = {xq[u].x, xq[u].y, xq[u].z, xq[u].w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                acc = fmaf(bf_lo(vw[e]), bf_lo(xw[e]), acc);
-                acc = fmaf(bf_hi(vw[e]), bf_hi(xw[e]), acc);
-              }
-            }
-          }
-        }
-      } else {
-        for (int j = j0 + lane; j < j1; j += 32)
-          acc = fmaf(ldx<__nv_bfloat16>(vrow + j), ldx<__nv_bfloat16>(xz + j), acc);
-      }
-#pragma unroll
-      for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (lane == 0) Pz.z[q * Pz.r_pad + c] = acc;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      __threadfence();
-      atomicAdd(&a.zsync[0], 1ull);
-    }
-  }
+  // U·z pass adds a row's pieces in order (deterministic).  A warp takes its
+  // pieces after its first S unit (its second is then in flight, and the other
+  // warps keep streaming); the CTA counts itself in once all its warps are done,
+  // and a CTA waits for the count to reach the grid only before its first U·z
+  // pass.  The launch is cooperative, so all CTAs are resident and the wait
+  // ends (it is bounded all the same).
+  bool z_pending = a.z_pieces > 0;
+  auto do_z = [&]() {
+    if (!z_pending) return;
+    z_pending = false;
+    b1_z_pieces(a, warp, lane, &zwarps);
+  };
   bool waited = false;
   while (row < row_end) {
     const ApplyProblem P = a.probs[p];
@@ -921,7 +911,9 @@ __global__ void __maxnreg__(112) k_apply_24_b1_tma(ApplyArgs a, B1Layout lay) {
     const uint32_t nsup_magic = nsup > 1 ? 0xFFFFFFFFu / uint32_t(nsup) + 1u : 0u;
     const int units = (l1 - l0) * nsup;
     const int nu = warp < units ? (units - warp + kB1Warps - 1) / kB1Warps : 0;
-    const int useg = kSegB1 * nsup / kB1Warps;  // units of a warp in one segment
+    // segments of equal length (at most kSegB1 rows): no short tail segment
+    const int nseg = (l1 - l0 + kSegB1 - 1) / kSegB1;
+    const int seg_rows = nseg > 0 ? (l1 - l0 + nseg - 1) / nseg : kSegB1;
     const uint32_t mstride = uint32_t(P.meta_stride) * 2u;
     const unsigned char* pval = static_cast<const unsigned char*>(P.pval);
     const unsigned char* pmeta = reinterpret_cast<const unsigned char*>(P.pmeta);
@@ -948,8 +940,7 @@ __global__ void __maxnreg__(112) k_apply_24_b1_tma(ApplyArgs a, B1Layout lay) {
       }
       pending |= 1u << sl;
     };
-    if (nu > 0 && !first_issued) issue(0);  // lands while x is staged
-    first_issued = false;
+    if (nu > 0) issue(0);  // lands while x is staged
     const __nv_bfloat16* x = x_of<__nv_bfloat16>(a, p) + int64_t(a.b0) * n;
     __syncthreads();
     if ((reinterpret_cast<uintptr_t>(x) & 15) == 0) {
@@ -966,19 +957,18 @@ __global__ void __maxnreg__(112) k_apply_24_b1_tma(ApplyArgs a, B1Layout lay) {
     const uint4* xwin_lo = xs4 + 2 * lane + xsw;
     const uint4* xwin_hi = xs4 + 2 * lane + 1 - xsw;
     __nv_bfloat16* y = y_of<__nv_bfloat16>(a, p) + int64_t(a.b0) * P.m;
-    for (int s0 = l0, seg = 0; s0 < l1; s0 += kSegB1, ++seg) {
-      const int s1 = min(s0 + kSegB1, l1);
-      // the segment's U rows: one bulk copy, landing while the S units stream
-      if (threadIdx.x == 0 && P.r_pad > 0 && !*abrt) {
-        const uint32_t ub = uint32_t(s1 - s0) * uint32_t(P.r_pad) * 2u;
-        tc::fence_async_smem();
-        tc::mbar_expect_tx(ubar, ub);
-        tc::bulk_load_hint(us, static_cast<const __nv_bfloat16*>(P.U) + int64_t(s0) * P.r_pad, ub,
-                           ubar, policy);
-        upending = true;
-      }
-      const int jend = min(nu, (seg + 1) * useg);
-      for (int j = seg * useg; j < jend; ++j) {
+    int jbeg = 0;  // this warp's first unit of the segment
+    for (int s0 = l0, seg = 0; s0 < l1; s0 += seg_rows, ++seg) {
+      const int s1 = min(s0 + seg_rows, l1);
+      // the segment's U rows into L2 while its S units stream (one bulk
+      // prefetch: the rows are contiguous), so the U·z pass reads them from L2
+      if (threadIdx.x == 0 && P.r_pad > 0)
+        tc::bulk_prefetch_l2(static_cast<const __nv_bfloat16*>(P.U) + int64_t(s0) * P.r_pad,
+                             uint32_t(s1 - s0) * uint32_t(P.r_pad) * 2u);
+      // units u = warp + 16·j of the segment: u < (s1 − l0)·nsup
+      const int ub = (s1 - l0) * nsup;
+      const int jend = min(nu, ub > warp ? (ub - warp + kB1Warps - 1) / kB1Warps : 0);
+      for (int j = jbeg; j < jend; ++j) {
         const int sl = j & 1;
         if (j + 1 < nu) issue(j + 1);
         bool ok = ((pending >> sl) & 1u) && !aborted();
@@ -1020,7 +1010,10 @@ __global__ void __maxnreg__(112) k_apply_24_b1_tma(ApplyArgs a, B1Layout lay) {
         for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
         if (lane == 0) ysp[(l0 + r - s0) * nsup + sp] = acc;
         __syncwarp();  // every lane is done with the slot before its next copy
+        do_z();        // after the warp's first unit (once)
       }
+      jbeg = jend;
+      do_z();  // a warp without units in this segment
       __syncthreads();
       // a row's partials, summed in super-chunk order
       float yrow = 0.f;
@@ -1050,22 +1043,17 @@ __global__ void __maxnreg__(112) k_apply_24_b1_tma(ApplyArgs a, B1Layout lay) {
         }
       }
       if (i < s1 - s0) ysp[i] = yrow;
-      if (threadIdx.x == 0 && upending) {
-        if (!tc::mbar_wait(ubar, uph, a.err)) *abrt = 1;
-        uph ^= 1u;
-        upending = false;
-      }
       __syncthreads();
-      urows<__nv_bfloat16, 1, kB1Threads>(P, zs, ysp, s0, s1, y, 1, us);
+      urows<__nv_bfloat16, 1, kB1Threads>(P, zs, ysp, s0, s1, y, 1);
       __syncthreads();
     }
     row = P.row0 + l1;
     ++p;
   }
+  do_z();  // a CTA without rows still computes its z pieces
   // after an abort, copies still in flight land before the CTA exits
   for (int sl = 0; sl < 2; ++sl)
     if ((pending >> sl) & 1u) tc::mbar_wait(mybar + sl, (ph >> sl) & 1u, a.err);
-  if (threadIdx.x == 0 && upending) tc::mbar_wait(ubar, uph, a.err);
   // the last CTA out resets the z counters for the next call on the stream
   __syncthreads();
   if (a.z_pieces > 0 && threadIdx.x == 0 &&
@@ -1095,6 +1083,11 @@ constexpr int kCsrWarps = kCsrThreads / 32;
 constexpr int kCsrChunk = 4096;
 constexpr int kCsrSeg = 1024;
 constexpr int kCsrProw = 8192;  // rows per staged window of row starts
+// Words the window takes in shared memory: its kCsrProw + 1 row starts,
+// padded so that the float arrays after it start on a 16-byte boundary.
+constexpr int kCsrProwWords = (kCsrProw + 1 + 3) & ~3;
+static_assert(kCsrProwWords * 4 % 16 == 0 && kCsrSeg * 4 % 16 == 0,
+              "z is read as 16-byte vectors from after the row starts and y partials");
 constexpr int kCsrMaxSlots = 6;
 
 struct CsrLayout {
@@ -1112,7 +1105,7 @@ CsrLayout csr_layout(int eb, int idx_bits, int n_max, int r_pad_max, int smem_ma
   L.bbytes = idx_bits == 8 ? kCsrChunk / 8 * 2 : 0;
   L.slot = L.vbytes + L.cbytes + L.bbytes;
   L.xs = int32_t(round_up(int64_t(n_max + 1) * eb, 16));
-  const int fixed = L.xs + (kCsrProw + 1) * 4 + kCsrSeg * 4 + r_pad_max * 4 + kCsrMaxSlots * 8 + 64;
+  const int fixed = L.xs + kCsrProwWords * 4 + kCsrSeg * 4 + r_pad_max * 4 + kCsrMaxSlots * 8 + 64;
   L.slots = std::min(kCsrMaxSlots, (smem_max - fixed) / L.slot);
   L.total = L.slots * L.slot + fixed;
   return L;
@@ -1165,7 +1158,7 @@ __global__ void __launch_bounds__(kCsrThreads, 1) k_apply_csr_b1(ApplyArgs a, Cs
   const int SL = lay.slots;
   T* xs = reinterpret_cast<T*>(smem + SL * lay.slot);
   int32_t* prow_s = reinterpret_cast<int32_t*>(smem + SL * lay.slot + lay.xs);
-  float* ysp = reinterpret_cast<float*>(prow_s + kCsrProw + 1);
+  float* ysp = reinterpret_cast<float*>(prow_s + kCsrProwWords);
   float* zs = ysp + kCsrSeg;
   uint64_t* bars = reinterpret_cast<uint64_t*>(
       (reinterpret_cast<uintptr_t>(zs + a.r_pad_max) + 7) & ~uintptr_t(7));

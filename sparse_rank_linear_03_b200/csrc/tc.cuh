@@ -100,6 +100,12 @@ __device__ __forceinline__ void bulk_load_hint(void* dst, const void* src, uint3
       "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
 }
+// Prefetch a contiguous range into L2 (16-byte aligned, size a multiple of 16).
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)),
+               "r"(bytes)
+               : "memory");
+}
 // Tiled load with an L2 eviction-priority policy (from make_policy_*).
 __device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* map, int32_t x,
                                                  int32_t y, uint64_t* bar, uint64_t policy) {
