@@ -28,9 +28,9 @@
 // 128×256 tile.  TMEM holds 2×192 accumulator columns plus 4-column-aligned
 // metadata slots (the sparse MMA requires that alignment).
 //
-// Warp roles (192 threads): warp 0 lane 0 issues TMA; warp 1 owns TMEM and
-// lane 0 issues MMAs; warps 2-5 move metadata (or expand S) and run the
-// epilogue.  All waits are bounded (kSpinLimit polls); a wait that gives up sets
+// Warp roles: warp 0 lane 0 issues TMA; warp 1 owns TMEM and lane 0 issues
+// MMAs; warps 2-5 move metadata (or expand S) and run the epilogue.  The
+// sparse kernel adds warps 6 and 7, which issue the X and metadata copies.  All waits are bounded (kSpinLimit polls); a wait that gives up sets
 // the error word and the CTA drains its copies, frees TMEM and exits.
 #include <cuda.h>
 
@@ -428,7 +428,11 @@ struct SpMaps {
   CUtensorMap zlo; // Z lo [T][r16]  box {32, 192} SW64
 };
 
-constexpr int SP_THREADS = 224;  // warps: 0 A copies, 1 MMA, 2-5 metadata + epilogue, 6 B copies
+// Warps: 0 A copies, 1 MMA, 2-5 metadata into TMEM + epilogue, 6 B copies,
+// 7 metadata copies.  A copy instruction holds its issuing thread for a
+// near-fixed time whatever its size, so the three streams of copies run on
+// three threads in parallel.
+constexpr int SP_THREADS = 256;
 __global__ void __launch_bounds__(SP_THREADS, 1)
     k_prefill_24sp(const __grid_constant__ SpMaps maps, const uint2* __restrict__ meta,
                    __nv_bfloat16* __restrict__ Y, int m, int n, int T, int r16, uint32_t* err) {
@@ -439,7 +443,8 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
   unsigned char* sB = sA + SP_STAGES * SP_A;
   unsigned char* sM = sB + SP_STAGES * SP_B;
   uint64_t* full = reinterpret_cast<uint64_t*>(sM + SP_STAGES * SP_M);
-  uint64_t* mfull = full + SP_STAGES;
+  uint64_t* mload = full + SP_STAGES;  // the stage's metadata has landed
+  uint64_t* mfull = mload + SP_STAGES; // ... and is in TMEM
   uint64_t* empty = mfull + SP_STAGES;
   uint64_t* accf = empty + SP_STAGES;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
@@ -457,7 +462,8 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
   if (threadIdx.x == 0) {
     abort_flag = 0;
     for (int s = 0; s < SP_STAGES; ++s) {
-      tc::mbar_init(&full[s], 2);  // the A issuer and the B issuer
+      tc::mbar_init(&full[s], 2);  // the A and B issuers
+      tc::mbar_init(&mload[s], 1);
       tc::mbar_init(&mfull[s], 128);
       tc::mbar_init(&empty[s], 1);
     }
@@ -480,34 +486,40 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
   const uint32_t tmem = *tmem_slot;
   volatile int* abrt = &abort_flag;
 
-  if (warp == 0 || warp == 6) {
+  if (warp == 0 || warp >= 6) {
     // warp 0: the A tile (S values, then U); warp 6: the B tile (X, then Z hi
-    // and lo) and the metadata
+    // and lo); warp 7: the metadata (none for the low-rank K-blocks)
     if (lane == 0) {
-      const bool bs = warp == 6;
+      const int role = warp == 0 ? 0 : warp - 5;  // 0 A, 1 B, 2 metadata
       const uint64_t keep = tc::make_policy_evict_last();
       const uint64_t stream = tc::make_policy_evict_first();
+      // the metadata issuer covers the 2:4 K-blocks only, on its own barrier,
+      // so the metadata reaches TMEM while the stage's A and X are in flight
+      const int nkr = role == 2 ? nkS : nk;
+      uint64_t* landed = role == 2 ? mload : full;
       int kb = 0;
-      for (; kb < nk; ++kb) {
+      for (; kb < nkr; ++kb) {
         const int s = kb % SP_STAGES;
         const uint32_t ph = (kb / SP_STAGES) & 1;
         if (!wait_or_abort(&empty[s], ph ^ 1, err, abrt)) break;
         unsigned char* a = sA + s * SP_A;
         unsigned char* b = sB + s * SP_B;
-        if (!bs) {
+        if (role == 0) {
           tc::mbar_expect_tx(&full[s], SP_A);
           if (kb < nkS) tc::tma_load_2d_hint(a, &maps.sv, kb * 32, i0, &full[s], stream);
           else tc::tma_load_2d_hint(a, &maps.u, (kb - nkS) * 32, i0, &full[s], stream);
-        } else if (kb < nkS) {
+        } else if (role == 2) {
           // the metadata of both halves (1 KB each)
           const int mt0 = i0 / 128;
           const int nmeta = (mt0 < mtiles128) + (mt0 + 1 < mtiles128);
-          tc::mbar_expect_tx(&full[s], SP_B + nmeta * 1024);
-          tc::tma_load_2d_hint(b, &maps.x, kb * 64, t0, &full[s], keep);
+          tc::mbar_expect_tx(&mload[s], nmeta * 1024);
           for (int h = 0; h < 2; ++h)
             if (mt0 + h < mtiles128)
               tc::bulk_load(sM + s * SP_M + h * 1024, meta + (int64_t(mt0 + h) * nkS + kb) * 128,
-                            1024, &full[s]);
+                            1024, &mload[s]);
+        } else if (kb < nkS) {
+          tc::mbar_expect_tx(&full[s], SP_B);
+          tc::tma_load_2d_hint(b, &maps.x, kb * 64, t0, &full[s], keep);
         } else {
           if (kb == nkS) pdl_wait();  // Z is written by the preceding kernel
           const int kl = kb - nkS;
@@ -517,9 +529,9 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
         }
       }
       // drain: the last stages this thread issued have landed (the other
-      // issuer's copies complete the same phases)
+      // issuer's copies complete the same phases of `full`)
       for (int j = kb > SP_STAGES ? kb - SP_STAGES : 0; j < kb; ++j)
-        tc::mbar_wait(&full[j % SP_STAGES], (j / SP_STAGES) & 1, err);
+        tc::mbar_wait(&landed[j % SP_STAGES], (j / SP_STAGES) & 1, err);
     }
     __syncwarp();  // lanes 1-31 wait here for lane 0: the warp meets the CTA barrier converged
   } else if (warp == 1) {
@@ -568,8 +580,9 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
     for (int kb = 0; kb < nkS; ++kb) {
       const int s = kb % SP_STAGES;
       const uint32_t ph = (kb / SP_STAGES) & 1;
-      // the stage's bytes (metadata included) have landed: its previous MMAs are done
-      if (!wait_or_abort(&full[s], ph, err, abrt)) break;
+      // the stage's metadata has landed, so its previous MMAs (the last
+      // readers of these TMEM slots) are done
+      if (!wait_or_abort(&mload[s], ph, err, abrt)) break;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int mt128 = i0 / 128 + h;

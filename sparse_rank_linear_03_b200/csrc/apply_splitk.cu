@@ -20,9 +20,9 @@
 //                16 KB per instruction streams about twice as fast as 8 KB),
 //                the two X blocks [TP tokens × 64] (128-byte swizzle, tokens
 //                past T zero-filled) and 2 KB of TMEM-ordered metadata by
-//                bulk copy, spread to one 16-byte row per TMEM lane and
-//                copied into TMEM by tcgen05.cp; four tcgen05.mma.sp of
-//                K = 32 into a 128×TP fp32 accumulator in TMEM.  A CTA's range covers the end
+//                bulk copy, written into TMEM by tcgen05.st; four
+//                tcgen05.mma.sp of K = 32 into a 128×TP fp32 accumulator in
+//                TMEM.  A CTA's range covers the end
 //                of one tile and the start of the next (or a whole tile), so it
 //                keeps two accumulators and hands each finished tile segment to
 //                its epilogue warps.
@@ -34,12 +34,12 @@
 //   the result is deterministic.  That CTA resets the counter for the next
 //   call.  Nobody waits on anybody: no spin on another CTA.
 //
-// Warp roles (352 threads): warp 0 lane 0 issues the S copies and warp 10
-// lane 0 the X and metadata copies (two issuers, both arriving on the stage's
-// barrier, so their copy instructions overlap); warp 1 owns TMEM and lane 0
-// copies each unit's metadata into TMEM (tcgen05.cp, ordered before its MMAs)
-// and issues the MMAs; warps 2-5 lay the metadata out for that copy; warps
-// 6-9 run the epilogues (TMEM lane quarter = warp % 4).  Every wait is
+// Warp roles (384 threads): lane 0 of warp 0 issues the S copies, of warp 10
+// the X copies and of warp 11 the metadata copy (three issuers, all arriving
+// on the stage's barrier, so their copy instructions overlap); warp 1 owns
+// TMEM and lane 0 issues the MMAs once the unit's metadata is in TMEM; warps
+// 2-5 write the metadata into TMEM (tcgen05.st); warps 6-9 run the epilogues
+// (TMEM lane quarter = warp % 4).  Every wait is
 // bounded; a wait that gives up sets the error word, and the CTA still drains
 // its copies, takes part in the tile counters and frees TMEM.
 #include <cuda.h>
@@ -54,19 +54,24 @@
 namespace hsl {
 namespace {
 
-constexpr int SK_THREADS = 352;    // 11 warps (roles below)
+constexpr int SK_THREADS = 384;    // 12 warps (roles below)
 constexpr int SK_A = 128 * 128;     // compressed values of a unit: 128 rows × 128 bytes (2 K-blocks)
 constexpr int SK_M = 2 * 128 * 8;   // TMEM-ordered metadata of the unit's 2 K-blocks (compact)
-constexpr int SK_MX = 4 * 128 * 16; // the same, one 16-byte row per TMEM lane and MMA (4 MMAs)
 constexpr uint32_t SK_TMEM_COLS = 256;
 // accumulator b at TMEM column 64·b
 __host__ __device__ constexpr uint32_t sk_acc_col(int b) { return 64u * uint32_t(b); }
 
 // stages per token padding: the ring and z (TP rows × up to 256 fp32, staged
-// once for the U·z sums of the tiles the CTA finishes) share the shared memory
-__host__ __device__ constexpr int sk_stages(int tp) { return tp <= 16 ? 6 : tp <= 32 ? 5 : tp <= 48 ? 4 : 3; }
-__host__ __device__ constexpr int sk_stage_bytes(int tp) { return SK_A + 2 * tp * 128 + SK_M + SK_MX; }
+// once for the U·z sums of the tiles the CTA finishes) share 200 KB of shared
+// memory; at most 8 stages (their metadata slots fill TMEM columns [128, 256))
+__host__ __device__ constexpr int sk_stage_bytes(int tp) { return SK_A + 2 * tp * 128 + SK_M; }
 __host__ __device__ constexpr int sk_zbytes(int tp) { return tp * 256 * 4; }
+__host__ __device__ constexpr int sk_stages(int tp) {
+  return (200 * 1024 - sk_zbytes(tp)) / sk_stage_bytes(tp) < 8
+             ? (200 * 1024 - sk_zbytes(tp)) / sk_stage_bytes(tp)
+             : 8;
+}
+static_assert(sk_stages(16) == 8 && sk_stages(64) >= 3, "stage counts");
 __host__ __device__ constexpr int sk_smem(int tp) {
   return sk_stages(tp) * sk_stage_bytes(tp) + sk_zbytes(tp) + 1024 + 256;
 }
@@ -232,7 +237,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
   if (threadIdx.x == 0) {
     abort_flag = 0;
     for (int s = 0; s < ST; ++s) {
-      tc::mbar_init(&full[s], 2);  // the S issuer and the X/metadata issuer
+      tc::mbar_init(&full[s], 3);  // the S, X and metadata issuers
       tc::mbar_init(&mfull[s], 128);
       tc::mbar_init(&empty[s], 1);
     }
@@ -254,10 +259,9 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
   const uint32_t tmem = *tmem_slot;
   volatile int* abrt = &abort_flag;
 
-  if (warp == 0 || warp == 10) {
-    // warp 0: the unit's S values; warp 10: its two X blocks and metadata
+  if (warp == 0 || warp >= 10) {
+    // warp 0: the unit's S values; warp 10: its two X blocks; warp 11: its metadata
     if (lane == 0) {
-      const bool xs = warp == 10;
       const uint64_t keep = tc::make_policy_evict_last();
       const uint64_t stream = tc::make_policy_evict_first();
       // (tile, K-block pair) of the unit advanced incrementally: a single
@@ -269,14 +273,16 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
       for (; k < nu; ++k) {
         if (!wait_or_abort(&empty[s], ph ^ 1, a.err, abrt)) break;
         unsigned char* st = smem + s * STAGE;
-        if (!xs) {
+        if (warp == 0) {
           tc::mbar_expect_tx(&full[s], SK_A);
           tc::tma_load_2d_hint(st, &maps.sv, kp * 64, tile * 128, &full[s], stream);
-        } else {
-          tc::mbar_expect_tx(&full[s], 2 * B_BYTES + SK_M);
+        } else if (warp == 10) {
+          tc::mbar_expect_tx(&full[s], 2 * B_BYTES);
           tc::tma_load_2d_hint(st + SK_A, &maps.x, kp * 128, 0, &full[s], keep);
           tc::tma_load_2d_hint(st + SK_A + B_BYTES, &maps.x, kp * 128 + 64, 0, &full[s], keep);
+        } else {
           // the metadata of K-blocks 2·kp and 2·kp + 1 lie next to each other
+          tc::mbar_expect_tx(&full[s], SK_M);
           tc::bulk_load(st + SK_A + 2 * B_BYTES, a.meta + ((long long)tile * nkb + kp) * 256, SK_M,
                         &full[s]);
         }
@@ -284,7 +290,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
         if (++s == ST) { s = 0; ph ^= 1u; }
       }
       // drain: the stages of the last (up to ST) units this thread issued have landed
-      // (the other issuer's copies complete the same phases)
+      // (the other issuers' copies complete the same phases)
       for (int j = k > ST ? k - ST : 0; j < k; ++j) tc::mbar_wait(&full[j % ST], (j / ST) & 1, a.err);
     }
     __syncwarp();  // lanes 1-31 wait here for lane 0: the warp meets the CTA barrier converged
@@ -311,10 +317,6 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
         const unsigned char* st = smem + s * STAGE;
         const uint64_t ad = tc::desc_sw128(st);
         const uint32_t d = tmem + sk_acc_col(seg & 1);
-        // the unit's metadata into its TMEM slots, ahead of the MMAs that read it
-        const unsigned char* mx = st + SK_A + 2 * B_BYTES + SK_M;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) tc::tmem_cp_128x128b(tmem + sk_meta_col(s, i), tc::desc_rows16(mx + i * 2048));
         // MMA i: K-block i / 2 (its X block), 32 logical columns (i % 2) of it;
         // the values advance 32 bytes per MMA within their 128-byte rows
 #pragma unroll
@@ -329,24 +331,28 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
     }
     __syncwarp();  // lanes 1-31 wait here for lane 0: the warp meets the CTA barrier converged
   } else if (warp < 6) {
-    // metadata of each unit, expanded to one 16-byte row per TMEM lane and MMA
-    // (the layout tcgen05.cp copies); the MMA thread moves it into TMEM
+    // metadata of each unit into its TMEM slots (one 32-bit column per lane and
+    // MMA), so the MMA thread only waits for it.  A warp reaches TMEM lanes
+    // 32·(warp % 4) onwards.
     const int L = ((warp & 3) << 5) | lane;
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    int s = 0;
+    uint32_t ph = 0;
     for (long long u = u0; u < u1; ++u) {
-      const int k = int(u - u0), s = k % ST;
-      const uint32_t ph = (k / ST) & 1;
-      // the stage's bytes have landed, so the MMAs of its previous use are done
+      // the stage's bytes have landed, so the MMAs of its previous use (the
+      // last readers of these TMEM slots) are done
       if (!wait_or_abort(&full[s], ph, a.err, abrt)) break;
-      unsigned char* st = smem + s * STAGE;
-      unsigned char* mx = st + SK_A + 2 * B_BYTES + SK_M;
+      const unsigned char* st = smem + s * STAGE;
 #pragma unroll
       for (int kb = 0; kb < 2; ++kb) {
         const uint2 w = *reinterpret_cast<const uint2*>(st + SK_A + 2 * B_BYTES + kb * 1024 + L * 8);
-        *reinterpret_cast<uint4*>(mx + (2 * kb) * 2048 + L * 16) = make_uint4(w.x, 0u, 0u, 0u);
-        *reinterpret_cast<uint4*>(mx + (2 * kb + 1) * 2048 + L * 16) = make_uint4(w.y, 0u, 0u, 0u);
+        tc::tmem_st1(tmem + lane_base + sk_meta_col(s, 2 * kb), w.x);
+        tc::tmem_st1(tmem + lane_base + sk_meta_col(s, 2 * kb + 1), w.y);
       }
-      tc::fence_async_smem();
+      tc::tmem_st_wait();
+      tc::tc_fence_before();
       tc::mbar_arrive(&mfull[s]);
+      if (++s == ST) { s = 0; ph ^= 1u; }
     }
   } else {
     // epilogue: one tile segment at a time; TMEM lane = row of the tile
