@@ -927,6 +927,18 @@ bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dt, int esize, const voi
                   int box_rows, CUtensorMapSwizzle sw) {
   return make_map(map, dt, esize, base, rows, cols, row_stride_elems, box_cols, box_rows, sw);
 }
+bool make_tmap_kblocks(CUtensorMap* map, const void* base, int64_t rows, int64_t cols,
+                       int box_rows, int box_kblocks) {
+  const EncodeTiledFn fn = encode_fn();
+  if (!fn || cols % 64 != 0) return false;
+  cuuint64_t dims[3] = {64, cuuint64_t(rows), cuuint64_t(cols / 64)};
+  cuuint64_t strides[2] = {cuuint64_t(cols * 2), 128};
+  cuuint32_t box[3] = {64, cuuint32_t(box_rows), cuuint32_t(box_kblocks)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 bool tmap_available() { return encode_fn() != nullptr; }
 
 // Z workspace and Vt come from the handle (Vt built when the factors are packed).

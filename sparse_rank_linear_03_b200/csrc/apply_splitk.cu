@@ -18,8 +18,8 @@
 //                one 16 KB TMA of the 128×64 compressed values (128-byte
 //                swizzle; a copy instruction costs a near-fixed time, so
 //                16 KB per instruction streams about twice as fast as 8 KB),
-//                the two X blocks [TP tokens × 64] (128-byte swizzle, tokens
-//                past T zero-filled) and 2 KB of TMEM-ordered metadata by
+//                the two X blocks [TP tokens × 64] in one 3-D box (128-byte
+//                swizzle, tokens past T zero-filled) and 2 KB of TMEM-ordered metadata by
 //                bulk copy, written into TMEM by tcgen05.st; four
 //                tcgen05.mma.sp of K = 32 into a 128×TP fp32 accumulator in
 //                TMEM.  A CTA's range covers the end
@@ -80,7 +80,7 @@ __device__ __forceinline__ uint32_t sk_meta_col(int s, int i) { return 128u + 16
 
 struct SkMaps {
   CUtensorMap sv;  // S values [m][n/2]  box {64, 128} SW128 (two K-blocks of 64 columns)
-  CUtensorMap x;   // X [T][n]           box {64, TP}  SW128
+  CUtensorMap x;   // X [T][n] as [n/64][T][64], box {64, TP, 2} SW128 (both X blocks of a unit)
 };
 
 struct SkArgs {
@@ -277,9 +277,10 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
           tc::mbar_expect_tx(&full[s], SK_A);
           tc::tma_load_2d_hint(st, &maps.sv, kp * 64, tile * 128, &full[s], stream);
         } else if (warp == 10) {
+          // one copy for both X blocks: a copy instruction holds its issuing
+          // thread for a near-fixed time whatever its size
           tc::mbar_expect_tx(&full[s], 2 * B_BYTES);
-          tc::tma_load_2d_hint(st + SK_A, &maps.x, kp * 128, 0, &full[s], keep);
-          tc::tma_load_2d_hint(st + SK_A + B_BYTES, &maps.x, kp * 128 + 64, 0, &full[s], keep);
+          tc::tma_load_3d_hint(st + SK_A, &maps.x, 0, 0, kp * 2, &full[s], keep);
         } else {
           // the metadata of K-blocks 2·kp and 2·kp + 1 lie next to each other
           tc::mbar_expect_tx(&full[s], SK_M);
@@ -522,7 +523,7 @@ hsl_status launch_tp(Handle& h, const void* X, void* Y, int64_t T, cudaStream_t 
   const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   if (!make_tmap_2d(&maps.sv, BF, 2, h.nm_val.p, m, n / 2, n / 2, 64, 128,
                     CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_tmap_2d(&maps.x, BF, 2, X, T, n, n, 64, TP, CU_TENSOR_MAP_SWIZZLE_128B)) {
+      !make_tmap_kblocks(&maps.x, X, T, n, TP, 2)) {
     set_message("tensor map encoding failed");
     return HSL_ERR_CUDA;
   }

@@ -162,6 +162,12 @@ hsl_status rcm_order(int64_t m, int64_t n, const int32_t* row_ptr, const int32_t
 bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dt, int esize, const void* base,
                   int64_t rows, int64_t cols, int64_t row_stride_elems, int box_cols,
                   int box_rows, CUtensorMapSwizzle sw);
+// 3-D TMA map over a row-major bf16 [rows][cols] matrix (cols a multiple of 64)
+// seen as [cols / 64][rows][64]: a box {64, box_rows, box_kblocks} brings
+// box_kblocks 64-column K-blocks of box_rows rows, each K-block's rows
+// contiguous (128-byte swizzle), in one copy (apply_prefill.cu).
+bool make_tmap_kblocks(CUtensorMap* map, const void* base, int64_t rows, int64_t cols,
+                       int box_rows, int box_kblocks);
 bool tmap_available();
 
 }  // namespace hsl
