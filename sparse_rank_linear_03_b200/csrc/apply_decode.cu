@@ -1370,7 +1370,7 @@ hsl_status launch_chunk(ApplyPlan& plan, ApplyArgs a, int num_sms, cudaStream_t 
         plan.n_max <= 16 * 2048) {
       auto bk = k_apply_24_b1_tma;
       if (cudaError_t e =
-              cudaFuncSetAttribute(bk, cudaFuncAttributeMaxDynamicSharedMemorySize, lay.total))
+              allow_dyn_smem(reinterpret_cast<const void*>(bk), lay.total))
         return cuda_fail(e, "apply smem attribute");
       // one CTA per SM, all resident (cooperative launch): z is computed inside
       cudaLaunchConfig_t cfg = {};
@@ -1397,8 +1397,7 @@ hsl_status launch_chunk(ApplyPlan& plan, ApplyArgs a, int num_sms, cudaStream_t 
     auto zk = k_lowrank_z<T, BC>;
     // the apply CTAs start beside the z CTAs (programmatic dependent launch):
     // an SM configured for a small shared-memory carveout could not take one
-    cudaFuncSetAttribute(zk, cudaFuncAttributePreferredSharedMemoryCarveout,
-                         cudaSharedmemCarveoutMaxShared);
+    prefer_carveout(reinterpret_cast<const void*>(zk), cudaSharedmemCarveoutMaxShared);
     const int64_t zgrid = std::min<int64_t>((int64_t(plan.z_items) * 32 + kZThreads - 1) / kZThreads,
                                             int64_t(num_sms) * 8);
     zk<<<unsigned(zgrid), kZThreads, 0, s>>>(a);
@@ -1417,7 +1416,7 @@ hsl_status launch_chunk(ApplyPlan& plan, ApplyArgs a, int num_sms, cudaStream_t 
     auto ck = plan.idx_bits == 8    ? k_apply_csr_b1<T, 8>
               : plan.idx_bits == 32 ? k_apply_csr_b1<T, 32>
                                     : k_apply_csr_b1<T, 16>;
-    if (cudaError_t e = cudaFuncSetAttribute(ck, cudaFuncAttributeMaxDynamicSharedMemorySize, clay.total))
+    if (cudaError_t e = allow_dyn_smem(reinterpret_cast<const void*>(ck), clay.total))
       return cuda_fail(e, "apply smem attribute");
     cfg.blockDim = dim3(kCsrThreads);
     cfg.gridDim = dim3(unsigned(std::min<int64_t>(num_sms, row_cap)));
@@ -1436,7 +1435,7 @@ hsl_status launch_chunk(ApplyPlan& plan, ApplyArgs a, int num_sms, cudaStream_t 
             : plan.idx_bits == 8    ? (vec ? k_apply_csr_vec<T, 8> : k_apply_decode<T, BC, true, 8>)
             : plan.idx_bits == 32   ? (vec ? k_apply_csr_vec<T, 32> : k_apply_decode<T, BC, true, 32>)
                                     : (vec ? k_apply_csr_vec<T, 16> : k_apply_decode<T, BC, true, 16>);
-  if (cudaError_t e = cudaFuncSetAttribute(ak, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm)))
+  if (cudaError_t e = allow_dyn_smem(reinterpret_cast<const void*>(ak), int(sm)))
     return cuda_fail(e, "apply smem attribute");
   int occ = 0;
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, ak, kThreads, sm);

@@ -968,7 +968,7 @@ hsl_status prefill_z_run(Handle& h, const void* X, int64_t T, cudaStream_t s) {
     set_message("tensor map encoding failed");
     return HSL_ERR_CUDA;
   }
-  if (cudaError_t e = cudaFuncSetAttribute(k_prefill_z, cudaFuncAttributeMaxDynamicSharedMemorySize, Z_SMEM))
+  if (cudaError_t e = allow_dyn_smem(reinterpret_cast<const void*>(k_prefill_z), Z_SMEM))
     return cuda_fail(e, "prefill z smem attribute");
   k_prefill_z<<<unsigned((T + 127) / 128), 192, Z_SMEM, s>>>(
       zm, static_cast<__nv_bfloat16*>(h.zpre.p), int(h.n), int(T), r16,
@@ -1013,8 +1013,7 @@ hsl_status apply_prefill_run(Handle& h, const void* X, void* Y, int64_t T, cudaS
       return HSL_ERR_CUDA;
     }
     if (r16 > 0) {
-      if (cudaError_t e = cudaFuncSetAttribute(k_prefill_z,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, Z_SMEM))
+      if (cudaError_t e = allow_dyn_smem(reinterpret_cast<const void*>(k_prefill_z), Z_SMEM))
         return cuda_fail(e, "prefill z smem attribute");
       k_prefill_z<<<unsigned((T + 127) / 128), 192, Z_SMEM, s>>>(
           zm, static_cast<__nv_bfloat16*>(h.zpre.p), int(n), int(T), r16, err0);
@@ -1038,8 +1037,7 @@ hsl_status apply_prefill_run(Handle& h, const void* X, void* Y, int64_t T, cudaS
         set_message("tensor map encoding failed");
         return HSL_ERR_CUDA;
       }
-      if (cudaError_t e = cudaFuncSetAttribute(k_prefill_24sp2,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, P2_SMEM))
+      if (cudaError_t e = allow_dyn_smem(reinterpret_cast<const void*>(k_prefill_24sp2), P2_SMEM))
         return cuda_fail(e, "prefill smem attribute");
       const int64_t pairs = ((m + 511) / 512) * ((T + P2_BN - 1) / P2_BN);
       cudaLaunchConfig_t cfg = {};
@@ -1059,8 +1057,7 @@ hsl_status apply_prefill_run(Handle& h, const void* X, void* Y, int64_t T, cudaS
                                           r16, err0),
                        "pair prefill launch");
     }
-    if (cudaError_t e = cudaFuncSetAttribute(k_prefill_24sp,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, SP_SMEM))
+    if (cudaError_t e = allow_dyn_smem(reinterpret_cast<const void*>(k_prefill_24sp), SP_SMEM))
       return cuda_fail(e, "prefill smem attribute");
     const int64_t tiles = ((m + 255) / 256) * ((T + SP_BN - 1) / SP_BN);
     cudaLaunchConfig_t cfg = {};
@@ -1100,16 +1097,14 @@ hsl_status apply_prefill_run(Handle& h, const void* X, void* Y, int64_t T, cudaS
   }
   uint32_t* err = static_cast<uint32_t*>(h.err.p);
   if (r16 > 0) {
-    if (cudaError_t e = cudaFuncSetAttribute(k_prefill_z,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, Z_SMEM))
+    if (cudaError_t e = allow_dyn_smem(reinterpret_cast<const void*>(k_prefill_z), Z_SMEM))
       return cuda_fail(e, "prefill z smem attribute");
     k_prefill_z<<<unsigned((T + 127) / 128), 192, Z_SMEM, s>>>(
         maps, static_cast<__nv_bfloat16*>(h.zpre.p), int(n), int(T), r16, err);
     note_launch();
     if (hsl_status e = cuda_fail(cudaGetLastError(), "prefill z launch")) return e;
   }
-  if (cudaError_t e = cudaFuncSetAttribute(k_prefill_24, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           PREFILL_SMEM))
+  if (cudaError_t e = allow_dyn_smem(reinterpret_cast<const void*>(k_prefill_24), PREFILL_SMEM))
     return cuda_fail(e, "prefill smem attribute");
   const int64_t tiles = ((m + BM - 1) / BM) * ((T + BN - 1) / BN);
   cudaLaunchConfig_t cfg = {};

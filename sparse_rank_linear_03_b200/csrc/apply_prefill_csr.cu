@@ -278,8 +278,7 @@ hsl_status apply_prefill_csr_run(Handle& h, const void* X, void* Y, int64_t T, c
     set_message("tensor map encoding failed");
     return HSL_ERR_CUDA;
   }
-  if (cudaError_t e = cudaFuncSetAttribute(k_prefill_csr, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           PC_SMEM))
+  if (cudaError_t e = allow_dyn_smem(reinterpret_cast<const void*>(k_prefill_csr), PC_SMEM))
     return cuda_fail(e, "CSR prefill smem attribute");
   const int64_t tiles = ((m + PC_BM - 1) / PC_BM) * ((T + PC_BN - 1) / PC_BN);
   cudaLaunchConfig_t cfg = {};

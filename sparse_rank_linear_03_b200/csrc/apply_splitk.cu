@@ -486,7 +486,7 @@ hsl_status launch_tp(Handle& h, const void* X, void* Y, int64_t T, cudaStream_t 
   const long long units = (long long)tiles * nkb;
   auto kern = k_apply_24_splitk<TP>;
   const int smem = sk_smem(TP);
-  if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))
+  if (cudaError_t e = allow_dyn_smem(reinterpret_cast<const void*>(kern), smem))
     return cuda_fail(e, "split-K smem attribute");
   // one CTA per SM (its stage ring takes most of the shared memory)
   const int grid = int(std::min<long long>(h.num_sms, units));

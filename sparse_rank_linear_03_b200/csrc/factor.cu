@@ -719,7 +719,7 @@ hsl_status gemm_tall(const uint16_t* A, int nA, int64_t M, const uint16_t* B, in
   g.splits = splits;
   g.stages = stages;
   g.stage_bytes = stage_bytes;
-  if (cudaError_t e = cudaFuncSetAttribute(k_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))
+  if (cudaError_t e = allow_dyn_smem(reinterpret_cast<const void*>(k_gemm_tc), smem))
     return cuda_fail(e, "factor gemm smem attribute");
   k_gemm_tc<<<unsigned(mtiles * splits), GT_THREADS, smem, s>>>(maps, g);
   note_launch();

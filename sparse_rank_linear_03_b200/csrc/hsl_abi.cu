@@ -26,6 +26,49 @@ hsl_status cuda_fail(cudaError_t e, const char* what) {
   return HSL_ERR_CUDA;
 }
 
+namespace {
+std::mutex g_attr_mu;
+struct AttrEntry {
+  int device;
+  const void* func;
+  int kind;  // 0 dynamic shared memory, 1 carveout
+  int value;
+};
+std::vector<AttrEntry> g_attrs;  // a few dozen kernels at most
+
+// The entry for (device, func, kind), or nullptr.
+AttrEntry* find_attr(int device, const void* func, int kind) {
+  for (AttrEntry& e : g_attrs)
+    if (e.device == device && e.func == func && e.kind == kind) return &e;
+  return nullptr;
+}
+}  // namespace
+
+cudaError_t allow_dyn_smem(const void* func, int bytes) {
+  int dev = 0;
+  if (cudaError_t e = cudaGetDevice(&dev)) return e;
+  std::lock_guard<std::mutex> lk(g_attr_mu);
+  AttrEntry* a = find_attr(dev, func, 0);
+  if (a && a->value >= bytes) return cudaSuccess;
+  if (cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes))
+    return e;
+  if (a) a->value = bytes;
+  else g_attrs.push_back({dev, func, 0, bytes});
+  return cudaSuccess;
+}
+
+cudaError_t prefer_carveout(const void* func, int percent) {
+  int dev = 0;
+  if (cudaError_t e = cudaGetDevice(&dev)) return e;
+  std::lock_guard<std::mutex> lk(g_attr_mu);
+  if (AttrEntry* a = find_attr(dev, func, 1); a && a->value == percent) return cudaSuccess;
+  if (cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributePreferredSharedMemoryCarveout, percent))
+    return e;
+  if (AttrEntry* a = find_attr(dev, func, 1)) a->value = percent;
+  else g_attrs.push_back({dev, func, 1, percent});
+  return cudaSuccess;
+}
+
 // HSL_FAULT_INJECT=alloc makes every device allocation fail; =zwait makes the
 // batch-1 2:4 decode's wait for z give up (host-side failure testing; no
 // device fault is involved).

@@ -20,6 +20,14 @@ hsl_status cuda_fail(cudaError_t e, const char* what);
 // HSL_FAULT_INJECT=<what> (read on every call): host-side failure testing.
 bool fault_injected(const char* what);
 
+// cudaFuncSetAttribute(func, MaxDynamicSharedMemorySize, bytes) on the current
+// device unless an earlier call already allowed at least `bytes` (grow-only), so
+// a launch path makes the driver call once per kernel rather than per call.
+cudaError_t allow_dyn_smem(const void* func, int bytes);
+// cudaFuncSetAttribute(func, PreferredSharedMemoryCarveout, percent), once per
+// device and function.
+cudaError_t prefer_carveout(const void* func, int percent);
+
 // Grow-only device allocation.
 struct DevBuf {
   void* p = nullptr;

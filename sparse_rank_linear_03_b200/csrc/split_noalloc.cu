@@ -111,8 +111,7 @@ hsl_status run_noalloc(const KT* W, int64_t m, int64_t n, int64_t k, int32_t* ro
     const size_t smem = (size_t(1) << bits[p]) * sizeof(unsigned);
     if (bits[p] == 15) {
       auto kern = k_split_hist<KT, 15>;
-      if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               int(smem)))
+      if (cudaError_t e = allow_dyn_smem(reinterpret_cast<const void*>(kern), int(smem)))
         return cuda_fail(e, "split histogram smem attribute");
       kern<<<d.sms, 1024, smem, s>>>(W, count, st, shifts[p], hist, err, vec_ok ? 1 : 0, skip);
     } else if (bits[p] == 11) {
@@ -139,8 +138,7 @@ hsl_status run_noalloc(const KT* W, int64_t m, int64_t n, int64_t k, int32_t* ro
     const int64_t ntiles = (count + TE - 1) / TE;
     const size_t smem = size_t(kStages) * kTileBytesLB;
     auto kern = k_split_emit_tile<KT, SB, kTileBytesLB>;
-    if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             int(smem)))
+    if (cudaError_t e = allow_dyn_smem(reinterpret_cast<const void*>(kern), int(smem)))
       return cuda_fail(e, "split emit smem attribute");
     int occ = 0;
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kTileThreads, smem);

@@ -52,8 +52,7 @@ hsl_status emit_tiles(Handle& h, const KT* W, int64_t k, KT* R, SelState* st, un
   const int64_t ntiles = (count + TE - 1) / TE;
   const size_t smem = size_t(kStages) * TB;
   auto kern = k_split_emit_tile<KT, SB, TB>;
-  if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           int(smem)))
+  if (cudaError_t e = allow_dyn_smem(reinterpret_cast<const void*>(kern), int(smem)))
     return cuda_fail(e, "split emit smem attribute");
   int occ = 0;
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kTileThreads, smem);
@@ -143,11 +142,9 @@ hsl_status run_typed(Handle& h, const KT* W, int64_t k, KT* R, cudaStream_t s) {
     const uint32_t r_lo = uint32_t(std::min(S + 1, std::ceil(ks + margin)));
     if (cudaError_t e = cudaMemsetAsync(hist, 0, 2 * hist_bytes, s)) return cuda_fail(e, "memset");
     const int smem = int(hist_bytes);
-    if (cudaError_t e = cudaFuncSetAttribute(k_sample_hist,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem))
+    if (cudaError_t e = allow_dyn_smem(reinterpret_cast<const void*>(k_sample_hist), smem))
       return cuda_fail(e, "split sample smem attribute");
-    if (cudaError_t e = cudaFuncSetAttribute(k_count_bracket,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem))
+    if (cudaError_t e = allow_dyn_smem(reinterpret_cast<const void*>(k_count_bracket), smem))
       return cuda_fail(e, "split count smem attribute");
     const uint16_t* W16 = reinterpret_cast<const uint16_t*>(W);
     // per emit tile: count above the bracket, bracket histogram, counts, prefixes
@@ -181,8 +178,7 @@ hsl_status run_typed(Handle& h, const KT* W, int64_t k, KT* R, cudaStream_t s) {
     const size_t smem = (size_t(1) << bits[p]) * sizeof(unsigned);
     if (bits[p] == 15) {
       auto kern = k_split_hist<KT, 15>;
-      if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               int(smem)))
+      if (cudaError_t e = allow_dyn_smem(reinterpret_cast<const void*>(kern), int(smem)))
         return cuda_fail(e, "split histogram smem attribute");
       kern<<<hist_grid, 1024, smem, s>>>(W, count, st, shifts[p], hist, err, vec_ok ? 1 : 0, skip);
     } else if (bits[p] == 11) {
