@@ -175,7 +175,7 @@ __global__ void __launch_bounds__(192, 1)
       for (int s = 0; s < STAGES; ++s)
         if (issued[s]) tc::mbar_wait(&full[s], (issued[s] - 1) & 1, err);
     }
-    __syncwarp();  // lanes 1-31 wait here for lane 0: the warp meets the CTA barrier converged
+    __syncwarp();  // lanes 1-31 wait here for lane 0
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = tc::idesc_bf16(BM, BN);
@@ -196,7 +196,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       tc::mma_commit(accf);
     }
-    __syncwarp();  // lanes 1-31 wait here for lane 0: the warp meets the CTA barrier converged
+    __syncwarp();  // lanes 1-31 wait here for lane 0
   } else {
     // warps 2..5: expansion of S, then the epilogue.  Row = TMEM lane.
     const int row = ((warp & 3) << 5) | lane;
@@ -258,7 +258,7 @@ __global__ void __launch_bounds__(192, 1)
     }
   }
   tc::tc_fence_before();
-  __syncthreads();
+  tc::cta_sync();
   if (warp == 1) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, BN);
@@ -323,7 +323,7 @@ __global__ void __launch_bounds__(192, 1)
       for (int s = 0; s < ZSTAGES; ++s)
         if (issued[s]) tc::mbar_wait(&full[s], (issued[s] - 1) & 1, err);
     }
-    __syncwarp();  // lanes 1-31 wait here for lane 0: the warp meets the CTA barrier converged
+    __syncwarp();  // lanes 1-31 wait here for lane 0
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = tc::idesc_bf16(128, r16);
@@ -342,7 +342,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       tc::mma_commit(accf);
     }
-    __syncwarp();  // lanes 1-31 wait here for lane 0: the warp meets the CTA barrier converged
+    __syncwarp();  // lanes 1-31 wait here for lane 0
   } else {
     const int row = ((warp & 3) << 5) | lane;  // token within the tile
     if (tc::mbar_wait(accf, 0, err) && !*abrt) {
@@ -381,7 +381,7 @@ __global__ void __launch_bounds__(192, 1)
     }
   }
   tc::tc_fence_before();
-  __syncthreads();
+  tc::cta_sync();
   if (warp == 1) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, ncols);
@@ -426,7 +426,11 @@ struct SpMaps {
   CUtensorMap u;   // U [m][r_pad]   box {32, 256} SW64
   CUtensorMap z;   // Z hi [T][r16]  box {32, 192} SW64
   CUtensorMap zlo; // Z lo [T][r16]  box {32, 192} SW64
+  CUtensorMap y;   // Y [T][m]       box {256, 192}, no swizzle (the epilogue's tile store)
 };
+// bytes of the staged output tile: [SP_BN tokens][256 rows] bf16, in the ring
+constexpr int SP_Y_STAGE = SP_BN * 256 * 2;
+static_assert(SP_Y_STAGE <= SP_STAGES * SP_STAGE, "output tile staging");
 
 // Warps: 0 A copies, 1 MMA, 2-5 metadata into TMEM + epilogue, 6 B copies,
 // 7 metadata copies.  A copy instruction holds its issuing thread for a
@@ -435,7 +439,8 @@ struct SpMaps {
 constexpr int SP_THREADS = 256;
 __global__ void __launch_bounds__(SP_THREADS, 1)
     k_prefill_24sp(const __grid_constant__ SpMaps maps, const uint2* __restrict__ meta,
-                   __nv_bfloat16* __restrict__ Y, int m, int n, int T, int r16, uint32_t* err) {
+                   __nv_bfloat16* __restrict__ Y, int m, int n, int T, int r16, int ystore,
+                   uint32_t* err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -533,7 +538,7 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
       for (int j = kb > SP_STAGES ? kb - SP_STAGES : 0; j < kb; ++j)
         tc::mbar_wait(&landed[j % SP_STAGES], (j / SP_STAGES) & 1, err);
     }
-    __syncwarp();  // lanes 1-31 wait here for lane 0: the warp meets the CTA barrier converged
+    __syncwarp();  // lanes 1-31 wait here for lane 0
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc_sp = tc::idesc_bf16(128, SP_BN) | (1u << 2);
@@ -572,7 +577,7 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
       }
       tc::mma_commit(accf);
     }
-    __syncwarp();  // lanes 1-31 wait here for lane 0: the warp meets the CTA barrier converged
+    __syncwarp();  // lanes 1-31 wait here for lane 0
   } else if (warp < 6) {
     // warps 2..5: metadata into TMEM, then the epilogue.  TMEM lane = L.
     const int L = ((warp & 3) << 5) | lane;
@@ -597,18 +602,43 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
     }
     if (tc::mbar_wait(accf, 0, err) && !*abrt) {
       tc::tc_fence_after();
+      if (ystore) {
+        // The tile, rounded to bf16, into shared memory as [token][row] (the ring
+        // is idle: every copy was consumed before the last MMAs), then one tiled
+        // store; rows past m and tokens past T are not written.  Scattered 2-byte
+        // stores straight from registers took ~13 µs per tile.
+        __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(smem);
 #pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        const int i = i0 + 128 * h + L;
+        for (int h = 0; h < 2; ++h) {
 #pragma unroll 1
-        for (int c0 = 0; c0 < SP_BN; c0 += 32) {
-          float v[32];
-          tc::tmem_ld32(tmem + lane_base + (h ? SP_ACC1_COL : 0u) + c0, v);
-          if (i < m) {
+          for (int c0 = 0; c0 < SP_BN; c0 += 32) {
+            float v[32];
+            tc::tmem_ld32(tmem + lane_base + (h ? SP_ACC1_COL : 0u) + c0, v);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int t = t0 + c0 + j;
-              if (c0 + j < SP_BN && t < T) __stcs(Y + int64_t(t) * m + i, __float2bfloat16_rn(v[j]));
+            for (int j = 0; j < 32; ++j) stg[(c0 + j) * 256 + 128 * h + L] = __float2bfloat16_rn(v[j]);
+          }
+        }
+        tc::fence_async_smem();
+        asm volatile("barrier.sync 1, 128;" ::: "memory");  // the four epilogue warps
+        if (L == 0) {
+          tc::tma_store_2d(&maps.y, stg, i0, t0);
+          tc::bulk_commit();
+          tc::bulk_wait_read_all();  // the CTA's shared memory is read before it ends
+        }
+      } else {
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          const int i = i0 + 128 * h + L;
+#pragma unroll 1
+          for (int c0 = 0; c0 < SP_BN; c0 += 32) {
+            float v[32];
+            tc::tmem_ld32(tmem + lane_base + (h ? SP_ACC1_COL : 0u) + c0, v);
+            if (i < m) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                const int t = t0 + c0 + j;
+                if (c0 + j < SP_BN && t < T) __stcs(Y + int64_t(t) * m + i, __float2bfloat16_rn(v[j]));
+              }
             }
           }
         }
@@ -618,7 +648,7 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
     }
   }
   tc::tc_fence_before();
-  __syncthreads();
+  tc::cta_sync();
   if (warp == 1) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, 512);
@@ -760,7 +790,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         }
       }
     }
-    __syncwarp();  // lanes 1-31 wait here for lane 0: the warp meets the CTA barrier converged
+    __syncwarp();  // lanes 1-31 wait here for lane 0
   } else if (warp == 1) {
     if (lane == 0 && leader) {
       const uint32_t idesc_sp = tc::idesc_bf16(256, P2_BN) | (1u << 2);
@@ -800,7 +830,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       }
       tc::mma_commit_pair(accf);
     }
-    __syncwarp();  // lanes 1-31 wait here for lane 0: the warp meets the CTA barrier converged
+    __syncwarp();  // lanes 1-31 wait here for lane 0
   } else {
     // warps 2..5: metadata into TMEM ahead of the MMAs, then the epilogue
     const int L = ((warp & 3) << 5) | lane;
@@ -847,7 +877,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         tc::tc_fence_before();
         // the four warps' stores are done: one arrival per CTA (cluster-scope
         // release), not one per thread
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        asm volatile("barrier.sync 1, 128;" ::: "memory");
         if (L == 0) tc::mbar_arrive_cluster(mready0 + uint32_t(set) * 8u);
         ring[d][0] = load_meta(kb + D, 0);
         ring[d][1] = load_meta(kb + D, 1);
@@ -876,7 +906,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     }
   }
   tc::tc_fence_before();
-  tc::cluster_sync();  // the pair is done with its TMEM and barriers
+  tc::cluster_sync_any();  // the pair is done with its TMEM and barriers
   if (warp == 1) {
     tc::tc_fence_after();
     tc::tmem_dealloc2(tmem, 512);
@@ -998,6 +1028,10 @@ hsl_status apply_prefill_run(Handle& h, const void* X, void* Y, int64_t T, cudaS
     bool ok = make_map(&sm.x, BFs, 2, X, T, n, n, 64, SP_BN, CU_TENSOR_MAP_SWIZZLE_128B) &&
               make_map(&sm.sv, BFs, 2, h.nm_val.p, m, n / 2, n / 2, 32, 256,
                        CU_TENSOR_MAP_SWIZZLE_64B);
+    // the epilogue's tiled store needs 16-byte row pitch and base
+    const int ystore = (m % 8 == 0 && reinterpret_cast<uintptr_t>(Y) % 16 == 0) ? 1 : 0;
+    if (ok && ystore)
+      ok = make_map(&sm.y, BFs, 2, Y, T, m, m, 256, SP_BN, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (ok && r16 > 0)
       ok = make_map(&sm.u, BFs, 2, h.U.p, m, h.r_pad, h.r_pad, 32, 256, CU_TENSOR_MAP_SWIZZLE_64B) &&
            make_map(&sm.z, BFs, 2, h.zpre.p, T, r16, r16, 32, SP_BN, CU_TENSOR_MAP_SWIZZLE_64B) &&
@@ -1074,7 +1108,7 @@ hsl_status apply_prefill_run(Handle& h, const void* X, void* Y, int64_t T, cudaS
     return cuda_fail(cudaLaunchKernelEx(&cfg, k_prefill_24sp, sm,
                                         static_cast<const uint2*>(h.pmeta_tc.p),
                                         static_cast<__nv_bfloat16*>(Y), int(m), int(n), int(T),
-                                        r16, err0),
+                                        r16, ystore, err0),
                      "sparse prefill launch");
   }
   PrefillMaps maps;

@@ -128,7 +128,7 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
 }
 
 // named barrier over the four epilogue warps
-__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void epi_sync() { asm volatile("barrier.sync 1, 128;" ::: "memory"); }
 
 // ---- z = Vᵀ x ------------------------------------------------------------------
 // Work items (row c of Vt, 8 tokens) are cut into pieces of 256 columns, a warp
@@ -294,7 +294,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
       // (the other issuers' copies complete the same phases)
       for (int j = k > ST ? k - ST : 0; j < k; ++j) tc::mbar_wait(&full[j % ST], (j / ST) & 1, a.err);
     }
-    __syncwarp();  // lanes 1-31 wait here for lane 0: the warp meets the CTA barrier converged
+    __syncwarp();  // lanes 1-31 wait here for lane 0
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc_sp = tc::idesc_bf16(128, TP) | (1u << 2);
@@ -330,7 +330,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
         if (last) tc::mma_commit(&accfull[seg & 1]);
       }
     }
-    __syncwarp();  // lanes 1-31 wait here for lane 0: the warp meets the CTA barrier converged
+    __syncwarp();  // lanes 1-31 wait here for lane 0
   } else if (warp < 6) {
     // metadata of each unit into its TMEM slots (one 32-bit column per lane and
     // MMA), so the MMA thread only waits for it.  A warp reaches TMEM lanes
@@ -471,7 +471,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
     }
   }
   tc::tc_fence_before();
-  __syncthreads();
+  tc::cta_sync();
   if (warp == 1) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, SK_TMEM_COLS);

@@ -208,7 +208,7 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
       for (int s = 0; s < ST; ++s)
         if (issued[s]) tc::mbar_wait(&full[s], (issued[s] - 1) & 1, g.err);
     }
-    __syncwarp();  // lanes 1-31 wait here for lane 0: the warp meets the CTA barrier converged
+    __syncwarp();  // lanes 1-31 wait here for lane 0
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = tc::idesc_bf16(128, g.BH);
@@ -230,7 +230,7 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
       }
       tc::mma_commit(accf);
     }
-    __syncwarp();  // lanes 1-31 wait here for lane 0: the warp meets the CTA barrier converged
+    __syncwarp();  // lanes 1-31 wait here for lane 0
   } else {
     // epilogue: TMEM lane = row of the tile
     const int q = warp & 3;
@@ -261,7 +261,7 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
     }
   }
   tc::tc_fence_before();
-  __syncthreads();
+  tc::cta_sync();
   if (warp == 1) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, ncols);

@@ -87,6 +87,16 @@ __device__ __forceinline__ void bulk_wait_read_all() {
 __device__ __forceinline__ void bulk_wait_read_but_one() {
   asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
+// Tiled store shared → global through a tensor map (coordinates x, y), tracked as
+// a bulk group of the issuing thread; parts of the box outside the tensor are
+// not written.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int32_t x,
+                                             int32_t y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(smem_u32(src))
+               : "memory");
+}
 // The issuing thread's bulk stores are complete.
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
@@ -285,6 +295,16 @@ __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
   return r;
+}
+// CTA-wide barrier for the end of kernels whose warps arrive from different role
+// branches (lane 0 of a warp in a loop, its other lanes waiting).  The
+// non-aligned form counts every thread; bar.sync (what __syncthreads emits) is
+// the aligned form, undefined for a warp that is not converged, and was measured
+// letting thread 0 through before the epilogue warps had arrived.
+__device__ __forceinline__ void cta_sync() { asm volatile("barrier.sync 0;" ::: "memory"); }
+// The same across a cluster (non-aligned arrive and wait).
+__device__ __forceinline__ void cluster_sync_any() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
 }
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" :::
