@@ -51,7 +51,9 @@ struct PcMaps {
   CUtensorMap u;    // U [m][r_pad]     box {64, 128} SW128
   CUtensorMap zhi;  // Z hi [T][r16]    box {64, 256} SW128
   CUtensorMap zlo;  // Z lo [T][r16]    box {64, 256} SW128
+  CUtensorMap y;    // Y [T][m]         box {256, 256}, no swizzle (the epilogue's tile store)
 };
+static_assert(PC_BN * PC_BM * 2 <= PC_STAGES * PC_STAGE, "output tile staging");
 
 __device__ __forceinline__ bool pc_wait(uint64_t* bar, uint32_t parity, uint32_t* err,
                                         volatile int* abort_flag) {
@@ -64,7 +66,8 @@ __device__ __forceinline__ bool pc_wait(uint64_t* bar, uint32_t parity, uint32_t
 __global__ void __launch_bounds__(PC_THREADS, 1)
     k_prefill_csr(const __grid_constant__ PcMaps maps, const int32_t* __restrict__ prow,
                   const uint16_t* __restrict__ pcol, const uint16_t* __restrict__ pval,
-                  __nv_bfloat16* __restrict__ Y, int m, int n, int T, int r16, uint32_t* err) {
+                  __nv_bfloat16* __restrict__ Y, int m, int n, int T, int r16, int ystore,
+                  uint32_t* err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -136,7 +139,7 @@ __global__ void __launch_bounds__(PC_THREADS, 1)
       for (int s = 0; s < PC_STAGES; ++s)
         if (issued[s]) tc::mbar_wait(&full[s], (issued[s] - 1) & 1, err);
     }
-    __syncwarp();  // lanes 1-31 wait here for lane 0: the warp meets the CTA barrier converged
+    __syncwarp();  // lanes 1-31 wait here for lane 0
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = tc::idesc_bf16(128, PC_BN);
@@ -160,7 +163,7 @@ __global__ void __launch_bounds__(PC_THREADS, 1)
       }
       tc::mma_commit(accf);
     }
-    __syncwarp();  // lanes 1-31 wait here for lane 0: the warp meets the CTA barrier converged
+    __syncwarp();  // lanes 1-31 wait here for lane 0
   } else {
     // decompression: thread R owns row i0 + R of the tile; rows 0..127 belong to
     // the first accumulator, 128..255 to the second (TMEM lane R mod 128; warp
@@ -228,15 +231,35 @@ __global__ void __launch_bounds__(PC_THREADS, 1)
     if (tc::mbar_wait(accf, 0, err) && !*abrt) {
       tc::tc_fence_after();
       const uint32_t tbase = tmem + (uint32_t((warp & 3) * 32) << 16) + (half ? PC_ACC1 : 0u);
+      if (ystore) {
+        // the rounded tile into the idle ring as [token][row], then one tiled
+        // store (rows past m and tokens past T are not written)
+        __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(smem);
 #pragma unroll 1
-      for (int c0 = 0; c0 < PC_BN; c0 += 32) {
-        float v[32];
-        tc::tmem_ld32(tbase + c0, v);
-        if (i < m) {
+        for (int c0 = 0; c0 < PC_BN; c0 += 32) {
+          float v[32];
+          tc::tmem_ld32(tbase + c0, v);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int t = t0 + c0 + j;
-            if (t < T) __stcs(Y + int64_t(t) * m + i, __float2bfloat16_rn(v[j]));
+          for (int j = 0; j < 32; ++j) stg[(c0 + j) * PC_BM + R] = __float2bfloat16_rn(v[j]);
+        }
+        tc::fence_async_smem();
+        asm volatile("barrier.sync 1, 256;" ::: "memory");  // the eight epilogue warps
+        if (R == 0) {
+          tc::tma_store_2d(&maps.y, stg, i0, t0);
+          tc::bulk_commit();
+          tc::bulk_wait_read_all();  // the CTA's shared memory is read before it ends
+        }
+      } else {
+#pragma unroll 1
+        for (int c0 = 0; c0 < PC_BN; c0 += 32) {
+          float v[32];
+          tc::tmem_ld32(tbase + c0, v);
+          if (i < m) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int t = t0 + c0 + j;
+              if (t < T) __stcs(Y + int64_t(t) * m + i, __float2bfloat16_rn(v[j]));
+            }
           }
         }
       }
@@ -245,7 +268,7 @@ __global__ void __launch_bounds__(PC_THREADS, 1)
     }
   }
   tc::tc_fence_before();
-  __syncthreads();
+  tc::cta_sync();
   if (warp == 1) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, 512);
@@ -268,6 +291,10 @@ hsl_status apply_prefill_csr_run(Handle& h, const void* X, void* Y, int64_t T, c
   const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
   bool ok = make_tmap_2d(&maps.x, BF, 2, X, T, n, n, 64, PC_BN, SW);
+  // the epilogue's tiled store needs 16-byte row pitch and base
+  const int ystore = (m % 8 == 0 && reinterpret_cast<uintptr_t>(Y) % 16 == 0) ? 1 : 0;
+  if (ok && ystore)
+    ok = make_tmap_2d(&maps.y, BF, 2, Y, T, m, m, PC_BM, PC_BN, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (ok && r16 > 0) {
     const __nv_bfloat16* z = static_cast<const __nv_bfloat16*>(h.zpre.p);
     ok = make_tmap_2d(&maps.u, BF, 2, h.U.p, m, h.r_pad, h.r_pad, 64, 128, SW) &&
@@ -296,7 +323,7 @@ hsl_status apply_prefill_csr_run(Handle& h, const void* X, void* Y, int64_t T, c
                                       static_cast<const uint16_t*>(h.pcol.p),
                                       static_cast<const uint16_t*>(h.pval.p),
                                       static_cast<__nv_bfloat16*>(Y), int(m), int(n), int(T), r16,
-                                      static_cast<uint32_t*>(h.err.p)),
+                                      ystore, static_cast<uint32_t*>(h.err.p)),
                    "CSR prefill launch");
 }
 
