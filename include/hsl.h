@@ -129,7 +129,8 @@ hsl_status hsl_split_topk(hsl_handle h, const void* W, hsl_dtype w_dtype,
  * HSL_ERR_UNSUPPORTED.  The first call on a device looks the array up with
  * that device current (make it before any stream capture).  All calls share
  * the array, so calls that can overlap on the GPU race: serialise them on one
- * stream.  Asynchronous on s, like the other entry points. */
+ * stream.  Asynchronous on s, like the other entry points.
+ * What it computes: [HSS] §Two-stage compression, Stage 1 (as hsl_split_topk). */
 hsl_status hsl_split_topk_noalloc(const void* W, int64_t m, int64_t n, hsl_dtype w_dtype,
                                   double frac, int32_t* row_ptr, int32_t* col, void* val,
                                   hsl_dtype val_dtype, void* residual, uint32_t* status,
@@ -223,7 +224,8 @@ hsl_status hsl_group_apply(hsl_group g, const void* const* X, void* const* Y, in
                            hsl_stream s);
 
 /* Release the group (synchronises its device first).  NULL is a no-op.
- * Same passage as hsl_group_create. */
+ * [HSS] §Implementation and operational patterns (the layers held for the
+ * forward pass), as hsl_group_create. */
 hsl_status hsl_group_destroy(hsl_group g);
 
 /* Stage 2 on the GPU: the rank-r factors of the residual R (device, m×n of
@@ -258,7 +260,8 @@ hsl_status hsl_factor(hsl_handle h, const void* R, hsl_dtype r_dtype, const floa
  * and bottom-right blocks of the 2×2 partition split at row ⌊m/2⌋ and column
  * ⌊n/2⌋; an all-zero W gives 0, a NaN in W gives NaN.  Sums in fp64 in a fixed
  * order (deterministic).  Writes *rho (host) and synchronises s.  Allocates a
- * small workspace for the call and frees it. */
+ * small workspace for the call and frees it.
+ * [HSS] §Permutation and hierarchical alignment (the ρ equation). */
 hsl_status hsl_concentration(const void* W, int64_t m, int64_t n, hsl_dtype dtype, double* rho,
                              hsl_stream s);
 
@@ -269,13 +272,15 @@ hsl_status hsl_concentration(const void* W, int64_t m, int64_t n, hsl_dtype dtyp
  * index first), visit breadth first taking neighbours by increasing degree
  * (same ties), reverse the whole order.  row_order[k] / col_order[k] (host,
  * m and n int32) receive the original row / column placed k-th.  Runs on the
- * host (a one-off graph step); HSL_ERR_INVALID_ARG for a bad pattern. */
+ * host (a one-off graph step); HSL_ERR_INVALID_ARG for a bad pattern.
+ * [HSS] §Permutation and hierarchical alignment (reverse Cuthill–McKee). */
 hsl_status hsl_rcm_order(int64_t m, int64_t n, const int32_t* row_ptr, const int32_t* col,
                          int32_t* row_order, int32_t* col_order);
 
 /* out[k][l] = W[row_order[k]][col_order[l]] (device arrays; bit copies).  The
  * orders are copied to the host and checked to be permutations first
- * (HSL_ERR_INVALID_ARG otherwise), which synchronises s. */
+ * (HSL_ERR_INVALID_ARG otherwise), which synchronises s.
+ * [HSS] §Permutation and hierarchical alignment (W permuted before the split). */
 hsl_status hsl_permute(const void* W, int64_t m, int64_t n, hsl_dtype dtype,
                        const int32_t* row_order, const int32_t* col_order, void* out,
                        hsl_stream s);
@@ -285,7 +290,8 @@ hsl_status hsl_permute(const void* W, int64_t m, int64_t n, hsl_dtype dtype,
  * layer's output: x' = x[col_order], y' = Ŵ' x', y[row_order[k]] = y'[k].
  * Device arrays, copied into the handle after a host-side permutation check
  * (synchronises s).  NULL for both clears it.  Groups do not take permuted
- * layers. */
+ * layers.  [HSS] §Permutation and hierarchical alignment (outputs in the
+ * original order). */
 hsl_status hsl_set_permutation(hsl_handle h, const int32_t* row_order, const int32_t* col_order,
                                hsl_stream s);
 
@@ -301,8 +307,9 @@ hsl_status hsl_check(hsl_handle h, hsl_stream s);
  * detection-and-fallback passage). */
 const char* hsl_status_str(hsl_status st);
 
-/* Detail of the last failing call on this thread ("" if none).  Same
- * passage as hsl_status_str. */
+/* Detail of the last failing call on this thread ("" if none).
+ * [HSS] §Risks and mitigations, risk 1 (detection of a misbehaving layer),
+ * as hsl_status_str. */
 const char* hsl_last_message(void);
 
 /* Number of kernels libhsl has launched in this process (all devices).
