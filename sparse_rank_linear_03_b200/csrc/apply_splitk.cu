@@ -35,11 +35,12 @@
 //   call.  Nobody waits on anybody: no spin on another CTA.
 //
 // Warp roles (384 threads): lane 0 of warp 0 issues the S copies, of warp 10
-// the X copies and of warp 11 the metadata copy (three issuers, all arriving
-// on the stage's barrier, so their copy instructions overlap); warp 1 owns
-// TMEM and lane 0 issues the MMAs once the unit's metadata is in TMEM; warps
-// 2-5 write the metadata into TMEM (tcgen05.st); warps 6-9 run the epilogues
-// (TMEM lane quarter = warp % 4).  Every wait is
+// the X copies and of warp 11 the metadata copy (three issuers, so their copy
+// instructions overlap); warps 2-5 write each unit's metadata into TMEM
+// (tcgen05.st) once it has landed; the S and X copies and those 128 threads
+// complete the unit's one `full` barrier, on which lane 0 of warp 1 (which owns
+// TMEM) waits before the unit's MMAs; warps 6-9 run the epilogues (TMEM lane
+// quarter = warp % 4).  Every wait is
 // bounded; a wait that gives up sets the error word, and the CTA still drains
 // its copies, takes part in the tile counters and frees TMEM.
 #include <cuda.h>
@@ -220,8 +221,8 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* zs = reinterpret_cast<float*>(smem + ST * STAGE);  // [TP][r_pad], staged once
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * STAGE + sk_zbytes(TP));
-  uint64_t* mfull = full + ST;
-  uint64_t* empty = mfull + ST;
+  uint64_t* mload = full + ST;  // the unit's metadata has landed
+  uint64_t* empty = mload + ST;
   uint64_t* accfull = empty + ST;   // [2]
   uint64_t* accempty = accfull + 2; // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accempty + 2);
@@ -237,8 +238,11 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
   if (threadIdx.x == 0) {
     abort_flag = 0;
     for (int s = 0; s < ST; ++s) {
-      tc::mbar_init(&full[s], 3);  // the S, X and metadata issuers
-      tc::mbar_init(&mfull[s], 128);
+      // the S and X issuers, and the 128 threads that put the unit's metadata
+      // into TMEM: the MMA thread waits on this one barrier per unit (a wait on a
+      // completed phase costs that thread a few hundred cycles after MMA issue)
+      tc::mbar_init(&full[s], 2 + 128);
+      tc::mbar_init(&mload[s], 1);
       tc::mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -283,16 +287,18 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
           tc::tma_load_3d_hint(st + SK_A, &maps.x, 0, 0, kp * 2, &full[s], keep);
         } else {
           // the metadata of K-blocks 2·kp and 2·kp + 1 lie next to each other
-          tc::mbar_expect_tx(&full[s], SK_M);
+          tc::mbar_expect_tx(&mload[s], SK_M);
           tc::bulk_load(st + SK_A + 2 * B_BYTES, a.meta + ((long long)tile * nkb + kp) * 256, SK_M,
-                        &full[s]);
+                        &mload[s]);
         }
         if (++kp == nkb) { kp = 0; ++tile; }
         if (++s == ST) { s = 0; ph ^= 1u; }
       }
       // drain: the stages of the last (up to ST) units this thread issued have landed
-      // (the other issuers' copies complete the same phases)
-      for (int j = k > ST ? k - ST : 0; j < k; ++j) tc::mbar_wait(&full[j % ST], (j / ST) & 1, a.err);
+      // (the S and X copies complete the same phases of `full`; the metadata
+      // completes on `mload`)
+      uint64_t* landed = warp == 11 ? mload : full;
+      for (int j = k > ST ? k - ST : 0; j < k; ++j) tc::mbar_wait(&landed[j % ST], (j / ST) & 1, a.err);
     }
     __syncwarp();  // lanes 1-31 wait here for lane 0
   } else if (warp == 1) {
@@ -313,7 +319,6 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
             break;
         }
         if (!wait_or_abort(&full[s], ph, a.err, abrt)) break;
-        if (!wait_or_abort(&mfull[s], ph, a.err, abrt)) break;
         tc::tc_fence_after();
         const unsigned char* st = smem + s * STAGE;
         const uint64_t ad = tc::desc_sw128(st);
@@ -333,16 +338,16 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
     __syncwarp();  // lanes 1-31 wait here for lane 0
   } else if (warp < 6) {
     // metadata of each unit into its TMEM slots (one 32-bit column per lane and
-    // MMA), so the MMA thread only waits for it.  A warp reaches TMEM lanes
-    // 32·(warp % 4) onwards.
+    // MMA), then an arrival on the unit's `full` barrier, so the MMA thread
+    // waits on that one barrier.  A warp reaches TMEM lanes 32·(warp % 4) onwards.
     const int L = ((warp & 3) << 5) | lane;
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     int s = 0;
     uint32_t ph = 0;
     for (long long u = u0; u < u1; ++u) {
-      // the stage's bytes have landed, so the MMAs of its previous use (the
-      // last readers of these TMEM slots) are done
-      if (!wait_or_abort(&full[s], ph, a.err, abrt)) break;
+      // the unit's metadata has landed, so the MMAs of its stage's previous use
+      // (the last readers of these TMEM slots) are done
+      if (!wait_or_abort(&mload[s], ph, a.err, abrt)) break;
       const unsigned char* st = smem + s * STAGE;
 #pragma unroll
       for (int kb = 0; kb < 2; ++kb) {
@@ -352,7 +357,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
       }
       tc::tmem_st_wait();
       tc::tc_fence_before();
-      tc::mbar_arrive(&mfull[s]);
+      tc::mbar_arrive(&full[s]);
       if (++s == ST) { s = 0; ph ^= 1u; }
     }
   } else {
