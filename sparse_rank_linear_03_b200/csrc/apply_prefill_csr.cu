@@ -72,8 +72,7 @@ __global__ void __launch_bounds__(PC_THREADS, 1)
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + PC_STAGES * PC_STAGE);
-  uint64_t* dense = full + PC_STAGES;
-  uint64_t* empty = dense + PC_STAGES;
+  uint64_t* empty = full + PC_STAGES;
   uint64_t* accf = empty + PC_STAGES;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
   __shared__ int abort_flag;
@@ -89,8 +88,10 @@ __global__ void __launch_bounds__(PC_THREADS, 1)
   if (threadIdx.x == 0) {
     abort_flag = 0;
     for (int s = 0; s < PC_STAGES; ++s) {
-      tc::mbar_init(&full[s], 1);
-      tc::mbar_init(&dense[s], 256);
+      // the copy issuer and the 256 threads that decompress the stage's A tile
+      // (none for the low-rank K-blocks, but they arrive all the same): the MMA
+      // thread waits on this one barrier per K-block
+      tc::mbar_init(&full[s], 1 + 256);
       tc::mbar_init(&empty[s], 1);
     }
     tc::mbar_init(accf, 1);
@@ -147,7 +148,6 @@ __global__ void __launch_bounds__(PC_THREADS, 1)
         const int s = kb % PC_STAGES;
         const uint32_t ph = (kb / PC_STAGES) & 1;
         if (!pc_wait(&full[s], ph, err, abrt)) break;
-        if (kb < nkS && !pc_wait(&dense[s], ph, err, abrt)) break;
         tc::tc_fence_after();
         unsigned char* a = smem + s * PC_STAGE;
         const uint64_t bd = tc::desc_sw128(a + PC_A);
@@ -188,11 +188,16 @@ __global__ void __launch_bounds__(PC_THREADS, 1)
       nv = ld_stream16(pval + e + 8);
     }
     int pos = 0;  // next unread entry of the current 8
-    for (int kb = 0; kb < nkS; ++kb) {
+    for (int kb = 0; kb < nk; ++kb) {
       const int s = kb % PC_STAGES;
       const uint32_t ph = (kb / PC_STAGES) & 1;
-      // the MMAs of this stage's previous use have read its A tile
+      // the MMAs of this stage's previous use have read its A tile (and so this
+      // arrival counts towards this K-block's phase)
       if (!pc_wait(&empty[s], ph ^ 1, err, abrt)) break;
+      if (kb >= nkS) {  // a low-rank K-block: its A tile (U) comes by copy
+        tc::mbar_arrive(&full[s]);
+        continue;
+      }
       unsigned char* arow = smem + s * PC_STAGE + half * PC_AH + (L >> 3) * 1024 + (L & 7) * 128;
 #pragma unroll
       for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(arow + c * 16) = make_uint4(0, 0, 0, 0);
@@ -225,7 +230,7 @@ __global__ void __launch_bounds__(PC_THREADS, 1)
         }
       }
       tc::fence_async_smem();
-      tc::mbar_arrive(&dense[s]);
+      tc::mbar_arrive(&full[s]);
     }
     // epilogue
     if (tc::mbar_wait(accf, 0, err) && !*abrt) {
