@@ -8,7 +8,7 @@
 //                  K = n, operands by TMA (128-byte swizzle), fp32 accumulator
 //                  in TMEM, bf16 epilogue.  Triggers the dependent launch at
 //                  its start.
-//   k_prefill_24sp the default: Yᵀ tile [256 rows of W × 192 tokens], two
+//   k_prefill_24sp the default: Yᵀ tile [256 rows of W × 224 tokens], two
 //                  128-row TMEM accumulators sharing every X tile; the 2:4
 //                  part runs on the sparse MMA (tcgen05.mma.sp, compressed
 //                  values straight from TMA, metadata in TMEM), the low-rank
@@ -22,11 +22,14 @@
 //   before the first Z tile, so the S·Xᵀ part overlaps it; the epilogue reads
 //   TMEM (tcgen05.ld), rounds to bf16 and stores Y[t][i] with streaming stores.
 //
-// Why 256×192 tiles: with a 2:4 sparse MMA the tensor work per byte of X halves,
+// Why 256×224 tiles: with a 2:4 sparse MMA the tensor work per byte of X halves,
 // so the X traffic per flop decides whether L2 can feed the MMAs; sharing each
 // X tile across 256 rows of W lowers the bytes per flop about 1.6× against a
-// 128×256 tile.  TMEM holds 2×192 accumulator columns plus 4-column-aligned
-// metadata slots (the sparse MMA requires that alignment).
+// 128×256 tile.  And the MMA thread's loop costs about the same per K-block
+// whatever N, so the widest tile TMEM allows pays: 2×224 accumulator columns
+// plus the 4-column-aligned metadata slots of four stages (the sparse MMA
+// requires that alignment); 1.15 ms against 1.25 ms with 192 tokens and five
+// stages on the 70B layer at 4096 tokens.
 //
 // Warp roles: warp 0 lane 0 issues TMA; warp 1 owns TMEM and lane 0 issues
 // MMAs; warps 2-5 move metadata (or expand S) and run the epilogue.  The
@@ -389,7 +392,7 @@ __global__ void __launch_bounds__(192, 1)
 }
 
 // ---- sparse tensor-core prefill -------------------------------------------------
-// Yᵀ tile [256 rows of W × 192 tokens]: two 128-row accumulators in TMEM share
+// Yᵀ tile [256 rows of W × 224 tokens]: two 128-row accumulators in TMEM share
 // every X tile (half the X traffic of one 128-row tile per flop).  K-blocks of
 // 64 logical columns: A = the compressed 2:4 values of all 256 rows in one TMA
 // (64-byte swizzle, 32 values per row, 16 KB: a copy instruction costs a
@@ -400,33 +403,36 @@ __global__ void __launch_bounds__(192, 1)
 // (tcgen05.st) from a layout built at pack time, one 8-byte word pair per TMEM
 // lane; each MMA's metadata column is 4-column aligned (a requirement of the
 // sparse MMA's metadata address).  The low-rank tail runs dense MMAs on
-// U [256 × 32] and Z [192 × 32] K-blocks (64-byte swizzle) into the same
+// U [256 × 32] and Z [224 × 32] K-blocks (64-byte swizzle) into the same
 // accumulators.
-constexpr int SP_BN = 192, SP_STAGES = 5;
+constexpr int SP_BN = 224, SP_STAGES = 4;
 constexpr int SP_A_HALF = 128 * 64;        // 128 rows × 64 bytes
 constexpr int SP_A = 2 * SP_A_HALF;        // 16 KB
-constexpr int SP_B = SP_BN * 128;          // 24 KB (X: 192 rows × 64 bf16)
-constexpr int SP_B_Z = SP_BN * 64;         // Z: 192 rows × 32 bf16
+constexpr int SP_B = SP_BN * 128;          // 28 KB (X: 224 rows × 64 bf16)
+constexpr int SP_B_Z = SP_BN * 64;         // Z: 224 rows × 32 bf16
 constexpr int SP_M = 2 * 128 * 8;           // metadata of the stage: 2 halves × 128 lanes × 8 B
 constexpr int SP_STAGE = SP_A + SP_B + SP_M;
 constexpr int SP_SMEM = SP_STAGES * SP_STAGE + 1024 + 256;
-// TMEM columns: accumulator 0 [0, 192), accumulator 1 [256, 448); metadata
-// slots of 4 columns, one per (stage, half, MMA): 16 in [192, 256), the rest in
-// [448, 512).
+// TMEM columns: accumulator 0 [0, SP_BN), accumulator 1 [256, 256 + SP_BN);
+// metadata slots of 4 columns, one per (stage, half, MMA), in the gaps
+// [SP_BN, 256) and [256 + SP_BN, 512).
 constexpr uint32_t SP_ACC1_COL = 256;
+constexpr int SP_GAP_SLOTS = (256 - SP_BN) / 4;  // slots in each gap
 __device__ __forceinline__ uint32_t sp_meta_col(int s, int h, int i) {
   const uint32_t slot = uint32_t(s * 4 + h * 2 + i);
-  return slot < 16 ? 192u + 4u * slot : 448u + 4u * (slot - 16u);
+  return slot < uint32_t(SP_GAP_SLOTS) ? uint32_t(SP_BN) + 4u * slot
+                                       : 256u + uint32_t(SP_BN) + 4u * (slot - SP_GAP_SLOTS);
 }
-static_assert(SP_STAGES * 4 <= 32, "metadata slots");
+static_assert(SP_BN % 16 == 0 && SP_BN <= 256 && SP_STAGES * 4 <= 2 * SP_GAP_SLOTS,
+              "accumulators and metadata slots fit TMEM");
 
 struct SpMaps {
-  CUtensorMap x;   // X [T][n]       box {64, 192} SW128
+  CUtensorMap x;   // X [T][n]       box {64, SP_BN} SW128
   CUtensorMap sv;  // S values [m][n/2] box {32, 256} SW64
   CUtensorMap u;   // U [m][r_pad]   box {32, 256} SW64
-  CUtensorMap z;   // Z hi [T][r16]  box {32, 192} SW64
-  CUtensorMap zlo; // Z lo [T][r16]  box {32, 192} SW64
-  CUtensorMap y;   // Y [T][m]       box {256, 192}, no swizzle (the epilogue's tile store)
+  CUtensorMap z;   // Z hi [T][r16]  box {32, SP_BN} SW64
+  CUtensorMap zlo; // Z lo [T][r16]  box {32, SP_BN} SW64
+  CUtensorMap y;   // Y [T][m]       box {256, SP_BN}, no swizzle (the epilogue's tile store)
 };
 // bytes of the staged output tile: [SP_BN tokens][256 rows] bf16, in the ring
 constexpr int SP_Y_STAGE = SP_BN * 256 * 2;
