@@ -397,12 +397,14 @@ __global__ void __launch_bounds__(192, 1)
 // 64 logical columns: A = the compressed 2:4 values of all 256 rows in one TMA
 // (64-byte swizzle, 32 values per row, 16 KB: a copy instruction costs a
 // near-fixed time, so two 8 KB copies took about twice as long), B = X (TMA,
-// 128-byte swizzle), two tcgen05.mma.sp of K = 32 per half.  Two threads issue
-// the copies of a stage, both arriving on its barrier: warp 0 the A tile,
-// warp 6 the B tile and the metadata, so their copy instructions overlap.  The metadata of a K-block is copied into TMEM by four warps
-// (tcgen05.st) from a layout built at pack time, one 8-byte word pair per TMEM
-// lane; each MMA's metadata column is 4-column aligned (a requirement of the
-// sparse MMA's metadata address).  The low-rank tail runs dense MMAs on
+// 128-byte swizzle), two tcgen05.mma.sp of K = 32 per half.  Three threads
+// issue the copies of a stage (warp 0 the A tile, warp 6 the B tile, warp 7 the
+// metadata on its own barrier), so their copy instructions overlap.  Four warps
+// put a K-block's metadata into TMEM (tcgen05.st) from a layout built at pack
+// time, one 8-byte word pair per TMEM lane, and arrive on the stage's data
+// barrier, so the MMA thread waits on one barrier per K-block; each MMA's
+// metadata column is 4-column aligned (a requirement of the sparse MMA's
+// metadata address).  The low-rank tail runs dense MMAs on
 // U [256 × 32] and Z [224 × 32] K-blocks (64-byte swizzle) into the same
 // accumulators.
 constexpr int SP_BN = 224, SP_STAGES = 4;
