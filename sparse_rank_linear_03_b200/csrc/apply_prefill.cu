@@ -994,7 +994,8 @@ bool tmap_available() { return encode_fn() != nullptr; }
 constexpr int64_t kPairMinTokens = 512;
 // HSL_PREFILL_PAIRS=1 selects the CTA-pair kernel.  It is exact (the parity
 // tests cover it) but measured slower than the single-CTA kernel on the 70B
-// layer (3.2 ms against 1.66 ms for 4096 tokens), so it is not the default.
+// layer (3.2 ms, measured against 1.66 ms for the single-CTA kernel of that time;
+// that kernel now takes 1.15 ms), so it is not the default.
 bool prefill_pairs_enabled() {
   const char* e = std::getenv("HSL_PREFILL_PAIRS");
   return e != nullptr && e[0] == '1';
